@@ -1,0 +1,277 @@
+/*
+ * mk.h -- C ABI of the persistent decode megakernel for B200 (sm_100a).
+ *
+ * One autoregressive decode step of a Llama-style decoder (dense, or with a
+ * routed mixture of experts) runs as ONE persistent kernel: exactly one CTA
+ * per SM stays resident for the whole step, CTAs pull per-tile tasks from a
+ * task list that the host builds once, and event counters in global memory
+ * take the place of kernel boundaries.
+ *
+ * Sources for the operation (titles of the pages this follows):
+ *  - "Cohere megakerneles kiszolgálót mutatott be a North Mini Code
+ *    modellhez", section "Egyetlen tartós kernelre épül a kiszolgálás": one
+ *    threadblock per SM resident for the whole decode step; blocks work from a
+ *    host-prepared task list; global-memory counters signal dependencies; the
+ *    scheduling unit is one tile of one operation.
+ *  - same page, section "Honnan jön a gyorsulás?": no per-operation wave
+ *    quantization; O-projection of a KV group may start when that group's
+ *    attention is done; expert down-projection depends only on its own up-
+ *    projection; weight tiles are prefetched before the activation dependency.
+ *  - same page, section "Folyamatos batchkezelés, paged attention ...":
+ *    continuous batching, paged attention, ragged sequences.
+ *  - "LLM को MegaKernel में compile करके low-latency inference हासिल करना"
+ *    (MPK digest), sections "Part 1. Compiler" (operator graph -> fine-grained
+ *    task graph; events as synchronisation points) and "Part 2. Runtime"
+ *    ("Event-आधारित execution तरीका": a finished task increments its event
+ *    counter; the event fires when the counter reaches its threshold).
+ *
+ * Conventions for every entry point:
+ *  - Return MK_OK or an error code; mk_last_error_string() describes the last
+ *    error of the calling thread.  No entry point aborts the process.
+ *  - "device pointer" = memory of the current CUDA device; "host pointer" =
+ *    ordinary host memory.  The library never frees memory it did not
+ *    allocate.
+ *  - Kernels run asynchronously on the given stream.  Errors that the host
+ *    can see (null pointers, sizes out of range) are returned before any
+ *    launch.  Errors found on the device (a wait that timed out, a position,
+ *    token id or page index out of range) set a device status word that the
+ *    next mk_sync() or mk_decode_step() on the same state returns.
+ *  - A state is not thread-safe: one host thread and one stream per state.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MK_OK = 0,
+    MK_ERR_INVALID_ARG = 1,   /* bad argument (host check) or bad index (device check) */
+    MK_ERR_CUDA = 2,          /* a CUDA runtime call failed */
+    MK_ERR_OOM = 3,           /* device allocation failed */
+    MK_ERR_UNSUPPORTED = 4,   /* shape or option this build does not support */
+    MK_ERR_TIMEOUT = 5,       /* a device-side wait exceeded its time limit */
+    MK_ERR_DEVICE_FAULT = 6   /* the device reported an inconsistent state */
+} mk_status;
+
+typedef struct mk_model mk_model;   /* weights (borrowed) + shape */
+typedef struct mk_graph mk_graph;   /* host-built task list + event table */
+typedef struct mk_state mk_state;   /* per-stream device state of one graph */
+
+/* Any cudaStream_t may be passed where an mk_stream is expected (0 = legacy default). */
+typedef struct CUstream_st* mk_stream;
+
+#define MK_DTYPE_BF16 0
+
+/* Flags of mk_model_desc.flags */
+#define MK_FLAG_TRACE 0x1u   /* record per-task timestamps (mk_state_read_trace) */
+
+/* Model shape.  n_experts == 0 selects the dense SiLU-gated FFN of width ffn;
+ * n_experts > 0 selects a routed MoE with top_k experts of width expert_ffn
+ * (router softmax over all experts; top-k ties to the lower expert index;
+ * selected weights renormalised to sum 1 when moe_renorm != 0). */
+typedef struct {
+    int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+    float rms_eps, rope_theta;
+    int n_experts, top_k, expert_ffn, moe_renorm;
+    int dtype;        /* MK_DTYPE_BF16 only */
+    unsigned flags;   /* MK_FLAG_* */
+} mk_model_desc;
+
+/* Paged KV cache, owned by the caller, device memory.
+ *   k_pages, v_pages: bf16 [n_layers][n_pages][n_kv_heads][page_size][head_dim]
+ *     (within a page, each KV head's page_size x head_dim block is contiguous)
+ *   page_table: int32 [batch][max_pages_per_seq]; entry j of row b is the
+ *     physical page holding positions 16j..16j+15 of sequence b.
+ * The library never allocates pages: the caller guarantees that every page
+ * the step touches (positions 0..positions[b]) is mapped. */
+typedef struct {
+    void* k_pages;
+    void* v_pages;
+    const int32_t* page_table;
+    int n_pages;
+    int page_size;          /* must be 16 */
+    int max_pages_per_seq;
+} mk_paged_kv;
+
+/* ---------------------------------------------------------------- model */
+
+/* Records the shape and the weight pointers (device, bf16, row-major
+ * [out][in]).  Order of weight_ptrs: tok_emb [vocab][hidden]; then per layer
+ * attn_norm [hidden], wq [n_q*d][hidden], wk [n_kv*d][hidden], wv
+ * [n_kv*d][hidden], wo [hidden][n_q*d], ffn_norm [hidden], then dense:
+ * w_gate [ffn][hidden], w_up [ffn][hidden], w_down [hidden][ffn]; or MoE:
+ * w_router [E][hidden], w_gate [E][Fe][hidden], w_up [E][Fe][hidden],
+ * w_down [E][hidden][Fe]; then final_norm [hidden], lm_head [vocab][hidden].
+ * n_ptrs must equal 1 + n_layers*(9 dense | 10 MoE) + 2.  Weights are
+ * borrowed: the caller keeps them alive and unchanged until
+ * mk_model_destroy.  Every pointer must be 16-byte aligned.
+ * Supported: head_dim in {64, 128}, n_q_heads a multiple of n_kv_heads,
+ * hidden, ffn, expert_ffn and n_q*d multiples of 8, top_k <= 16. */
+mk_status mk_load_model(const mk_model_desc* desc, const void* const* weight_ptrs, int n_ptrs,
+                        mk_model** out);
+void mk_model_destroy(mk_model* model);
+
+/* ---------------------------------------------------------------- task graph */
+
+/* Builds the task list for batches up to max_batch and contexts up to max_ctx
+ * tokens (positions 0..max_ctx-1) on the current device (its SM count sets
+ * the tile sizes and the grid) and uploads it.  Operator graph -> per-tile
+ * tasks; a task depends on the tasks whose output rows overlap its input
+ * rows (MPK digest, "Part 1. Compiler"; HN thread answer on task granularity
+ * and dependency analysis). */
+mk_status mk_build_taskgraph(mk_model* model, int max_batch, int max_ctx, mk_graph** out);
+
+/* The same plan on the host only (no device memory, no CUDA call), for an
+ * SM count given by the caller: for inspecting and checking the graph. */
+mk_status mk_plan_taskgraph(const mk_model_desc* desc, int max_batch, int max_ctx, int n_sm,
+                            mk_graph** out);
+void mk_graph_destroy(mk_graph* graph);
+
+typedef struct {
+    int n_tasks, n_events, n_sm, max_batch, max_ctx;
+    int attn_splits;       /* split-K factor of decode attention per (sequence, kv head) */
+    int n_ops;             /* operator kinds used (see mk_task_info.op) */
+    int64_t weight_bytes_per_step;   /* bf16 weight bytes streamed by one B=1 step (dense: all
+                                        but the embedding table; MoE: router + top_k experts) */
+} mk_graph_info;
+mk_status mk_graph_get_info(const mk_graph* graph, mk_graph_info* info);
+
+/* Operator kinds of a task. */
+enum {
+    MK_OP_QKV = 1,        /* rows of [Wq;Wk;Wv] . rmsnorm(x)           */
+    MK_OP_ATTN = 2,       /* decode attention split (b, kv head, split) */
+    MK_OP_OPROJ = 3,      /* rows of Wo . o, plus the residual          */
+    MK_OP_GATEUP = 4,     /* rows of silu(Wg h) * (Wu h)                */
+    MK_OP_DOWN = 5,       /* rows of Wd . a, plus the residual          */
+    MK_OP_LMHEAD = 6,     /* rows of Wlm . rmsnorm(x)                   */
+    MK_OP_ROUTER = 7,     /* rows of Wr . rmsnorm(x); last tile: top-k  */
+    MK_OP_EXP_GATEUP = 8, /* expert slot k: rows of silu(Wg_e h)*(Wu_e h) */
+    MK_OP_EXP_DOWN = 9    /* expert slot k: rows of Wd_e . a_e          */
+};
+
+#define MK_NO_EVENT 0xFFFFFFFFu
+
+/* One task as the device sees it.  Rows [r0, r1) of the operator's output;
+ * for MK_OP_ATTN r0 is the split index and r1 the split count; b is the batch
+ * row (MK_OP_ATTN / expert ops) and aux the kv head or expert slot.  The task
+ * waits until counter[wait[i]] >= threshold[wait[i]] * epoch, then signals
+ * counter[signal] += 1 (attention splits: only the last split of a
+ * (b, kv head) signals, after merging the partial results; router tiles: only
+ * the last tile of a layer, after selecting the experts).  Expert tasks also
+ * wait on pointer_wait (the router's event) before the weight address of the
+ * routed expert is read; MK_NO_EVENT elsewhere. */
+typedef struct {
+    int op, layer, b, aux;
+    uint32_t r0, r1;
+    uint32_t wait[2];
+    uint32_t signal;
+    uint32_t pointer_wait;
+} mk_task_info;
+
+/* Copies min(cap, n_tasks) tasks in list order; returns the count written via *n. */
+mk_status mk_graph_export_tasks(const mk_graph* graph, mk_task_info* out, int cap, int* n);
+/* thresholds[e] for e < n_events (per step). */
+mk_status mk_graph_export_thresholds(const mk_graph* graph, uint32_t* out, int cap, int* n);
+
+/* Wave-quantisation arithmetic used by the tile sizer: n_tiles equal tiles on
+ * n_sm SMs take ceil(n_tiles / n_sm) waves and leave idle SMs in the last
+ * wave (Cohere page, "Honnan jön a gyorsulás?": 200 tiles on 132 SMs -> 2
+ * waves, 64 SMs idle). */
+mk_status mk_wave_stats(int n_tiles, int n_sm, int* waves, int* idle_sms_last_wave);
+
+/* ---------------------------------------------------------------- state and steps */
+
+/* Allocates the device state of a graph (event counters, work-queue head,
+ * activation buffers, attention partials): library-owned until
+ * mk_state_destroy. */
+mk_status mk_state_create(mk_graph* graph, mk_state** out);
+void mk_state_destroy(mk_state* state);
+
+/* Device-side wait limit in nanoseconds (default 2e9).  A wait that exceeds
+ * it sets MK_ERR_TIMEOUT; the kernel then drains and returns. */
+mk_status mk_state_set_timeout(mk_state* state, int64_t timeout_ns);
+
+/* Test hook for failure detection: adds `offset` to the target of every
+ * device-side event wait of later steps (0 = normal).  With offset 1 no wait
+ * can be satisfied, so the step ends with MK_ERR_TIMEOUT after the state's
+ * timeout, without faulting or hanging the device. */
+mk_status mk_state_debug_wait_offset(mk_state* state, uint32_t offset);
+
+/* One decode step for `batch` sequences (1 <= batch <= max_batch).
+ *   token_ids  device int32 [batch]: the token fed to each sequence
+ *   positions  device int32 [batch]: its position = tokens already cached
+ *              (0 <= positions[b] < max_ctx); the step writes K/V at that
+ *              position and attends to positions 0..positions[b]
+ *   kv         paged cache (see mk_paged_kv); page_table rows 0..batch-1
+ *   logits_out device fp32 [batch][vocab]
+ * One kernel launch on `stream`.  Returns a device error recorded by an
+ * earlier step of this state, if any (the state is then reset). */
+mk_status mk_decode_step(mk_state* state, const int32_t* token_ids, const int32_t* positions,
+                         int batch, const mk_paged_kv* kv, float* logits_out, mk_stream stream);
+
+/* Same step with HOST inputs and outputs: copies token_ids and positions
+ * (host int32 [batch]) to the device, runs the step, copies the logits back
+ * to logits_host (host fp32 [batch][vocab]) and waits for the stream. */
+mk_status mk_decode_step_host(mk_state* state, const int32_t* token_ids, const int32_t* positions,
+                              int batch, const mk_paged_kv* kv, float* logits_host,
+                              mk_stream stream);
+
+/* Runs a prompt through the same graph, one token per step, for ONE sequence
+ * whose page-table row is kv->page_table[0]: tokens (device int32
+ * [n_tokens]) at positions pos0 .. pos0+n_tokens-1.  Writes the logits of
+ * the last prompt token to last_logits (device fp32 [vocab]); the LM head is
+ * skipped for the other tokens. */
+mk_status mk_prefill(mk_state* state, const int32_t* tokens, int n_tokens, int pos0,
+                     const mk_paged_kv* kv, float* last_logits, mk_stream stream);
+
+/* Waits for the stream and returns the device status word of the last step
+ * (MK_OK, MK_ERR_TIMEOUT, MK_ERR_INVALID_ARG, ...). */
+mk_status mk_sync(mk_state* state, mk_stream stream);
+
+/* ---------------------------------------------------------------- inspection */
+
+typedef struct {
+    uint32_t epoch;            /* steps completed since creation or reset */
+    uint32_t done;             /* tasks completed, total (= n_tasks * epoch) */
+    uint64_t queue_head;       /* work-queue head (= (n_tasks + n_sm) * epoch) */
+    int32_t error;             /* device status word */
+    int32_t error_info[4];     /* where: task, event, value, detail */
+} mk_state_counters;
+
+/* Synchronises the stream, then copies the counters; events (host uint32
+ * [n_events]) may be NULL. */
+mk_status mk_state_read_counters(mk_state* state, mk_stream stream, mk_state_counters* c,
+                                 uint32_t* events, int cap);
+
+/* Copies an activation buffer of the last step to host fp32 memory.
+ *   which 0: residual after attention  [batch][hidden] of `layer`
+ *         1: residual after the FFN    [batch][hidden] of `layer`
+ *            (MoE: combined on the host side of this call is NOT done; the
+ *            buffer holds the dense residual only for dense models)
+ *         2: merged attention output   [batch][n_q*d]  of `layer`
+ *         3: MoE selected experts of `layer` as fp32 [batch][top_k]
+ *         4: MoE combine weights of `layer`          [batch][top_k]
+ * n = number of floats to copy. */
+mk_status mk_state_read_buffer(mk_state* state, int which, int layer, float* host, size_t n,
+                               mk_stream stream);
+
+/* Per-task trace of the last step (needs MK_FLAG_TRACE): host uint64
+ * [n_tasks][4] = {wait start ns, compute start ns, end ns, sm id}. */
+mk_status mk_state_read_trace(mk_state* state, uint64_t* host, int cap_tasks, mk_stream stream);
+
+/* Text of the last error of the calling thread ("" if none). */
+const char* mk_last_error_string(void);
+
+/* Library version string. */
+const char* mk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MK_H */

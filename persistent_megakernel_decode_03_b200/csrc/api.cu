@@ -1,0 +1,606 @@
+// C ABI of the decode megakernel (declared in include/mk.h): model
+// registration, task-graph build and upload, per-stream state, decode steps.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "graph.h"
+#include "megakernel.h"
+#include "mk_internal.h"
+
+using mk::GraphPlan;
+
+struct mk_model {
+    mk_model_desc desc{};
+    int device = 0;
+    std::vector<const void*> w;
+    std::vector<mk::LayerW> h_layers;
+    mk::LayerW* d_layers = nullptr;
+};
+
+struct mk_graph {
+    GraphPlan plan;
+    mk_model* model = nullptr;   // null for a host-only plan
+    int device = -1;
+    mk::Task* d_tasks = nullptr;
+    uint32_t* d_thr = nullptr;
+    float* d_rope = nullptr;
+};
+
+struct mk_state {
+    mk_graph* g = nullptr;
+    uint32_t epoch = 0;
+    bool needs_reset = false;
+    long long timeout_ns = 2000000000LL;
+    uint32_t wait_offset = 0;
+    // device memory
+    uint32_t* events = nullptr;
+    unsigned long long* queue = nullptr;
+    uint32_t* done = nullptr;
+    int* err = nullptr;
+    uint32_t* merge_cnt = nullptr;
+    uint32_t* router_cnt = nullptr;
+    float *x_mid = nullptr, *x_out = nullptr, *qkv = nullptr, *o = nullptr, *act = nullptr;
+    float *part = nullptr, *rlogits = nullptr, *moe_w = nullptr, *ypart = nullptr;
+    int* moe_sel = nullptr;
+    int32_t* tokpos = nullptr;     // host-input variant: [2][max_batch]
+    float* logits = nullptr;       // host-output variant: [max_batch][vocab]
+    unsigned long long* trace = nullptr;
+    std::vector<void*> allocs;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+mk_status fail(mk_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+mk_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(e == cudaErrorMemoryAllocation ? MK_ERR_OOM : MK_ERR_CUDA, "%s: %s", what,
+                cudaGetErrorString(e));
+}
+
+int slots_per_layer(const mk_model_desc& d) { return d.n_experts > 0 ? 10 : 9; }
+
+template <typename T>
+mk_status dev_alloc(mk_state* s, T** p, size_t count) {
+    if (count == 0) count = 1;
+    void* v = nullptr;
+    cudaError_t e = cudaMalloc(&v, count * sizeof(T));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc");
+    e = cudaMemset(v, 0, count * sizeof(T));
+    if (e != cudaSuccess) {
+        cudaFree(v);
+        return cuda_fail(e, "cudaMemset");
+    }
+    s->allocs.push_back(v);
+    *p = static_cast<T*>(v);
+    return MK_OK;
+}
+
+void free_state_memory(mk_state* s) {
+    for (void* v : s->allocs) cudaFree(v);
+    s->allocs.clear();
+}
+
+mk_status reset_counters(mk_state* s, cudaStream_t st) {
+    const GraphPlan& P = s->g->plan;
+    const mk_model_desc& d = P.desc;
+    cudaError_t e = cudaMemsetAsync(s->events, 0, sizeof(uint32_t) * std::max(1, P.n_events), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s->queue, 0, sizeof(unsigned long long), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s->done, 0, sizeof(uint32_t), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s->err, 0, sizeof(int) * 8, st);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(s->merge_cnt, 0,
+                            sizeof(uint32_t) * (size_t)d.n_layers * P.max_batch * d.n_kv_heads, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s->router_cnt, 0, sizeof(uint32_t) * d.n_layers, st);
+    if (e != cudaSuccess) return cuda_fail(e, "reset");
+    s->epoch = 0;
+    s->needs_reset = false;
+    return MK_OK;
+}
+
+mk_status check_kv(const mk_state* s, const mk_paged_kv* kv) {
+    if (!kv || !kv->k_pages || !kv->v_pages || !kv->page_table)
+        return fail(MK_ERR_INVALID_ARG, "paged KV: null pointer");
+    if (kv->page_size != mk::kPageSize) return fail(MK_ERR_INVALID_ARG, "paged KV: page_size must be 16");
+    if (kv->n_pages < 1 || kv->max_pages_per_seq < 1)
+        return fail(MK_ERR_INVALID_ARG, "paged KV: n_pages and max_pages_per_seq must be >= 1");
+    if (((uintptr_t)kv->k_pages | (uintptr_t)kv->v_pages) & 15)
+        return fail(MK_ERR_INVALID_ARG, "paged KV: pools must be 16-byte aligned");
+    (void)s;
+    return MK_OK;
+}
+
+mk::Params base_params(mk_state* s) {
+    const GraphPlan& P = s->g->plan;
+    const mk_model_desc& d = P.desc;
+    const mk_model* m = s->g->model;
+    mk::Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.tasks = s->g->d_tasks;
+    p.n_tasks = (uint32_t)P.tasks.size();
+    p.thr = s->g->d_thr;
+    p.events = s->events;
+    p.queue = s->queue;
+    p.done = s->done;
+    p.err = s->err;
+    p.merge_cnt = s->merge_cnt;
+    p.router_cnt = s->router_cnt;
+    p.timeout_ns = s->timeout_ns;
+    p.wait_offset = s->wait_offset;
+    p.trace = s->trace;
+    p.layers = m->d_layers;
+    const int L = d.n_layers;
+    p.tok_emb = static_cast<const uint16_t*>(m->w[0]);
+    p.final_norm = static_cast<const uint16_t*>(m->w[1 + L * slots_per_layer(d)]);
+    p.lm_head = static_cast<const uint16_t*>(m->w[2 + L * slots_per_layer(d)]);
+    p.L = L;
+    p.H = d.hidden;
+    p.nq = d.n_q_heads;
+    p.nkv = d.n_kv_heads;
+    p.hd = d.head_dim;
+    p.F = d.ffn;
+    p.V = d.vocab;
+    p.E = d.n_experts;
+    p.topk = d.top_k;
+    p.Fe = d.expert_ffn;
+    p.renorm = d.moe_renorm;
+    p.eps = d.rms_eps;
+    p.max_ctx = P.max_ctx;
+    p.max_batch = P.max_batch;
+    p.S = P.S;
+    p.n_router_tiles = P.n_router_tiles;
+    p.rope = s->g->d_rope;
+    p.x_mid = s->x_mid;
+    p.x_out = s->x_out;
+    p.qkv = s->qkv;
+    p.o = s->o;
+    p.act = s->act;
+    p.part = s->part;
+    p.rlogits = s->rlogits;
+    p.moe_w = s->moe_w;
+    p.moe_sel = s->moe_sel;
+    p.ypart = s->ypart;
+    return p;
+}
+
+mk_status launch_step(mk_state* s, mk::Params& p, cudaStream_t st) {
+    if (s->needs_reset) {
+        mk_status r = reset_counters(s, st);
+        if (r != MK_OK) return r;
+    }
+    const GraphPlan& P = s->g->plan;
+    s->epoch += 1;
+    p.epoch = s->epoch;
+    p.queue_base = (unsigned long long)(s->epoch - 1) * (P.tasks.size() + (size_t)P.n_sm);
+    cudaError_t e = mk::megakernel_launch(p, P.n_sm, st);
+    if (e != cudaSuccess) {
+        s->needs_reset = true;
+        return cuda_fail(e, "megakernel launch");
+    }
+    return MK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mk_last_error_string(void) { return g_err.c_str(); }
+const char* mk_version(void) { return "mk 0.1 (sm_100a persistent decode megakernel)"; }
+
+mk_status mk_wave_stats(int n_tiles, int n_sm, int* waves, int* idle) {
+    if (n_tiles < 0 || n_sm < 1 || !waves || !idle) return fail(MK_ERR_INVALID_ARG, "wave_stats: bad argument");
+    mk::wave_stats(n_tiles, n_sm, waves, idle);
+    return MK_OK;
+}
+
+// ---------------------------------------------------------------- model
+
+mk_status mk_load_model(const mk_model_desc* desc, const void* const* wp, int n_ptrs, mk_model** out) {
+    if (!desc || !wp || !out) return fail(MK_ERR_INVALID_ARG, "mk_load_model: null argument");
+    *out = nullptr;
+    const mk_model_desc& d = *desc;
+    std::string err;
+    if (!mk::validate_desc(d, err)) return fail(MK_ERR_UNSUPPORTED, "mk_load_model: %s", err.c_str());
+    if (!mk::megakernel_supports(d.n_q_heads / d.n_kv_heads, d.head_dim))
+        return fail(MK_ERR_UNSUPPORTED, "mk_load_model: heads per group must be 1, 2, 4 or 8");
+    const int need = 1 + d.n_layers * slots_per_layer(d) + 2;
+    if (n_ptrs != need) return fail(MK_ERR_INVALID_ARG, "mk_load_model: expected %d weight pointers, got %d", need, n_ptrs);
+    for (int i = 0; i < n_ptrs; ++i) {
+        if (!wp[i]) return fail(MK_ERR_INVALID_ARG, "mk_load_model: weight pointer %d is null", i);
+        if ((uintptr_t)wp[i] & 15) return fail(MK_ERR_INVALID_ARG, "mk_load_model: weight pointer %d is not 16-byte aligned", i);
+    }
+    mk_model* m = new (std::nothrow) mk_model;
+    if (!m) return fail(MK_ERR_OOM, "mk_load_model: host allocation");
+    m->desc = d;
+    cudaGetDevice(&m->device);
+    m->w.assign(wp, wp + n_ptrs);
+    const int S = slots_per_layer(d);
+    for (int l = 0; l < d.n_layers; ++l) {
+        const void* const* q = wp + 1 + l * S;
+        mk::LayerW lw;
+        std::memset(&lw, 0, sizeof(lw));
+        lw.attn_norm = (const uint16_t*)q[0];
+        lw.wq = (const uint16_t*)q[1];
+        lw.wk = (const uint16_t*)q[2];
+        lw.wv = (const uint16_t*)q[3];
+        lw.wo = (const uint16_t*)q[4];
+        lw.ffn_norm = (const uint16_t*)q[5];
+        if (d.n_experts > 0) {
+            lw.w_router = (const uint16_t*)q[6];
+            lw.w_gate = (const uint16_t*)q[7];
+            lw.w_up = (const uint16_t*)q[8];
+            lw.w_down = (const uint16_t*)q[9];
+        } else {
+            lw.w_gate = (const uint16_t*)q[6];
+            lw.w_up = (const uint16_t*)q[7];
+            lw.w_down = (const uint16_t*)q[8];
+        }
+        m->h_layers.push_back(lw);
+    }
+    cudaError_t e = cudaMalloc(&m->d_layers, sizeof(mk::LayerW) * d.n_layers);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(m->d_layers, m->h_layers.data(), sizeof(mk::LayerW) * d.n_layers, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        if (m->d_layers) cudaFree(m->d_layers);
+        delete m;
+        return cuda_fail(e, "mk_load_model");
+    }
+    *out = m;
+    return MK_OK;
+}
+
+void mk_model_destroy(mk_model* m) {
+    if (!m) return;
+    if (m->d_layers) cudaFree(m->d_layers);
+    delete m;
+}
+
+// ---------------------------------------------------------------- graph
+
+mk_status mk_plan_taskgraph(const mk_model_desc* desc, int max_batch, int max_ctx, int n_sm, mk_graph** out) {
+    if (!desc || !out) return fail(MK_ERR_INVALID_ARG, "mk_plan_taskgraph: null argument");
+    *out = nullptr;
+    mk_graph* g = new (std::nothrow) mk_graph;
+    if (!g) return fail(MK_ERR_OOM, "mk_plan_taskgraph: host allocation");
+    std::string err;
+    if (!mk::plan_graph(*desc, max_batch, max_ctx, n_sm, g->plan, err)) {
+        delete g;
+        return fail(MK_ERR_UNSUPPORTED, "mk_plan_taskgraph: %s", err.c_str());
+    }
+    *out = g;
+    return MK_OK;
+}
+
+mk_status mk_build_taskgraph(mk_model* model, int max_batch, int max_ctx, mk_graph** out) {
+    if (!model || !out) return fail(MK_ERR_INVALID_ARG, "mk_build_taskgraph: null argument");
+    *out = nullptr;
+    int dev = 0, n_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_build_taskgraph: device query");
+    int coop = 0;
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+    if (!coop) return fail(MK_ERR_UNSUPPORTED, "mk_build_taskgraph: device lacks cooperative launch");
+    const mk_model_desc& d = model->desc;
+    int per_sm = 0;
+    e = mk::megakernel_occupancy(d.n_q_heads / d.n_kv_heads, d.head_dim, &per_sm);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_build_taskgraph: occupancy query");
+    if (per_sm < 1) return fail(MK_ERR_UNSUPPORTED, "mk_build_taskgraph: megakernel does not fit on one SM");
+    mk_graph* g = nullptr;
+    mk_status st = mk_plan_taskgraph(&d, max_batch, max_ctx, n_sm, &g);
+    if (st != MK_OK) return st;
+    g->model = model;
+    g->device = dev;
+    const GraphPlan& P = g->plan;
+    // RoPE table: cos/sin of pos * theta^(-2i/d), computed in double, stored fp32
+    const int half = d.head_dim / 2;
+    std::vector<float> rope((size_t)max_ctx * half * 2);
+    for (int pos = 0; pos < max_ctx; ++pos)
+        for (int i = 0; i < half; ++i) {
+            double inv = std::pow((double)d.rope_theta, -2.0 * i / (double)d.head_dim);
+            double a = (double)pos * inv;
+            rope[((size_t)pos * half + i) * 2 + 0] = (float)std::cos(a);
+            rope[((size_t)pos * half + i) * 2 + 1] = (float)std::sin(a);
+        }
+    e = cudaMalloc(&g->d_tasks, sizeof(mk::Task) * P.tasks.size());
+    if (e == cudaSuccess) e = cudaMalloc(&g->d_thr, sizeof(uint32_t) * std::max<size_t>(1, P.thr.size()));
+    if (e == cudaSuccess) e = cudaMalloc(&g->d_rope, sizeof(float) * rope.size());
+    if (e == cudaSuccess)
+        e = cudaMemcpy(g->d_tasks, P.tasks.data(), sizeof(mk::Task) * P.tasks.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !P.thr.empty())
+        e = cudaMemcpy(g->d_thr, P.thr.data(), sizeof(uint32_t) * P.thr.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(g->d_rope, rope.data(), sizeof(float) * rope.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        mk_graph_destroy(g);
+        return cuda_fail(e, "mk_build_taskgraph: upload");
+    }
+    *out = g;
+    return MK_OK;
+}
+
+void mk_graph_destroy(mk_graph* g) {
+    if (!g) return;
+    if (g->d_tasks) cudaFree(g->d_tasks);
+    if (g->d_thr) cudaFree(g->d_thr);
+    if (g->d_rope) cudaFree(g->d_rope);
+    delete g;
+}
+
+mk_status mk_graph_get_info(const mk_graph* g, mk_graph_info* info) {
+    if (!g || !info) return fail(MK_ERR_INVALID_ARG, "mk_graph_get_info: null argument");
+    const GraphPlan& P = g->plan;
+    info->n_tasks = (int)P.tasks.size();
+    info->n_events = P.n_events;
+    info->n_sm = P.n_sm;
+    info->max_batch = P.max_batch;
+    info->max_ctx = P.max_ctx;
+    info->attn_splits = P.S;
+    info->n_ops = P.desc.n_experts > 0 ? 7 : 6;
+    info->weight_bytes_per_step = P.weight_bytes;
+    return MK_OK;
+}
+
+mk_status mk_graph_export_tasks(const mk_graph* g, mk_task_info* out, int cap, int* n) {
+    if (!g || !n || (cap > 0 && !out)) return fail(MK_ERR_INVALID_ARG, "mk_graph_export_tasks: bad argument");
+    const auto& T = g->plan.tasks;
+    int k = std::min<int>(cap, (int)T.size());
+    for (int i = 0; i < k; ++i) {
+        out[i].op = T[i].op;
+        out[i].layer = T[i].layer;
+        out[i].b = T[i].b;
+        out[i].aux = T[i].aux;
+        out[i].r0 = T[i].r0;
+        out[i].r1 = T[i].r1;
+        out[i].wait[0] = T[i].wait0;
+        out[i].wait[1] = T[i].wait1;
+        out[i].signal = T[i].sig;
+        out[i].pointer_wait = T[i].pad;
+    }
+    *n = k;
+    return MK_OK;
+}
+
+mk_status mk_graph_export_thresholds(const mk_graph* g, uint32_t* out, int cap, int* n) {
+    if (!g || !n || (cap > 0 && !out)) return fail(MK_ERR_INVALID_ARG, "mk_graph_export_thresholds: bad argument");
+    int k = std::min<int>(cap, (int)g->plan.thr.size());
+    for (int i = 0; i < k; ++i) out[i] = g->plan.thr[i];
+    *n = k;
+    return MK_OK;
+}
+
+// ---------------------------------------------------------------- state
+
+mk_status mk_state_create(mk_graph* g, mk_state** out) {
+    if (!g || !out) return fail(MK_ERR_INVALID_ARG, "mk_state_create: null argument");
+    if (!g->model || !g->d_tasks) return fail(MK_ERR_INVALID_ARG, "mk_state_create: graph was planned on the host only");
+    *out = nullptr;
+    mk_state* s = new (std::nothrow) mk_state;
+    if (!s) return fail(MK_ERR_OOM, "mk_state_create: host allocation");
+    s->g = g;
+    const GraphPlan& P = g->plan;
+    const mk_model_desc& d = P.desc;
+    const size_t L = d.n_layers, B = P.max_batch, H = d.hidden;
+    const size_t qkvw = (size_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim;
+    const size_t hpg = d.n_q_heads / d.n_kv_heads;
+    mk_status st = MK_OK;
+#define ALLOC(ptr, n) if (st == MK_OK) st = dev_alloc(s, &s->ptr, (n))
+    ALLOC(events, (size_t)std::max(1, P.n_events));
+    ALLOC(queue, 1);
+    ALLOC(done, 1);
+    ALLOC(err, 8);
+    ALLOC(merge_cnt, L * B * d.n_kv_heads);
+    ALLOC(router_cnt, L);
+    ALLOC(x_mid, L * B * H);
+    ALLOC(x_out, L * B * H);
+    ALLOC(qkv, L * B * qkvw);
+    ALLOC(o, L * B * d.n_q_heads * d.head_dim);
+    if (d.n_experts > 0) {
+        ALLOC(act, L * B * d.top_k * d.expert_ffn);
+        ALLOC(rlogits, L * B * d.n_experts);
+        ALLOC(moe_w, L * B * d.top_k);
+        ALLOC(moe_sel, L * B * d.top_k);
+        ALLOC(ypart, L * B * d.top_k * H);
+    } else {
+        ALLOC(act, L * B * d.ffn);
+    }
+    ALLOC(part, L * B * d.n_kv_heads * P.S * hpg * (d.head_dim + 2));
+    ALLOC(tokpos, 2 * B);
+    ALLOC(logits, B * (size_t)d.vocab);
+    if (d.flags & MK_FLAG_TRACE) ALLOC(trace, P.tasks.size() * 4);
+#undef ALLOC
+    if (st != MK_OK) {
+        free_state_memory(s);
+        delete s;
+        return st;
+    }
+    *out = s;
+    return MK_OK;
+}
+
+void mk_state_destroy(mk_state* s) {
+    if (!s) return;
+    free_state_memory(s);
+    delete s;
+}
+
+mk_status mk_state_set_timeout(mk_state* s, int64_t ns) {
+    if (!s || ns < 1000) return fail(MK_ERR_INVALID_ARG, "mk_state_set_timeout: bad argument");
+    s->timeout_ns = ns;
+    return MK_OK;
+}
+
+mk_status mk_state_debug_wait_offset(mk_state* s, uint32_t offset) {
+    if (!s) return fail(MK_ERR_INVALID_ARG, "mk_state_debug_wait_offset: null state");
+    s->wait_offset = offset;
+    return MK_OK;
+}
+
+mk_status mk_decode_step(mk_state* s, const int32_t* token_ids, const int32_t* positions, int batch,
+                         const mk_paged_kv* kv, float* logits_out, mk_stream stream) {
+    if (!s || !token_ids || !positions || !logits_out) return fail(MK_ERR_INVALID_ARG, "mk_decode_step: null argument");
+    if (batch < 1 || batch > s->g->plan.max_batch)
+        return fail(MK_ERR_INVALID_ARG, "mk_decode_step: batch %d outside 1..%d", batch, s->g->plan.max_batch);
+    mk_status r = check_kv(s, kv);
+    if (r != MK_OK) return r;
+    mk::Params p = base_params(s);
+    p.tokens = token_ids;
+    p.positions = positions;
+    p.pos_offset = 0;
+    p.batch = batch;
+    p.skip_lm = 0;
+    p.k_pages = static_cast<uint16_t*>(kv->k_pages);
+    p.v_pages = static_cast<uint16_t*>(kv->v_pages);
+    p.page_table = kv->page_table;
+    p.n_pages = kv->n_pages;
+    p.max_pages = kv->max_pages_per_seq;
+    p.logits = logits_out;
+    return launch_step(s, p, (cudaStream_t)stream);
+}
+
+mk_status mk_decode_step_host(mk_state* s, const int32_t* token_ids, const int32_t* positions, int batch,
+                              const mk_paged_kv* kv, float* logits_host, mk_stream stream) {
+    if (!s || !token_ids || !positions || !logits_host) return fail(MK_ERR_INVALID_ARG, "mk_decode_step_host: null argument");
+    if (batch < 1 || batch > s->g->plan.max_batch)
+        return fail(MK_ERR_INVALID_ARG, "mk_decode_step_host: batch %d outside 1..%d", batch, s->g->plan.max_batch);
+    cudaStream_t st = (cudaStream_t)stream;
+    const int B = s->g->plan.max_batch;
+    cudaError_t e = cudaMemcpyAsync(s->tokpos, token_ids, sizeof(int32_t) * batch, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(s->tokpos + B, positions, sizeof(int32_t) * batch, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_decode_step_host: H2D");
+    mk_status r = mk_decode_step(s, s->tokpos, s->tokpos + B, batch, kv, s->logits, stream);
+    if (r != MK_OK) return r;
+    e = cudaMemcpyAsync(logits_host, s->logits, sizeof(float) * (size_t)batch * s->g->plan.desc.vocab,
+                        cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_decode_step_host: D2H");
+    return MK_OK;
+}
+
+mk_status mk_prefill(mk_state* s, const int32_t* tokens, int n_tokens, int pos0, const mk_paged_kv* kv,
+                     float* last_logits, mk_stream stream) {
+    if (!s || !tokens || !last_logits) return fail(MK_ERR_INVALID_ARG, "mk_prefill: null argument");
+    if (n_tokens < 1 || pos0 < 0 || pos0 + n_tokens > s->g->plan.max_ctx)
+        return fail(MK_ERR_INVALID_ARG, "mk_prefill: positions %d..%d outside the graph's context", pos0, pos0 + n_tokens - 1);
+    mk_status r = check_kv(s, kv);
+    if (r != MK_OK) return r;
+    for (int i = 0; i < n_tokens; ++i) {
+        mk::Params p = base_params(s);
+        p.tokens = tokens + i;
+        p.positions = nullptr;
+        p.pos_offset = pos0 + i;
+        p.batch = 1;
+        p.skip_lm = (i + 1 < n_tokens) ? 1 : 0;
+        p.k_pages = static_cast<uint16_t*>(kv->k_pages);
+        p.v_pages = static_cast<uint16_t*>(kv->v_pages);
+        p.page_table = kv->page_table;
+        p.n_pages = kv->n_pages;
+        p.max_pages = kv->max_pages_per_seq;
+        p.logits = last_logits;
+        r = launch_step(s, p, (cudaStream_t)stream);
+        if (r != MK_OK) return r;
+    }
+    return MK_OK;
+}
+
+mk_status mk_sync(mk_state* s, mk_stream stream) {
+    if (!s) return fail(MK_ERR_INVALID_ARG, "mk_sync: null state");
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_sync");
+    int err[8];
+    e = cudaMemcpy(err, s->err, sizeof(err), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_sync: status read");
+    if (err[0] != 0) {
+        s->needs_reset = true;
+        return fail((mk_status)err[0], "device status %d (task %d, event/where %d, value %d, detail %d)", err[0],
+                    err[1], err[2], err[3], err[4]);
+    }
+    return MK_OK;
+}
+
+// ---------------------------------------------------------------- inspection
+
+mk_status mk_state_read_counters(mk_state* s, mk_stream stream, mk_state_counters* c, uint32_t* events, int cap) {
+    if (!s || !c) return fail(MK_ERR_INVALID_ARG, "mk_state_read_counters: null argument");
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    int err[8];
+    unsigned long long q = 0;
+    uint32_t done = 0;
+    if (e == cudaSuccess) e = cudaMemcpy(err, s->err, sizeof(err), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(&q, s->queue, sizeof(q), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(&done, s->done, sizeof(done), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && events && cap > 0)
+        e = cudaMemcpy(events, s->events, sizeof(uint32_t) * std::min(cap, s->g->plan.n_events), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_state_read_counters");
+    c->epoch = s->epoch;
+    c->done = done;
+    c->queue_head = q;
+    c->error = err[0];
+    for (int i = 0; i < 4; ++i) c->error_info[i] = err[1 + i];
+    return MK_OK;
+}
+
+mk_status mk_state_read_buffer(mk_state* s, int which, int layer, float* host, size_t n, mk_stream stream) {
+    if (!s || !host) return fail(MK_ERR_INVALID_ARG, "mk_state_read_buffer: null argument");
+    const GraphPlan& P = s->g->plan;
+    const mk_model_desc& d = P.desc;
+    if (layer < 0 || layer >= d.n_layers) return fail(MK_ERR_INVALID_ARG, "mk_state_read_buffer: bad layer");
+    const size_t B = P.max_batch;
+    const void* src = nullptr;
+    size_t avail = 0;
+    std::vector<int> tmp;
+    switch (which) {
+        case 0: src = s->x_mid + layer * B * d.hidden; avail = B * d.hidden; break;
+        case 1: src = s->x_out + layer * B * d.hidden; avail = B * d.hidden; break;
+        case 2: src = s->o + layer * B * d.n_q_heads * d.head_dim; avail = B * d.n_q_heads * d.head_dim; break;
+        case 3:
+        case 4:
+            if (d.n_experts == 0) return fail(MK_ERR_INVALID_ARG, "mk_state_read_buffer: not an MoE model");
+            avail = B * d.top_k;
+            src = (which == 3) ? (const void*)(s->moe_sel + layer * avail) : (const void*)(s->moe_w + layer * avail);
+            break;
+        default: return fail(MK_ERR_INVALID_ARG, "mk_state_read_buffer: bad buffer id");
+    }
+    if (n > avail) return fail(MK_ERR_INVALID_ARG, "mk_state_read_buffer: %zu floats requested, %zu available", n, avail);
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess) {
+        if (which == 3) {
+            tmp.resize(n);
+            e = cudaMemcpy(tmp.data(), src, sizeof(int) * n, cudaMemcpyDeviceToHost);
+            for (size_t i = 0; i < n; ++i) host[i] = (float)tmp[i];
+        } else {
+            e = cudaMemcpy(host, src, sizeof(float) * n, cudaMemcpyDeviceToHost);
+        }
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "mk_state_read_buffer");
+    return MK_OK;
+}
+
+mk_status mk_state_read_trace(mk_state* s, uint64_t* host, int cap_tasks, mk_stream stream) {
+    if (!s || !host) return fail(MK_ERR_INVALID_ARG, "mk_state_read_trace: null argument");
+    if (!s->trace) return fail(MK_ERR_INVALID_ARG, "mk_state_read_trace: model was loaded without MK_FLAG_TRACE");
+    int n = std::min<int>(cap_tasks, (int)s->g->plan.tasks.size());
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaMemcpy(host, s->trace, sizeof(uint64_t) * 4 * n, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_state_read_trace");
+    return MK_OK;
+}
+
+}  // extern "C"

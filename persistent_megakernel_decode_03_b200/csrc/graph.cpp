@@ -1,0 +1,333 @@
+// Host task-graph compiler: operator graph of one decode step -> per-tile
+// tasks in a topological list + event counters with per-step thresholds.
+//
+// Follows the MPK digest ("LLM को MegaKernel में compile करके low-latency
+// inference हासिल करना", section "Part 1. Compiler"): each operator is split
+// into tasks of about one threadblock's work, events are the synchronisation
+// points between tasks, and (HN thread "Compiling LLMs into a MegaKernel",
+// answer #58) task B depends on task A when A's output elements overlap B's
+// inputs.  Tile sizes avoid per-operator wave quantisation on the device's SM
+// count (Cohere page, section "Honnan jön a gyorsulás?"), and dependencies
+// stay at producer granularity: attention of one KV head waits only for the
+// QKV tiles of that head's rows, an expert's down-projection only for its own
+// gate/up tiles.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <numeric>
+#include <string>
+#include <vector>
+
+#include "graph.h"
+
+namespace mk {
+
+namespace {
+
+// Tensor kinds for the region-overlap analysis.
+enum TensorKind { T_XIN = 1, T_QKV, T_O, T_XMID, T_ACT, T_ACTE, T_SEL, T_LOGITS };
+
+struct Region {
+    int tensor;         // encoded (kind, layer, slot)
+    int b_lo, b_hi;     // batch rows [b_lo, b_hi)
+    int64_t lo, hi;     // element rows [lo, hi)
+};
+
+struct Entity {         // a producer: one task, or a merge / router-final reached by the last of several tasks
+    std::vector<int> tasks;  // tasks that may signal on its behalf
+    std::vector<Region> outs;
+};
+
+int tensor_key(int kind, int layer, int slot) { return (kind * 4096 + layer) * 64 + slot; }
+
+bool overlaps(const Region& a, const Region& b) {
+    return a.tensor == b.tensor && a.b_lo < b.b_hi && b.b_lo < a.b_hi && a.lo < b.hi && b.lo < a.hi;
+}
+
+struct UnionFind {
+    std::vector<int> p;
+    int add() { p.push_back((int)p.size()); return (int)p.size() - 1; }
+    int find(int x) { while (p[x] != x) { p[x] = p[p[x]]; x = p[x]; } return x; }
+    void unite(int a, int b) { a = find(a); b = find(b); if (a != b) p[std::max(a, b)] = std::min(a, b); }
+};
+
+int largest_divisor_at_most(int n, int cap) {
+    for (int r = std::min(n, cap); r >= 1; --r)
+        if (n % r == 0) return r;
+    return 1;
+}
+
+}  // namespace
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+void wave_stats(int n_tiles, int n_sm, int* waves, int* idle) {
+    int w = (int)ceil_div(n_tiles, n_sm);
+    *waves = w;
+    *idle = (n_tiles == 0) ? 0 : w * n_sm - n_tiles;
+}
+
+// Rows per GEMV tile.  Aims at `target` bytes per task; shrinks the tile while
+// the operator would leave SMs without a tile; when `divide` > 0 the row count
+// divides it (QKV tiles never straddle two heads, so each feeds one KV head).
+int choose_tile_rows(int64_t rows, int64_t row_bytes, int n_blocks, int n_sm, int64_t target,
+                     int divide) {
+    int cap = kMaxTaskRows / n_blocks;
+    int R = (int)std::max<int64_t>(1, std::min<int64_t>(cap, target / (row_bytes * n_blocks)));
+    if (divide > 0) R = largest_divisor_at_most(divide, R);
+    const int64_t min_bytes = 16 * 1024;
+    while (R > 1 && ceil_div(rows, R) < n_sm) {
+        int next = (divide > 0) ? largest_divisor_at_most(divide, R - 1) : R - 1;
+        if ((int64_t)next * row_bytes * n_blocks < min_bytes) break;
+        R = next;
+    }
+    return R;
+}
+
+bool validate_desc(const mk_model_desc& d, std::string& err) {
+    auto fail = [&](const std::string& m) { err = m; return false; };
+    const int L = d.n_layers, H = d.hidden, nq = d.n_q_heads, nkv = d.n_kv_heads, hd = d.head_dim;
+    const bool moe = d.n_experts > 0;
+    if (moe && d.n_experts > 1024) return fail("at most 1024 experts");
+    if (L <= 0 || H <= 0 || nq <= 0 || nkv <= 0 || hd <= 0 || d.vocab <= 0)
+        return fail("model shape has a non-positive dimension");
+    if (hd != 64 && hd != 128) return fail("head_dim must be 64 or 128");
+    if (nq % nkv != 0) return fail("n_q_heads must be a multiple of n_kv_heads");
+    if (nq / nkv > kMaxHeadsPerGroup) return fail("more than 8 q heads per kv head");
+    if (H % 8 || (nq * hd) % 8) return fail("hidden and n_q*head_dim must be multiples of 8");
+    if (H > 16384 || nq * hd > 16384) return fail("hidden and n_q*head_dim must be <= 16384");
+    if (moe) {
+        if (d.top_k <= 0 || d.top_k > kMaxTopK || d.top_k > d.n_experts)
+            return fail("top_k must be in 1..min(16, n_experts)");
+        if (d.expert_ffn <= 0 || d.expert_ffn % 8 || d.expert_ffn > 16384)
+            return fail("expert_ffn must be a positive multiple of 8, <= 16384");
+    } else {
+        if (d.ffn <= 0 || d.ffn % 8 || d.ffn > 16384)
+            return fail("ffn must be a positive multiple of 8, <= 16384");
+    }
+    if (d.dtype != MK_DTYPE_BF16) return fail("only bf16 weights are supported");
+
+    return true;
+}
+
+bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, GraphPlan& g,
+                std::string& err) {
+    auto fail = [&](const std::string& m) { err = m; return false; };
+    if (!validate_desc(d, err)) return false;
+    const int L = d.n_layers, H = d.hidden, nq = d.n_q_heads, nkv = d.n_kv_heads, hd = d.head_dim;
+    const bool moe = d.n_experts > 0;
+    if (max_batch < 1) return fail("max_batch must be >= 1");
+    if (max_batch > 1) return fail("max_batch > 1 is not supported by this build");
+    if (max_ctx < 1 || max_ctx > (1 << 22)) return fail("max_ctx must be in 1..4194304");
+    if (n_sm < 1) return fail("n_sm must be >= 1");
+
+    g = GraphPlan();
+    g.desc = d;
+    g.max_batch = max_batch;
+    g.max_ctx = max_ctx;
+    g.n_sm = n_sm;
+    const int B = max_batch;
+    const int hpg = nq / nkv;
+    const int64_t qkv_rows = (int64_t)(nq + 2 * nkv) * hd;
+    const int64_t target = 128 * 1024;
+
+    // attention split-K: enough (sequence, kv head, split) tasks to cover the SMs,
+    // but at most one split per 64 positions of context.
+    int S = (int)ceil_div(n_sm, (int64_t)B * nkv);
+    S = std::max(1, std::min<int>(S, (int)ceil_div(max_ctx, 64)));
+    g.S = S;
+
+    const int R_qkv = choose_tile_rows(qkv_rows, 2LL * H, 1, n_sm, target, hd);
+    const int R_o = choose_tile_rows(H, 2LL * nq * hd, 1, n_sm, target, 0);
+    const int R_lm = choose_tile_rows(d.vocab, 2LL * H, 1, n_sm, target, 0);
+    int R_gu = 0, R_dn = 0, R_rt = 0, R_egu = 0, R_edn = 0;
+    if (!moe) {
+        R_gu = choose_tile_rows(d.ffn, 2LL * H, 2, n_sm, target, 0);
+        R_dn = choose_tile_rows(H, 2LL * d.ffn, 1, n_sm, target, 0);
+    } else {
+        R_rt = choose_tile_rows(d.n_experts, 2LL * H, 1, n_sm, 64 * 1024, 0);
+        // expert tiles: all top_k slots share the SMs
+        R_egu = choose_tile_rows(d.expert_ffn, 2LL * H, 2, std::max(1, n_sm / d.top_k), target, 0);
+        R_edn = choose_tile_rows(H, 2LL * d.expert_ffn, 1, std::max(1, n_sm / d.top_k), target, 0);
+    }
+    g.n_router_tiles = moe ? (int)ceil_div(d.n_experts, R_rt) : 0;
+    g.tile_rows = {R_qkv, R_o, R_gu, R_dn, R_lm, R_rt, R_egu, R_edn};
+
+    std::vector<Task>& T = g.tasks;
+    std::vector<Entity> ent;                     // producer entities
+    std::vector<int> task_entity;                // entity a task belongs to
+    std::vector<std::vector<Region>> task_in;    // primary input regions per task
+    std::vector<int> router_ent(L, -1);          // router-final entity per layer (MoE)
+
+    auto new_task = [&](int op, int layer, int b, int aux, uint32_t r0, uint32_t r1) {
+        Task t;
+        std::memset(&t, 0, sizeof(t));
+        t.op = (uint8_t)op;
+        t.layer = (uint16_t)layer;
+        t.b = (uint16_t)b;
+        t.aux = (uint16_t)aux;
+        t.r0 = r0;
+        t.r1 = r1;
+        t.wait0 = t.wait1 = MK_NO_EVENT;
+        t.sig = MK_NO_EVENT;
+        t.pad = MK_NO_EVENT;
+        T.push_back(t);
+        task_entity.push_back(-1);
+        task_in.emplace_back();
+        return (int)T.size() - 1;
+    };
+    auto own_entity = [&](int task, std::vector<Region> outs) {
+        Entity e;
+        e.tasks = {task};
+        e.outs = std::move(outs);
+        ent.push_back(std::move(e));
+        task_entity[task] = (int)ent.size() - 1;
+    };
+    auto all_rows = [&](int kind, int layer, int slot, int64_t n) {
+        return Region{tensor_key(kind, layer, slot), 0, B, 0, n};
+    };
+    auto gemv_op = [&](int op, int layer, int64_t rows, int R, int out_kind, int out_layer,
+                       std::vector<Region> in) {
+        for (int64_t r0 = 0; r0 < rows; r0 += R) {
+            int64_t r1 = std::min<int64_t>(rows, r0 + R);
+            int t = new_task(op, layer, 0, 0, (uint32_t)r0, (uint32_t)r1);
+            task_in[t] = in;
+            own_entity(t, {Region{tensor_key(out_kind, out_layer, 0), 0, B, r0, r1}});
+        }
+    };
+
+    for (int l = 0; l < L; ++l) {
+        // QKV: primary input is the residual stream entering the layer.
+        gemv_op(MK_OP_QKV, l, qkv_rows, R_qkv, T_QKV, l, {all_rows(T_XIN, l, 0, H)});
+        // attention: per (sequence, kv head, split); the merge entity is signalled by the last split.
+        for (int b = 0; b < B; ++b)
+            for (int kh = 0; kh < nkv; ++kh) {
+                Entity m;
+                m.outs = {Region{tensor_key(T_O, l, 0), b, b + 1, (int64_t)kh * hpg * hd,
+                                 (int64_t)(kh + 1) * hpg * hd}};
+                int eid = (int)ent.size();
+                ent.push_back(m);
+                for (int s = 0; s < S; ++s) {
+                    int t = new_task(MK_OP_ATTN, l, b, kh, (uint32_t)s, (uint32_t)S);
+                    int key = tensor_key(T_QKV, l, 0);
+                    task_in[t] = {Region{key, 0, B, (int64_t)kh * hpg * hd, (int64_t)(kh + 1) * hpg * hd},
+                                  Region{key, 0, B, (int64_t)nq * hd + kh * hd, (int64_t)nq * hd + (kh + 1) * hd},
+                                  Region{key, 0, B, (int64_t)(nq + nkv) * hd + kh * hd,
+                                         (int64_t)(nq + nkv) * hd + (kh + 1) * hd}};
+                    task_entity[t] = eid;
+                    ent[eid].tasks.push_back(t);
+                }
+            }
+        gemv_op(MK_OP_OPROJ, l, H, R_o, T_XMID, l, {all_rows(T_O, l, 0, (int64_t)nq * hd)});
+        if (!moe) {
+            gemv_op(MK_OP_GATEUP, l, d.ffn, R_gu, T_ACT, l, {all_rows(T_XMID, l, 0, H)});
+            gemv_op(MK_OP_DOWN, l, H, R_dn, T_XIN, l + 1, {all_rows(T_ACT, l, 0, d.ffn)});
+        } else {
+            Entity rf;
+            rf.outs = {all_rows(T_SEL, l, 0, d.top_k)};
+            int rid = (int)ent.size();
+            ent.push_back(rf);
+            router_ent[l] = rid;
+            for (int r0 = 0; r0 < d.n_experts; r0 += R_rt) {
+                int t = new_task(MK_OP_ROUTER, l, 0, 0, (uint32_t)r0,
+                                 (uint32_t)std::min(d.n_experts, r0 + R_rt));
+                task_in[t] = {all_rows(T_XMID, l, 0, H)};
+                task_entity[t] = rid;
+                ent[rid].tasks.push_back(t);
+            }
+            for (int b = 0; b < B; ++b)
+                for (int k = 0; k < d.top_k; ++k)
+                    for (int r0 = 0; r0 < d.expert_ffn; r0 += R_egu) {
+                        int r1 = std::min(d.expert_ffn, r0 + R_egu);
+                        int t = new_task(MK_OP_EXP_GATEUP, l, b, k, (uint32_t)r0, (uint32_t)r1);
+                        task_in[t] = {all_rows(T_SEL, l, 0, d.top_k)};
+                        own_entity(t, {Region{tensor_key(T_ACTE, l, k), b, b + 1, r0, r1}});
+                    }
+            for (int b = 0; b < B; ++b)
+                for (int k = 0; k < d.top_k; ++k)
+                    for (int r0 = 0; r0 < H; r0 += R_edn) {
+                        int r1 = std::min(H, r0 + R_edn);
+                        int t = new_task(MK_OP_EXP_DOWN, l, b, k, (uint32_t)r0, (uint32_t)r1);
+                        task_in[t] = {Region{tensor_key(T_ACTE, l, k), b, b + 1, 0, d.expert_ffn}};
+                        own_entity(t, {Region{tensor_key(T_XIN, l + 1, 0), b, b + 1, r0, r1}});
+                    }
+        }
+    }
+    gemv_op(MK_OP_LMHEAD, L, d.vocab, R_lm, T_LOGITS, 0, {all_rows(T_XIN, L, 0, H)});
+
+    // ---- dependency analysis: producers overlapping each task's primary input
+    std::map<int, std::vector<int>> by_tensor;   // tensor -> entities writing it
+    for (int e = 0; e < (int)ent.size(); ++e)
+        for (const Region& r : ent[e].outs) by_tensor[r.tensor].push_back(e);
+    UnionFind uf;
+    for (size_t e = 0; e < ent.size(); ++e) uf.add();
+    std::vector<int> first_dep(T.size(), -1);
+    for (size_t t = 0; t < T.size(); ++t) {
+        int first = -1;
+        for (const Region& in : task_in[t]) {
+            auto it = by_tensor.find(in.tensor);
+            if (it == by_tensor.end()) continue;       // e.g. the embedding: no producer task
+            for (int e : it->second)
+                for (const Region& o : ent[e].outs)
+                    if (overlaps(in, o)) {
+                        if (first < 0) first = e;
+                        else uf.unite(first, e);
+                    }
+        }
+        first_dep[t] = first;
+    }
+    // events = connected components of producer entities that some task waits on
+    std::map<int, int> comp_event;
+    std::vector<uint32_t>& thr = g.thr;
+    auto event_of = [&](int e) -> int {
+        int c = uf.find(e);
+        auto it = comp_event.find(c);
+        if (it != comp_event.end()) return it->second;
+        int id = (int)thr.size();
+        comp_event[c] = id;
+        thr.push_back(0);
+        return id;
+    };
+    for (size_t t = 0; t < T.size(); ++t)
+        if (first_dep[t] >= 0) T[t].wait0 = (uint32_t)event_of(first_dep[t]);
+    // producers signal their component's event; thresholds count entities
+    for (int e = 0; e < (int)ent.size(); ++e) {
+        int c = uf.find(e);
+        auto it = comp_event.find(c);
+        if (it == comp_event.end()) continue;          // nobody waits on it (e.g. LM head)
+        thr[it->second] += 1;
+        for (int t : ent[e].tasks) T[t].sig = (uint32_t)it->second;
+    }
+    // expert tasks: the producer warp waits on the router event before it reads the expert id
+    for (size_t t = 0; t < T.size(); ++t)
+        if (T[t].op == MK_OP_EXP_GATEUP || T[t].op == MK_OP_EXP_DOWN) {
+            int c = uf.find(router_ent[T[t].layer]);
+            T[t].pad = (uint32_t)comp_event.at(c);
+        }
+    // ---- checks: every wait is satisfied only by tasks earlier in the list
+    std::vector<int> last_signaler(thr.size(), -1);
+    for (int t = 0; t < (int)T.size(); ++t)
+        if (T[t].sig != MK_NO_EVENT) last_signaler[T[t].sig] = t;
+    for (int t = 0; t < (int)T.size(); ++t) {
+        uint32_t w = T[t].wait0;
+        if (w != MK_NO_EVENT && last_signaler[w] >= t)
+            return fail("internal: task list is not topologically ordered");
+    }
+    g.n_events = (int)thr.size();
+
+    // ---- bytes streamed per B=1 step
+    int64_t wb = 2LL * H;                               // one embedding row
+    for (int l = 0; l < L; ++l) {
+        wb += 2LL * H * 2;                              // norm gains
+        wb += 2LL * qkv_rows * H + 2LL * H * nq * hd;
+        if (!moe) wb += 2LL * 3 * d.ffn * H;
+        else wb += 2LL * d.n_experts * H + 2LL * 3 * d.top_k * d.expert_ffn * H;
+    }
+    wb += 2LL * H + 2LL * d.vocab * H;
+    g.weight_bytes = wb;
+    return true;
+}
+
+}  // namespace mk

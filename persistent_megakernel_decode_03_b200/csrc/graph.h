@@ -1,0 +1,33 @@
+// Host task-graph compiler interface.
+#pragma once
+
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "mk_internal.h"
+
+namespace mk {
+
+struct GraphPlan {
+    mk_model_desc desc{};
+    int max_batch = 0, max_ctx = 0, n_sm = 0;
+    int S = 1;                   // attention splits per (sequence, kv head)
+    int n_router_tiles = 0;
+    int n_events = 0;
+    int64_t weight_bytes = 0;    // bf16 bytes streamed per B=1 step
+    std::vector<int> tile_rows;  // qkv, o, gate/up, down, lm, router, expert gate/up, expert down
+    std::vector<Task> tasks;     // topological order
+    std::vector<uint32_t> thr;   // per-event threshold per step
+};
+
+int64_t ceil_div(int64_t a, int64_t b);
+void wave_stats(int n_tiles, int n_sm, int* waves, int* idle);
+int choose_tile_rows(int64_t rows, int64_t row_bytes, int n_blocks, int n_sm, int64_t target,
+                     int divide);
+bool validate_desc(const mk_model_desc& d, std::string& err);
+bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, GraphPlan& g,
+                std::string& err);
+
+}  // namespace mk

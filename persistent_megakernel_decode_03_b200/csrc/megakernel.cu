@@ -1,0 +1,1204 @@
+// The persistent decode megakernel for sm_100a.
+//
+// One CTA per SM stays resident for the whole decode step and pulls tasks from
+// the host-built list through one global atomic work-queue head (Cohere page
+// "Cohere megakerneles kiszolgálót mutatott be a North Mini Code modellhez",
+// section "Egyetlen tartós kernelre épül a kiszolgálás").  A task waits on an
+// event counter in global memory until it reaches threshold * epoch, computes
+// one tile, and increments its own event (MPK digest "LLM को MegaKernel में
+// compile करके low-latency inference हासिल करना", section "Part 2. Runtime":
+// worker loop fetch -> execute -> notify; event fires at its threshold).
+//
+// Warp roles inside a CTA:
+//   warps 0-7  consumers: dependency wait, prologue (RMSNorm / RoPE), dot
+//              products out of shared memory, epilogue, reductions
+//   warp 8     producer: dequeues the next tasks and streams their weight rows
+//              and KV pages into an 11-stage shared-memory ring with bulk
+//              asynchronous copies (cp.async.bulk, mbarrier completion).
+//              Weights never depend on activations, so the producer runs ahead
+//              of the consumers across task and layer boundaries: the next
+//              layer's weights are in flight while this layer's tail finishes
+//              (Cohere page, "Honnan jön a gyorsulás?": weight tiles are
+//              prefetched before the activation dependency is met).
+//   warp 9     signal: publishes completions (fence + release add) so that the
+//              consumers do not stall on the gpu-scope fence.
+//
+// Deadlock freedom: tasks are dequeued in list order, the list is topological
+// and each CTA runs its tasks in dequeue order, so the lowest unfinished task
+// always has its producers finished and its CTA free to run it.
+// Every wait (event counter, ring slot, signal slot) gives up after
+// Params::timeout_ns, records MK_ERR_TIMEOUT and the kernel drains its own
+// copies in flight and returns.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "megakernel.h"
+#include "mk_internal.h"
+
+namespace mk {
+
+// ----------------------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t tx) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(tx)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// Bulk async copy global -> this CTA's shared memory; completion counted on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ int ld_relaxed_int(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+// fp32 -> bf16 round-to-nearest-even (finite values)
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+    uint32_t u = __float_as_uint(f);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+__device__ __forceinline__ void set_error(const Params& p, int code, int a, int b, int c, int d) {
+    if (atomicCAS(p.err, 0, code) == 0) {
+        p.err[1] = a;
+        p.err[2] = b;
+        p.err[3] = c;
+        p.err[4] = d;
+    }
+}
+
+// ----------------------------------------------------------------------------- shared memory
+
+struct StageInfo {
+    int task;      // task index, -1 = end of work
+    int chunk;     // chunk index within the task
+    int nchunks;   // chunks of the task (0 for a task without streamed data)
+    int aux;       // attention: first logical page of this chunk
+};
+
+constexpr int kAttnScratch = kConsumerWarps * kMaxHeadsPerGroup * (128 + 2);
+
+struct __align__(128) Smem {
+    uint8_t ring[kStages][kStageBytes];
+    float red[2][kMaxTaskRows][kConsumerWarps];
+    float attn[kAttnScratch];                 // per-warp (m, l, o) partials
+    float qs[kMaxHeadsPerGroup * 128];        // rotated, pre-scaled q of one kv group
+    float kn[128], vn[128];                   // the new token's k, v (bf16-rounded)
+    float rlog[1024];                         // router logits of one sequence
+    float bcast[kConsumerWarps + 8];
+    uint64_t full[kStages], empty[kStages];
+    uint64_t sig_full[kSigSlots], sig_empty[kSigSlots];
+    StageInfo info[kStages];
+    uint32_t sig_evt[kSigSlots];
+    int sig_task[kSigSlots];
+    int flag[4];
+};
+
+// ----------------------------------------------------------------------------- geometry
+
+__device__ __forceinline__ int hpg_of(const Params& p) { return p.nq / p.nkv; }
+
+// Token position of batch row b this step (validated by the caller).
+__device__ __forceinline__ int position_of(const Params& p, int b) {
+    return (p.positions ? p.positions[b] : 0) + p.pos_offset;
+}
+
+struct GemvGeom {
+    int K;            // columns
+    int rows;         // rows per weight block
+    int nblk;         // 1 or 2 weight blocks (gate/up)
+    const uint16_t* w[2];
+};
+
+// Weight blocks of a GEMV task.  Expert ops read the routed expert id (producer
+// side only; the consumer needs just K and rows).
+__device__ __forceinline__ void gemv_geom(const Params& p, const Task& t, GemvGeom& g, bool want_ptr) {
+    const int H = p.H;
+    g.rows = (int)(t.r1 - t.r0);
+    g.nblk = 1;
+    g.w[0] = g.w[1] = nullptr;
+    const LayerW* lw = (t.op == MK_OP_LMHEAD) ? nullptr : &p.layers[t.layer];
+    switch (t.op) {
+        case MK_OP_QKV: {
+            g.K = H;
+            if (want_ptr) {
+                int qr = p.nq * p.hd, kr = p.nkv * p.hd;
+                int r = (int)t.r0;
+                const uint16_t* base;
+                if (r < qr) base = lw->wq + (size_t)r * H;
+                else if (r < qr + kr) base = lw->wk + (size_t)(r - qr) * H;
+                else base = lw->wv + (size_t)(r - qr - kr) * H;
+                g.w[0] = base;
+            }
+            break;
+        }
+        case MK_OP_OPROJ:
+            g.K = p.nq * p.hd;
+            if (want_ptr) g.w[0] = lw->wo + (size_t)t.r0 * g.K;
+            break;
+        case MK_OP_GATEUP:
+            g.K = H;
+            g.nblk = 2;
+            if (want_ptr) {
+                g.w[0] = lw->w_gate + (size_t)t.r0 * H;
+                g.w[1] = lw->w_up + (size_t)t.r0 * H;
+            }
+            break;
+        case MK_OP_DOWN:
+            g.K = p.F;
+            if (want_ptr) g.w[0] = lw->w_down + (size_t)t.r0 * p.F;
+            break;
+        case MK_OP_LMHEAD:
+            g.K = H;
+            if (want_ptr) g.w[0] = p.lm_head + (size_t)t.r0 * H;
+            break;
+        case MK_OP_ROUTER:
+            g.K = H;
+            if (want_ptr) g.w[0] = lw->w_router + (size_t)t.r0 * H;
+            break;
+        case MK_OP_EXP_GATEUP: {
+            g.K = H;
+            g.nblk = 2;
+            if (want_ptr) {
+                int e = __ldcg(p.moe_sel + ((size_t)t.layer * p.max_batch + t.b) * p.topk + t.aux);
+                if (e < 0 || e >= p.E) { set_error(p, kErrFault, -1, -7, e, t.layer); e = 0; }
+                size_t off = ((size_t)e * p.Fe + t.r0) * H;
+                g.w[0] = lw->w_gate + off;
+                g.w[1] = lw->w_up + off;
+            }
+            break;
+        }
+        case MK_OP_EXP_DOWN: {
+            g.K = p.Fe;
+            if (want_ptr) {
+                int e = __ldcg(p.moe_sel + ((size_t)t.layer * p.max_batch + t.b) * p.topk + t.aux);
+                if (e < 0 || e >= p.E) { set_error(p, kErrFault, -1, -7, e, t.layer); e = 0; }
+                g.w[0] = lw->w_down + ((size_t)e * H + t.r0) * p.Fe;
+            }
+            break;
+        }
+        default:
+            g.K = 8;
+            g.rows = 0;
+            break;
+    }
+}
+
+__device__ __forceinline__ bool is_gemv(int op) { return op != MK_OP_ATTN; }
+
+// Chunks of one weight block: kStageBytes pieces of the contiguous rows.
+__device__ __forceinline__ int block_chunks(const GemvGeom& g) {
+    int64_t bytes = (int64_t)g.rows * g.K * 2;
+    return (int)((bytes + kStageBytes - 1) / kStageBytes);
+}
+
+// Attention split range [j0, j1) of positions (inclusive of the new token).
+__device__ __forceinline__ void attn_range(int n_ctx, int S, int s, int& j0, int& j1) {
+    int per = (n_ctx + S - 1) / S;
+    per = (per + kPageSize - 1) / kPageSize * kPageSize;
+    j0 = s * per;
+    j1 = min(n_ctx, j0 + per);
+    if (j0 > n_ctx) j0 = n_ctx;
+}
+
+__device__ __forceinline__ int pages_per_stage(const Params& p) {
+    return kStageBytes / (2 * kPageSize * p.hd * 2);
+}
+
+// ----------------------------------------------------------------------------- waits
+
+struct Waiter {
+    uint64_t t0;
+    int spins;
+};
+
+// true when the deadline has passed or another CTA has recorded an error
+__device__ __forceinline__ bool wait_should_stop(const Params& p, Waiter& w) {
+    if (++w.spins & 63) return false;
+    if (ld_relaxed_int(p.err) != 0) return true;
+    if (w.t0 == 0) w.t0 = globaltimer();
+    else if ((long long)(globaltimer() - w.t0) > p.timeout_ns) return true;
+    return false;
+}
+
+__device__ bool mbar_wait_bounded(const Params& p, uint64_t* bar, uint32_t parity, int where) {
+    Waiter w{0, 0};
+    while (!mbar_try_wait(bar, parity)) {
+        if (wait_should_stop(p, w)) {
+            if (ld_relaxed_int(p.err) == 0) set_error(p, kErrTimeout, -1, -1, where, (int)blockIdx.x);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Wait on a phase that another thread of this CTA has already seen complete
+// (so it returns at once); bounded anyway: on failure it records a fault and
+// raises the CTA's abort flag, which every consumer reads after its next barrier.
+__device__ __forceinline__ void seen_complete_wait(const Params& p, uint64_t* bar, uint32_t parity, int* abort_flag) {
+    for (int i = 0; i < (1 << 22); ++i)
+        if (mbar_try_wait(bar, parity)) return;
+    set_error(p, kErrFault, -1, -6, (int)parity, (int)blockIdx.x);
+    *abort_flag = 1;
+}
+
+// Spin (acquire) until events[e] >= target.  Single thread.
+__device__ bool event_wait(const Params& p, uint32_t e, uint32_t target, int task) {
+    Waiter w{0, 0};
+    while (true) {
+        uint32_t v = ld_acquire(&p.events[e]);
+        if ((int32_t)(v - target) >= 0) return true;
+        if (wait_should_stop(p, w)) {
+            if (ld_relaxed_int(p.err) == 0) set_error(p, kErrTimeout, task, (int)e, (int)v, (int)target);
+            return false;
+        }
+        __nanosleep(32);
+    }
+}
+
+// ----------------------------------------------------------------------------- producer
+
+__device__ void producer_loop(const Params& p, Smem& sm) {
+    const uint64_t pol = l2_evict_first_policy();
+    int stage = 0;
+    uint32_t issued[kStages];           // fills issued per stage
+    for (int s = 0; s < kStages; ++s) issued[s] = 0;
+    bool ok = true;
+
+    auto acquire_slot = [&]() -> bool {
+        // first lap: slots start empty
+        if (issued[stage] == 0) return true;
+        return mbar_wait_bounded(p, &sm.empty[stage], (issued[stage] - 1) & 1, 1);
+    };
+    auto advance = [&]() {
+        issued[stage] += 1;
+        stage = (stage + 1 == kStages) ? 0 : stage + 1;
+    };
+
+    uint32_t last_router_evt = MK_NO_EVENT;
+    while (ok) {
+        if (ld_relaxed_int(p.err) != 0) { ok = false; break; }
+        unsigned long long q = atomicAdd(p.queue, 1ull) - p.queue_base;
+        if (q >= p.n_tasks) break;
+        const int ti = (int)q;
+        const Task t = p.tasks[ti];
+        if (t.op == MK_OP_ATTN) {
+            const int b = t.b;
+            int npages = 0, lp0 = 0;
+            if (b < p.batch) {
+                int pos = position_of(p, b);
+                if (pos >= 0 && pos < p.max_ctx && pos / kPageSize < p.max_pages) {
+                    int j0, j1;
+                    attn_range(pos + 1, (int)t.r1, (int)t.r0, j0, j1);
+                    int jc = min(j1, pos);          // cached positions only; the new token is fresh
+                    if (jc > j0) {
+                        lp0 = j0 / kPageSize;
+                        npages = (jc - 1) / kPageSize - lp0 + 1;
+                    }
+                }
+            }
+            const int pps = pages_per_stage(p);
+            const int nch = (npages + pps - 1) / pps;
+            const uint32_t blk = (uint32_t)(kPageSize * p.hd * 2);
+            if (nch == 0) {
+                if (!acquire_slot()) { ok = false; break; }
+                sm.info[stage] = StageInfo{ti, 0, 0, 0};
+                mbar_arrive(&sm.full[stage]);
+                advance();
+            }
+            for (int c = 0; c < nch && ok; ++c) {
+                if (!acquire_slot()) { ok = false; break; }
+                int first = lp0 + c * pps;
+                int n = min(pps, lp0 + npages - first);
+                sm.info[stage] = StageInfo{ti, c, nch, first};
+                // validate page indices before issuing any copy
+                const int* prow = p.page_table + (size_t)b * p.max_pages;
+                bool bad = false;
+                for (int i = 0; i < n; ++i) {
+                    int ph = prow[first + i];
+                    if (ph < 0 || ph >= p.n_pages) bad = true;
+                }
+                if (bad) {
+                    set_error(p, kErrInvalid, ti, -2, first, b);
+                    mbar_arrive(&sm.full[stage]);
+                    advance();
+                    continue;
+                }
+                mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)n * 2u * blk);
+                for (int i = 0; i < n; ++i) {
+                    int ph = prow[first + i];
+                    size_t off = (((size_t)t.layer * p.n_pages + ph) * p.nkv + t.aux) * (size_t)kPageSize * p.hd;
+                    uint8_t* dst = sm.ring[stage] + (size_t)i * 2 * blk;
+                    bulk_g2s(dst, p.k_pages + off, blk, &sm.full[stage], pol);
+                    bulk_g2s(dst + blk, p.v_pages + off, blk, &sm.full[stage], pol);
+                }
+                advance();
+            }
+            continue;
+        }
+        // GEMV-type task
+        bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
+        if ((t.op == MK_OP_EXP_GATEUP || t.op == MK_OP_EXP_DOWN) && t.pad != MK_NO_EVENT &&
+            t.pad != last_router_evt) {
+            // the expert id comes from the router: wait for it before computing addresses
+            if (!event_wait(p, t.pad, p.thr[t.pad] * p.epoch + p.wait_offset, ti)) { ok = false; break; }
+            last_router_evt = t.pad;
+        }
+        GemvGeom g;
+        gemv_geom(p, t, g, !skip);
+        int nch_blk = skip ? 0 : block_chunks(g);
+        int nch = nch_blk * g.nblk;
+        if (nch == 0) {
+            if (!acquire_slot()) { ok = false; break; }
+            sm.info[stage] = StageInfo{ti, 0, 0, 0};
+            mbar_arrive(&sm.full[stage]);
+            advance();
+            continue;
+        }
+        const int64_t blk_bytes = (int64_t)g.rows * g.K * 2;
+        for (int c = 0; c < nch; ++c) {
+            if (!acquire_slot()) { ok = false; break; }
+            int bi = c / nch_blk, ci = c % nch_blk;
+            int64_t off = (int64_t)ci * kStageBytes;
+            uint32_t bytes = (uint32_t)((blk_bytes - off < (int64_t)kStageBytes) ? (blk_bytes - off) : (int64_t)kStageBytes);
+            sm.info[stage] = StageInfo{ti, c, nch, 0};
+            mbar_arrive_expect_tx(&sm.full[stage], bytes);
+            bulk_g2s(sm.ring[stage], (const uint8_t*)g.w[bi] + off, bytes, &sm.full[stage], pol);
+            advance();
+        }
+    }
+    // end-of-work marker (best effort when aborting)
+    if (acquire_slot()) {
+        sm.info[stage] = StageInfo{-1, 0, 0, 0};
+        mbar_arrive(&sm.full[stage]);
+        advance();
+    }
+    // drain: every issued fill must have landed before the CTA's shared memory goes away
+    for (int s = 0; s < kStages; ++s) {
+        if (issued[s] == 0) continue;
+        Waiter w{0, 0};
+        while (!mbar_try_wait(&sm.full[s], (issued[s] - 1) & 1)) {
+            if (++w.spins > (1 << 26)) break;   // copies of valid memory always land; hard cap only
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- signal warp
+
+__device__ void signal_loop(const Params& p, Smem& sm) {
+    int slot = 0;
+    uint32_t lap = 0;
+    while (true) {
+        if (!mbar_wait_bounded(p, &sm.sig_full[slot], lap & 1, 2)) return;
+        uint32_t e = sm.sig_evt[slot];
+        int task = sm.sig_task[slot];
+        if (e == 0xFFFFFFFEu) return;   // end of work
+        __threadfence();
+        if (e != MK_NO_EVENT) red_release_add(&p.events[e], 1u);
+        atomicAdd(p.done, 1u);
+        if (p.trace && task >= 0) p.trace[(size_t)task * 4 + 2] = globaltimer();
+        mbar_arrive(&sm.sig_empty[slot]);
+        if (++slot == kSigSlots) { slot = 0; ++lap; }
+    }
+}
+
+// ----------------------------------------------------------------------------- consumer helpers
+
+// Residual stream entering layer l (l == L: after the last layer), element i of batch row b.
+__device__ __forceinline__ float x_in(const Params& p, int l, int b, int i) {
+    if (l == 0) {
+        int tok = p.tokens[b];
+        if (tok < 0 || tok >= p.V) tok = 0;   // recorded as an error by the prologue
+        return bf16_to_f32(p.tok_emb[(size_t)tok * p.H + i]);
+    }
+    if (p.E == 0) return __ldcg(p.x_out + ((size_t)(l - 1) * p.max_batch + b) * p.H + i);
+    const size_t lb = (size_t)(l - 1) * p.max_batch + b;
+    float v = __ldcg(p.x_mid + lb * p.H + i);
+    for (int k = 0; k < p.topk; ++k)
+        v += __ldcg(p.moe_w + lb * p.topk + k) * __ldcg(p.ypart + (lb * p.topk + k) * p.H + i);
+    return v;
+}
+
+__device__ __forceinline__ float x_mid_at(const Params& p, int l, int b, int i) {
+    return __ldcg(p.x_mid + ((size_t)l * p.max_batch + b) * p.H + i);
+}
+
+// Input element i of a GEMV task (before normalisation).
+__device__ __forceinline__ float gemv_input(const Params& p, const Task& t, int i) {
+    const int l = t.layer, b = t.b;
+    switch (t.op) {
+        case MK_OP_QKV: return x_in(p, l, 0, i);
+        case MK_OP_OPROJ: return __ldcg(p.o + ((size_t)l * p.max_batch) * (p.nq * p.hd) + i);
+        case MK_OP_GATEUP:
+        case MK_OP_ROUTER: return x_mid_at(p, l, 0, i);
+        case MK_OP_EXP_GATEUP: return x_mid_at(p, l, b, i);
+        case MK_OP_DOWN: return __ldcg(p.act + ((size_t)l * p.max_batch) * p.F + i);
+        case MK_OP_EXP_DOWN:
+            return __ldcg(p.act + (((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.Fe + i);
+        case MK_OP_LMHEAD: return x_in(p, p.L, 0, i);
+        default: return 0.0f;
+    }
+}
+
+__device__ __forceinline__ const uint16_t* gemv_norm_gain(const Params& p, const Task& t) {
+    switch (t.op) {
+        case MK_OP_QKV: return p.layers[t.layer].attn_norm;
+        case MK_OP_GATEUP:
+        case MK_OP_ROUTER:
+        case MK_OP_EXP_GATEUP: return p.layers[t.layer].ffn_norm;
+        case MK_OP_LMHEAD: return p.final_norm;
+        default: return nullptr;
+    }
+}
+
+// Sum over all consumer threads, same order in every CTA.
+__device__ __forceinline__ float block_sum(Smem& sm, float v) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    v = warp_sum(v);
+    consumer_sync();
+    if (lane == 0) sm.bcast[warp] = v;
+    consumer_sync();
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) s += sm.bcast[w];
+    consumer_sync();
+    return s;
+}
+
+struct ThreadMap {
+    int nvec, wpg, G, grp, lig, gstride, vpt;
+    bool active;
+};
+
+__device__ __forceinline__ ThreadMap thread_map(int K) {
+    ThreadMap m;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    m.nvec = K / 8;
+    int wneed = (m.nvec + 31) / 32;
+    m.wpg = min(kConsumerWarps, wneed);
+    m.G = kConsumerWarps / m.wpg;
+    m.grp = warp / m.wpg;
+    m.lig = (warp % m.wpg) * 32 + lane;
+    m.gstride = m.wpg * 32;
+    m.vpt = (m.nvec + m.gstride - 1) / m.gstride;
+    m.active = m.grp < m.G;
+    return m;
+}
+
+// Loads this thread's slice of the (normalised) input into registers.
+__device__ void gemv_prologue(const Params& p, Smem& sm, const Task& t, const ThreadMap& m, int K,
+                              float (&xr)[kMaxVecPerThread][8]) {
+    const uint16_t* gain = gemv_norm_gain(p, t);
+    float rstd = 1.0f;
+    if (gain) {
+        float ss = 0.0f;
+        for (int i = threadIdx.x; i < K; i += kConsumerThreads) {
+            float v = gemv_input(p, t, i);
+            ss = fmaf(v, v, ss);
+        }
+        float tot = block_sum(sm, ss);
+        rstd = 1.0f / sqrtf(tot / (float)K + p.eps);
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxVecPerThread; ++j) {
+        int v = m.lig + j * m.gstride;
+        if (j < m.vpt && v < m.nvec && m.active) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                int col = v * 8 + e;
+                float x = gemv_input(p, t, col);
+                if (gain) x = (x * rstd) * bf16_to_f32(gain[col]);
+                xr[j][e] = x;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[j][e] = 0.0f;
+        }
+    }
+}
+
+__device__ __forceinline__ float dot8(const uint4 q, const float (&x)[8], float acc) {
+    acc = fmaf(bf_lo(q.x), x[0], acc);
+    acc = fmaf(bf_hi(q.x), x[1], acc);
+    acc = fmaf(bf_lo(q.y), x[2], acc);
+    acc = fmaf(bf_hi(q.y), x[3], acc);
+    acc = fmaf(bf_lo(q.z), x[4], acc);
+    acc = fmaf(bf_hi(q.z), x[5], acc);
+    acc = fmaf(bf_lo(q.w), x[6], acc);
+    acc = fmaf(bf_hi(q.w), x[7], acc);
+    return acc;
+}
+
+// Dot products of one chunk (vectors [c0, c1) of weight block `blk`) against x.
+__device__ __forceinline__ void gemv_chunk(Smem& sm, int buf, const uint8_t* stage, const ThreadMap& m,
+                                           int rows, int blk, int c0, int c1,
+                                           const float (&xr)[kMaxVecPerThread][8]) {
+    if (!m.active) return;
+    const int lane = threadIdx.x & 31, wig = (threadIdx.x >> 5) % m.wpg;
+    const int nvec = m.nvec;
+    const int row_first = c0 / nvec, row_last = (c1 - 1) / nvec;
+    int r = row_first + (((m.grp - row_first) % m.G) + m.G) % m.G;
+    const uint4* sv = reinterpret_cast<const uint4*>(stage);
+    for (; r <= row_last; r += m.G) {
+        const int rb = r * nvec;
+        const int vs = max(c0, rb) - rb, ve = min(c1, rb + nvec) - rb;
+        const uint4* rowp = sv + (rb - c0);
+        float acc = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kMaxVecPerThread; ++j) {
+            int v = m.lig + j * m.gstride;
+            if (j < m.vpt && v >= vs && v < ve) acc = dot8(rowp[v], xr[j], acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) {
+            float* slot = &sm.red[buf][blk * rows + r][wig];
+            if (rb >= c0) *slot = acc;
+            else *slot += acc;
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- consumer: attention
+
+template <int HPG, int DPL>
+struct AttnState {
+    float q[HPG][DPL];
+    float o[HPG][DPL];
+    float m[HPG], l[HPG];
+};
+
+template <int HPG, int DPL>
+__device__ __forceinline__ void attn_token(AttnState<HPG, DPL>& st, const float (&k)[DPL],
+                                           const float (&v)[DPL]) {
+#pragma unroll
+    for (int h = 0; h < HPG; ++h) {
+        float s = 0.0f;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) s = fmaf(st.q[h][d], k[d], s);
+        s = warp_sum(s);                       // log2-domain score (q pre-scaled)
+        float mn = fmaxf(st.m[h], s);
+        float corr = exp2f(st.m[h] - mn);
+        float pw = exp2f(s - mn);
+        st.l[h] = fmaf(st.l[h], corr, pw);
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) st.o[h][d] = fmaf(st.o[h][d], corr, pw * v[d]);
+        st.m[h] = mn;
+    }
+}
+
+template <int DPL>
+__device__ __forceinline__ void load_bf16_dpl(const uint16_t* src, float (&out)[DPL]) {
+    if (DPL == 4) {
+        uint2 u = *reinterpret_cast<const uint2*>(src);
+        out[0] = bf_lo(u.x); out[1] = bf_hi(u.x);
+        out[2 % DPL] = bf_lo(u.y); out[3 % DPL] = bf_hi(u.y);
+    } else {
+        uint32_t u = *reinterpret_cast<const uint32_t*>(src);
+        out[0] = bf_lo(u); out[1 % DPL] = bf_hi(u);
+    }
+}
+
+// Split partial layout: [L][B][nkv][S][HPG][hd + 2] = (m, l, o[hd]) per head.
+__device__ __forceinline__ float* attn_part(const Params& p, int l, int b, int g, int s, int h) {
+    const int hpg = hpg_of(p);
+    size_t idx = ((((size_t)l * p.max_batch + b) * p.nkv + g) * p.S + s) * hpg + h;
+    return p.part + idx * (p.hd + 2);
+}
+
+template <int HPG, int DPL>
+__device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti, int& stage,
+                               uint32_t& lap, bool& abort_all) {
+    constexpr int HD = DPL * 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = t.b, g = t.aux, s = (int)t.r0, S = (int)t.r1, l = t.layer;
+    const bool active_row = b < p.batch;
+    int pos = active_row ? position_of(p, b) : 0;
+    bool valid = active_row && pos >= 0 && pos < p.max_ctx && pos / kPageSize < p.max_pages;
+    if (active_row && !valid && tid == 0) set_error(p, kErrInvalid, ti, -3, pos, b);
+    int j0 = 0, j1 = 0;
+    if (valid) attn_range(pos + 1, S, s, j0, j1);
+    const bool has_new = valid && pos >= j0 && pos < j1;
+    const float qscale = 1.4426950408889634f / sqrtf((float)HD);   // log2(e) / sqrt(d)
+
+    AttnState<HPG, DPL> st;
+#pragma unroll
+    for (int h = 0; h < HPG; ++h) {
+        st.m[h] = -INFINITY;
+        st.l[h] = 0.0f;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) st.o[h][d] = 0.0f;
+    }
+    if (valid && j1 > j0) {
+        // q of the group's heads, k and v of the new token, rotated at `pos`
+        const float* qkv = p.qkv + ((size_t)l * p.max_batch + b) * ((p.nq + 2 * p.nkv) * HD);
+        const float* rope = p.rope + (size_t)pos * HD;   // [HD/2][2]
+        for (int idx = tid; idx < (HPG + 1) * (HD / 2); idx += kConsumerThreads) {
+            int h = idx / (HD / 2), i = idx % (HD / 2);
+            float c = rope[2 * i], sn = rope[2 * i + 1];
+            const float* src = (h < HPG) ? qkv + (size_t)(g * HPG + h) * HD : qkv + (size_t)(p.nq + g) * HD;
+            float x0 = __ldcg(src + i), x1 = __ldcg(src + i + HD / 2);
+            float r0 = x0 * c - x1 * sn, r1 = x1 * c + x0 * sn;
+            if (h < HPG) {
+                sm.qs[h * HD + i] = r0 * qscale;
+                sm.qs[h * HD + i + HD / 2] = r1 * qscale;
+            } else {
+                sm.kn[i] = bf16_to_f32(f32_to_bf16_rne(r0));
+                sm.kn[i + HD / 2] = bf16_to_f32(f32_to_bf16_rne(r1));
+            }
+        }
+        for (int i = tid; i < HD; i += kConsumerThreads) {
+            float v = __ldcg(qkv + (size_t)(p.nq + p.nkv + g) * HD + i);
+            sm.vn[i] = bf16_to_f32(f32_to_bf16_rne(v));
+        }
+        consumer_sync();
+        // KV append: the split that owns the new position writes it
+        if (has_new) {
+            const int* prow = p.page_table + (size_t)b * p.max_pages;
+            int ph = prow[pos / kPageSize];
+            if (ph >= 0 && ph < p.n_pages) {
+                size_t off = ((((size_t)l * p.n_pages + ph) * p.nkv + g) * kPageSize + pos % kPageSize) * HD;
+                for (int i = tid; i < HD; i += kConsumerThreads) {
+                    p.k_pages[off + i] = f32_to_bf16_rne(sm.kn[i]);
+                    p.v_pages[off + i] = f32_to_bf16_rne(sm.vn[i]);
+                }
+            } else if (tid == 0) {
+                set_error(p, kErrInvalid, ti, -2, pos / kPageSize, b);
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < HPG; ++h)
+#pragma unroll
+            for (int d = 0; d < DPL; ++d) st.q[h][d] = sm.qs[h * HD + lane * DPL + d];
+    }
+
+    // streamed chunks of cached pages (the first stage was seen complete by thread 0)
+    const int jc = min(j1, pos);
+    const int pps = pages_per_stage(p);
+    const int blk_elems = kPageSize * HD;
+    for (int c = 0;; ++c) {
+        if (c == 0) {
+            seen_complete_wait(p, &sm.full[stage], lap & 1, &sm.flag[3]);
+        } else if (!mbar_wait_bounded(p, &sm.full[stage], lap & 1, 3)) {
+            sm.flag[3] = 1;
+            break;
+        }
+        const StageInfo inf = sm.info[stage];
+        if (inf.task != ti) {
+            set_error(p, kErrFault, ti, -4, inf.task, 0);
+            sm.flag[3] = 1;
+            break;
+        }
+        if (inf.nchunks > 0) {
+            const uint16_t* base = reinterpret_cast<const uint16_t*>(sm.ring[stage]);
+            const int first_page = inf.aux;
+            const int tok_lo = max(j0, first_page * kPageSize);
+            const int tok_hi = min(jc, (first_page + pps) * kPageSize);
+            for (int pos_t = tok_lo + warp; pos_t < tok_hi; pos_t += kConsumerWarps) {
+                int pi = pos_t / kPageSize - first_page, slot = pos_t % kPageSize;
+                const uint16_t* kb = base + (size_t)pi * 2 * blk_elems + slot * HD + lane * DPL;
+                float kf[DPL], vf[DPL];
+                load_bf16_dpl<DPL>(kb, kf);
+                load_bf16_dpl<DPL>(kb + blk_elems, vf);
+                attn_token<HPG, DPL>(st, kf, vf);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        const bool last = inf.nchunks == 0 || inf.chunk == inf.nchunks - 1;
+        if (++stage == kStages) { stage = 0; ++lap; }
+        if (last) break;
+    }
+    if (has_new && warp == 0) {
+        float kf[DPL], vf[DPL];
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) {
+            kf[d] = sm.kn[lane * DPL + d];
+            vf[d] = sm.vn[lane * DPL + d];
+        }
+        attn_token<HPG, DPL>(st, kf, vf);
+    }
+    // combine the 8 warps' partials
+    float* sc = sm.attn;
+#pragma unroll
+    for (int h = 0; h < HPG; ++h) {
+        float* w = sc + ((size_t)warp * HPG + h) * (HD + 2);
+        if (lane == 0) { w[0] = st.m[h]; w[1] = st.l[h]; }
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) w[2 + lane * DPL + d] = st.o[h][d];
+    }
+    consumer_sync();
+    if (sm.flag[3]) { abort_all = true; return; }   // same decision in every consumer thread
+    if (valid || !active_row) {
+        for (int idx = tid; idx < HPG * (HD + 2); idx += kConsumerThreads) {
+            int h = idx / (HD + 2), c = idx % (HD + 2);
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sc[((size_t)w * HPG + h) * (HD + 2)]);
+            float val;
+            if (c == 0) {
+                val = M;
+            } else {
+                float acc = 0.0f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        const float* ww = sc + ((size_t)w * HPG + h) * (HD + 2);
+                        float f = (ww[0] == -INFINITY) ? 0.0f : exp2f(ww[0] - M);
+                        acc = fmaf(ww[c], f, acc);
+                    }
+                }
+                val = acc;
+            }
+            attn_part(p, l, b, g, s, h)[c] = val;
+        }
+    }
+    // arrival; the last split of (layer, b, kv head) merges and signals
+    consumer_sync();
+    if (tid == 0) {
+        __threadfence();
+        uint32_t* cnt = p.merge_cnt + ((size_t)l * p.max_batch + b) * p.nkv + g;
+        uint32_t old = atomicAdd(cnt, 1u);
+        __threadfence();
+        sm.flag[0] = (old == (uint32_t)S * p.epoch - 1u) ? 1 : 0;
+        atomicAdd(p.done, 1u);
+    }
+    consumer_sync();
+    if (sm.flag[0]) {
+        if (valid) {
+            for (int idx = tid; idx < HPG * HD; idx += kConsumerThreads) {
+                int h = idx / HD, i = idx % HD;
+                float M = -INFINITY;
+                for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(attn_part(p, l, b, g, sp, h)));
+                float Ls = 0.0f, O = 0.0f;
+                for (int sp = 0; sp < S; ++sp) {
+                    const float* pp = attn_part(p, l, b, g, sp, h);
+                    float m = __ldcg(pp);
+                    float f = (m == -INFINITY) ? 0.0f : exp2f(m - M);
+                    Ls = fmaf(__ldcg(pp + 1), f, Ls);
+                    O = fmaf(__ldcg(pp + 2 + i), f, O);
+                }
+                p.o[((size_t)l * p.max_batch + b) * (p.nq * HD) + (size_t)(g * HPG + h) * HD + i] = O / Ls;
+            }
+        }
+        consumer_sync();
+        if (tid == 0) {
+            __threadfence();
+            if (t.sig != MK_NO_EVENT) red_release_add(&p.events[t.sig], 1u);
+        }
+    }
+    if (tid == 0 && p.trace) p.trace[(size_t)ti * 4 + 2] = globaltimer();
+}
+
+// ----------------------------------------------------------------------------- consumer: router top-k
+
+// Last router tile of a layer: softmax over the experts, top-k (ties to the
+// lower index), optional renormalisation.  Warp 0 does the work.
+__device__ void router_finalize(const Params& p, Smem& sm, int l) {
+    const int lane = threadIdx.x & 31;
+    if ((threadIdx.x >> 5) != 0) return;
+    for (int b = 0; b < p.max_batch; ++b) {
+        const float* lg = p.rlogits + ((size_t)l * p.max_batch + b) * p.E;
+        float mx = -INFINITY;
+        for (int e = lane; e < p.E; e += 32) {
+            float v = __ldcg(lg + e);
+            sm.rlog[e] = v;
+            mx = fmaxf(mx, v);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        float sum = 0.0f;
+        for (int e = lane; e < p.E; e += 32) {
+            float v = expf(sm.rlog[e] - mx);
+            sm.rlog[e] = v;
+            sum += v;
+        }
+        sum = warp_sum(sum);
+        __syncwarp();
+        float selw[kMaxTopK];
+        int sel[kMaxTopK];
+        float wsum = 0.0f;
+        for (int k = 0; k < p.topk; ++k) {
+            float best = -1.0f;
+            int bi = 0x7FFFFFFF;
+            for (int e = lane; e < p.E; e += 32) {
+                float v = sm.rlog[e];
+                if (v > best || (v == best && e < bi)) { best = v; bi = e; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                float ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+                int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+                if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+            }
+            sel[k] = bi;
+            selw[k] = best / sum;
+            wsum += selw[k];
+            __syncwarp();
+            if (lane == 0) sm.rlog[bi] = -2.0f;   // taken (probabilities are >= 0)
+            __syncwarp();
+        }
+        if (lane == 0) {
+            for (int k = 0; k < p.topk; ++k) {
+                size_t o = ((size_t)l * p.max_batch + b) * p.topk + k;
+                p.moe_sel[o] = sel[k];
+                p.moe_w[o] = p.renorm ? selw[k] / wsum : selw[k];
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// ----------------------------------------------------------------------------- consumer loop
+
+template <int HPG, int DPL>
+__device__ void consumer_loop(const Params& p, Smem& sm) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    int stage = 0;
+    uint32_t lap = 0;
+    int sig_slot = 0;
+    uint32_t sig_lap = 0;
+    int buf = 0;
+    float xr[kMaxVecPerThread][8];
+    int x_key_op = -1, x_key_layer = -1, x_key_b = -1, x_key_aux = -1;
+    uint32_t ok_evt[4] = {MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT};   // thread 0
+
+    // Every exit decision below is taken by thread 0 (or written to sm.flag[3]
+    // before a consumer barrier) and read by all consumer threads after that
+    // barrier, so all 256 consumer threads always pass the same named barriers.
+    while (true) {
+        if (tid == 0) {
+            int st = 1;                                   // 1 run, 0 abort, 2 end of work
+            if (sm.flag[3] || !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 4)) {
+                st = 0;
+            } else {
+                const int ti = sm.info[stage].task;
+                if (ti < 0) {
+                    st = 2;
+                } else {
+                    const uint32_t e = p.tasks[ti].wait0;
+                    if (p.trace) p.trace[(size_t)ti * 4 + 0] = globaltimer();
+                    if (e != MK_NO_EVENT && e != ok_evt[0] && e != ok_evt[1] && e != ok_evt[2] &&
+                        e != ok_evt[3]) {
+                        if (event_wait(p, e, p.thr[e] * p.epoch + p.wait_offset, ti)) {
+                            __threadfence();
+                            ok_evt[3] = ok_evt[2]; ok_evt[2] = ok_evt[1]; ok_evt[1] = ok_evt[0]; ok_evt[0] = e;
+                        } else {
+                            st = 0;
+                        }
+                    }
+                    if (p.trace) {
+                        p.trace[(size_t)ti * 4 + 1] = globaltimer();
+                        p.trace[(size_t)ti * 4 + 3] = (uint64_t)blockIdx.x;
+                    }
+                }
+            }
+            sm.flag[1] = st;
+        }
+        consumer_sync();
+        const int st = sm.flag[1];
+        if (st == 0) break;
+        seen_complete_wait(p, &sm.full[stage], lap & 1, &sm.flag[3]);   // seen complete by thread 0
+        const int ti = sm.info[stage].task;
+        if (st == 2) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);
+            break;
+        }
+        const Task t = p.tasks[ti];
+
+        if (t.op == MK_OP_ATTN) {
+            bool abort_all = false;
+            attention_task<HPG, DPL>(p, sm, t, ti, stage, lap, abort_all);
+            if (abort_all) break;
+            // the input slice in registers is dead across an attention task (saves registers)
+            x_key_op = -1;
+#pragma unroll
+            for (int j = 0; j < kMaxVecPerThread; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) xr[j][e] = 0.0f;
+            continue;
+        }
+
+        // ---- GEMV task
+        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
+        GemvGeom g;
+        gemv_geom(p, t, g, false);
+        const ThreadMap m = thread_map(g.K);
+        if (!skip) {
+            if (t.op == MK_OP_QKV && t.layer == 0 && tid == 0) {
+                int tok = p.tokens[0];
+                if (tok < 0 || tok >= p.V) set_error(p, kErrInvalid, ti, -5, tok, 0);
+            }
+            if (!(x_key_op == t.op && x_key_layer == t.layer && x_key_b == t.b &&
+                  (x_key_aux == t.aux || t.op != MK_OP_EXP_DOWN))) {
+                gemv_prologue(p, sm, t, m, g.K, xr);
+                x_key_op = t.op; x_key_layer = t.layer; x_key_b = t.b; x_key_aux = t.aux;
+            }
+        }
+        const int rows_total = g.rows * g.nblk;
+        for (int c = 0;; ++c) {
+            if (c > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) {
+                sm.flag[3] = 1;
+                break;
+            }
+            const StageInfo inf = sm.info[stage];
+            if (inf.task != ti) {
+                set_error(p, kErrFault, ti, -4, inf.task, 1);
+                sm.flag[3] = 1;
+                break;
+            }
+            if (inf.nchunks > 0) {
+                const int nch_blk = inf.nchunks / g.nblk;
+                const int blk = inf.chunk / nch_blk, ci = inf.chunk % nch_blk;
+                const int64_t blk_vecs = (int64_t)g.rows * m.nvec;
+                const int c0 = ci * (kStageBytes / 16);
+                const int c1 = (int)((blk_vecs < (int64_t)c0 + kStageBytes / 16) ? blk_vecs : (int64_t)c0 + kStageBytes / 16);
+                gemv_chunk(sm, buf, sm.ring[stage], m, g.rows, blk, c0, c1, xr);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);
+            const bool last = inf.nchunks == 0 || inf.chunk == inf.nchunks - 1;
+            if (++stage == kStages) { stage = 0; ++lap; }
+            if (last) break;
+        }
+        consumer_sync();   // all partial sums of this task are in red[buf]
+        if (sm.flag[3]) break;
+
+        // ---- epilogue: reduce the warps' partials in fixed order, apply the op's output rule
+        if (!skip) {
+            const int l = t.layer, b = t.b;
+            const int nout = (g.nblk == 2) ? g.rows : rows_total;
+            for (int r = tid; r < nout; r += kConsumerThreads) {
+                float y = 0.0f;
+                for (int w = 0; w < m.wpg; ++w) y += sm.red[buf][r][w];
+                const int row = (int)t.r0 + r;
+                switch (t.op) {
+                    case MK_OP_QKV:
+                        p.qkv[((size_t)l * p.max_batch) * ((p.nq + 2 * p.nkv) * p.hd) + row] = y;
+                        break;
+                    case MK_OP_OPROJ:
+                        p.x_mid[((size_t)l * p.max_batch) * p.H + row] = x_in(p, l, 0, row) + y;
+                        break;
+                    case MK_OP_GATEUP: {
+                        float u = 0.0f;
+                        for (int w = 0; w < m.wpg; ++w) u += sm.red[buf][g.rows + r][w];
+                        p.act[((size_t)l * p.max_batch) * p.F + row] = silu_f(y) * u;
+                        break;
+                    }
+                    case MK_OP_DOWN:
+                        p.x_out[((size_t)l * p.max_batch) * p.H + row] = x_mid_at(p, l, 0, row) + y;
+                        break;
+                    case MK_OP_LMHEAD:
+                        p.logits[row] = y;
+                        break;
+                    case MK_OP_ROUTER:
+                        p.rlogits[((size_t)l * p.max_batch) * p.E + row] = y;
+                        break;
+                    case MK_OP_EXP_GATEUP: {
+                        float u = 0.0f;
+                        for (int w = 0; w < m.wpg; ++w) u += sm.red[buf][g.rows + r][w];
+                        p.act[(((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.Fe + row] = silu_f(y) * u;
+                        break;
+                    }
+                    case MK_OP_EXP_DOWN:
+                        p.ypart[(((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.H + row] = y;
+                        break;
+                    default:
+                        break;
+                }
+            }
+        }
+        buf ^= 1;
+
+        if (t.op == MK_OP_ROUTER) {
+            // arrival; the last router tile of the layer selects the experts and signals
+            consumer_sync();
+            if (tid == 0) {
+                __threadfence();
+                uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
+                __threadfence();
+                sm.flag[0] = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
+                atomicAdd(p.done, 1u);
+            }
+            consumer_sync();
+            if (sm.flag[0]) {
+                router_finalize(p, sm, t.layer);
+                consumer_sync();
+                if (tid == 0) {
+                    __threadfence();
+                    if (t.sig != MK_NO_EVENT) red_release_add(&p.events[t.sig], 1u);
+                }
+            }
+            if (tid == 0 && p.trace) p.trace[(size_t)ti * 4 + 2] = globaltimer();
+            continue;
+        }
+
+        // ---- hand the completion to the signal warp (its fence does not stall the consumers)
+        if (tid == 0) {
+            if (sig_lap > 0 && !mbar_wait_bounded(p, &sm.sig_empty[sig_slot], (sig_lap - 1) & 1, 6))
+                sm.flag[3] = 1;
+            sm.sig_evt[sig_slot] = t.sig;
+            sm.sig_task[sig_slot] = ti;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sig_full[sig_slot]);
+        if (++sig_slot == kSigSlots) { sig_slot = 0; ++sig_lap; }
+    }
+    // end of work for the signal warp
+    consumer_sync();
+    if (tid == 0) {
+        if (sig_lap > 0) (void)mbar_wait_bounded(p, &sm.sig_empty[sig_slot], (sig_lap - 1) & 1, 7);
+        sm.sig_evt[sig_slot] = 0xFFFFFFFEu;
+        sm.sig_task[sig_slot] = -1;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.sig_full[sig_slot]);
+}
+
+// ----------------------------------------------------------------------------- kernel
+
+template <int HPG, int DPL>
+__global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], kConsumerWarps);
+        }
+        for (int s = 0; s < kSigSlots; ++s) {
+            mbar_init(&sm.sig_full[s], kConsumerWarps);
+            mbar_init(&sm.sig_empty[s], 1);
+        }
+        for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp < kConsumerWarps) {
+        consumer_loop<HPG, DPL>(p, sm);
+    } else if (warp == kProducerWarp) {
+        if (lane == 0) producer_loop(p, sm);
+    } else {
+        if (lane == 0) signal_loop(p, sm);
+    }
+}
+
+// ----------------------------------------------------------------------------- host launch
+
+template <int HPG, int DPL>
+static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream) {
+    auto kern = megakernel<HPG, DPL>;
+    static bool attr_set = false;   // per instantiation; set before first launch on each device use
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(Smem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+    (void)attr_set;
+    void* args[] = {const_cast<Params*>(&p)};
+    return cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kThreads), args,
+                                       sizeof(Smem), stream);
+}
+
+size_t megakernel_smem_bytes() { return sizeof(Smem); }
+
+cudaError_t megakernel_launch(const Params& p, int grid, cudaStream_t stream) {
+    const int hpg = p.nq / p.nkv;
+    const int dpl = p.hd / 32;
+    if (dpl == 4) {
+        switch (hpg) {
+            case 1: return launch_t<1, 4>(p, grid, stream);
+            case 2: return launch_t<2, 4>(p, grid, stream);
+            case 4: return launch_t<4, 4>(p, grid, stream);
+            case 8: return launch_t<8, 4>(p, grid, stream);
+        }
+    } else if (dpl == 2) {
+        switch (hpg) {
+            case 1: return launch_t<1, 2>(p, grid, stream);
+            case 2: return launch_t<2, 2>(p, grid, stream);
+            case 4: return launch_t<4, 2>(p, grid, stream);
+            case 8: return launch_t<8, 2>(p, grid, stream);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+bool megakernel_supports(int hpg, int hd) {
+    return (hd == 64 || hd == 128) && (hpg == 1 || hpg == 2 || hpg == 4 || hpg == 8);
+}
+
+cudaError_t megakernel_occupancy(int hpg, int hd, int* blocks_per_sm) {
+    const int dpl = hd / 32;
+    const void* f = nullptr;
+    if (dpl == 4) {
+        if (hpg == 1) f = (const void*)megakernel<1, 4>;
+        if (hpg == 2) f = (const void*)megakernel<2, 4>;
+        if (hpg == 4) f = (const void*)megakernel<4, 4>;
+        if (hpg == 8) f = (const void*)megakernel<8, 4>;
+    } else {
+        if (hpg == 1) f = (const void*)megakernel<1, 2>;
+        if (hpg == 2) f = (const void*)megakernel<2, 2>;
+        if (hpg == 4) f = (const void*)megakernel<4, 2>;
+        if (hpg == 8) f = (const void*)megakernel<8, 2>;
+    }
+    if (!f) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, f, kThreads, sizeof(Smem));
+}
+
+}  // namespace mk

@@ -1,0 +1,113 @@
+// Internal layout shared by the host task-graph compiler and the megakernel.
+// Plain C++ (no CUDA types) so the host compiler can include it.
+#pragma once
+
+#include <stdint.h>
+
+#include "../../include/mk.h"
+
+namespace mk {
+
+// Kernel geometry.  One CTA per SM: 8 consumer warps compute, 1 producer warp
+// streams weights and KV pages into a shared-memory ring with bulk async copies,
+// 1 signal warp publishes task completions.
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kProducerWarp = kConsumerWarps;        // warp 8
+constexpr int kSignalWarp = kConsumerWarps + 1;      // warp 9
+constexpr int kThreads = (kConsumerWarps + 2) * 32;  // 320
+constexpr int kStageBytes = 16 * 1024;
+constexpr int kStages = 11;
+constexpr int kMaxTaskRows = 64;        // rows (all weight blocks) of one GEMV task
+constexpr int kMaxVecPerThread = 8;     // 16-byte vectors of x per consumer thread (K <= 16384)
+constexpr int kSigSlots = 8;            // signal queue depth
+constexpr int kMaxHeadsPerGroup = 8;
+constexpr int kMaxTopK = 16;
+constexpr int kPageSize = 16;
+
+// Device task record (32 bytes).
+struct Task {
+    uint8_t op;
+    uint8_t flags;
+    uint16_t layer;
+    uint16_t b;      // batch row (attention / expert tasks)
+    uint16_t aux;    // kv head (attention) or expert slot (expert tasks)
+    uint32_t r0, r1; // output rows; attention: split index, split count
+    uint32_t wait0, wait1;
+    uint32_t sig;
+    uint32_t pad;
+};
+static_assert(sizeof(Task) == 32, "task record is 32 bytes");
+
+// Per-layer weight pointers (bf16 bits).
+struct LayerW {
+    const uint16_t* attn_norm;
+    const uint16_t* wq;
+    const uint16_t* wk;
+    const uint16_t* wv;
+    const uint16_t* wo;
+    const uint16_t* ffn_norm;
+    const uint16_t* w_router;
+    const uint16_t* w_gate;
+    const uint16_t* w_up;
+    const uint16_t* w_down;
+};
+
+struct Params {
+    // task list and synchronisation
+    const Task* tasks;
+    uint32_t n_tasks;
+    uint32_t epoch;              // 1-based step counter; thresholds are thr * epoch
+    const uint32_t* thr;         // per-event threshold per step
+    uint32_t* events;
+    unsigned long long* queue;   // global work-queue head
+    unsigned long long queue_base;
+    uint32_t* done;              // completed-task counter
+    int* err;                    // [0] status, [1..4] info
+    uint32_t* merge_cnt;         // [L][max_batch][n_kv] attention split arrivals
+    uint32_t* router_cnt;        // [L] router tile arrivals
+    long long timeout_ns;
+    uint32_t wait_offset;        // added to every wait target (0; tests set 1 to force a timeout)
+    unsigned long long* trace;   // [n_tasks][4] or null
+
+    // model
+    const LayerW* layers;
+    const uint16_t* tok_emb;
+    const uint16_t* final_norm;
+    const uint16_t* lm_head;
+    int L, H, nq, nkv, hd, F, V, E, topk, Fe, renorm;
+    float eps;
+    int max_ctx, max_batch, S, n_router_tiles;
+    const float* rope;           // [max_ctx][hd/2][2] = cos, sin (fp32)
+
+    // activations (fp32), per layer
+    float* x_mid;    // [L][B][H]   residual after attention
+    float* x_out;    // [L][B][H]   residual after the dense FFN
+    float* qkv;      // [L][B][(nq+2nkv)*hd]
+    float* o;        // [L][B][nq*hd] merged attention output
+    float* act;      // dense: [L][B][F]; MoE: [L][B][topk][Fe]
+    float* part;     // [L][B][nkv][S][hpg][hd+2] attention partials
+    float* rlogits;  // [L][B][E]
+    float* moe_w;    // [L][B][topk]
+    int* moe_sel;    // [L][B][topk]
+    float* ypart;    // [L][B][topk][H]
+
+    // per step
+    const int* tokens;
+    const int* positions;        // may be null (then position = pos_offset)
+    int pos_offset;
+    int batch;
+    int skip_lm;                 // 1: LM-head tasks do nothing
+    uint16_t* k_pages;
+    uint16_t* v_pages;
+    const int* page_table;
+    int n_pages, max_pages;
+    float* logits;
+};
+
+// Error status values written by the device (match mk_status).
+constexpr int kErrInvalid = MK_ERR_INVALID_ARG;
+constexpr int kErrTimeout = MK_ERR_TIMEOUT;
+constexpr int kErrFault = MK_ERR_DEVICE_FAULT;
+
+}  // namespace mk

@@ -1,0 +1,208 @@
+"""CPU executor of an exported task graph, in random valid orders (test support).
+
+Each task is executed symbolically: it reads the tensor elements the kernel's
+tile for that task reads and writes a 64-bit digest of (task, inputs) to the
+elements it writes.  A task may run only when its events have reached their
+thresholds (the kernel's rule).  Reading an element nobody has written yet,
+or writing one twice, is a violation.  If the events are sufficient for every
+read, every valid order produces the same final digests ("identical bits").
+
+Read/write sets per operator mirror the megakernel's tiles:
+  qkv      reads x_in[l] (all)                 writes qkv[l][rows]
+  attn     reads qkv[l] rows of its kv head    writes part[l,b,g,s]; the last split
+           of (l,b,g) reads all its parts and writes o[l][b][rows of g]
+  oproj    reads o[l] (all), x_in[l][rows]     writes x_mid[l][rows]
+  gateup   reads x_mid[l] (all)                writes act[l][rows]
+  down     reads act[l] (all), x_mid[l][rows]  writes x_in[l+1][rows]
+  router   reads x_mid[l] (all)                writes rlog[l][rows]; the last tile reads
+           rlog[l] (all) and writes sel[l]
+  exp_gu   reads sel[l], x_mid[l] (all)        writes acte[l][k][rows]
+  exp_dn   reads sel[l], acte[l][k] (all)      writes ypart[l][k][rows]
+  lmhead   reads x_in[L] (all)                 writes logits[rows]
+For MoE models x_in[l+1][i] is x_mid[l][i] combined with ypart[l][k][i] for all k
+and the routing weights sel[l].
+"""
+from __future__ import annotations
+
+import random
+from collections import defaultdict
+from typing import Dict, List
+
+import numpy as np
+
+OP = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
+      8: "exp_gu", 9: "exp_dn"}
+NO_EVENT = 0xFFFFFFFF
+M64 = (1 << 64) - 1
+
+
+class Violation(AssertionError):
+    pass
+
+
+def _mix(a: int) -> int:
+    a = (a + 0x9E3779B97F4A7C15) & M64
+    a = ((a ^ (a >> 30)) * 0xBF58476D1CE4E5B9) & M64
+    a = ((a ^ (a >> 27)) * 0x94D049BB133111EB) & M64
+    return a ^ (a >> 31)
+
+
+class Tensor:
+    def __init__(self, n: int, ready: bool = False):
+        self.val = np.zeros(n, dtype=np.uint64)
+        self.ok = np.full(n, ready, dtype=bool)
+        if ready:
+            self.val[:] = np.arange(n, dtype=np.uint64) * np.uint64(2654435761)
+
+    def read(self, lo: int, hi: int, who: str) -> int:
+        if not self.ok[lo:hi].all():
+            raise Violation(f"{who} read unwritten elements [{lo},{hi})")
+        return int(self.val[lo:hi].sum(dtype=np.uint64))
+
+    def write(self, lo: int, hi: int, digest: int, who: str) -> None:
+        if self.ok[lo:hi].any():
+            raise Violation(f"{who} wrote [{lo},{hi}) twice")
+        self.ok[lo:hi] = True
+        self.val[lo:hi] = (np.arange(lo, hi, dtype=np.uint64) * np.uint64(0x100000001B3)) ^ np.uint64(digest)
+
+
+def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
+    """Executes all tasks once in a random valid order; returns final digests."""
+    L, H, nq, nkv, hd = shape["L"], shape["H"], shape["nq"], shape["nkv"], shape["hd"]
+    B, E, K, Fe, F, V = shape["B"], shape["E"], shape["topk"], shape["Fe"], shape["F"], shape["V"]
+    hpg = nq // nkv
+    qkv_rows = (nq + 2 * nkv) * hd
+    moe = E > 0
+    T: Dict[tuple, Tensor] = {}
+
+    def t(*key) -> Tensor:
+        return T[key]
+
+    T[("x_in", 0)] = Tensor(B * H, ready=True)      # embedding rows: inputs of the step
+    for l in range(L):
+        T[("qkv", l)] = Tensor(qkv_rows)
+        T[("o", l)] = Tensor(B * nq * hd)
+        T[("x_mid", l)] = Tensor(B * H)
+        if moe:
+            T[("rlog", l)] = Tensor(E)
+            T[("sel", l)] = Tensor(B * K)
+            for k in range(K):
+                T[("acte", l, k)] = Tensor(B * Fe)
+                T[("ypart", l, k)] = Tensor(B * H)
+        else:
+            T[("act", l)] = Tensor(F)
+            T[("x_in", l + 1)] = Tensor(B * H)
+    T[("logits",)] = Tensor(V)
+    parts = defaultdict(int)          # (l,b,g) -> arrivals
+    part_digest = defaultdict(int)
+    router_arr = defaultdict(int)
+    n_router = defaultdict(int)
+    for tk in tasks:
+        if tk.op == 7:
+            n_router[tk.layer] += 1
+
+    def read_xin(l: int, lo: int, hi: int, who: str) -> int:
+        if l == 0 or not moe:
+            return t("x_in", l).read(lo, hi, who)
+        d = t("x_mid", l - 1).read(lo, hi, who) + t("sel", l - 1).read(0, B * K, who)
+        for k in range(K):
+            d += t("ypart", l - 1, k).read(lo, hi, who)
+        return d & M64
+
+    counters = [0] * len(thr)
+    pending = [0] * len(tasks)
+    waiters = defaultdict(list)
+    for i, tk in enumerate(tasks):
+        evs = {e for e in (tk.wait[0], tk.wait[1]) if e != NO_EVENT}
+        pad = tk.pointer_wait
+        if pad != NO_EVENT:
+            evs.add(pad)
+        pending[i] = len(evs)
+        for e in evs:
+            waiters[e].append(i)
+    rng = random.Random(seed)
+    ready = [i for i in range(len(tasks)) if pending[i] == 0]
+    done = 0
+
+    def signal(e: int) -> None:
+        if e == NO_EVENT:
+            return
+        counters[e] += 1
+        if counters[e] == thr[e]:
+            for w in waiters[e]:
+                pending[w] -= 1
+                if pending[w] == 0:
+                    ready.append(w)
+        if counters[e] > thr[e]:
+            raise Violation(f"event {e} signalled beyond its threshold")
+
+    while ready:
+        j = rng.randrange(len(ready))
+        ready[j], ready[-1] = ready[-1], ready[j]
+        i = ready.pop()
+        tk = tasks[i]
+        op, l, r0, r1 = OP[tk.op], tk.layer, tk.r0, tk.r1
+        who = f"task {i} ({op} l{l} b{tk.b} aux{tk.aux} {r0}:{r1})"
+        base = _mix(i + 1)
+        if op == "qkv":
+            d = read_xin(l, 0, H, who)
+            t("qkv", l).write(r0, r1, _mix(base ^ d), who)
+            signal(tk.signal)
+        elif op == "attn":
+            g, b = tk.aux, tk.b
+            qkv = t("qkv", l)
+            d = qkv.read(g * hpg * hd, (g + 1) * hpg * hd, who)
+            d += qkv.read(nq * hd + g * hd, nq * hd + (g + 1) * hd, who)
+            d += qkv.read((nq + nkv) * hd + g * hd, (nq + nkv) * hd + (g + 1) * hd, who)
+            key = (l, b, g)
+            part_digest[key] = (part_digest[key] + _mix(base ^ d)) & M64
+            parts[key] += 1
+            if parts[key] == r1:                      # last split merges and signals
+                lo = b * nq * hd + g * hpg * hd
+                t("o", l).write(lo, lo + hpg * hd, part_digest[key], who)
+                signal(tk.signal)
+        elif op == "oproj":
+            d = t("o", l).read(0, B * nq * hd, who) + read_xin(l, r0, r1, who)
+            t("x_mid", l).write(r0, r1, _mix(base ^ (d & M64)), who)
+            signal(tk.signal)
+        elif op == "gateup":
+            d = t("x_mid", l).read(0, B * H, who)
+            t("act", l).write(r0, r1, _mix(base ^ d), who)
+            signal(tk.signal)
+        elif op == "down":
+            d = t("act", l).read(0, F, who) + t("x_mid", l).read(r0, r1, who)
+            t("x_in", l + 1).write(r0, r1, _mix(base ^ (d & M64)), who)
+            signal(tk.signal)
+        elif op == "router":
+            d = t("x_mid", l).read(0, B * H, who)
+            t("rlog", l).write(r0, r1, _mix(base ^ d), who)
+            router_arr[l] += 1
+            if router_arr[l] == n_router[l]:
+                d2 = t("rlog", l).read(0, E, who)
+                t("sel", l).write(0, B * K, _mix(d2), who)
+                signal(tk.signal)
+        elif op == "exp_gu":
+            d = t("sel", l).read(0, B * K, who) + t("x_mid", l).read(0, B * H, who)
+            lo = tk.b * Fe
+            t("acte", l, tk.aux).write(lo + r0, lo + r1, _mix(base ^ (d & M64)), who)
+            signal(tk.signal)
+        elif op == "exp_dn":
+            d = t("sel", l).read(0, B * K, who) + t("acte", l, tk.aux).read(tk.b * Fe, (tk.b + 1) * Fe, who)
+            lo = tk.b * H
+            t("ypart", l, tk.aux).write(lo + r0, lo + r1, _mix(base ^ (d & M64)), who)
+            signal(tk.signal)
+        elif op == "lmhead":
+            d = read_xin(L, 0, H, who)
+            t("logits").write(r0, r1, _mix(base ^ d), who)
+            signal(tk.signal)
+        else:
+            raise Violation(f"unknown op {tk.op}")
+        done += 1
+    if done != len(tasks):
+        raise Violation(f"only {done} of {len(tasks)} tasks could run (deadlock)")
+    for e, (c, th) in enumerate(zip(counters, thr)):
+        if c != th:
+            raise Violation(f"event {e}: counter {c} != threshold {th}")
+    if not T[("logits",)].ok.all():
+        raise Violation("logits not fully written")
+    return {"logits": T[("logits",)].val.copy()}
