@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Decode throughput of the persistent megakernel on B200.
+
+Default workload: an 8B-class dense decoder (32 layers, hidden 4096, 32/8
+heads, head_dim 128, FFN 14336, vocab 128256; bf16 weights ~N(0, 0.02)),
+batch 1, a 39-token prompt and 512 decode steps over a contiguous KV cache
+(the workload of the MPK digest, section "MPK का मुख्य मूल्य").  One step =
+one decode step = one launch of the megakernel.  Tokens are seeded synthetic
+ids fed teacher-forced; positions cycle over 39..550.
+
+Metric: decode tokens/s at batch 1, and its fraction of the HBM
+speed-of-light bound  tokens/s_SoL = 8e12 B/s / (weight bytes + KV bytes per
+step)  (Cohere page, section "A szűk keresztmetszet a memória-sávszélesség").
+
+Multi-GPU: replicas only (each rank decodes its own sequence with its own full
+weight copy; no collective on the data path); value = all ranks' tokens / the
+slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s at batch 1 and % of HBM speed-of-light (bytes/step ÷ peak)"
+SOL_BW = 8.0e12            # nominal B200 HBM bandwidth used for the speed-of-light bound
+PROMPT = 39
+GEN = 512
+
+
+# ----------------------------------------------------------------------------- arithmetic
+
+def sol_tokens_per_s(bytes_per_step: float, bandwidth: float, batch: int = 1) -> float:
+    """Speed-of-light decode rate: every step must read its bytes once at `bandwidth`."""
+    return batch * bandwidth / bytes_per_step
+
+
+def kv_read_bytes(cfg, positions) -> float:
+    """Mean KV bytes read per step: (p+1) cached tokens x layers x (K,V) x heads x dim x 2 B."""
+    per_tok = cfg.n_layers * 2 * cfg.n_kv_heads * cfg.head_dim * 2
+    return sum((p + 1) * per_tok for p in positions) / len(positions)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.out,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+        mhz = [num(r[1]) for r in rows]
+        mx = max(num(r[2]) for r in rows)
+        power = [num(r[3]) for r in rows]
+        loaded = [m for m, pw in zip(mhz, power) if pw > 250.0] or mhz
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def workload(name: str):
+    import synthetic as syn
+    if name == "llama8b":
+        return dict(cfg=syn.LLAMA8B, seed=2, prompt=PROMPT, gen=GEN, ctx0=0,
+                    desc="llama-8b-class dense decode, batch 1, 39-token prompt + 512 steps, "
+                         "contiguous KV")
+    if name == "tiny":
+        return dict(cfg=syn.TINY, seed=1, prompt=PROMPT, gen=16, ctx0=0,
+                    desc="tiny 2-layer decoder, batch 1, 39-token prompt + 16 steps")
+    if name == "moe30b":
+        return dict(cfg=syn.MOE30B, seed=3, prompt=8192, gen=256, ctx0=8192,
+                    desc="30B-total/3.3B-active MoE decode, batch 1, 8192-token synthetic KV, "
+                         "256 steps")
+    if name == "long131k":
+        return dict(cfg=syn.LLAMA8B, seed=5, prompt=131072, gen=64, ctx0=131072,
+                    desc="llama-8b-class decode, batch 1, 131072-token synthetic paged KV "
+                         "(shuffled 16-token pages), 64 steps")
+    raise SystemExit(f"unknown workload {name}")
+
+
+def dist_info():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def oracle_rate(W: dict, max_steps: int, budget_s: float, warmup: int = 1):
+    """Times the CPU oracle on a bounded sample of the workload; returns (tok/s, steps, desc)."""
+    import numpy as np
+    import oracle
+    import synthetic as syn
+    cfg = W["cfg"]
+    seed = syn.SEED_WEIGHTS + W["seed"]
+    ctx = W["prompt"]
+    cap = ctx + max_steps + warmup + 1
+    specs = syn.tensor_specs(cfg)
+    names = [s.name for s in specs]
+    if cfg.is_moe:
+        # experts are regenerated on demand (all 128 per layer do not fit host memory)
+        by_name = {s.name: s for s in specs}
+        experts = ("w_gate", "w_up", "w_down")
+        host_w = {s.name: syn.host_tensor(s, seed) for s in specs
+                  if not any(s.name.endswith(e) for e in experts)}
+        n = cfg.expert_ffn * cfg.hidden
+
+        def prov(l, e, which):
+            s = by_name[f"layers.{l}.{experts[which]}"]
+            return syn.host_bf16(n, seed, s.tensor_id, s.sigma, s.mean, offset=e * n)
+        model = oracle.Model(cfg, host_w, cap, names, expert_provider=prov)
+    else:
+        model = oracle.Model(cfg, syn.host_weights(cfg, seed), cap, names)
+    for l in range(cfg.n_layers):     # synthetic context standing in for the prompt
+        model.k[l][:ctx] = syn.host_kv(cfg, syn.SEED_KV + W["seed"], l, "k", 0, 0, ctx)
+        model.v[l][:ctx] = syn.host_kv(cfg, syn.SEED_KV + W["seed"], l, "v", 0, 0, ctx)
+    toks = syn.host_tokens(warmup + max_steps, syn.SEED_PROMPT + W["seed"], cfg.vocab)
+    for i in range(warmup):
+        model.decode_step(int(toks[i]), ctx + i)
+    t0 = time.perf_counter()
+    n = 0
+    while n < max_steps:
+        model.decode_step(int(toks[warmup + n]), ctx + warmup + n)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    sample = (f"{n} decode step(s) of the same model at positions {ctx + warmup}..{ctx + warmup + n - 1} "
+              f"over a {ctx}-token synthetic context, after {warmup} warm-up step(s)")
+    return n / dt, n, sample, oracle.num_threads()
+
+
+def run_reference(args, W):
+    rank, world, _ = dist_info()
+    if rank != 0:
+        return
+    rate, n, sample, cores = oracle_rate(W, max(1, args.steps), budget_s=float(args.ref_budget),
+                                         warmup=min(args.warmup, 1))
+    line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
+            "n_gpus": world, "steps": n, "warmup": min(args.warmup, 1),
+            "ms_per_step": 1000.0 / rate, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": W["desc"], "batch": 1},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, W):
+    import numpy as np
+    import torch
+    import synthetic as syn
+    import persistent_megakernel_decode_03_b200 as mk
+    from persistent_megakernel_decode_03_b200.runner import Decoder
+
+    rank, world, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+        pg = dist
+    cfg = W["cfg"]
+    seed = syn.SEED_WEIGHTS + W["seed"]
+    specs = syn.tensor_specs(cfg)
+    ts = []
+    for s in specs:
+        t = torch.empty(s.shape, dtype=torch.bfloat16, device=dev)
+        syn.dev_fill_tensor(t, s, seed)
+        ts.append(t)
+    n_steps_total = args.warmup + args.steps
+    ctx0 = W["ctx0"]
+    span = W["gen"]                       # positions cycle over [prompt, prompt + gen)
+    max_ctx = W["prompt"] + span
+    desc = dict(n_layers=cfg.n_layers, hidden=cfg.hidden, n_q_heads=cfg.n_q_heads,
+                n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, ffn=cfg.ffn, vocab=cfg.vocab,
+                rms_eps=cfg.rms_eps, rope_theta=cfg.rope_theta, n_experts=cfg.n_experts,
+                top_k=cfg.top_k, expert_ffn=cfg.expert_ffn, moe_renorm=cfg.moe_renorm)
+    page_table = None
+    n_pages = None
+    if args.workload == "long131k":
+        pages = (max_ctx + 15) // 16
+        perm = syn.page_permutation(pages, syn.SEED_KV + W["seed"])
+        page_table = torch.tensor(perm, dtype=torch.int32, device=dev).view(1, pages)
+        n_pages = pages
+    dec = Decoder(desc, [t.data_ptr() for t in ts], 1, max_ctx, page_table=page_table,
+                  n_pages=n_pages, device=f"cuda:{local}")
+    stream = torch.cuda.current_stream(dev)
+    prompt_toks = torch.tensor(syn.host_tokens(W["prompt"], syn.SEED_PROMPT + W["seed"], cfg.vocab),
+                               dtype=torch.int32, device=dev)
+    if ctx0 > 0:
+        for l in range(cfg.n_layers):
+            syn.dev_fill_kv_paged(dec.k_pages[l], dec.page_table[0], 0, 0, ctx0, cfg, 16,
+                                  syn.SEED_KV + W["seed"], syn.TID_K_BASE + l)
+            syn.dev_fill_kv_paged(dec.v_pages[l], dec.page_table[0], 0, 0, ctx0, cfg, 16,
+                                  syn.SEED_KV + W["seed"], syn.TID_V_BASE + l)
+    else:
+        dec.prefill(prompt_toks)          # the 39-token prompt through the same megakernel
+    dec.check()
+    gen_toks = syn.host_tokens(n_steps_total, syn.SEED_PROMPT + 100 + W["seed"], cfg.vocab)
+    positions = [W["prompt"] + (i % span) for i in range(n_steps_total)]
+    toks_d = torch.tensor(gen_toks, dtype=torch.int32, device=dev)
+    pos_d = torch.tensor(positions, dtype=torch.int32, device=dev)
+
+    def launch(i):
+        mk.mk_decode_step(dec.state, toks_d[i:].data_ptr(), pos_d[i:].data_ptr(), 1, dec.kv,
+                          dec.logits.data_ptr(), stream.cuda_stream)
+
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize(dev)
+    st = dec.sync()
+    if st != mk.MK_OK:
+        raise SystemExit(f"warm-up failed: {mk.mk_last_error_string()}")
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    clocks = ClockSampler(local)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    torch.cuda.nvtx.range_push("timed")
+    events[0].record(stream)
+    for k in range(args.steps):
+        launch(args.warmup + k)
+        events[k + 1].record(stream)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if pg:
+        pg.barrier()
+    st = dec.sync()
+    if st != mk.MK_OK:
+        raise SystemExit(f"timed steps failed: {mk.mk_last_error_string()}")
+    per = [events[k].elapsed_time(events[k + 1]) for k in range(args.steps)]
+    total_ms = events[0].elapsed_time(events[-1])
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    timed_pos = positions[args.warmup:]
+    info = dec.info
+    bytes_step = float(info.weight_bytes_per_step) + kv_read_bytes(cfg, timed_pos)
+    tok_s = world * args.steps / (total_ms / 1e3)
+    sol = sol_tokens_per_s(bytes_step, SOL_BW)
+    peak, peak_kind = measured_peaks()
+    launch_ms = statistics.mean(per)
+    achieved = bytes_step / (launch_ms / 1e3) / 1e9
+
+    # end to end through the host-buffer entry point: H2D of token+position, D2H of logits
+    e2e = None
+    if not args.no_e2e:
+        k_e2e = min(args.steps, 100)
+        tok_h = torch.tensor(gen_toks, dtype=torch.int32).pin_memory()
+        pos_h = torch.tensor(positions, dtype=torch.int32).pin_memory()
+        logits_h = torch.empty((1, cfg.vocab), dtype=torch.float32).pin_memory()
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in range(k_e2e):
+            i = args.warmup + k
+            mk.mk_decode_step_host(dec.state, tok_h[i:].data_ptr(), pos_h[i:].data_ptr(), 1, dec.kv,
+                                   logits_h.data_ptr(), stream.cuda_stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([e2e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        if dec.sync() != mk.MK_OK:
+            raise SystemExit(f"e2e steps failed: {mk.mk_last_error_string()}")
+        e2e = {"value": world * k_e2e / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": 8, "d2h_bytes_per_step": 4 * cfg.vocab, "steps": k_e2e,
+               "api": "mk_decode_step_host"}
+
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tr = json.load(f)
+        ent = tr.get(args.workload)
+        if ent and ent.get("kernel_source_sha") == kernel_source_sha():
+            traffic = ent["bytes_per_launch"]
+    line = {
+        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": W["desc"], "batch": 1, "weights": "bf16", "activations": "f32",
+                   "kv_cache": "bf16", "positions": [timed_pos[0], max(timed_pos)],
+                   "l2": "inputs larger than L2 (every step streams all weights)",
+                   "parallelism": "replicas" if world > 1 else "single-gpu"},
+        "sol_pct": 100.0 * tok_s / world / sol,
+        "sol_tokens_per_s": sol,
+        "bytes_per_step": bytes_step,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+                     "kernel": "mk::megakernel", "launch_ms": launch_ms},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, sample, cores = oracle_rate(W, 3 if cfg.n_layers > 2 else 16, budget_s=25.0)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dec.close()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def kernel_source_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("megakernel.cu", "mk_internal.h", "graph.cpp"):
+        with open(os.path.join(ROOT, "persistent_megakernel_decode_03_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=507)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mk", "reference"], default="mk")
+    ap.add_argument("--workload", default="llama8b", choices=["llama8b", "tiny", "moe30b", "long131k"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of CPU time the reference arm may spend on timed steps")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "mk":
+        raise SystemExit("at least 3 warm-up steps")
+    W = workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, W)
+    else:
+        run_gpu(args, W)
+
+
+if __name__ == "__main__":
+    main()
