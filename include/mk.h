@@ -264,6 +264,12 @@ mk_status mk_state_read_buffer(mk_state* state, int which, int layer, float* hos
  * [n_tasks][4] = {wait start ns, compute start ns, end ns, sm id}. */
 mk_status mk_state_read_trace(mk_state* state, uint64_t* host, int cap_tasks, mk_stream stream);
 
+/* Per-CTA cycle counters accumulated since the last read (needs
+ * MK_FLAG_TRACE), then cleared: host uint64 [n_sm][8] = {producer waits for a
+ * free ring slot, consumer waits for streamed data, dependency waits, kernel
+ * cycles, -, signal-slot waits, -, -}. */
+mk_status mk_state_read_stats(mk_state* state, uint64_t* host, int cap, mk_stream stream);
+
 /* Text of the last error of the calling thread ("" if none). */
 const char* mk_last_error_string(void);
 

@@ -40,7 +40,8 @@ SYMBOLS = (
     "mk_wave_stats", "mk_state_create", "mk_state_destroy", "mk_state_set_timeout",
     "mk_state_debug_wait_offset",
     "mk_decode_step", "mk_decode_step_host", "mk_prefill", "mk_sync", "mk_state_read_counters",
-    "mk_state_read_buffer", "mk_state_read_trace", "mk_last_error_string", "mk_version",
+    "mk_state_read_buffer", "mk_state_read_trace", "mk_state_read_stats", "mk_last_error_string",
+    "mk_version",
 )
 
 
@@ -118,6 +119,7 @@ def lib() -> ctypes.CDLL:
             "mk_state_read_counters": ([vp, vp, P(mk_state_counters), vp, i32], st),
             "mk_state_read_buffer": ([vp, i32, i32, vp, ctypes.c_size_t, vp], st),
             "mk_state_read_trace": ([vp, vp, i32, vp], st),
+            "mk_state_read_stats": ([vp, vp, i32, vp], st),
             "mk_last_error_string": ([], ctypes.c_char_p),
             "mk_version": ([], ctypes.c_char_p),
         }
@@ -250,6 +252,12 @@ def mk_state_read_counters(state: int, n_events: int = 0, stream: int = 0):
 def mk_state_read_buffer(state: int, which: int, layer: int, n: int, stream: int = 0):
     buf = (ctypes.c_float * n)()
     _check(lib().mk_state_read_buffer(state, which, layer, buf, n, stream))
+    return list(buf)
+
+
+def mk_state_read_stats(state: int, n_sm: int, stream: int = 0):
+    buf = (ctypes.c_uint64 * (8 * n_sm))()
+    _check(lib().mk_state_read_stats(state, buf, 8 * n_sm, stream))
     return list(buf)
 
 

@@ -12,6 +12,7 @@ HEADERS = ["mk_internal.h", "graph.h", "megakernel.h"]
 
 def nvcc_cmd(ptxas_verbose: bool = False):
     cmd = ["nvcc", "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+           "-maxrregcount=200",
            "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(HERE, "..", "include")]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]

@@ -52,6 +52,7 @@ struct mk_state {
     int32_t* tokpos = nullptr;     // host-input variant: [2][max_batch]
     float* logits = nullptr;       // host-output variant: [max_batch][vocab]
     unsigned long long* trace = nullptr;
+    unsigned long long* stats = nullptr;
     std::vector<void*> allocs;
 };
 
@@ -144,6 +145,7 @@ mk::Params base_params(mk_state* s) {
     p.timeout_ns = s->timeout_ns;
     p.wait_offset = s->wait_offset;
     p.trace = s->trace;
+    p.stats = s->stats;
     p.layers = m->d_layers;
     const int L = d.n_layers;
     p.tok_emb = static_cast<const uint16_t*>(m->w[0]);
@@ -424,6 +426,7 @@ mk_status mk_state_create(mk_graph* g, mk_state** out) {
     ALLOC(tokpos, 2 * B);
     ALLOC(logits, B * (size_t)d.vocab);
     if (d.flags & MK_FLAG_TRACE) ALLOC(trace, P.tasks.size() * 4);
+    if (d.flags & MK_FLAG_TRACE) ALLOC(stats, (size_t)P.n_sm * 8);
 #undef ALLOC
     if (st != MK_OK) {
         free_state_memory(s);
@@ -590,6 +593,17 @@ mk_status mk_state_read_buffer(mk_state* s, int which, int layer, float* host, s
         }
     }
     if (e != cudaSuccess) return cuda_fail(e, "mk_state_read_buffer");
+    return MK_OK;
+}
+
+mk_status mk_state_read_stats(mk_state* s, uint64_t* host, int cap, mk_stream stream) {
+    if (!s || !host) return fail(MK_ERR_INVALID_ARG, "mk_state_read_stats: null argument");
+    if (!s->stats) return fail(MK_ERR_INVALID_ARG, "mk_state_read_stats: model was loaded without MK_FLAG_TRACE");
+    int n = std::min<int>(cap, s->g->plan.n_sm * 8);
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaMemcpy(host, s->stats, sizeof(uint64_t) * n, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(s->stats, 0, sizeof(uint64_t) * s->g->plan.n_sm * 8);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_state_read_stats");
     return MK_OK;
 }
 

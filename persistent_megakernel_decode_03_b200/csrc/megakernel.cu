@@ -240,10 +240,18 @@ __device__ __forceinline__ void gemv_geom(const Params& p, const Task& t, GemvGe
 
 __device__ __forceinline__ bool is_gemv(int op) { return op != MK_OP_ATTN; }
 
-// Chunks of one weight block: kStageBytes pieces of the contiguous rows.
-__device__ __forceinline__ int block_chunks(const GemvGeom& g) {
-    int64_t bytes = (int64_t)g.rows * g.K * 2;
-    return (int)((bytes + kStageBytes - 1) / kStageBytes);
+// Chunks of a GEMV task: per weight block, groups of whole rows that fit one
+// stage, or (rows longer than a stage) each row in stage-sized segments.
+__device__ __forceinline__ int gemv_chunks(const GemvGeom& g) {
+    const int64_t RB = (int64_t)g.K * 2;
+    int per_blk;
+    if (RB <= kStageBytes) {
+        const int rps = (int)(kStageBytes / RB);
+        per_blk = (g.rows + rps - 1) / rps;
+    } else {
+        per_blk = g.rows * (int)((RB + kStageBytes - 1) / kStageBytes);
+    }
+    return per_blk * g.nblk;
 }
 
 // Attention split range [j0, j1) of positions (inclusive of the new token).
@@ -275,14 +283,33 @@ __device__ __forceinline__ bool wait_should_stop(const Params& p, Waiter& w) {
     return false;
 }
 
+// Per-CTA cycle counters (tracing builds of the state only): [0] producer waits for a
+// free ring slot, [1] consumer thread 0 waits for data, [2] dependency waits,
+// [3] kernel cycles, [4] tasks run, [5] signal-slot waits.
+__device__ __forceinline__ void stat_add(const Params& p, int i, unsigned long long v) {
+    if (p.stats) p.stats[(size_t)blockIdx.x * 8 + i] += v;
+}
+
+__device__ __forceinline__ void wait_stat(const Params& p, int where, long long c0) {
+    if (!p.stats) return;
+    const unsigned long long d = (unsigned long long)(clock64() - c0);
+    if (where == 1) stat_add(p, 0, d);                                   // producer: ring full
+    else if ((where == 3 || where == 4 || where == 5) && threadIdx.x == 0) stat_add(p, 1, d);
+    else if (where == 6) stat_add(p, 5, d);
+}
+
 __device__ bool mbar_wait_bounded(const Params& p, uint64_t* bar, uint32_t parity, int where) {
+    if (mbar_try_wait(bar, parity)) return true;
     Waiter w{0, 0};
+    const long long c0 = p.stats ? clock64() : 0;
     while (!mbar_try_wait(bar, parity)) {
         if (wait_should_stop(p, w)) {
             if (ld_relaxed_int(p.err) == 0) set_error(p, kErrTimeout, -1, -1, where, (int)blockIdx.x);
+            wait_stat(p, where, c0);
             return false;
         }
     }
+    wait_stat(p, where, c0);
     return true;
 }
 
@@ -299,15 +326,20 @@ __device__ __forceinline__ void seen_complete_wait(const Params& p, uint64_t* ba
 // Spin (acquire) until events[e] >= target.  Single thread.
 __device__ bool event_wait(const Params& p, uint32_t e, uint32_t target, int task) {
     Waiter w{0, 0};
+    const long long c0 = p.stats ? clock64() : 0;
+    bool ok = true;
     while (true) {
         uint32_t v = ld_acquire(&p.events[e]);
-        if ((int32_t)(v - target) >= 0) return true;
+        if ((int32_t)(v - target) >= 0) break;
         if (wait_should_stop(p, w)) {
             if (ld_relaxed_int(p.err) == 0) set_error(p, kErrTimeout, task, (int)e, (int)v, (int)target);
-            return false;
+            ok = false;
+            break;
         }
         __nanosleep(32);
     }
+    if (p.stats && threadIdx.x == 0) stat_add(p, 2, (unsigned long long)(clock64() - c0));
+    return ok;
 }
 
 // ----------------------------------------------------------------------------- producer
@@ -400,8 +432,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         }
         GemvGeom g;
         gemv_geom(p, t, g, !skip);
-        int nch_blk = skip ? 0 : block_chunks(g);
-        int nch = nch_blk * g.nblk;
+        const int nch = skip ? 0 : gemv_chunks(g);
         if (nch == 0) {
             if (!acquire_slot()) { ok = false; break; }
             sm.info[stage] = StageInfo{ti, 0, 0, 0};
@@ -409,17 +440,37 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
             advance();
             continue;
         }
-        const int64_t blk_bytes = (int64_t)g.rows * g.K * 2;
-        for (int c = 0; c < nch; ++c) {
-            if (!acquire_slot()) { ok = false; break; }
-            int bi = c / nch_blk, ci = c % nch_blk;
-            int64_t off = (int64_t)ci * kStageBytes;
-            uint32_t bytes = (uint32_t)((blk_bytes - off < (int64_t)kStageBytes) ? (blk_bytes - off) : (int64_t)kStageBytes);
+        // chunk sequence (the consumer walks the same one): per weight block, either
+        // groups of whole rows that fit one stage, or one row in stage-sized segments
+        const int64_t RB = (int64_t)g.K * 2;
+        int c = 0;
+        auto issue = [&](const uint8_t* src, uint32_t bytes) -> bool {
+            if (!acquire_slot()) return false;
             sm.info[stage] = StageInfo{ti, c, nch, 0};
             mbar_arrive_expect_tx(&sm.full[stage], bytes);
-            bulk_g2s(sm.ring[stage], (const uint8_t*)g.w[bi] + off, bytes, &sm.full[stage], pol);
+            bulk_g2s(sm.ring[stage], src, bytes, &sm.full[stage], pol);
             advance();
+            ++c;
+            return true;
+        };
+        for (int bi = 0; bi < g.nblk && ok; ++bi) {
+            const uint8_t* base = reinterpret_cast<const uint8_t*>(g.w[bi]);
+            if (RB <= kStageBytes) {
+                const int rps = (int)(kStageBytes / RB);
+                for (int r0 = 0; r0 < g.rows && ok; r0 += rps) {
+                    const int n = min(rps, g.rows - r0);
+                    ok = issue(base + (int64_t)r0 * RB, (uint32_t)(n * RB));
+                }
+            } else {
+                for (int r = 0; r < g.rows && ok; ++r)
+                    for (int64_t off = 0; off < RB && ok; off += kStageBytes) {
+                        const int64_t left = RB - off;
+                        ok = issue(base + (int64_t)r * RB + off,
+                                   (uint32_t)(left < kStageBytes ? left : (int64_t)kStageBytes));
+                    }
+            }
         }
+        if (!ok) break;
     }
     // end-of-work marker (best effort when aborting)
     if (acquire_slot()) {
@@ -571,44 +622,157 @@ __device__ void gemv_prologue(const Params& p, Smem& sm, const Task& t, const Th
     }
 }
 
-__device__ __forceinline__ float dot8(const uint4 q, const float (&x)[8], float acc) {
-    acc = fmaf(bf_lo(q.x), x[0], acc);
-    acc = fmaf(bf_hi(q.x), x[1], acc);
-    acc = fmaf(bf_lo(q.y), x[2], acc);
-    acc = fmaf(bf_hi(q.y), x[3], acc);
-    acc = fmaf(bf_lo(q.z), x[4], acc);
-    acc = fmaf(bf_hi(q.z), x[5], acc);
-    acc = fmaf(bf_lo(q.w), x[6], acc);
-    acc = fmaf(bf_hi(q.w), x[7], acc);
-    return acc;
+// Two interleaved accumulators (even / odd elements) halve the FMA chain.
+__device__ __forceinline__ void dot8(const uint4 q, const float (&x)[8], float& a0, float& a1) {
+    a0 = fmaf(bf_lo(q.x), x[0], a0);
+    a1 = fmaf(bf_hi(q.x), x[1], a1);
+    a0 = fmaf(bf_lo(q.y), x[2], a0);
+    a1 = fmaf(bf_hi(q.y), x[3], a1);
+    a0 = fmaf(bf_lo(q.z), x[4], a0);
+    a1 = fmaf(bf_hi(q.z), x[5], a1);
+    a0 = fmaf(bf_lo(q.w), x[6], a0);
+    a1 = fmaf(bf_hi(q.w), x[7], a1);
 }
 
-// Dot products of one chunk (vectors [c0, c1) of weight block `blk`) against x.
-__device__ __forceinline__ void gemv_chunk(Smem& sm, int buf, const uint8_t* stage, const ThreadMap& m,
-                                           int rows, int blk, int c0, int c1,
-                                           const float (&xr)[kMaxVecPerThread][8]) {
-    if (!m.active) return;
+// Whole rows [r0, r0+n) of block `blk` sit in `sv` back to back (nvec vectors each).
+template <int VPT>
+__device__ __forceinline__ void gemv_rows(Smem& sm, int buf, const uint4* sv, const ThreadMap& m,
+                                          int rows, int blk, int r0, int n,
+                                          const float (&xr)[kMaxVecPerThread][8]) {
     const int lane = threadIdx.x & 31, wig = (threadIdx.x >> 5) % m.wpg;
     const int nvec = m.nvec;
-    const int row_first = c0 / nvec, row_last = (c1 - 1) / nvec;
-    int r = row_first + (((m.grp - row_first) % m.G) + m.G) % m.G;
-    const uint4* sv = reinterpret_cast<const uint4*>(stage);
-    for (; r <= row_last; r += m.G) {
-        const int rb = r * nvec;
-        const int vs = max(c0, rb) - rb, ve = min(c1, rb + nvec) - rb;
-        const uint4* rowp = sv + (rb - c0);
-        float acc = 0.0f;
+    float* red = &sm.red[buf][blk * rows + r0][0];
+    if (m.G == 1) {
+        int rr = 0;
+        for (; rr + 1 < n; rr += 2) {
+            const uint4* p0 = sv + rr * nvec;
+            const uint4* p1 = p0 + nvec;
+            float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < kMaxVecPerThread; ++j) {
-            int v = m.lig + j * m.gstride;
-            if (j < m.vpt && v >= vs && v < ve) acc = dot8(rowp[v], xr[j], acc);
+            for (int j = 0; j < VPT; ++j) {
+                const int v = m.lig + j * m.gstride;
+                if (v < nvec) {
+                    const uint4 q0 = p0[v], q1 = p1[v];
+                    dot8(q0, xr[j], a0, a1);
+                    dot8(q1, xr[j], b0, b1);
+                }
+            }
+            float a = a0 + a1, b = b0 + b1;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+                b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
+            }
+            if (lane == 0) {
+                red[rr * kConsumerWarps + wig] = a;
+                red[(rr + 1) * kConsumerWarps + wig] = b;
+            }
         }
-        acc = warp_sum(acc);
-        if (lane == 0) {
-            float* slot = &sm.red[buf][blk * rows + r][wig];
-            if (rb >= c0) *slot = acc;
-            else *slot += acc;
+        if (rr < n) {
+            const uint4* p0 = sv + rr * nvec;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) {
+                const int v = m.lig + j * m.gstride;
+                if (v < nvec) dot8(p0[v], xr[j], a0, a1);
+            }
+            float a = warp_sum(a0 + a1);
+            if (lane == 0) red[rr * kConsumerWarps + wig] = a;
         }
+    } else {
+        if (!m.active) return;
+        int rr = ((m.grp - r0 % m.G) % m.G + m.G) % m.G;
+        for (; rr < n; rr += m.G) {
+            const uint4* p0 = sv + rr * nvec;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) {
+                const int v = m.lig + j * m.gstride;
+                if (v < nvec) dot8(p0[v], xr[j], a0, a1);
+            }
+            float a = warp_sum(a0 + a1);
+            if (lane == 0) red[rr * kConsumerWarps + wig] = a;
+        }
+    }
+}
+
+// Streams one GEMV task's chunks out of the ring (same sequence as the producer)
+// and leaves the warps' partial row sums in red[buf].  Returns false on abort.
+template <int VPT>
+__device__ bool gemv_task_body(const Params& p, Smem& sm, int ti, const GemvGeom& g,
+                               const ThreadMap& m, const float (&xr)[kMaxVecPerThread][8], int buf,
+                               int& stage, uint32_t& lap, bool skip) {
+    const int lane = threadIdx.x & 31, wig = (threadIdx.x >> 5) % m.wpg;
+    bool first = true;
+    auto next_stage = [&]() -> bool {
+        if (!first && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) {
+            sm.flag[3] = 1;
+            return false;
+        }
+        first = false;
+        if (sm.info[stage].task != ti) {
+            set_error(p, kErrFault, ti, -4, sm.info[stage].task, 1);
+            sm.flag[3] = 1;
+            return false;
+        }
+        return true;
+    };
+    auto release = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        if (++stage == kStages) { stage = 0; ++lap; }
+    };
+    if (skip) {
+        if (!next_stage()) return false;
+        release();
+        return true;
+    }
+    const int64_t RB = (int64_t)g.K * 2;
+    for (int blk = 0; blk < g.nblk; ++blk) {
+        if (RB <= kStageBytes) {
+            const int rps = (int)(kStageBytes / RB);
+            for (int r0 = 0; r0 < g.rows; r0 += rps) {
+                if (!next_stage()) return false;
+                gemv_rows<VPT>(sm, buf, reinterpret_cast<const uint4*>(sm.ring[stage]), m, g.rows, blk,
+                               r0, min(rps, g.rows - r0), xr);
+                release();
+            }
+        } else {
+            constexpr int kSegVec = kStageBytes / 16;
+            for (int r = 0; r < g.rows; ++r) {
+                float a0 = 0.f, a1 = 0.f;
+                for (int vs = 0; vs < m.nvec; vs += kSegVec) {
+                    if (!next_stage()) return false;
+                    const int ve = min(m.nvec, vs + kSegVec);
+                    const uint4* sv = reinterpret_cast<const uint4*>(sm.ring[stage]) - vs;
+#pragma unroll
+                    for (int j = 0; j < VPT; ++j) {
+                        const int v = m.lig + j * m.gstride;
+                        if (v >= vs && v < ve) dot8(sv[v], xr[j], a0, a1);
+                    }
+                    release();
+                }
+                const float a = warp_sum(a0 + a1);
+                if (lane == 0) sm.red[buf][blk * g.rows + r][wig] = a;
+            }
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool gemv_task_dispatch(const Params& p, Smem& sm, int ti, const GemvGeom& g,
+                                                   const ThreadMap& m,
+                                                   const float (&xr)[kMaxVecPerThread][8], int buf,
+                                                   int& stage, uint32_t& lap, bool skip) {
+    switch (m.vpt) {
+        case 1: return gemv_task_body<1>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        case 2: return gemv_task_body<2>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        case 3: return gemv_task_body<3>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        case 4: return gemv_task_body<4>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        case 5: return gemv_task_body<5>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        case 6: return gemv_task_body<6>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        case 7: return gemv_task_body<7>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        default: return gemv_task_body<8>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
     }
 }
 
@@ -990,31 +1154,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             }
         }
         const int rows_total = g.rows * g.nblk;
-        for (int c = 0;; ++c) {
-            if (c > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) {
-                sm.flag[3] = 1;
-                break;
-            }
-            const StageInfo inf = sm.info[stage];
-            if (inf.task != ti) {
-                set_error(p, kErrFault, ti, -4, inf.task, 1);
-                sm.flag[3] = 1;
-                break;
-            }
-            if (inf.nchunks > 0) {
-                const int nch_blk = inf.nchunks / g.nblk;
-                const int blk = inf.chunk / nch_blk, ci = inf.chunk % nch_blk;
-                const int64_t blk_vecs = (int64_t)g.rows * m.nvec;
-                const int c0 = ci * (kStageBytes / 16);
-                const int c1 = (int)((blk_vecs < (int64_t)c0 + kStageBytes / 16) ? blk_vecs : (int64_t)c0 + kStageBytes / 16);
-                gemv_chunk(sm, buf, sm.ring[stage], m, g.rows, blk, c0, c1, xr);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[stage]);
-            const bool last = inf.nchunks == 0 || inf.chunk == inf.nchunks - 1;
-            if (++stage == kStages) { stage = 0; ++lap; }
-            if (last) break;
-        }
+        (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
         consumer_sync();   // all partial sums of this task are in red[buf]
         if (sm.flag[3]) break;
 
@@ -1129,8 +1269,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+    const long long k0 = clock64();
     if (warp < kConsumerWarps) {
         consumer_loop<HPG, DPL>(p, sm);
+        if (threadIdx.x == 0) stat_add(p, 3, (unsigned long long)(clock64() - k0));
     } else if (warp == kProducerWarp) {
         if (lane == 0) producer_loop(p, sm);
     } else {

@@ -69,6 +69,7 @@ struct Params {
     long long timeout_ns;
     uint32_t wait_offset;        // added to every wait target (0; tests set 1 to force a timeout)
     unsigned long long* trace;   // [n_tasks][4] or null
+    unsigned long long* stats;   // [grid][8] per-CTA cycle counters (with trace) or null
 
     // model
     const LayerW* layers;
