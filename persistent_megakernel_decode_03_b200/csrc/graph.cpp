@@ -74,7 +74,7 @@ void wave_stats(int n_tiles, int n_sm, int* waves, int* idle) {
 // divides it (QKV tiles never straddle two heads, so each feeds one KV head).
 int choose_tile_rows(int64_t rows, int64_t row_bytes, int n_blocks, int n_sm, int64_t target,
                      int divide) {
-    int cap = kMaxTaskRows / n_blocks;
+    int cap = 16 / n_blocks;   // <= 16 rows per task: the fast GEMV path keeps row sums in registers
     int R = (int)std::max<int64_t>(1, std::min<int64_t>(cap, target / (row_bytes * n_blocks)));
     if (divide > 0) R = largest_divisor_at_most(divide, R);
     const int64_t min_bytes = 16 * 1024;

@@ -520,7 +520,7 @@ __device__ __forceinline__ float x_in(const Params& p, int l, int b, int i) {
     const size_t lb = (size_t)(l - 1) * p.max_batch + b;
     float v = __ldcg(p.x_mid + lb * p.H + i);
     for (int k = 0; k < p.topk; ++k)
-        v += __ldcg(p.moe_w + lb * p.topk + k) * __ldcg(p.ypart + (lb * p.topk + k) * p.H + i);
+        v = fmaf(__ldcg(p.moe_w + lb * p.topk + k), __ldcg(p.ypart + (lb * p.topk + k) * p.H + i), v);
     return v;
 }
 
@@ -591,54 +591,181 @@ __device__ __forceinline__ ThreadMap thread_map(int K) {
 }
 
 // Loads this thread's slice of the (normalised) input into registers.
-__device__ void gemv_prologue(const Params& p, Smem& sm, const Task& t, const ThreadMap& m, int K,
-                              float (&xr)[kMaxVecPerThread][8]) {
-    const uint16_t* gain = gemv_norm_gain(p, t);
-    float rstd = 1.0f;
-    if (gain) {
-        float ss = 0.0f;
-        for (int i = threadIdx.x; i < K; i += kConsumerThreads) {
-            float v = gemv_input(p, t, i);
-            ss = fmaf(v, v, ss);
-        }
-        float tot = block_sum(sm, ss);
-        rstd = 1.0f / sqrtf(tot / (float)K + p.eps);
+// Where a GEMV task's input vector lives: an fp32 row, a bf16 embedding row, and
+// for an MoE residual the routed experts' outputs with their combine weights.
+struct InSrc {
+    const float* base;
+    const uint16_t* emb;
+    const float* parts;   // [nparts][pstride]
+    const float* pw;      // [nparts]
+    int nparts, pstride;
+};
+
+__device__ __forceinline__ InSrc xin_src(const Params& p, int l, int b) {
+    InSrc s{nullptr, nullptr, nullptr, nullptr, 0, 0};
+    if (l == 0) {
+        int tok = p.tokens[b];
+        if (tok < 0 || tok >= p.V) tok = 0;   // recorded as an error by the QKV task
+        s.emb = p.tok_emb + (size_t)tok * p.H;
+    } else if (p.E == 0) {
+        s.base = p.x_out + ((size_t)(l - 1) * p.max_batch + b) * p.H;
+    } else {
+        const size_t lb = (size_t)(l - 1) * p.max_batch + b;
+        s.base = p.x_mid + lb * p.H;
+        s.parts = p.ypart + lb * p.topk * p.H;
+        s.pw = p.moe_w + lb * p.topk;
+        s.nparts = p.topk;
+        s.pstride = p.H;
     }
+    return s;
+}
+
+__device__ __forceinline__ InSrc gemv_src(const Params& p, const Task& t) {
+    const int l = t.layer, b = t.b;
+    InSrc s{nullptr, nullptr, nullptr, nullptr, 0, 0};
+    switch (t.op) {
+        case MK_OP_QKV: return xin_src(p, l, 0);
+        case MK_OP_LMHEAD: return xin_src(p, p.L, 0);
+        case MK_OP_OPROJ: s.base = p.o + ((size_t)l * p.max_batch) * (p.nq * p.hd); break;
+        case MK_OP_GATEUP:
+        case MK_OP_ROUTER: s.base = p.x_mid + ((size_t)l * p.max_batch) * p.H; break;
+        case MK_OP_EXP_GATEUP: s.base = p.x_mid + ((size_t)l * p.max_batch + b) * p.H; break;
+        case MK_OP_DOWN: s.base = p.act + ((size_t)l * p.max_batch) * p.F; break;
+        case MK_OP_EXP_DOWN:
+            s.base = p.act + (((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.Fe;
+            break;
+        default: break;
+    }
+    return s;
+}
+
+// Eight consecutive input elements starting at col (a multiple of 8), as four
+// pairs; every load is independent so a thread's whole slice is in flight at once.
+template <bool PARTS>
+__device__ __forceinline__ void load8(const InSrc& s, int col, float2 (&x)[4]) {
+    if (s.emb) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(s.emb + col));
+        x[0] = make_float2(bf_lo(u.x), bf_hi(u.x));
+        x[1] = make_float2(bf_lo(u.y), bf_hi(u.y));
+        x[2] = make_float2(bf_lo(u.z), bf_hi(u.z));
+        x[3] = make_float2(bf_lo(u.w), bf_hi(u.w));
+        return;
+    }
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(s.base + col));
+    const float4 c = __ldcg(reinterpret_cast<const float4*>(s.base + col + 4));
+    x[0] = make_float2(a.x, a.y);
+    x[1] = make_float2(a.z, a.w);
+    x[2] = make_float2(c.x, c.y);
+    x[3] = make_float2(c.z, c.w);
+    if (!PARTS) return;
+    for (int k = 0; k < s.nparts; ++k) {
+        const float w = __ldcg(s.pw + k);
+        const float4 pa = __ldcg(reinterpret_cast<const float4*>(s.parts + (size_t)k * s.pstride + col));
+        const float4 pc = __ldcg(reinterpret_cast<const float4*>(s.parts + (size_t)k * s.pstride + col + 4));
+        x[0] = make_float2(fmaf(w, pa.x, x[0].x), fmaf(w, pa.y, x[0].y));
+        x[1] = make_float2(fmaf(w, pa.z, x[1].x), fmaf(w, pa.w, x[1].y));
+        x[2] = make_float2(fmaf(w, pc.x, x[2].x), fmaf(w, pc.y, x[2].y));
+        x[3] = make_float2(fmaf(w, pc.z, x[3].x), fmaf(w, pc.w, x[3].y));
+    }
+}
+
+// Loads this thread's slice of the (RMS-normalised) input into registers in one
+// pass: the sum of squares comes from the slices of group 0, which together
+// cover every column exactly once, so every CTA reduces in the same order.
+template <bool PARTS>
+__device__ void gemv_prologue_t(const Params& p, Smem& sm, const Task& t, const ThreadMap& m, int K,
+                                const InSrc& src, float2 (&xr)[kMaxVecPerThread][4]) {
+    const uint16_t* gain = gemv_norm_gain(p, t);
+    float ss = 0.0f;
 #pragma unroll
     for (int j = 0; j < kMaxVecPerThread; ++j) {
-        int v = m.lig + j * m.gstride;
+        const int v = m.lig + j * m.gstride;
         if (j < m.vpt && v < m.nvec && m.active) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                int col = v * 8 + e;
-                float x = gemv_input(p, t, col);
-                if (gain) x = (x * rstd) * bf16_to_f32(gain[col]);
-                xr[j][e] = x;
-            }
+            load8<PARTS>(src, v * 8, xr[j]);
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) xr[j][e] = 0.0f;
+            for (int e = 0; e < 4; ++e) xr[j][e] = make_float2(0.0f, 0.0f);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxVecPerThread; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ss = fmaf(xr[j][e].y, xr[j][e].y, fmaf(xr[j][e].x, xr[j][e].x, ss));
+    if (gain) {
+        const float tot = block_sum(sm, (m.grp == 0 && m.active) ? ss : 0.0f);
+        const float rstd = 1.0f / sqrtf(tot / (float)K + p.eps);
+#pragma unroll
+        for (int j = 0; j < kMaxVecPerThread; ++j) {
+            const int v = m.lig + j * m.gstride;
+            if (j < m.vpt && v < m.nvec && m.active) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4*>(gain + v * 8));
+                const float g[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
+                                    bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    xr[j][e] = make_float2((xr[j][e].x * rstd) * g[2 * e], (xr[j][e].y * rstd) * g[2 * e + 1]);
+            }
         }
     }
 }
 
-// Two interleaved accumulators (even / odd elements) halve the FMA chain.
-__device__ __forceinline__ void dot8(const uint4 q, const float (&x)[8], float& a0, float& a1) {
-    a0 = fmaf(bf_lo(q.x), x[0], a0);
-    a1 = fmaf(bf_hi(q.x), x[1], a1);
-    a0 = fmaf(bf_lo(q.y), x[2], a0);
-    a1 = fmaf(bf_hi(q.y), x[3], a1);
-    a0 = fmaf(bf_lo(q.z), x[4], a0);
-    a1 = fmaf(bf_hi(q.z), x[5], a1);
-    a0 = fmaf(bf_lo(q.w), x[6], a0);
-    a1 = fmaf(bf_hi(q.w), x[7], a1);
+__device__ __forceinline__ void gemv_prologue(const Params& p, Smem& sm, const Task& t, const ThreadMap& m,
+                                              int K, float2 (&xr)[kMaxVecPerThread][4]) {
+    const InSrc src = gemv_src(p, t);
+    if (src.nparts > 0) gemv_prologue_t<true>(p, sm, t, m, K, src, xr);
+    else gemv_prologue_t<false>(p, sm, t, m, K, src, xr);
+}
+
+// Packed fp32x2 fused multiply-add (sm_100): d = a * b + c, lane-wise on two floats.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+        " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// acc.x accumulates the even elements of 8 bf16 weights times x, acc.y the odd ones.
+__device__ __forceinline__ void dot8(const uint4 q, const float2 (&x)[4], float2& acc) {
+    acc = ffma2(make_float2(bf_lo(q.x), bf_hi(q.x)), x[0], acc);
+    acc = ffma2(make_float2(bf_lo(q.y), bf_hi(q.y)), x[1], acc);
+    acc = ffma2(make_float2(bf_lo(q.z), bf_hi(q.z)), x[2], acc);
+    acc = ffma2(make_float2(bf_lo(q.w), bf_hi(q.w)), x[3], acc);
+}
+__device__ __forceinline__ void dot8(const uint4 q, const float2 (&x)[4], float& a0, float& a1) {
+    float2 acc = make_float2(a0, a1);
+    dot8(q, x, acc);
+    a0 = acc.x;
+    a1 = acc.y;
+}
+
+// Sums N per-lane values over the warp at once (reduce-scatter: N/2 + N/4 + ... + 1
+// shuffles, then log2(32/N) more).  Lane l returns the total of value l / (32/N).
+template <int N>
+__device__ __forceinline__ float warp_reduce_rows(float (&v)[N]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int cnt = N, o = 16; cnt > 1; cnt >>= 1, o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < cnt / 2; ++i) {
+            const float send = up ? v[i] : v[i + cnt / 2];
+            const float keep = up ? v[i + cnt / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+        }
+    }
+    float r = v[0];
+#pragma unroll
+    for (int o = 16 / N; o >= 1; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+    return r;
 }
 
 // Whole rows [r0, r0+n) of block `blk` sit in `sv` back to back (nvec vectors each).
 template <int VPT>
 __device__ __forceinline__ void gemv_rows(Smem& sm, int buf, const uint4* sv, const ThreadMap& m,
                                           int rows, int blk, int r0, int n,
-                                          const float (&xr)[kMaxVecPerThread][8]) {
+                                          const float2 (&xr)[kMaxVecPerThread][4]) {
     const int lane = threadIdx.x & 31, wig = (threadIdx.x >> 5) % m.wpg;
     const int nvec = m.nvec;
     float* red = &sm.red[buf][blk * rows + r0][0];
@@ -700,7 +827,7 @@ __device__ __forceinline__ void gemv_rows(Smem& sm, int buf, const uint4* sv, co
 // and leaves the warps' partial row sums in red[buf].  Returns false on abort.
 template <int VPT>
 __device__ bool gemv_task_body(const Params& p, Smem& sm, int ti, const GemvGeom& g,
-                               const ThreadMap& m, const float (&xr)[kMaxVecPerThread][8], int buf,
+                               const ThreadMap& m, const float2 (&xr)[kMaxVecPerThread][4], int buf,
                                int& stage, uint32_t& lap, bool skip) {
     const int lane = threadIdx.x & 31, wig = (threadIdx.x >> 5) % m.wpg;
     bool first = true;
@@ -760,9 +887,115 @@ __device__ bool gemv_task_body(const Params& p, Smem& sm, int ti, const GemvGeom
     return true;
 }
 
+// Fast paths for rows whose 16-byte vectors split evenly over the 256 consumer
+// threads (hidden sizes that are multiples of 2048): every thread owns VPT
+// vectors of every row, the NROWS row sums stay in registers across the task's
+// stages, and the warp reduces them once at the end.
+
+// Rows that fit a stage: RPS rows per stage, NROWS / RPS stages.
+template <int VPT, int RPS, int NROWS>
+__device__ bool gemv_fast_rows(const Params& p, Smem& sm, int ti, const float2 (&xr)[kMaxVecPerThread][4],
+                               int buf, int& stage, uint32_t& lap) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float2 acc[NROWS];
+#pragma unroll
+    for (int r = 0; r < NROWS; ++r) acc[r] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int st = 0; st < NROWS / RPS; ++st) {
+        if (st > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) { sm.flag[3] = 1; return false; }
+        if (sm.info[stage].task != ti) { set_error(p, kErrFault, ti, -4, sm.info[stage].task, 2); sm.flag[3] = 1; return false; }
+        const uint4* sv = reinterpret_cast<const uint4*>(sm.ring[stage]) + threadIdx.x;
+        uint4 q[RPS][VPT];
+#pragma unroll
+        for (int rr = 0; rr < RPS; ++rr)
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) q[rr][j] = sv[(rr * VPT + j) * kConsumerThreads];
+#pragma unroll
+        for (int rr = 0; rr < RPS; ++rr)
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) dot8(q[rr][j], xr[j], acc[st * RPS + rr]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        if (++stage == kStages) { stage = 0; ++lap; }
+    }
+    float v[NROWS];
+#pragma unroll
+    for (int r = 0; r < NROWS; ++r) v[r] = acc[r].x + acc[r].y;
+    const float tot = warp_reduce_rows<NROWS>(v);
+    if ((lane & (32 / NROWS - 1)) == 0) sm.red[buf][lane / (32 / NROWS)][warp] = tot;
+    return true;
+}
+
+// Rows longer than a stage: each row arrives as segments of SEGJ*256 vectors
+// (the last segment holds the rest); NROWS rows.
+template <int VPT, int SEGJ, int NROWS>
+__device__ bool gemv_fast_segs(const Params& p, Smem& sm, int ti, const float2 (&xr)[kMaxVecPerThread][4],
+                               int buf, int& stage, uint32_t& lap, bool first_seen) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NSEG = (VPT + SEGJ - 1) / SEGJ;
+    float2 acc[NROWS];
+#pragma unroll
+    for (int r = 0; r < NROWS; ++r) acc[r] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < NROWS; ++r) {
+#pragma unroll
+        for (int sg = 0; sg < NSEG; ++sg) {
+            if ((r > 0 || sg > 0 || !first_seen) && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) {
+                sm.flag[3] = 1;
+                return false;
+            }
+            if (sm.info[stage].task != ti) { set_error(p, kErrFault, ti, -4, sm.info[stage].task, 3); sm.flag[3] = 1; return false; }
+            const uint4* sv = reinterpret_cast<const uint4*>(sm.ring[stage]) + threadIdx.x;
+            constexpr int J0 = 0;
+            uint4 q[SEGJ];
+#pragma unroll
+            for (int j = 0; j < SEGJ; ++j)
+                if (sg * SEGJ + j < VPT) q[j] = sv[j * kConsumerThreads];
+#pragma unroll
+            for (int j = J0; j < SEGJ; ++j)
+                if (sg * SEGJ + j < VPT) dot8(q[j], xr[sg * SEGJ + j], acc[r]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);
+            if (++stage == kStages) { stage = 0; ++lap; }
+        }
+    }
+    float v[NROWS];
+#pragma unroll
+    for (int r = 0; r < NROWS; ++r) v[r] = acc[r].x + acc[r].y;
+    const float tot = warp_reduce_rows<NROWS>(v);
+    if ((lane & (32 / NROWS - 1)) == 0) sm.red[buf][lane / (32 / NROWS)][warp] = tot;
+    return true;
+}
+
+// Returns 1 when a fast path handled the task, 0 when the generic path must, -1 on abort.
+__device__ __forceinline__ int gemv_fast_dispatch(const Params& p, Smem& sm, int ti, const GemvGeom& g,
+                                                  const ThreadMap& m,
+                                                  const float2 (&xr)[kMaxVecPerThread][4], int buf,
+                                                  int& stage, uint32_t& lap) {
+    if (m.nvec % kConsumerThreads != 0) return 0;
+    const int vpt = m.nvec / kConsumerThreads;
+    const int rows = g.rows * g.nblk;
+    const int64_t RB = (int64_t)g.K * 2;
+    bool ok;
+    if (RB <= kStageBytes) {
+        const int rps = (int)(kStageBytes / RB);
+        if (g.rows % rps != 0) return 0;
+        if (vpt == 2 && rps == 2 && rows == 16) ok = gemv_fast_rows<2, 2, 16>(p, sm, ti, xr, buf, stage, lap);
+        else if (vpt == 2 && rps == 2 && rows == 8) ok = gemv_fast_rows<2, 2, 8>(p, sm, ti, xr, buf, stage, lap);
+        else if (vpt == 1 && rps == 4 && rows == 16) ok = gemv_fast_rows<1, 4, 16>(p, sm, ti, xr, buf, stage, lap);
+        else if (vpt == 1 && rps == 4 && rows == 8) ok = gemv_fast_rows<1, 4, 8>(p, sm, ti, xr, buf, stage, lap);
+        else return 0;
+    } else {
+        if (vpt == 7 && rows == 4) ok = gemv_fast_segs<7, 4, 4>(p, sm, ti, xr, buf, stage, lap, true);
+        else if (vpt == 7 && rows == 2) ok = gemv_fast_segs<7, 4, 2>(p, sm, ti, xr, buf, stage, lap, true);
+        else return 0;
+    }
+    return ok ? 1 : -1;
+}
+
 __device__ __forceinline__ bool gemv_task_dispatch(const Params& p, Smem& sm, int ti, const GemvGeom& g,
                                                    const ThreadMap& m,
-                                                   const float (&xr)[kMaxVecPerThread][8], int buf,
+                                                   const float2 (&xr)[kMaxVecPerThread][4], int buf,
                                                    int& stage, uint32_t& lap, bool skip) {
     switch (m.vpt) {
         case 1: return gemv_task_body<1>(p, sm, ti, g, m, xr, buf, stage, lap, skip);
@@ -1076,7 +1309,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
     int sig_slot = 0;
     uint32_t sig_lap = 0;
     int buf = 0;
-    float xr[kMaxVecPerThread][8];
+    float2 xr[kMaxVecPerThread][4];
     int x_key_op = -1, x_key_layer = -1, x_key_b = -1, x_key_aux = -1;
     uint32_t ok_evt[4] = {MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT};   // thread 0
 
@@ -1133,7 +1366,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
 #pragma unroll
             for (int j = 0; j < kMaxVecPerThread; ++j)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) xr[j][e] = 0.0f;
+                for (int e = 0; e < 4; ++e) xr[j][e] = make_float2(0.0f, 0.0f);
             continue;
         }
 
@@ -1154,7 +1387,14 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             }
         }
         const int rows_total = g.rows * g.nblk;
-        (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        // residual rows for the epilogue, fetched now so the load overlaps the streaming
+        float resid = 0.0f;
+        if (!skip && tid < rows_total) {
+            if (t.op == MK_OP_OPROJ) resid = x_in(p, t.layer, 0, (int)t.r0 + tid);
+            else if (t.op == MK_OP_DOWN) resid = x_mid_at(p, t.layer, 0, (int)t.r0 + tid);
+        }
+        int handled = skip ? 0 : gemv_fast_dispatch(p, sm, ti, g, m, xr, buf, stage, lap);
+        if (handled == 0) (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
         consumer_sync();   // all partial sums of this task are in red[buf]
         if (sm.flag[3]) break;
 
@@ -1171,7 +1411,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
                         p.qkv[((size_t)l * p.max_batch) * ((p.nq + 2 * p.nkv) * p.hd) + row] = y;
                         break;
                     case MK_OP_OPROJ:
-                        p.x_mid[((size_t)l * p.max_batch) * p.H + row] = x_in(p, l, 0, row) + y;
+                        p.x_mid[((size_t)l * p.max_batch) * p.H + row] = resid + y;
                         break;
                     case MK_OP_GATEUP: {
                         float u = 0.0f;
@@ -1180,7 +1420,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
                         break;
                     }
                     case MK_OP_DOWN:
-                        p.x_out[((size_t)l * p.max_batch) * p.H + row] = x_mid_at(p, l, 0, row) + y;
+                        p.x_out[((size_t)l * p.max_batch) * p.H + row] = resid + y;
                         break;
                     case MK_OP_LMHEAD:
                         p.logits[row] = y;
