@@ -126,6 +126,11 @@ void mk_model_destroy(mk_model* model);
  * and dependency analysis). */
 mk_status mk_build_taskgraph(mk_model* model, int max_batch, int max_ctx, mk_graph** out);
 
+/* Profiling aid: the graph's tasks of one dense operator kind only (op in
+ * MK_OP_QKV..MK_OP_LMHEAD, every layer), with no dependencies, so one tile type
+ * can be timed and profiled alone.  Its outputs are not a decode step. */
+mk_status mk_build_taskgraph_solo(mk_model* model, int max_batch, int max_ctx, int op, mk_graph** out);
+
 /* The same plan on the host only (no device memory, no CUDA call), for an
  * SM count given by the caller: for inspecting and checking the graph. */
 mk_status mk_plan_taskgraph(const mk_model_desc* desc, int max_batch, int max_ctx, int n_sm,
@@ -196,6 +201,10 @@ void mk_state_destroy(mk_state* state);
  * it sets MK_ERR_TIMEOUT; the kernel then drains and returns. */
 mk_status mk_state_set_timeout(mk_state* state, int64_t timeout_ns);
 
+/* L2 prefetch distance, in tasks ahead of the work-queue head (default 0 =
+ * off).  A hint only: results do not depend on it. */
+mk_status mk_state_set_prefetch(mk_state* state, int tasks_ahead);
+
 /* Test hook for failure detection: adds `offset` to the target of every
  * device-side event wait of later steps (0 = normal).  With offset 1 no wait
  * can be satisfied, so the step ends with MK_ERR_TIMEOUT after the state's
@@ -249,13 +258,11 @@ mk_status mk_state_read_counters(mk_state* state, mk_stream stream, mk_state_cou
                                  uint32_t* events, int cap);
 
 /* Copies an activation buffer of the last step to host fp32 memory.
- *   which 0: residual after attention  [batch][hidden] of `layer`
- *         1: residual after the FFN    [batch][hidden] of `layer`
- *            (MoE: combined on the host side of this call is NOT done; the
- *            buffer holds the dense residual only for dense models)
- *         2: merged attention output   [batch][n_q*d]  of `layer`
- *         3: MoE selected experts of `layer` as fp32 [batch][top_k]
- *         4: MoE combine weights of `layer`          [batch][top_k]
+ *   which 0: residual stream after attention [batch][hidden] of `layer`
+ *         1: residual stream after the FFN   [batch][hidden] of `layer`
+ *            (dense models; an MoE layer keeps its FFN output per expert slot)
+ *         3: MoE selected experts of `layer`, as fp32 [batch][top_k]
+ *         4: MoE combine weights of `layer`           [batch][top_k]
  * n = number of floats to copy. */
 mk_status mk_state_read_buffer(mk_state* state, int which, int layer, float* host, size_t n,
                                mk_stream stream);

@@ -16,7 +16,8 @@ import os
 from typing import List, Optional, Sequence, Tuple
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmk.so")
+# MK_LIBRARY may name another build of the same C ABI (e.g. an experimental one).
+LIB_PATH = os.environ.get("MK_LIBRARY") or os.path.join(_HERE, "libmk.so")
 
 MK_OK = 0
 MK_ERR_INVALID_ARG = 1
@@ -35,10 +36,11 @@ OP_NAMES = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead"
 
 # Exported symbols (declared in include/mk.h).
 SYMBOLS = (
-    "mk_load_model", "mk_model_destroy", "mk_build_taskgraph", "mk_plan_taskgraph",
+    "mk_load_model", "mk_model_destroy", "mk_build_taskgraph", "mk_build_taskgraph_solo",
+    "mk_plan_taskgraph",
     "mk_graph_destroy", "mk_graph_get_info", "mk_graph_export_tasks", "mk_graph_export_thresholds",
     "mk_wave_stats", "mk_state_create", "mk_state_destroy", "mk_state_set_timeout",
-    "mk_state_debug_wait_offset",
+    "mk_state_debug_wait_offset", "mk_state_set_prefetch",
     "mk_decode_step", "mk_decode_step_host", "mk_prefill", "mk_sync", "mk_state_read_counters",
     "mk_state_read_buffer", "mk_state_read_trace", "mk_state_read_stats", "mk_last_error_string",
     "mk_version",
@@ -103,6 +105,7 @@ def lib() -> ctypes.CDLL:
             "mk_model_destroy": ([vp], None),
             "mk_build_taskgraph": ([vp, i32, i32, P(vp)], st),
             "mk_plan_taskgraph": ([P(mk_model_desc), i32, i32, i32, P(vp)], st),
+            "mk_build_taskgraph_solo": ([vp, i32, i32, i32, P(vp)], st),
             "mk_graph_destroy": ([vp], None),
             "mk_graph_get_info": ([vp, P(mk_graph_info)], st),
             "mk_graph_export_tasks": ([vp, P(mk_task_info), i32, P(i32)], st),
@@ -112,6 +115,7 @@ def lib() -> ctypes.CDLL:
             "mk_state_destroy": ([vp], None),
             "mk_state_set_timeout": ([vp, ctypes.c_int64], st),
             "mk_state_debug_wait_offset": ([vp, ctypes.c_uint32], st),
+            "mk_state_set_prefetch": ([vp, i32], st),
             "mk_decode_step": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_decode_step_host": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_prefill": ([vp, vp, i32, i32, P(mk_paged_kv), vp, vp], st),
@@ -160,6 +164,12 @@ def mk_model_destroy(model: int) -> None:
 def mk_build_taskgraph(model: int, max_batch: int, max_ctx: int) -> int:
     out = ctypes.c_void_p()
     _check(lib().mk_build_taskgraph(model, max_batch, max_ctx, ctypes.byref(out)))
+    return out.value
+
+
+def mk_build_taskgraph_solo(model: int, max_batch: int, max_ctx: int, op: int) -> int:
+    out = ctypes.c_void_p()
+    _check(lib().mk_build_taskgraph_solo(model, max_batch, max_ctx, op, ctypes.byref(out)))
     return out.value
 
 
@@ -217,6 +227,10 @@ def mk_state_set_timeout(state: int, timeout_ns: int) -> None:
 
 def mk_state_debug_wait_offset(state: int, offset: int) -> None:
     _check(lib().mk_state_debug_wait_offset(state, int(offset)))
+
+
+def mk_state_set_prefetch(state: int, tasks_ahead: int) -> None:
+    _check(lib().mk_state_set_prefetch(state, int(tasks_ahead)))
 
 
 def mk_decode_step(state: int, token_ids: int, positions: int, batch: int, kv: mk_paged_kv,

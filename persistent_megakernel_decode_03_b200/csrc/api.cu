@@ -41,12 +41,12 @@ struct mk_state {
     uint32_t wait_offset = 0;
     // device memory
     uint32_t* events = nullptr;
-    unsigned long long* queue = nullptr;
+    unsigned long long* queue = nullptr;   // [0] work queue, [1] L2-prefetch cursor
+    uint32_t pf_dist = 0;
     uint32_t* done = nullptr;
     int* err = nullptr;
-    uint32_t* merge_cnt = nullptr;
     uint32_t* router_cnt = nullptr;
-    float *x_mid = nullptr, *x_out = nullptr, *qkv = nullptr, *o = nullptr, *act = nullptr;
+    float *x_mid = nullptr, *x_out = nullptr, *qkv = nullptr, *act = nullptr;
     float *part = nullptr, *rlogits = nullptr, *moe_w = nullptr, *ypart = nullptr;
     int* moe_sel = nullptr;
     int32_t* tokpos = nullptr;     // host-input variant: [2][max_batch]
@@ -102,12 +102,9 @@ mk_status reset_counters(mk_state* s, cudaStream_t st) {
     const GraphPlan& P = s->g->plan;
     const mk_model_desc& d = P.desc;
     cudaError_t e = cudaMemsetAsync(s->events, 0, sizeof(uint32_t) * std::max(1, P.n_events), st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(s->queue, 0, sizeof(unsigned long long), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s->queue, 0, 2 * sizeof(unsigned long long), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(s->done, 0, sizeof(uint32_t), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(s->err, 0, sizeof(int) * 8, st);
-    if (e == cudaSuccess)
-        e = cudaMemsetAsync(s->merge_cnt, 0,
-                            sizeof(uint32_t) * (size_t)d.n_layers * P.max_batch * d.n_kv_heads, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(s->router_cnt, 0, sizeof(uint32_t) * d.n_layers, st);
     if (e != cudaSuccess) return cuda_fail(e, "reset");
     s->epoch = 0;
@@ -138,9 +135,10 @@ mk::Params base_params(mk_state* s) {
     p.thr = s->g->d_thr;
     p.events = s->events;
     p.queue = s->queue;
+    p.pf_head = s->queue + 1;
+    p.pf_dist = s->pf_dist;
     p.done = s->done;
     p.err = s->err;
-    p.merge_cnt = s->merge_cnt;
     p.router_cnt = s->router_cnt;
     p.timeout_ns = s->timeout_ns;
     p.wait_offset = s->wait_offset;
@@ -171,7 +169,6 @@ mk::Params base_params(mk_state* s) {
     p.x_mid = s->x_mid;
     p.x_out = s->x_out;
     p.qkv = s->qkv;
-    p.o = s->o;
     p.act = s->act;
     p.part = s->part;
     p.rlogits = s->rlogits;
@@ -289,7 +286,20 @@ mk_status mk_plan_taskgraph(const mk_model_desc* desc, int max_batch, int max_ct
     return MK_OK;
 }
 
+static mk_status build_graph(mk_model* model, int max_batch, int max_ctx, int solo_op, mk_graph** out);
+
 mk_status mk_build_taskgraph(mk_model* model, int max_batch, int max_ctx, mk_graph** out) {
+    return build_graph(model, max_batch, max_ctx, 0, out);
+}
+
+mk_status mk_build_taskgraph_solo(mk_model* model, int max_batch, int max_ctx, int op, mk_graph** out) {
+    if (op < MK_OP_QKV || op > MK_OP_EXP_DOWN || op == MK_OP_ROUTER || op == MK_OP_EXP_GATEUP ||
+        op == MK_OP_EXP_DOWN)
+        return fail(MK_ERR_INVALID_ARG, "mk_build_taskgraph_solo: op must be a dense operator (1..6)");
+    return build_graph(model, max_batch, max_ctx, op, out);
+}
+
+static mk_status build_graph(mk_model* model, int max_batch, int max_ctx, int solo_op, mk_graph** out) {
     if (!model || !out) return fail(MK_ERR_INVALID_ARG, "mk_build_taskgraph: null argument");
     *out = nullptr;
     int dev = 0, n_sm = 0;
@@ -309,6 +319,7 @@ mk_status mk_build_taskgraph(mk_model* model, int max_batch, int max_ctx, mk_gra
     if (st != MK_OK) return st;
     g->model = model;
     g->device = dev;
+    if (solo_op) mk::make_solo(g->plan, solo_op);
     const GraphPlan& P = g->plan;
     // RoPE table: cos/sin of pos * theta^(-2i/d), computed in double, stored fp32
     const int half = d.head_dim / 2;
@@ -404,15 +415,13 @@ mk_status mk_state_create(mk_graph* g, mk_state** out) {
     mk_status st = MK_OK;
 #define ALLOC(ptr, n) if (st == MK_OK) st = dev_alloc(s, &s->ptr, (n))
     ALLOC(events, (size_t)std::max(1, P.n_events));
-    ALLOC(queue, 1);
+    ALLOC(queue, 2);
     ALLOC(done, 1);
     ALLOC(err, 8);
-    ALLOC(merge_cnt, L * B * d.n_kv_heads);
     ALLOC(router_cnt, L);
     ALLOC(x_mid, L * B * H);
     ALLOC(x_out, L * B * H);
     ALLOC(qkv, L * B * qkvw);
-    ALLOC(o, L * B * d.n_q_heads * d.head_dim);
     if (d.n_experts > 0) {
         ALLOC(act, L * B * d.top_k * d.expert_ffn);
         ALLOC(rlogits, L * B * d.n_experts);
@@ -446,6 +455,12 @@ void mk_state_destroy(mk_state* s) {
 mk_status mk_state_set_timeout(mk_state* s, int64_t ns) {
     if (!s || ns < 1000) return fail(MK_ERR_INVALID_ARG, "mk_state_set_timeout: bad argument");
     s->timeout_ns = ns;
+    return MK_OK;
+}
+
+mk_status mk_state_set_prefetch(mk_state* s, int tasks_ahead) {
+    if (!s || tasks_ahead < 0) return fail(MK_ERR_INVALID_ARG, "mk_state_set_prefetch: bad argument");
+    s->pf_dist = (uint32_t)tasks_ahead;
     return MK_OK;
 }
 
@@ -572,7 +587,6 @@ mk_status mk_state_read_buffer(mk_state* s, int which, int layer, float* host, s
     switch (which) {
         case 0: src = s->x_mid + layer * B * d.hidden; avail = B * d.hidden; break;
         case 1: src = s->x_out + layer * B * d.hidden; avail = B * d.hidden; break;
-        case 2: src = s->o + layer * B * d.n_q_heads * d.head_dim; avail = B * d.n_q_heads * d.head_dim; break;
         case 3:
         case 4:
             if (d.n_experts == 0) return fail(MK_ERR_INVALID_ARG, "mk_state_read_buffer: not an MoE model");

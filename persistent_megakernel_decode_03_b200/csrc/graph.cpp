@@ -97,7 +97,8 @@ bool validate_desc(const mk_model_desc& d, std::string& err) {
     if (nq % nkv != 0) return fail("n_q_heads must be a multiple of n_kv_heads");
     if (nq / nkv > kMaxHeadsPerGroup) return fail("more than 8 q heads per kv head");
     if (H % 8 || (nq * hd) % 8) return fail("hidden and n_q*head_dim must be multiples of 8");
-    if (H > 16384 || nq * hd > 16384) return fail("hidden and n_q*head_dim must be <= 16384");
+    if (H > 16384) return fail("hidden must be <= 16384");
+    if (nq * hd > 8192) return fail("n_q*head_dim must be <= 8192");
     if (moe) {
         if (d.top_k <= 0 || d.top_k > kMaxTopK || d.top_k > d.n_experts)
             return fail("top_k must be in 1..min(16, n_experts)");
@@ -201,14 +202,10 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     for (int l = 0; l < L; ++l) {
         // QKV: primary input is the residual stream entering the layer.
         gemv_op(MK_OP_QKV, l, qkv_rows, R_qkv, T_QKV, l, {all_rows(T_XIN, l, 0, H)});
-        // attention: per (sequence, kv head, split); the merge entity is signalled by the last split.
+        // attention: per (sequence, kv head, split); each split writes its softmax partial,
+        // and the O-projection's input stage merges the splits.
         for (int b = 0; b < B; ++b)
-            for (int kh = 0; kh < nkv; ++kh) {
-                Entity m;
-                m.outs = {Region{tensor_key(T_O, l, 0), b, b + 1, (int64_t)kh * hpg * hd,
-                                 (int64_t)(kh + 1) * hpg * hd}};
-                int eid = (int)ent.size();
-                ent.push_back(m);
+            for (int kh = 0; kh < nkv; ++kh)
                 for (int s = 0; s < S; ++s) {
                     int t = new_task(MK_OP_ATTN, l, b, kh, (uint32_t)s, (uint32_t)S);
                     int key = tensor_key(T_QKV, l, 0);
@@ -216,10 +213,9 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
                                   Region{key, 0, B, (int64_t)nq * hd + kh * hd, (int64_t)nq * hd + (kh + 1) * hd},
                                   Region{key, 0, B, (int64_t)(nq + nkv) * hd + kh * hd,
                                          (int64_t)(nq + nkv) * hd + (kh + 1) * hd}};
-                    task_entity[t] = eid;
-                    ent[eid].tasks.push_back(t);
+                    own_entity(t, {Region{tensor_key(T_O, l, 0), b, b + 1, (int64_t)kh * hpg * hd,
+                                          (int64_t)(kh + 1) * hpg * hd}});
                 }
-            }
         gemv_op(MK_OP_OPROJ, l, H, R_o, T_XMID, l, {all_rows(T_O, l, 0, (int64_t)nq * hd)});
         if (!moe) {
             gemv_op(MK_OP_GATEUP, l, d.ffn, R_gu, T_ACT, l, {all_rows(T_XMID, l, 0, H)});
@@ -328,6 +324,21 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     wb += 2LL * H + 2LL * d.vocab * H;
     g.weight_bytes = wb;
     return true;
+}
+
+void make_solo(GraphPlan& g, int op) {
+    std::vector<Task> kept;
+    for (const Task& t : g.tasks)
+        if (t.op == op) {
+            Task u = t;
+            u.wait0 = u.wait1 = MK_NO_EVENT;
+            u.sig = MK_NO_EVENT;
+            u.pad = MK_NO_EVENT;
+            kept.push_back(u);
+        }
+    g.tasks.swap(kept);
+    g.thr.clear();
+    g.n_events = 0;
 }
 
 }  // namespace mk

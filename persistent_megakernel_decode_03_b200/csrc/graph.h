@@ -29,5 +29,8 @@ int choose_tile_rows(int64_t rows, int64_t row_bytes, int n_blocks, int n_sm, in
 bool validate_desc(const mk_model_desc& d, std::string& err);
 bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, GraphPlan& g,
                 std::string& err);
+// Keeps only the tasks of operator `op` (all layers), without dependencies:
+// a list for timing and profiling one tile type alone.
+void make_solo(GraphPlan& g, int op);
 
 }  // namespace mk

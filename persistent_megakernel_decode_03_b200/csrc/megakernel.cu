@@ -30,6 +30,7 @@
 // Params::timeout_ns, records MK_ERR_TIMEOUT and the kernel drains its own
 // copies in flight and returns.
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "megakernel.h"
@@ -76,6 +77,15 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
+// Hint: bring [src, src+bytes) into L2 (16-byte aligned, multiple of 16 bytes).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -94,7 +104,7 @@ __device__ __forceinline__ int ld_relaxed_int(const int* p) {
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
@@ -128,9 +138,10 @@ struct StageInfo {
     int chunk;     // chunk index within the task
     int nchunks;   // chunks of the task (0 for a task without streamed data)
     int aux;       // attention: first logical page of this chunk
+    Task rec;      // the task record (read once, by the producer)
 };
 
-constexpr int kAttnScratch = kConsumerWarps * kMaxHeadsPerGroup * (128 + 2);
+constexpr int kAttnScratch = kConsumerWarps * kMaxHeadsPerGroup * (128 + 2);   // >= n_q * head_dim floats too
 
 struct __align__(128) Smem {
     uint8_t ring[kStages][kStageBytes];
@@ -142,11 +153,15 @@ struct __align__(128) Smem {
     float bcast[kConsumerWarps + 8];
     uint64_t full[kStages], empty[kStages];
     uint64_t sig_full[kSigSlots], sig_empty[kSigSlots];
+    uint64_t csync;                          // all-consumer-warp sync (arrival count 8)
     StageInfo info[kStages];
     uint32_t sig_evt[kSigSlots];
     int sig_task[kSigSlots];
     int flag[4];
+    unsigned long long stat[8];              // per-CTA counters (tracing only), flushed at exit
 };
+
+constexpr size_t kStatsOffset = offsetof(Smem, stat);
 
 // ----------------------------------------------------------------------------- geometry
 
@@ -254,6 +269,14 @@ __device__ __forceinline__ int gemv_chunks(const GemvGeom& g) {
     return per_blk * g.nblk;
 }
 
+// Splits of one (sequence, kv head) actually used this step: about one per
+// kAttnSplitTokens positions of context, at most the graph's split count S.
+constexpr int kAttnSplitTokens = 128;
+__device__ __forceinline__ int attn_active_splits(int n_ctx, int S) {
+    int a = (n_ctx + kAttnSplitTokens - 1) / kAttnSplitTokens;
+    return a < 1 ? 1 : (a > S ? S : a);
+}
+
 // Attention split range [j0, j1) of positions (inclusive of the new token).
 __device__ __forceinline__ void attn_range(int n_ctx, int S, int s, int& j0, int& j1) {
     int per = (n_ctx + S - 1) / S;
@@ -287,7 +310,9 @@ __device__ __forceinline__ bool wait_should_stop(const Params& p, Waiter& w) {
 // free ring slot, [1] consumer thread 0 waits for data, [2] dependency waits,
 // [3] kernel cycles, [4] tasks run, [5] signal-slot waits.
 __device__ __forceinline__ void stat_add(const Params& p, int i, unsigned long long v) {
-    if (p.stats) p.stats[(size_t)blockIdx.x * 8 + i] += v;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    unsigned long long* acc = reinterpret_cast<unsigned long long*>(smem_raw + kStatsOffset);
+    if (p.stats) atomicAdd(&acc[i], v);
 }
 
 __device__ __forceinline__ void wait_stat(const Params& p, int where, long long c0) {
@@ -298,8 +323,7 @@ __device__ __forceinline__ void wait_stat(const Params& p, int where, long long 
     else if (where == 6) stat_add(p, 5, d);
 }
 
-__device__ bool mbar_wait_bounded(const Params& p, uint64_t* bar, uint32_t parity, int where) {
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ bool mbar_wait_slow(const Params& p, uint64_t* bar, uint32_t parity, int where) {
     Waiter w{0, 0};
     const long long c0 = p.stats ? clock64() : 0;
     while (!mbar_try_wait(bar, parity)) {
@@ -311,6 +335,23 @@ __device__ bool mbar_wait_bounded(const Params& p, uint64_t* bar, uint32_t parit
     }
     wait_stat(p, where, c0);
     return true;
+}
+
+// Bounded wait on an mbarrier phase; the common case (phase complete) stays inline.
+__device__ __forceinline__ bool mbar_wait_bounded(const Params& p, uint64_t* bar, uint32_t parity, int where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(p, bar, parity, where);
+}
+
+// Sync of the 8 consumer warps through an mbarrier (one arrival per warp, after
+// __syncwarp).  Every wait is bounded: on a timeout the CTA's abort flag is
+// raised instead of hanging, so no path can stall a consumer forever.  Each
+// consumer thread keeps its own copy of the phase parity.
+__device__ __forceinline__ void csync(const Params& p, Smem& sm, uint32_t& phase) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.csync);
+    if (!mbar_wait_bounded(p, &sm.csync, phase, 8)) sm.flag[3] = 1;
+    phase ^= 1;
 }
 
 // Wait on a phase that another thread of this CTA has already seen complete
@@ -364,18 +405,21 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
     uint32_t last_router_evt = MK_NO_EVENT;
     while (ok) {
         if (ld_relaxed_int(p.err) != 0) { ok = false; break; }
+        const long long c_dq = p.stats ? clock64() : 0;
         unsigned long long q = atomicAdd(p.queue, 1ull) - p.queue_base;
         if (q >= p.n_tasks) break;
         const int ti = (int)q;
         const Task t = p.tasks[ti];
+        if (p.stats) { const uint32_t w0 = t.wait0; stat_add(p, 4, (unsigned long long)(clock64() - c_dq) + (w0 & 0)); }
         if (t.op == MK_OP_ATTN) {
             const int b = t.b;
             int npages = 0, lp0 = 0;
             if (b < p.batch) {
                 int pos = position_of(p, b);
                 if (pos >= 0 && pos < p.max_ctx && pos / kPageSize < p.max_pages) {
-                    int j0, j1;
-                    attn_range(pos + 1, (int)t.r1, (int)t.r0, j0, j1);
+                    int j0 = 0, j1 = 0;
+                    const int sa = attn_active_splits(pos + 1, (int)t.r1);
+                    if ((int)t.r0 < sa) attn_range(pos + 1, sa, (int)t.r0, j0, j1);
                     int jc = min(j1, pos);          // cached positions only; the new token is fresh
                     if (jc > j0) {
                         lp0 = j0 / kPageSize;
@@ -388,7 +432,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
             const uint32_t blk = (uint32_t)(kPageSize * p.hd * 2);
             if (nch == 0) {
                 if (!acquire_slot()) { ok = false; break; }
-                sm.info[stage] = StageInfo{ti, 0, 0, 0};
+                sm.info[stage] = StageInfo{ti, 0, 0, 0, t};
                 mbar_arrive(&sm.full[stage]);
                 advance();
             }
@@ -396,7 +440,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
                 if (!acquire_slot()) { ok = false; break; }
                 int first = lp0 + c * pps;
                 int n = min(pps, lp0 + npages - first);
-                sm.info[stage] = StageInfo{ti, c, nch, first};
+                sm.info[stage] = StageInfo{ti, c, nch, first, t};
                 // validate page indices before issuing any copy
                 const int* prow = p.page_table + (size_t)b * p.max_pages;
                 bool bad = false;
@@ -435,7 +479,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         const int nch = skip ? 0 : gemv_chunks(g);
         if (nch == 0) {
             if (!acquire_slot()) { ok = false; break; }
-            sm.info[stage] = StageInfo{ti, 0, 0, 0};
+            sm.info[stage] = StageInfo{ti, 0, 0, 0, t};
             mbar_arrive(&sm.full[stage]);
             advance();
             continue;
@@ -446,7 +490,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         int c = 0;
         auto issue = [&](const uint8_t* src, uint32_t bytes) -> bool {
             if (!acquire_slot()) return false;
-            sm.info[stage] = StageInfo{ti, c, nch, 0};
+            sm.info[stage] = StageInfo{ti, c, nch, 0, t};
             mbar_arrive_expect_tx(&sm.full[stage], bytes);
             bulk_g2s(sm.ring[stage], src, bytes, &sm.full[stage], pol);
             advance();
@@ -474,7 +518,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
     }
     // end-of-work marker (best effort when aborting)
     if (acquire_slot()) {
-        sm.info[stage] = StageInfo{-1, 0, 0, 0};
+        sm.info[stage].task = -1;
         mbar_arrive(&sm.full[stage]);
         advance();
     }
@@ -485,6 +529,60 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         while (!mbar_try_wait(&sm.full[s], (issued[s] - 1) & 1)) {
             if (++w.spins > (1 << 26)) break;   // copies of valid memory always land; hard cap only
         }
+    }
+}
+
+// ----------------------------------------------------------------------------- L2 prefetcher
+
+// Walks the task list a bounded distance ahead of the work-queue head and asks
+// L2 to fetch the weight rows (and KV pages) of upcoming tasks, so HBM keeps
+// streaming while the consumers wait on a dependency; the ring copies then hit
+// L2.  Routed-expert weights are unknown until the router runs and are skipped.
+__device__ void prefetch_loop(const Params& p) {
+    if (p.pf_dist == 0 || p.pf_head == nullptr) return;
+    while (true) {
+        const unsigned long long i = atomicAdd(p.pf_head, 1ull) - p.queue_base;
+        if (i >= p.n_tasks) return;
+        Waiter w{0, 0};
+        while (true) {
+            const unsigned long long h = ld_relaxed_u64(p.queue) - p.queue_base;
+            if (h + p.pf_dist > i) break;
+            if (wait_should_stop(p, w)) return;   // an error elsewhere; a slow step is not one
+            __nanosleep(200);
+        }
+        const Task t = p.tasks[i];
+        if (t.op == MK_OP_ATTN) {
+            const int b = t.b;
+            if (b >= p.batch) continue;
+            const int pos = position_of(p, b);
+            if (pos < 0 || pos >= p.max_ctx || pos / kPageSize >= p.max_pages) continue;
+            const int sa = attn_active_splits(pos + 1, (int)t.r1);
+            if ((int)t.r0 >= sa) continue;
+            int j0, j1;
+            attn_range(pos + 1, sa, (int)t.r0, j0, j1);
+            const int jc = min(j1, pos);
+            if (jc <= j0) continue;
+            const int* prow = p.page_table + (size_t)b * p.max_pages;
+            const uint32_t blk = (uint32_t)(kPageSize * p.hd * 2);
+            for (int lp = j0 / kPageSize; lp <= (jc - 1) / kPageSize; ++lp) {
+                const int ph = prow[lp];
+                if (ph < 0 || ph >= p.n_pages) break;
+                const size_t off = (((size_t)t.layer * p.n_pages + ph) * p.nkv + t.aux) * (size_t)kPageSize * p.hd;
+                prefetch_l2(p.k_pages + off, blk);
+                prefetch_l2(p.v_pages + off, blk);
+            }
+            continue;
+        }
+        if (t.op == MK_OP_EXP_GATEUP || t.op == MK_OP_EXP_DOWN) continue;
+        if (t.op == MK_OP_LMHEAD && p.skip_lm) continue;
+        GemvGeom g;
+        gemv_geom(p, t, g, true);
+        const int64_t bytes = (int64_t)g.rows * g.K * 2;
+        for (int bi = 0; bi < g.nblk; ++bi)
+            for (int64_t off = 0; off < bytes; off += 32768) {
+                const int64_t n = bytes - off < 32768 ? bytes - off : 32768;
+                prefetch_l2(reinterpret_cast<const uint8_t*>(g.w[bi]) + off, (uint32_t)n);
+            }
     }
 }
 
@@ -528,23 +626,6 @@ __device__ __forceinline__ float x_mid_at(const Params& p, int l, int b, int i) 
     return __ldcg(p.x_mid + ((size_t)l * p.max_batch + b) * p.H + i);
 }
 
-// Input element i of a GEMV task (before normalisation).
-__device__ __forceinline__ float gemv_input(const Params& p, const Task& t, int i) {
-    const int l = t.layer, b = t.b;
-    switch (t.op) {
-        case MK_OP_QKV: return x_in(p, l, 0, i);
-        case MK_OP_OPROJ: return __ldcg(p.o + ((size_t)l * p.max_batch) * (p.nq * p.hd) + i);
-        case MK_OP_GATEUP:
-        case MK_OP_ROUTER: return x_mid_at(p, l, 0, i);
-        case MK_OP_EXP_GATEUP: return x_mid_at(p, l, b, i);
-        case MK_OP_DOWN: return __ldcg(p.act + ((size_t)l * p.max_batch) * p.F + i);
-        case MK_OP_EXP_DOWN:
-            return __ldcg(p.act + (((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.Fe + i);
-        case MK_OP_LMHEAD: return x_in(p, p.L, 0, i);
-        default: return 0.0f;
-    }
-}
-
 __device__ __forceinline__ const uint16_t* gemv_norm_gain(const Params& p, const Task& t) {
     switch (t.op) {
         case MK_OP_QKV: return p.layers[t.layer].attn_norm;
@@ -557,16 +638,15 @@ __device__ __forceinline__ const uint16_t* gemv_norm_gain(const Params& p, const
 }
 
 // Sum over all consumer threads, same order in every CTA.
-__device__ __forceinline__ float block_sum(Smem& sm, float v) {
+__device__ __forceinline__ float block_sum(const Params& p, Smem& sm, uint32_t& cph, float v) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     v = warp_sum(v);
-    consumer_sync();
     if (lane == 0) sm.bcast[warp] = v;
-    consumer_sync();
+    csync(p, sm, cph);
     float s = 0.0f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) s += sm.bcast[w];
-    consumer_sync();
+    csync(p, sm, cph);   // bcast is free again
     return s;
 }
 
@@ -591,6 +671,43 @@ __device__ __forceinline__ ThreadMap thread_map(int K) {
 }
 
 // Loads this thread's slice of the (normalised) input into registers.
+// Split partial layout: [L][B][nkv][S][HPG][hd + 2] = (m, l, o[hd]) per head, with
+// m in the log2 domain and o not yet divided by l.
+__device__ __forceinline__ float* attn_part(const Params& p, int l, int b, int g, int s, int h) {
+    const int hpg = hpg_of(p);
+    size_t idx = ((((size_t)l * p.max_batch + b) * p.nkv + g) * p.S + s) * hpg + h;
+    return p.part + idx * (p.hd + 2);
+}
+
+// Input of the O-projection: the attention output, merged over the active splits
+// of every (sequence, kv head) in split order.  Eight consecutive columns lie in
+// one q head.
+__device__ __forceinline__ void load8_attn_merge(const Params& p, int l, int b, int col,
+                                                 float2 (&x)[4]) {
+    const int hd = p.hd, hpg = hpg_of(p);
+    const int head = col / hd, i = col % hd;
+    const int g = head / hpg, h = head % hpg;
+    int pos = position_of(p, b);
+    if (pos < 0 || pos >= p.max_ctx) pos = 0;
+    const int sa = attn_active_splits(pos + 1, p.S);
+    float M = -INFINITY;
+    for (int sp = 0; sp < sa; ++sp) M = fmaxf(M, __ldcg(attn_part(p, l, b, g, sp, h)));
+    float L = 0.0f;
+    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int sp = 0; sp < sa; ++sp) {
+        const float* pp = attn_part(p, l, b, g, sp, h);
+        const float m = __ldcg(pp);
+        if (m == -INFINITY) continue;
+        const float f = exp2f(m - M);
+        L = fmaf(__ldcg(pp + 1), f, L);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = fmaf(__ldcg(pp + 2 + i + e), f, o[e]);
+    }
+    const float inv = 1.0f / L;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = make_float2(o[2 * e] * inv, o[2 * e + 1] * inv);
+}
+
 // Where a GEMV task's input vector lives: an fp32 row, a bf16 embedding row, and
 // for an MoE residual the routed experts' outputs with their combine weights.
 struct InSrc {
@@ -626,7 +743,7 @@ __device__ __forceinline__ InSrc gemv_src(const Params& p, const Task& t) {
     switch (t.op) {
         case MK_OP_QKV: return xin_src(p, l, 0);
         case MK_OP_LMHEAD: return xin_src(p, p.L, 0);
-        case MK_OP_OPROJ: s.base = p.o + ((size_t)l * p.max_batch) * (p.nq * p.hd); break;
+        case MK_OP_OPROJ: break;   // merged from the attention partials (load8_attn_merge)
         case MK_OP_GATEUP:
         case MK_OP_ROUTER: s.base = p.x_mid + ((size_t)l * p.max_batch) * p.H; break;
         case MK_OP_EXP_GATEUP: s.base = p.x_mid + ((size_t)l * p.max_batch + b) * p.H; break;
@@ -657,7 +774,7 @@ __device__ __forceinline__ void load8(const InSrc& s, int col, float2 (&x)[4]) {
     x[1] = make_float2(a.z, a.w);
     x[2] = make_float2(c.x, c.y);
     x[3] = make_float2(c.z, c.w);
-    if (!PARTS) return;
+    if constexpr (!PARTS) return;
     for (int k = 0; k < s.nparts; ++k) {
         const float w = __ldcg(s.pw + k);
         const float4 pa = __ldcg(reinterpret_cast<const float4*>(s.parts + (size_t)k * s.pstride + col));
@@ -673,8 +790,8 @@ __device__ __forceinline__ void load8(const InSrc& s, int col, float2 (&x)[4]) {
 // pass: the sum of squares comes from the slices of group 0, which together
 // cover every column exactly once, so every CTA reduces in the same order.
 template <bool PARTS>
-__device__ void gemv_prologue_t(const Params& p, Smem& sm, const Task& t, const ThreadMap& m, int K,
-                                const InSrc& src, float2 (&xr)[kMaxVecPerThread][4]) {
+__device__ void gemv_prologue_t(const Params& p, Smem& sm, uint32_t& cph, const Task& t, const ThreadMap& m,
+                                int K, const InSrc& src, float2 (&xr)[kMaxVecPerThread][4]) {
     const uint16_t* gain = gemv_norm_gain(p, t);
     float ss = 0.0f;
 #pragma unroll
@@ -692,7 +809,7 @@ __device__ void gemv_prologue_t(const Params& p, Smem& sm, const Task& t, const 
 #pragma unroll
         for (int e = 0; e < 4; ++e) ss = fmaf(xr[j][e].y, xr[j][e].y, fmaf(xr[j][e].x, xr[j][e].x, ss));
     if (gain) {
-        const float tot = block_sum(sm, (m.grp == 0 && m.active) ? ss : 0.0f);
+        const float tot = block_sum(p, sm, cph, (m.grp == 0 && m.active) ? ss : 0.0f);
         const float rstd = 1.0f / sqrtf(tot / (float)K + p.eps);
 #pragma unroll
         for (int j = 0; j < kMaxVecPerThread; ++j) {
@@ -709,11 +826,40 @@ __device__ void gemv_prologue_t(const Params& p, Smem& sm, const Task& t, const 
     }
 }
 
-__device__ __forceinline__ void gemv_prologue(const Params& p, Smem& sm, const Task& t, const ThreadMap& m,
-                                              int K, float2 (&xr)[kMaxVecPerThread][4]) {
+__device__ __forceinline__ void gemv_prologue(const Params& p, Smem& sm, uint32_t& cph, const Task& t,
+                                              const ThreadMap& m, int K,
+                                              float2 (&xr)[kMaxVecPerThread][4]) {
+    if (t.op == MK_OP_OPROJ) {
+        // merged attention output -> shared memory (K <= the scratch size) -> registers
+        float* ob = sm.attn;
+        csync(p, sm, cph);                       // the scratch is free
+        for (int v = threadIdx.x; v < K / 8; v += kConsumerThreads) {
+            float2 x[4];
+            load8_attn_merge(p, t.layer, 0, v * 8, x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ob[v * 8 + 2 * e] = x[e].x;
+                ob[v * 8 + 2 * e + 1] = x[e].y;
+            }
+        }
+        csync(p, sm, cph);
+#pragma unroll
+        for (int j = 0; j < kMaxVecPerThread; ++j) {
+            const int v = m.lig + j * m.gstride;
+            if (j < m.vpt && v < m.nvec && m.active) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xr[j][e] = make_float2(ob[v * 8 + 2 * e], ob[v * 8 + 2 * e + 1]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xr[j][e] = make_float2(0.0f, 0.0f);
+            }
+        }
+        csync(p, sm, cph);                       // everyone has its slice
+        return;
+    }
     const InSrc src = gemv_src(p, t);
-    if (src.nparts > 0) gemv_prologue_t<true>(p, sm, t, m, K, src, xr);
-    else gemv_prologue_t<false>(p, sm, t, m, K, src, xr);
+    if (src.nparts > 0) gemv_prologue_t<true>(p, sm, cph, t, m, K, src, xr);
+    else gemv_prologue_t<false>(p, sm, cph, t, m, K, src, xr);
 }
 
 // Packed fp32x2 fused multiply-add (sm_100): d = a * b + c, lane-wise on two floats.
@@ -897,9 +1043,9 @@ template <int VPT, int RPS, int NROWS>
 __device__ bool gemv_fast_rows(const Params& p, Smem& sm, int ti, const float2 (&xr)[kMaxVecPerThread][4],
                                int buf, int& stage, uint32_t& lap) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float2 acc[NROWS];
+    float acc[NROWS];
 #pragma unroll
-    for (int r = 0; r < NROWS; ++r) acc[r] = make_float2(0.f, 0.f);
+    for (int r = 0; r < NROWS; ++r) acc[r] = 0.f;
 #pragma unroll
     for (int st = 0; st < NROWS / RPS; ++st) {
         if (st > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) { sm.flag[3] = 1; return false; }
@@ -911,17 +1057,17 @@ __device__ bool gemv_fast_rows(const Params& p, Smem& sm, int ti, const float2 (
 #pragma unroll
             for (int j = 0; j < VPT; ++j) q[rr][j] = sv[(rr * VPT + j) * kConsumerThreads];
 #pragma unroll
-        for (int rr = 0; rr < RPS; ++rr)
+        for (int rr = 0; rr < RPS; ++rr) {
+            float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) dot8(q[rr][j], xr[j], acc[st * RPS + rr]);
+            for (int j = 0; j < VPT; ++j) dot8(q[rr][j], xr[j], a);
+            acc[st * RPS + rr] += a.x + a.y;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[stage]);
         if (++stage == kStages) { stage = 0; ++lap; }
     }
-    float v[NROWS];
-#pragma unroll
-    for (int r = 0; r < NROWS; ++r) v[r] = acc[r].x + acc[r].y;
-    const float tot = warp_reduce_rows<NROWS>(v);
+    const float tot = warp_reduce_rows<NROWS>(acc);
     if ((lane & (32 / NROWS - 1)) == 0) sm.red[buf][lane / (32 / NROWS)][warp] = tot;
     return true;
 }
@@ -933,9 +1079,9 @@ __device__ bool gemv_fast_segs(const Params& p, Smem& sm, int ti, const float2 (
                                int buf, int& stage, uint32_t& lap, bool first_seen) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int NSEG = (VPT + SEGJ - 1) / SEGJ;
-    float2 acc[NROWS];
+    float acc[NROWS];
 #pragma unroll
-    for (int r = 0; r < NROWS; ++r) acc[r] = make_float2(0.f, 0.f);
+    for (int r = 0; r < NROWS; ++r) acc[r] = 0.f;
 #pragma unroll
     for (int r = 0; r < NROWS; ++r) {
 #pragma unroll
@@ -946,23 +1092,21 @@ __device__ bool gemv_fast_segs(const Params& p, Smem& sm, int ti, const float2 (
             }
             if (sm.info[stage].task != ti) { set_error(p, kErrFault, ti, -4, sm.info[stage].task, 3); sm.flag[3] = 1; return false; }
             const uint4* sv = reinterpret_cast<const uint4*>(sm.ring[stage]) + threadIdx.x;
-            constexpr int J0 = 0;
             uint4 q[SEGJ];
 #pragma unroll
             for (int j = 0; j < SEGJ; ++j)
                 if (sg * SEGJ + j < VPT) q[j] = sv[j * kConsumerThreads];
+            float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = J0; j < SEGJ; ++j)
-                if (sg * SEGJ + j < VPT) dot8(q[j], xr[sg * SEGJ + j], acc[r]);
+            for (int j = 0; j < SEGJ; ++j)
+                if (sg * SEGJ + j < VPT) dot8(q[j], xr[sg * SEGJ + j], a);
+            acc[r] += a.x + a.y;
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
             if (++stage == kStages) { stage = 0; ++lap; }
         }
     }
-    float v[NROWS];
-#pragma unroll
-    for (int r = 0; r < NROWS; ++r) v[r] = acc[r].x + acc[r].y;
-    const float tot = warp_reduce_rows<NROWS>(v);
+    const float tot = warp_reduce_rows<NROWS>(acc);
     if ((lane & (32 / NROWS - 1)) == 0) sm.red[buf][lane / (32 / NROWS)][warp] = tot;
     return true;
 }
@@ -1018,22 +1162,52 @@ struct AttnState {
     float m[HPG], l[HPG];
 };
 
-template <int HPG, int DPL>
-__device__ __forceinline__ void attn_token(AttnState<HPG, DPL>& st, const float (&k)[DPL],
-                                           const float (&v)[DPL]) {
+// T tokens at once: the T*HPG partial dot products are summed over the warp
+// together (independent shuffle chains), then one online-softmax update per head.
+// ok[t] masks tokens beyond the range.
+template <int HPG, int DPL, int T>
+__device__ __forceinline__ void attn_tokens(AttnState<HPG, DPL>& st, const float (&k)[T][DPL],
+                                            const float (&v)[T][DPL], const bool (&ok)[T]) {
+    float sc[T][HPG];
+#pragma unroll
+    for (int t = 0; t < T; ++t)
+#pragma unroll
+        for (int h = 0; h < HPG; ++h) {
+            float a = 0.0f;
+#pragma unroll
+            for (int d = 0; d < DPL; ++d) a = fmaf(st.q[h][d], k[t][d], a);
+            sc[t][h] = a;
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int t = 0; t < T; ++t)
+#pragma unroll
+            for (int h = 0; h < HPG; ++h) sc[t][h] += __shfl_xor_sync(0xFFFFFFFFu, sc[t][h], o);
 #pragma unroll
     for (int h = 0; h < HPG; ++h) {
-        float s = 0.0f;
+        float mx = st.m[h];
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) s = fmaf(st.q[h][d], k[d], s);
-        s = warp_sum(s);                       // log2-domain score (q pre-scaled)
-        float mn = fmaxf(st.m[h], s);
-        float corr = exp2f(st.m[h] - mn);
-        float pw = exp2f(s - mn);
-        st.l[h] = fmaf(st.l[h], corr, pw);
+        for (int t = 0; t < T; ++t)
+            if (ok[t]) mx = fmaxf(mx, sc[t][h]);
+        if (mx == -INFINITY) continue;                   // no token yet
+        const float corr = exp2f(st.m[h] - mx);          // 0 when m was -inf
+        float pw[T];
+        float ps = 0.0f;
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) st.o[h][d] = fmaf(st.o[h][d], corr, pw * v[d]);
-        st.m[h] = mn;
+        for (int t = 0; t < T; ++t) {
+            pw[t] = ok[t] ? exp2f(sc[t][h] - mx) : 0.0f;
+            ps += pw[t];
+        }
+        st.l[h] = fmaf(st.l[h], corr, ps);
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) {
+            float acc = st.o[h][d] * corr;
+#pragma unroll
+            for (int t = 0; t < T; ++t) acc = fmaf(pw[t], v[t][d], acc);
+            st.o[h][d] = acc;
+        }
+        st.m[h] = mx;
     }
 }
 
@@ -1049,17 +1223,16 @@ __device__ __forceinline__ void load_bf16_dpl(const uint16_t* src, float (&out)[
     }
 }
 
-// Split partial layout: [L][B][nkv][S][HPG][hd + 2] = (m, l, o[hd]) per head.
-__device__ __forceinline__ float* attn_part(const Params& p, int l, int b, int g, int s, int h) {
-    const int hpg = hpg_of(p);
-    size_t idx = ((((size_t)l * p.max_batch + b) * p.nkv + g) * p.S + s) * hpg + h;
-    return p.part + idx * (p.hd + 2);
-}
-
+// One split of decode attention for (layer, sequence b, kv head g): RoPE on the
+// group's q heads and the new k, KV-cache append (the split that owns the new
+// position), softmax partial over the split's positions streamed from the paged
+// cache.  Writes the partial and hands the completion to the signal warp; the
+// O-projection's input stage merges the splits in a fixed order.
 template <int HPG, int DPL>
-__device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti, int& stage,
+__device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti, int& stage,
                                uint32_t& lap, bool& abort_all) {
     constexpr int HD = DPL * 32;
+    constexpr int TB = (HPG >= 8) ? 2 : 4;               // tokens per warp step
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = t.b, g = t.aux, s = (int)t.r0, S = (int)t.r1, l = t.layer;
     const bool active_row = b < p.batch;
@@ -1067,7 +1240,10 @@ __device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti,
     bool valid = active_row && pos >= 0 && pos < p.max_ctx && pos / kPageSize < p.max_pages;
     if (active_row && !valid && tid == 0) set_error(p, kErrInvalid, ti, -3, pos, b);
     int j0 = 0, j1 = 0;
-    if (valid) attn_range(pos + 1, S, s, j0, j1);
+    if (valid) {
+        const int sa = attn_active_splits(pos + 1, S);
+        if (s < sa) attn_range(pos + 1, sa, s, j0, j1);
+    }
     const bool has_new = valid && pos >= j0 && pos < j1;
     const float qscale = 1.4426950408889634f / sqrtf((float)HD);   // log2(e) / sqrt(d)
 
@@ -1079,38 +1255,57 @@ __device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti,
 #pragma unroll
         for (int d = 0; d < DPL; ++d) st.o[h][d] = 0.0f;
     }
-    if (valid && j1 > j0) {
-        // q of the group's heads, k and v of the new token, rotated at `pos`
+    const bool work = valid && j1 > j0;
+    csync(p, sm, cph);                                   // shared scratch of the previous task is free
+    if (work) {
+        // q of the group's heads and the new k (rotated at `pos`), the new v; all loads
+        // of a thread are issued before any is used
         const float* qkv = p.qkv + ((size_t)l * p.max_batch + b) * ((p.nq + 2 * p.nkv) * HD);
-        const float* rope = p.rope + (size_t)pos * HD;   // [HD/2][2]
-        for (int idx = tid; idx < (HPG + 1) * (HD / 2); idx += kConsumerThreads) {
-            int h = idx / (HD / 2), i = idx % (HD / 2);
-            float c = rope[2 * i], sn = rope[2 * i + 1];
-            const float* src = (h < HPG) ? qkv + (size_t)(g * HPG + h) * HD : qkv + (size_t)(p.nq + g) * HD;
-            float x0 = __ldcg(src + i), x1 = __ldcg(src + i + HD / 2);
-            float r0 = x0 * c - x1 * sn, r1 = x1 * c + x0 * sn;
-            if (h < HPG) {
-                sm.qs[h * HD + i] = r0 * qscale;
-                sm.qs[h * HD + i + HD / 2] = r1 * qscale;
-            } else {
-                sm.kn[i] = bf16_to_f32(f32_to_bf16_rne(r0));
-                sm.kn[i + HD / 2] = bf16_to_f32(f32_to_bf16_rne(r1));
+        const float* rope = p.rope + (size_t)pos * HD;   // [HD/2][2] = cos, sin
+        constexpr int NPAIR = (HPG + 1) * (HD / 2);
+        constexpr int IT = (NPAIR + kConsumerThreads - 1) / kConsumerThreads;
+        float x0[IT], x1[IT], cs[IT], sn[IT];
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+            const int idx = tid + it * kConsumerThreads;
+            if (idx < NPAIR) {
+                const int h = idx / (HD / 2), i = idx % (HD / 2);
+                const float* src = (h < HPG) ? qkv + (size_t)(g * HPG + h) * HD : qkv + (size_t)(p.nq + g) * HD;
+                x0[it] = __ldcg(src + i);
+                x1[it] = __ldcg(src + i + HD / 2);
+                const float2 r = __ldg(reinterpret_cast<const float2*>(rope) + i);
+                cs[it] = r.x;
+                sn[it] = r.y;
             }
         }
-        for (int i = tid; i < HD; i += kConsumerThreads) {
-            float v = __ldcg(qkv + (size_t)(p.nq + p.nkv + g) * HD + i);
-            sm.vn[i] = bf16_to_f32(f32_to_bf16_rne(v));
+        float vv = 0.0f;
+        if (tid < HD) vv = __ldcg(qkv + (size_t)(p.nq + p.nkv + g) * HD + tid);
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+            const int idx = tid + it * kConsumerThreads;
+            if (idx < NPAIR) {
+                const int h = idx / (HD / 2), i = idx % (HD / 2);
+                const float r0 = x0[it] * cs[it] - x1[it] * sn[it], r1 = x1[it] * cs[it] + x0[it] * sn[it];
+                if (h < HPG) {
+                    sm.qs[h * HD + i] = r0 * qscale;
+                    sm.qs[h * HD + i + HD / 2] = r1 * qscale;
+                } else {
+                    sm.kn[i] = bf16_to_f32(f32_to_bf16_rne(r0));
+                    sm.kn[i + HD / 2] = bf16_to_f32(f32_to_bf16_rne(r1));
+                }
+            }
         }
-        consumer_sync();
+        if (tid < HD) sm.vn[tid] = bf16_to_f32(f32_to_bf16_rne(vv));
+        csync(p, sm, cph);
         // KV append: the split that owns the new position writes it
         if (has_new) {
             const int* prow = p.page_table + (size_t)b * p.max_pages;
-            int ph = prow[pos / kPageSize];
+            const int ph = prow[pos / kPageSize];
             if (ph >= 0 && ph < p.n_pages) {
                 size_t off = ((((size_t)l * p.n_pages + ph) * p.nkv + g) * kPageSize + pos % kPageSize) * HD;
-                for (int i = tid; i < HD; i += kConsumerThreads) {
-                    p.k_pages[off + i] = f32_to_bf16_rne(sm.kn[i]);
-                    p.v_pages[off + i] = f32_to_bf16_rne(sm.vn[i]);
+                if (tid < HD) {
+                    p.k_pages[off + tid] = f32_to_bf16_rne(sm.kn[tid]);
+                    p.v_pages[off + tid] = f32_to_bf16_rne(sm.vn[tid]);
                 }
             } else if (tid == 0) {
                 set_error(p, kErrInvalid, ti, -2, pos / kPageSize, b);
@@ -1144,13 +1339,20 @@ __device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti,
             const int first_page = inf.aux;
             const int tok_lo = max(j0, first_page * kPageSize);
             const int tok_hi = min(jc, (first_page + pps) * kPageSize);
-            for (int pos_t = tok_lo + warp; pos_t < tok_hi; pos_t += kConsumerWarps) {
-                int pi = pos_t / kPageSize - first_page, slot = pos_t % kPageSize;
-                const uint16_t* kb = base + (size_t)pi * 2 * blk_elems + slot * HD + lane * DPL;
-                float kf[DPL], vf[DPL];
-                load_bf16_dpl<DPL>(kb, kf);
-                load_bf16_dpl<DPL>(kb + blk_elems, vf);
-                attn_token<HPG, DPL>(st, kf, vf);
+            for (int t0 = tok_lo + warp * TB; t0 < tok_hi; t0 += kConsumerWarps * TB) {
+                float kf[TB][DPL], vf[TB][DPL];
+                bool ok[TB];
+#pragma unroll
+                for (int u = 0; u < TB; ++u) {
+                    const int pt = t0 + u;
+                    ok[u] = pt < tok_hi;
+                    const int ptc = ok[u] ? pt : t0;
+                    const int pi = ptc / kPageSize - first_page, slot = ptc % kPageSize;
+                    const uint16_t* kb = base + (size_t)pi * 2 * blk_elems + slot * HD + lane * DPL;
+                    load_bf16_dpl<DPL>(kb, kf[u]);
+                    load_bf16_dpl<DPL>(kb + blk_elems, vf[u]);
+                }
+                attn_tokens<HPG, DPL, TB>(st, kf, vf, ok);
             }
         }
         __syncwarp();
@@ -1160,15 +1362,16 @@ __device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti,
         if (last) break;
     }
     if (has_new && warp == 0) {
-        float kf[DPL], vf[DPL];
+        float kf[1][DPL], vf[1][DPL];
+        const bool ok[1] = {true};
 #pragma unroll
         for (int d = 0; d < DPL; ++d) {
-            kf[d] = sm.kn[lane * DPL + d];
-            vf[d] = sm.vn[lane * DPL + d];
+            kf[0][d] = sm.kn[lane * DPL + d];
+            vf[0][d] = sm.vn[lane * DPL + d];
         }
-        attn_token<HPG, DPL>(st, kf, vf);
+        attn_tokens<HPG, DPL, 1>(st, kf, vf, ok);
     }
-    // combine the 8 warps' partials
+    // combine the warps' partials (fixed order) into this split's partial
     float* sc = sm.attn;
 #pragma unroll
     for (int h = 0; h < HPG; ++h) {
@@ -1177,11 +1380,11 @@ __device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti,
 #pragma unroll
         for (int d = 0; d < DPL; ++d) w[2 + lane * DPL + d] = st.o[h][d];
     }
-    consumer_sync();
-    if (sm.flag[3]) { abort_all = true; return; }   // same decision in every consumer thread
-    if (valid || !active_row) {
+    csync(p, sm, cph);
+    if (sm.flag[3]) { abort_all = true; return; }
+    if (valid) {
         for (int idx = tid; idx < HPG * (HD + 2); idx += kConsumerThreads) {
-            int h = idx / (HD + 2), c = idx % (HD + 2);
+            const int h = idx / (HD + 2), c = idx % (HD + 2);
             float M = -INFINITY;
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sc[((size_t)w * HPG + h) * (HD + 2)]);
@@ -1194,7 +1397,7 @@ __device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti,
 #pragma unroll
                     for (int w = 0; w < kConsumerWarps; ++w) {
                         const float* ww = sc + ((size_t)w * HPG + h) * (HD + 2);
-                        float f = (ww[0] == -INFINITY) ? 0.0f : exp2f(ww[0] - M);
+                        const float f = (ww[0] == -INFINITY) ? 0.0f : exp2f(ww[0] - M);
                         acc = fmaf(ww[c], f, acc);
                     }
                 }
@@ -1203,41 +1406,6 @@ __device__ void attention_task(const Params& p, Smem& sm, const Task& t, int ti,
             attn_part(p, l, b, g, s, h)[c] = val;
         }
     }
-    // arrival; the last split of (layer, b, kv head) merges and signals
-    consumer_sync();
-    if (tid == 0) {
-        __threadfence();
-        uint32_t* cnt = p.merge_cnt + ((size_t)l * p.max_batch + b) * p.nkv + g;
-        uint32_t old = atomicAdd(cnt, 1u);
-        __threadfence();
-        sm.flag[0] = (old == (uint32_t)S * p.epoch - 1u) ? 1 : 0;
-        atomicAdd(p.done, 1u);
-    }
-    consumer_sync();
-    if (sm.flag[0]) {
-        if (valid) {
-            for (int idx = tid; idx < HPG * HD; idx += kConsumerThreads) {
-                int h = idx / HD, i = idx % HD;
-                float M = -INFINITY;
-                for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(attn_part(p, l, b, g, sp, h)));
-                float Ls = 0.0f, O = 0.0f;
-                for (int sp = 0; sp < S; ++sp) {
-                    const float* pp = attn_part(p, l, b, g, sp, h);
-                    float m = __ldcg(pp);
-                    float f = (m == -INFINITY) ? 0.0f : exp2f(m - M);
-                    Ls = fmaf(__ldcg(pp + 1), f, Ls);
-                    O = fmaf(__ldcg(pp + 2 + i), f, O);
-                }
-                p.o[((size_t)l * p.max_batch + b) * (p.nq * HD) + (size_t)(g * HPG + h) * HD + i] = O / Ls;
-            }
-        }
-        consumer_sync();
-        if (tid == 0) {
-            __threadfence();
-            if (t.sig != MK_NO_EVENT) red_release_add(&p.events[t.sig], 1u);
-        }
-    }
-    if (tid == 0 && p.trace) p.trace[(size_t)ti * 4 + 2] = globaltimer();
 }
 
 // ----------------------------------------------------------------------------- consumer: router top-k
@@ -1309,93 +1477,105 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
     int sig_slot = 0;
     uint32_t sig_lap = 0;
     int buf = 0;
+    uint32_t cph = 0;                                   // phase of sm.csync
     float2 xr[kMaxVecPerThread][4];
     int x_key_op = -1, x_key_layer = -1, x_key_b = -1, x_key_aux = -1;
-    uint32_t ok_evt[4] = {MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT};   // thread 0
+    uint32_t ok_evt[4] = {MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT};   // per warp
 
-    // Every exit decision below is taken by thread 0 (or written to sm.flag[3]
-    // before a consumer barrier) and read by all consumer threads after that
-    // barrier, so all 256 consumer threads always pass the same named barriers.
+    // Each warp waits for its own data and dependencies; the warps meet once per
+    // task, after the chunk loop (csync, bounded).  Every failure raises
+    // sm.flag[3], which all consumer threads read after that meeting, so they
+    // leave the loop together.
     while (true) {
-        if (tid == 0) {
-            int st = 1;                                   // 1 run, 0 abort, 2 end of work
-            if (sm.flag[3] || !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 4)) {
-                st = 0;
-            } else {
-                const int ti = sm.info[stage].task;
-                if (ti < 0) {
-                    st = 2;
-                } else {
-                    const uint32_t e = p.tasks[ti].wait0;
-                    if (p.trace) p.trace[(size_t)ti * 4 + 0] = globaltimer();
-                    if (e != MK_NO_EVENT && e != ok_evt[0] && e != ok_evt[1] && e != ok_evt[2] &&
-                        e != ok_evt[3]) {
-                        if (event_wait(p, e, p.thr[e] * p.epoch + p.wait_offset, ti)) {
-                            __threadfence();
-                            ok_evt[3] = ok_evt[2]; ok_evt[2] = ok_evt[1]; ok_evt[1] = ok_evt[0]; ok_evt[0] = e;
-                        } else {
-                            st = 0;
-                        }
-                    }
-                    if (p.trace) {
-                        p.trace[(size_t)ti * 4 + 1] = globaltimer();
-                        p.trace[(size_t)ti * 4 + 3] = (uint64_t)blockIdx.x;
-                    }
-                }
-            }
-            sm.flag[1] = st;
-        }
-        consumer_sync();
-        const int st = sm.flag[1];
-        if (st == 0) break;
-        seen_complete_wait(p, &sm.full[stage], lap & 1, &sm.flag[3]);   // seen complete by thread 0
-        const int ti = sm.info[stage].task;
-        if (st == 2) {
+        bool ok = mbar_wait_bounded(p, &sm.full[stage], lap & 1, 4);
+        int ti = ok ? sm.info[stage].task : -2;
+        if (ti == -1) {                                  // end of work (same stage for every warp)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
             break;
         }
-        const Task t = p.tasks[ti];
+        Task t;
+        if (ok) t = sm.info[stage].rec;
+        if (p.trace && tid == 0 && ok) p.trace[(size_t)ti * 4 + 0] = globaltimer();
+        if (ok) {
+            const uint32_t e = t.wait0;
+            if (e != MK_NO_EVENT && e != ok_evt[0] && e != ok_evt[1] && e != ok_evt[2] && e != ok_evt[3]) {
+                int r = 1;
+                if (lane == 0) {
+                    r = event_wait(p, e, p.thr[e] * p.epoch + p.wait_offset, ti) ? 1 : 0;
+                    if (r) __threadfence();
+                }
+                r = __shfl_sync(0xFFFFFFFFu, r, 0);
+                if (r) {
+                    ok_evt[3] = ok_evt[2]; ok_evt[2] = ok_evt[1]; ok_evt[1] = ok_evt[0]; ok_evt[0] = e;
+                } else {
+                    ok = false;
+                }
+            }
+        }
+        if (!ok) sm.flag[3] = 1;
+        if (p.trace && tid == 0 && ok) {
+            p.trace[(size_t)ti * 4 + 1] = globaltimer();
+            p.trace[(size_t)ti * 4 + 3] = (uint64_t)blockIdx.x;
+        }
 
-        if (t.op == MK_OP_ATTN) {
+        if (ok && t.op == MK_OP_ATTN) {
             bool abort_all = false;
-            attention_task<HPG, DPL>(p, sm, t, ti, stage, lap, abort_all);
+            attention_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
             if (abort_all) break;
-            // the input slice in registers is dead across an attention task (saves registers)
             x_key_op = -1;
+            // the input slice in registers is dead across an attention task (saves registers)
 #pragma unroll
             for (int j = 0; j < kMaxVecPerThread; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) xr[j][e] = make_float2(0.0f, 0.0f);
+            // hand the completion to the signal warp once this warp's stores are issued
+            if (tid == 0) {
+                if (sig_lap > 0 && !mbar_wait_bounded(p, &sm.sig_empty[sig_slot], (sig_lap - 1) & 1, 6))
+                    sm.flag[3] = 1;
+                sm.sig_evt[sig_slot] = t.sig;
+                sm.sig_task[sig_slot] = ti;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sig_full[sig_slot]);
+            if (++sig_slot == kSigSlots) { sig_slot = 0; ++sig_lap; }
             continue;
         }
 
         // ---- GEMV task
-        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
         GemvGeom g;
-        gemv_geom(p, t, g, false);
-        const ThreadMap m = thread_map(g.K);
-        if (!skip) {
-            if (t.op == MK_OP_QKV && t.layer == 0 && tid == 0) {
-                int tok = p.tokens[0];
-                if (tok < 0 || tok >= p.V) set_error(p, kErrInvalid, ti, -5, tok, 0);
-            }
-            if (!(x_key_op == t.op && x_key_layer == t.layer && x_key_b == t.b &&
-                  (x_key_aux == t.aux || t.op != MK_OP_EXP_DOWN))) {
-                gemv_prologue(p, sm, t, m, g.K, xr);
-                x_key_op = t.op; x_key_layer = t.layer; x_key_b = t.b; x_key_aux = t.aux;
-            }
-        }
-        const int rows_total = g.rows * g.nblk;
-        // residual rows for the epilogue, fetched now so the load overlaps the streaming
+        ThreadMap m;
+        bool skip = false;
+        int rows_total = 0;
         float resid = 0.0f;
-        if (!skip && tid < rows_total) {
-            if (t.op == MK_OP_OPROJ) resid = x_in(p, t.layer, 0, (int)t.r0 + tid);
-            else if (t.op == MK_OP_DOWN) resid = x_mid_at(p, t.layer, 0, (int)t.r0 + tid);
+        if (ok) {
+            skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
+            gemv_geom(p, t, g, false);
+            m = thread_map(g.K);
+            rows_total = g.rows * g.nblk;
+            if (!skip) {
+                if (t.op == MK_OP_QKV && t.layer == 0 && tid == 0) {
+                    const int tok = p.tokens[0];
+                    if (tok < 0 || tok >= p.V) set_error(p, kErrInvalid, ti, -5, tok, 0);
+                }
+                if (!(x_key_op == t.op && x_key_layer == t.layer && x_key_b == t.b &&
+                      (x_key_aux == t.aux || t.op != MK_OP_EXP_DOWN))) {
+                    gemv_prologue(p, sm, cph, t, m, g.K, xr);
+                    x_key_op = t.op; x_key_layer = t.layer; x_key_b = t.b; x_key_aux = t.aux;
+                }
+                // residual rows for the epilogue, fetched now so the load overlaps the streaming
+                if (tid < rows_total) {
+                    if (t.op == MK_OP_OPROJ) resid = x_in(p, t.layer, 0, (int)t.r0 + tid);
+                    else if (t.op == MK_OP_DOWN) resid = x_mid_at(p, t.layer, 0, (int)t.r0 + tid);
+                }
+            }
+            const long long c_ch = (p.stats && tid == 0) ? clock64() : 0;
+            const int handled = skip ? 0 : gemv_fast_dispatch(p, sm, ti, g, m, xr, buf, stage, lap);
+            if (handled == 0) (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+            if (p.stats && tid == 0) stat_add(p, 6, (unsigned long long)(clock64() - c_ch));
         }
-        int handled = skip ? 0 : gemv_fast_dispatch(p, sm, ti, g, m, xr, buf, stage, lap);
-        if (handled == 0) (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
-        consumer_sync();   // all partial sums of this task are in red[buf]
+        const long long c_ep = (p.stats && tid == 0) ? clock64() : 0;
+        csync(p, sm, cph);                               // all partial sums are in red[buf]
         if (sm.flag[3]) break;
 
         // ---- epilogue: reduce the warps' partials in fixed order, apply the op's output rule
@@ -1446,18 +1626,20 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
 
         if (t.op == MK_OP_ROUTER) {
             // arrival; the last router tile of the layer selects the experts and signals
-            consumer_sync();
+            csync(p, sm, cph);
             if (tid == 0) {
                 __threadfence();
-                uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
+                const uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
                 __threadfence();
                 sm.flag[0] = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
                 atomicAdd(p.done, 1u);
             }
-            consumer_sync();
-            if (sm.flag[0]) {
+            csync(p, sm, cph);
+            const int last = sm.flag[0];
+            csync(p, sm, cph);                           // flag[0] read by everyone
+            if (last) {
                 router_finalize(p, sm, t.layer);
-                consumer_sync();
+                csync(p, sm, cph);
                 if (tid == 0) {
                     __threadfence();
                     if (t.sig != MK_NO_EVENT) red_release_add(&p.events[t.sig], 1u);
@@ -1477,9 +1659,10 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.sig_full[sig_slot]);
         if (++sig_slot == kSigSlots) { sig_slot = 0; ++sig_lap; }
+        if (p.stats && tid == 0) stat_add(p, 7, (unsigned long long)(clock64() - c_ep));
     }
     // end of work for the signal warp
-    consumer_sync();
+    csync(p, sm, cph);
     if (tid == 0) {
         if (sig_lap > 0) (void)mbar_wait_bounded(p, &sm.sig_empty[sig_slot], (sig_lap - 1) & 1, 7);
         sm.sig_evt[sig_slot] = 0xFFFFFFFEu;
@@ -1505,7 +1688,9 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&sm.sig_full[s], kConsumerWarps);
             mbar_init(&sm.sig_empty[s], 1);
         }
+        mbar_init(&sm.csync, kConsumerWarps);
         for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
+        for (int i = 0; i < 8; ++i) sm.stat[i] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -1515,8 +1700,14 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         if (threadIdx.x == 0) stat_add(p, 3, (unsigned long long)(clock64() - k0));
     } else if (warp == kProducerWarp) {
         if (lane == 0) producer_loop(p, sm);
-    } else {
+    } else if (warp == kSignalWarp) {
         if (lane == 0) signal_loop(p, sm);
+    } else {
+        if (lane == 0) prefetch_loop(p);
+    }
+    if (p.stats) {
+        __syncthreads();
+        if (threadIdx.x < 8) p.stats[(size_t)blockIdx.x * 8 + threadIdx.x] += sm.stat[threadIdx.x];
     }
 }
 

@@ -15,7 +15,8 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kProducerWarp = kConsumerWarps;        // warp 8
 constexpr int kSignalWarp = kConsumerWarps + 1;      // warp 9
-constexpr int kThreads = (kConsumerWarps + 2) * 32;  // 320
+constexpr int kPrefetchWarp = kConsumerWarps + 2;    // warp 10
+constexpr int kThreads = (kConsumerWarps + 3) * 32;  // 352
 constexpr int kStageBytes = 16 * 1024;
 constexpr int kStages = 11;
 constexpr int kMaxTaskRows = 64;        // rows (all weight blocks) of one GEMV task
@@ -62,9 +63,10 @@ struct Params {
     uint32_t* events;
     unsigned long long* queue;   // global work-queue head
     unsigned long long queue_base;
+    unsigned long long* pf_head; // L2-prefetch cursor over the task list (same base as the queue)
+    uint32_t pf_dist;            // prefetch at most this many tasks ahead of the queue head (0: off)
     uint32_t* done;              // completed-task counter
     int* err;                    // [0] status, [1..4] info
-    uint32_t* merge_cnt;         // [L][max_batch][n_kv] attention split arrivals
     uint32_t* router_cnt;        // [L] router tile arrivals
     long long timeout_ns;
     uint32_t wait_offset;        // added to every wait target (0; tests set 1 to force a timeout)
@@ -85,9 +87,8 @@ struct Params {
     float* x_mid;    // [L][B][H]   residual after attention
     float* x_out;    // [L][B][H]   residual after the dense FFN
     float* qkv;      // [L][B][(nq+2nkv)*hd]
-    float* o;        // [L][B][nq*hd] merged attention output
     float* act;      // dense: [L][B][F]; MoE: [L][B][topk][Fe]
-    float* part;     // [L][B][nkv][S][hpg][hd+2] attention partials
+    float* part;     // [L][B][nkv][S][hpg][hd+2] attention split partials (m, l, o)
     float* rlogits;  // [L][B][E]
     float* moe_w;    // [L][B][topk]
     int* moe_sel;    // [L][B][topk]

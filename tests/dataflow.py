@@ -9,9 +9,8 @@ read, every valid order produces the same final digests ("identical bits").
 
 Read/write sets per operator mirror the megakernel's tiles:
   qkv      reads x_in[l] (all)                 writes qkv[l][rows]
-  attn     reads qkv[l] rows of its kv head    writes part[l,b,g,s]; the last split
-           of (l,b,g) reads all its parts and writes o[l][b][rows of g]
-  oproj    reads o[l] (all), x_in[l][rows]     writes x_mid[l][rows]
+  attn     reads qkv[l] rows of its kv head    writes part[l][b,g,s]
+  oproj    reads part[l] (all), x_in[l][rows]  writes x_mid[l][rows] (merging the splits)
   gateup   reads x_mid[l] (all)                writes act[l][rows]
   down     reads act[l] (all), x_mid[l][rows]  writes x_in[l+1][rows]
   router   reads x_mid[l] (all)                writes rlog[l][rows]; the last tile reads
@@ -81,7 +80,7 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
     T[("x_in", 0)] = Tensor(B * H, ready=True)      # embedding rows: inputs of the step
     for l in range(L):
         T[("qkv", l)] = Tensor(qkv_rows)
-        T[("o", l)] = Tensor(B * nq * hd)
+        T[("part", l)] = Tensor(B * nkv * 4096)
         T[("x_mid", l)] = Tensor(B * H)
         if moe:
             T[("rlog", l)] = Tensor(E)
@@ -93,8 +92,7 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
             T[("act", l)] = Tensor(F)
             T[("x_in", l + 1)] = Tensor(B * H)
     T[("logits",)] = Tensor(V)
-    parts = defaultdict(int)          # (l,b,g) -> arrivals
-    part_digest = defaultdict(int)
+    tasks_split = {tk.layer: tk.r1 for tk in tasks if tk.op == 2}
     router_arr = defaultdict(int)
     n_router = defaultdict(int)
     for tk in tasks:
@@ -154,15 +152,16 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
             d = qkv.read(g * hpg * hd, (g + 1) * hpg * hd, who)
             d += qkv.read(nq * hd + g * hd, nq * hd + (g + 1) * hd, who)
             d += qkv.read((nq + nkv) * hd + g * hd, (nq + nkv) * hd + (g + 1) * hd, who)
-            key = (l, b, g)
-            part_digest[key] = (part_digest[key] + _mix(base ^ d)) & M64
-            parts[key] += 1
-            if parts[key] == r1:                      # last split merges and signals
-                lo = b * nq * hd + g * hpg * hd
-                t("o", l).write(lo, lo + hpg * hd, part_digest[key], who)
-                signal(tk.signal)
+            idx = (b * nkv + g) * 4096 + r0            # r0 = split index
+            t("part", l).write(idx, idx + 1, _mix(base ^ (d & M64)), who)
+            signal(tk.signal)
         elif op == "oproj":
-            d = t("o", l).read(0, B * nq * hd, who) + read_xin(l, r0, r1, who)
+            n_split = tasks_split[l]
+            d = read_xin(l, r0, r1, who)
+            for bb in range(B):
+                for gg in range(nkv):
+                    lo = (bb * nkv + gg) * 4096
+                    d += t("part", l).read(lo, lo + n_split, who)
             t("x_mid", l).write(r0, r1, _mix(base ^ (d & M64)), who)
             signal(tk.signal)
         elif op == "gateup":

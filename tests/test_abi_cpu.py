@@ -73,12 +73,10 @@ def test_plan_is_topological_and_thresholds_match_signals(cfg):
     for i, t in enumerate(tasks):
         if t.signal != mk.MK_NO_EVENT:
             last_signal[t.signal] = i
-    # attention splits and router tiles signal once per group / layer
+    # router tiles signal once per layer (the last tile, after the top-k)
     groups = {}
     for i, t in enumerate(tasks):
-        if t.op == mk.MK_OP_ATTN:
-            groups.setdefault(("a", t.layer, t.b, t.aux), t.signal)
-        elif t.op == mk.MK_OP_ROUTER:
+        if t.op == mk.MK_OP_ROUTER:
             groups.setdefault(("r", t.layer), t.signal)
         elif t.signal != mk.MK_NO_EVENT:
             signalled[t.signal] += 1
