@@ -313,6 +313,21 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     }
     g.n_events = (int)thr.size();
 
+    // ---- GEMV fast-path variant per task (the device dispatches on it without any
+    //      geometry arithmetic)
+    for (Task& t : T) {
+        int K = 0, nblk = 1;
+        switch (t.op) {
+            case MK_OP_QKV: case MK_OP_LMHEAD: case MK_OP_ROUTER: K = H; break;
+            case MK_OP_GATEUP: case MK_OP_EXP_GATEUP: K = H; nblk = 2; break;
+            case MK_OP_OPROJ: K = nq * hd; break;
+            case MK_OP_DOWN: K = d.ffn; break;
+            case MK_OP_EXP_DOWN: K = d.expert_ffn; break;
+            default: break;
+        }
+        t.flags = K ? fast_path_for(K, (int)(t.r1 - t.r0), nblk) : 0;
+    }
+
     // ---- bytes streamed per B=1 step
     int64_t wb = 2LL * H;                               // one embedding row
     for (int l = 0; l < L; ++l) {

@@ -142,18 +142,24 @@ struct StageInfo {
 };
 
 constexpr int kAttnScratch = kConsumerWarps * kMaxHeadsPerGroup * (128 + 2);   // >= n_q * head_dim floats too
+// Rotating buffers of per-warp row sums.  A consumer warp runs at most one ring's
+// worth of stages (< 2 tasks) ahead of the slowest, so 4 buffers never collide.
+constexpr int kRedBufs = 4;
 
 struct __align__(128) Smem {
     uint8_t ring[kStages][kStageBytes];
-    float red[2][kMaxTaskRows][kConsumerWarps];
-    float attn[kAttnScratch];                 // per-warp (m, l, o) partials
+    float red[kRedBufs][kMaxTaskRows][kConsumerWarps];   // per-warp row sums, rotating per task
+    union {
+        float attn[kAttnScratch];             // per-warp (m, l, o) partials; O-proj merge scratch
+        float rlog[1024];                     // router logits of one sequence
+    };
     float qs[kMaxHeadsPerGroup * 128];        // rotated, pre-scaled q of one kv group
     float kn[128], vn[128];                   // the new token's k, v (bf16-rounded)
-    float rlog[1024];                         // router logits of one sequence
     float bcast[kConsumerWarps + 8];
     uint64_t full[kStages], empty[kStages];
     uint64_t sig_full[kSigSlots], sig_empty[kSigSlots];
     uint64_t csync;                          // all-consumer-warp sync (arrival count 8)
+    uint32_t arrive[kRedBufs];               // per-task warp arrivals (monotone, 8 per use)
     StageInfo info[kStages];
     uint32_t sig_evt[kSigSlots];
     int sig_task[kSigSlots];
@@ -298,8 +304,9 @@ struct Waiter {
 };
 
 // true when the deadline has passed or another CTA has recorded an error
+// (polled every 256 spins: each poll is an L2 round trip)
 __device__ __forceinline__ bool wait_should_stop(const Params& p, Waiter& w) {
-    if (++w.spins & 63) return false;
+    if (++w.spins & 255) return false;
     if (ld_relaxed_int(p.err) != 0) return true;
     if (w.t0 == 0) w.t0 = globaltimer();
     else if ((long long)(globaltimer() - w.t0) > p.timeout_ns) return true;
@@ -354,6 +361,20 @@ __device__ __forceinline__ void csync(const Params& p, Smem& sm, uint32_t& phase
     phase ^= 1;
 }
 
+// Every consumer warp calls this once per task after depositing its share;
+// returns true in the warp that arrives last (acquire: it sees every other
+// warp's shared-memory writes), which then finishes the task alone.
+__device__ __forceinline__ bool last_warp_arrival(uint32_t* cnt) {
+    __syncwarp();
+    uint32_t old = 0;
+    if ((threadIdx.x & 31) == 0)
+        asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                     : "=r"(old) : "r"(smem_u32(cnt)) : "memory");
+    old = __shfl_sync(0xFFFFFFFFu, old, 0);
+    __syncwarp();
+    return (old % kConsumerWarps) == kConsumerWarps - 1;
+}
+
 // Wait on a phase that another thread of this CTA has already seen complete
 // (so it returns at once); bounded anyway: on failure it records a fault and
 // raises the CTA's abort flag, which every consumer reads after its next barrier.
@@ -387,29 +408,36 @@ __device__ bool event_wait(const Params& p, uint32_t e, uint32_t target, int tas
 
 __device__ void producer_loop(const Params& p, Smem& sm) {
     const uint64_t pol = l2_evict_first_policy();
+    // Ring position in registers: fill number n goes to stage n % kStages on lap
+    // n / kStages; a slot of lap k > 0 is free once the consumers released lap k-1.
     int stage = 0;
-    uint32_t issued[kStages];           // fills issued per stage
-    for (int s = 0; s < kStages; ++s) issued[s] = 0;
+    uint32_t lap = 0;
     bool ok = true;
 
     auto acquire_slot = [&]() -> bool {
-        // first lap: slots start empty
-        if (issued[stage] == 0) return true;
-        return mbar_wait_bounded(p, &sm.empty[stage], (issued[stage] - 1) & 1, 1);
+        if (lap == 0) return true;                       // first lap: slots start empty
+        return mbar_wait_bounded(p, &sm.empty[stage], (lap - 1) & 1, 1);
     };
     auto advance = [&]() {
-        issued[stage] += 1;
-        stage = (stage + 1 == kStages) ? 0 : stage + 1;
+        if (++stage == kStages) { stage = 0; ++lap; }
     };
 
     uint32_t last_router_evt = MK_NO_EVENT;
+    // The next task is claimed while the current one's copies are issued, so the
+    // atomic's round trip overlaps useful work.  Still exactly one failing claim
+    // per CTA, which keeps the queue head at (n_tasks + grid) per step.
+    unsigned long long q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
+    uint32_t n_claimed = 0;
     while (ok) {
-        if (ld_relaxed_int(p.err) != 0) { ok = false; break; }
+        // abort checks: the CTA's own flag every task, the grid's status word (an L2
+        // round trip) every 32 tasks; waits below poll it too
+        if (sm.flag[3] != 0 || ((++n_claimed & 31) == 0 && ld_relaxed_int(p.err) != 0)) { ok = false; break; }
         const long long c_dq = p.stats ? clock64() : 0;
-        unsigned long long q = atomicAdd(p.queue, 1ull) - p.queue_base;
+        const unsigned long long q = q_next;
         if (q >= p.n_tasks) break;
         const int ti = (int)q;
         const Task t = p.tasks[ti];
+        q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
         if (p.stats) { const uint32_t w0 = t.wait0; stat_add(p, 4, (unsigned long long)(clock64() - c_dq) + (w0 & 0)); }
         if (t.op == MK_OP_ATTN) {
             const int b = t.b;
@@ -440,7 +468,9 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
                 if (!acquire_slot()) { ok = false; break; }
                 int first = lp0 + c * pps;
                 int n = min(pps, lp0 + npages - first);
-                sm.info[stage] = StageInfo{ti, c, nch, first, t};
+                sm.info[stage].task = ti; sm.info[stage].chunk = c; sm.info[stage].nchunks = nch;
+                sm.info[stage].aux = first;
+                if (c == 0) sm.info[stage].rec = t;
                 // validate page indices before issuing any copy
                 const int* prow = p.page_table + (size_t)b * p.max_pages;
                 bool bad = false;
@@ -490,7 +520,8 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         int c = 0;
         auto issue = [&](const uint8_t* src, uint32_t bytes) -> bool {
             if (!acquire_slot()) return false;
-            sm.info[stage] = StageInfo{ti, c, nch, 0, t};
+            sm.info[stage].task = ti; sm.info[stage].chunk = c; sm.info[stage].nchunks = nch;
+            if (c == 0) sm.info[stage].rec = t;
             mbar_arrive_expect_tx(&sm.full[stage], bytes);
             bulk_g2s(sm.ring[stage], src, bytes, &sm.full[stage], pol);
             advance();
@@ -523,10 +554,12 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         advance();
     }
     // drain: every issued fill must have landed before the CTA's shared memory goes away
+    // (stage s has had lap + (s < stage) fills; the last one has parity fills - 1)
     for (int s = 0; s < kStages; ++s) {
-        if (issued[s] == 0) continue;
+        const uint32_t fills = lap + (s < stage ? 1u : 0u);
+        if (fills == 0) continue;
         Waiter w{0, 0};
-        while (!mbar_try_wait(&sm.full[s], (issued[s] - 1) & 1)) {
+        while (!mbar_try_wait(&sm.full[s], (fills - 1) & 1)) {
             if (++w.spins > (1 << 26)) break;   // copies of valid memory always land; hard cap only
         }
     }
@@ -774,7 +807,7 @@ __device__ __forceinline__ void load8(const InSrc& s, int col, float2 (&x)[4]) {
     x[1] = make_float2(a.z, a.w);
     x[2] = make_float2(c.x, c.y);
     x[3] = make_float2(c.z, c.w);
-    if constexpr (!PARTS) return;
+    if constexpr (PARTS) {
     for (int k = 0; k < s.nparts; ++k) {
         const float w = __ldcg(s.pw + k);
         const float4 pa = __ldcg(reinterpret_cast<const float4*>(s.parts + (size_t)k * s.pstride + col));
@@ -783,6 +816,7 @@ __device__ __forceinline__ void load8(const InSrc& s, int col, float2 (&x)[4]) {
         x[1] = make_float2(fmaf(w, pa.z, x[1].x), fmaf(w, pa.w, x[1].y));
         x[2] = make_float2(fmaf(w, pc.x, x[2].x), fmaf(w, pc.y, x[2].y));
         x[3] = make_float2(fmaf(w, pc.z, x[3].x), fmaf(w, pc.w, x[3].y));
+    }
     }
 }
 
@@ -1111,30 +1145,18 @@ __device__ bool gemv_fast_segs(const Params& p, Smem& sm, int ti, const float2 (
     return true;
 }
 
-// Returns 1 when a fast path handled the task, 0 when the generic path must, -1 on abort.
-__device__ __forceinline__ int gemv_fast_dispatch(const Params& p, Smem& sm, int ti, const GemvGeom& g,
-                                                  const ThreadMap& m,
-                                                  const float2 (&xr)[kMaxVecPerThread][4], int buf,
-                                                  int& stage, uint32_t& lap) {
-    if (m.nvec % kConsumerThreads != 0) return 0;
-    const int vpt = m.nvec / kConsumerThreads;
-    const int rows = g.rows * g.nblk;
-    const int64_t RB = (int64_t)g.K * 2;
-    bool ok;
-    if (RB <= kStageBytes) {
-        const int rps = (int)(kStageBytes / RB);
-        if (g.rows % rps != 0) return 0;
-        if (vpt == 2 && rps == 2 && rows == 16) ok = gemv_fast_rows<2, 2, 16>(p, sm, ti, xr, buf, stage, lap);
-        else if (vpt == 2 && rps == 2 && rows == 8) ok = gemv_fast_rows<2, 2, 8>(p, sm, ti, xr, buf, stage, lap);
-        else if (vpt == 1 && rps == 4 && rows == 16) ok = gemv_fast_rows<1, 4, 16>(p, sm, ti, xr, buf, stage, lap);
-        else if (vpt == 1 && rps == 4 && rows == 8) ok = gemv_fast_rows<1, 4, 8>(p, sm, ti, xr, buf, stage, lap);
-        else return 0;
-    } else {
-        if (vpt == 7 && rows == 4) ok = gemv_fast_segs<7, 4, 4>(p, sm, ti, xr, buf, stage, lap, true);
-        else if (vpt == 7 && rows == 2) ok = gemv_fast_segs<7, 4, 2>(p, sm, ti, xr, buf, stage, lap, true);
-        else return 0;
+// Runs the task's fast path (variant chosen by the planner); false on abort.
+__device__ __forceinline__ bool gemv_fast_dispatch(const Params& p, Smem& sm, int ti, int variant,
+                                                   const float2 (&xr)[kMaxVecPerThread][4], int buf,
+                                                   int& stage, uint32_t& lap) {
+    switch (variant) {
+        case kFastV2R2N16: return gemv_fast_rows<2, 2, 16>(p, sm, ti, xr, buf, stage, lap);
+        case kFastV2R2N8: return gemv_fast_rows<2, 2, 8>(p, sm, ti, xr, buf, stage, lap);
+        case kFastV1R4N16: return gemv_fast_rows<1, 4, 16>(p, sm, ti, xr, buf, stage, lap);
+        case kFastV1R4N8: return gemv_fast_rows<1, 4, 8>(p, sm, ti, xr, buf, stage, lap);
+        case kFastV7S4N4: return gemv_fast_segs<7, 4, 4>(p, sm, ti, xr, buf, stage, lap, true);
+        default: return gemv_fast_segs<7, 4, 2>(p, sm, ti, xr, buf, stage, lap, true);
     }
-    return ok ? 1 : -1;
 }
 
 __device__ __forceinline__ bool gemv_task_dispatch(const Params& p, Smem& sm, int ti, const GemvGeom& g,
@@ -1411,10 +1433,9 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
 // ----------------------------------------------------------------------------- consumer: router top-k
 
 // Last router tile of a layer: softmax over the experts, top-k (ties to the
-// lower index), optional renormalisation.  Warp 0 does the work.
+// lower index), optional renormalisation.  One warp (the caller) does the work.
 __device__ void router_finalize(const Params& p, Smem& sm, int l) {
     const int lane = threadIdx.x & 31;
-    if ((threadIdx.x >> 5) != 0) return;
     for (int b = 0; b < p.max_batch; ++b) {
         const float* lg = p.rlogits + ((size_t)l * p.max_batch + b) * p.E;
         float mx = -INFINITY;
@@ -1474,52 +1495,59 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
     const int tid = threadIdx.x, lane = tid & 31;
     int stage = 0;
     uint32_t lap = 0;
-    int sig_slot = 0;
-    uint32_t sig_lap = 0;
-    int buf = 0;
+    uint32_t seq = 0;                                   // tasks finished by this CTA (same in every warp)
     uint32_t cph = 0;                                   // phase of sm.csync
     float2 xr[kMaxVecPerThread][4];
     int x_key_op = -1, x_key_layer = -1, x_key_b = -1, x_key_aux = -1;
     uint32_t ok_evt[4] = {MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT};   // per warp
 
-    // Each warp waits for its own data and dependencies; the warps meet once per
-    // task, after the chunk loop (csync, bounded).  Every failure raises
-    // sm.flag[3], which all consumer threads read after that meeting, so they
-    // leave the loop together.
+    // Hands task `ti` to the signal warp: called by one lane-0 thread (the warp that
+    // finished the task last) after its warp's stores; slots are used in task order.
+    auto hand_off = [&](uint32_t evt, int ti) {
+        const int slot = (int)(seq % kSigSlots);
+        const uint32_t slap = seq / kSigSlots;
+        if (slap > 0 && !mbar_wait_bounded(p, &sm.sig_empty[slot], (slap - 1) & 1, 6)) sm.flag[3] = 1;
+        sm.sig_evt[slot] = evt;
+        sm.sig_task[slot] = ti;
+        mbar_arrive(&sm.sig_full[slot]);
+    };
+
+    // Each warp waits for its own data and dependencies and runs its share of the
+    // task; the last warp to finish a task reduces the shares, stores the output
+    // and hands the completion to the signal warp.  Warps meet only inside
+    // prologues and attention tasks (bounded mbarrier syncs).  A failure raises
+    // sm.flag[3]; every warp checks it before its next task.
     while (true) {
+        if (sm.flag[3]) break;
         bool ok = mbar_wait_bounded(p, &sm.full[stage], lap & 1, 4);
-        int ti = ok ? sm.info[stage].task : -2;
+        const int ti = ok ? sm.info[stage].task : -2;
         if (ti == -1) {                                  // end of work (same stage for every warp)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
             break;
         }
-        Task t;
-        if (ok) t = sm.info[stage].rec;
-        if (p.trace && tid == 0 && ok) p.trace[(size_t)ti * 4 + 0] = globaltimer();
-        if (ok) {
-            const uint32_t e = t.wait0;
-            if (e != MK_NO_EVENT && e != ok_evt[0] && e != ok_evt[1] && e != ok_evt[2] && e != ok_evt[3]) {
-                int r = 1;
-                if (lane == 0) {
-                    r = event_wait(p, e, p.thr[e] * p.epoch + p.wait_offset, ti) ? 1 : 0;
-                    if (r) __threadfence();
-                }
-                r = __shfl_sync(0xFFFFFFFFu, r, 0);
-                if (r) {
-                    ok_evt[3] = ok_evt[2]; ok_evt[2] = ok_evt[1]; ok_evt[1] = ok_evt[0]; ok_evt[0] = e;
-                } else {
-                    ok = false;
-                }
+        if (!ok) { sm.flag[3] = 1; break; }
+        const Task t = sm.info[stage].rec;
+        if (p.trace && tid == 0) p.trace[(size_t)ti * 4 + 0] = globaltimer();
+        const uint32_t e = t.wait0;
+        if (e != MK_NO_EVENT && e != ok_evt[0] && e != ok_evt[1] && e != ok_evt[2] && e != ok_evt[3]) {
+            int r = 1;
+            if (lane == 0) {
+                r = event_wait(p, e, p.thr[e] * p.epoch + p.wait_offset, ti) ? 1 : 0;
+                if (r) __threadfence();
             }
+            r = __shfl_sync(0xFFFFFFFFu, r, 0);
+            if (!r) { sm.flag[3] = 1; break; }
+            ok_evt[3] = ok_evt[2]; ok_evt[2] = ok_evt[1]; ok_evt[1] = ok_evt[0]; ok_evt[0] = e;
         }
-        if (!ok) sm.flag[3] = 1;
-        if (p.trace && tid == 0 && ok) {
+        if (p.trace && tid == 0) {
             p.trace[(size_t)ti * 4 + 1] = globaltimer();
             p.trace[(size_t)ti * 4 + 3] = (uint64_t)blockIdx.x;
         }
+        uint32_t* arrive = &sm.arrive[seq % kRedBufs];
+        const int buf = (int)(seq % kRedBufs);
 
-        if (ok && t.op == MK_OP_ATTN) {
+        if (t.op == MK_OP_ATTN) {
             bool abort_all = false;
             attention_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
             if (abort_all) break;
@@ -1528,64 +1556,64 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
 #pragma unroll
             for (int j = 0; j < kMaxVecPerThread; ++j)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) xr[j][e] = make_float2(0.0f, 0.0f);
-            // hand the completion to the signal warp once this warp's stores are issued
-            if (tid == 0) {
-                if (sig_lap > 0 && !mbar_wait_bounded(p, &sm.sig_empty[sig_slot], (sig_lap - 1) & 1, 6))
-                    sm.flag[3] = 1;
-                sm.sig_evt[sig_slot] = t.sig;
-                sm.sig_task[sig_slot] = ti;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.sig_full[sig_slot]);
-            if (++sig_slot == kSigSlots) { sig_slot = 0; ++sig_lap; }
+                for (int q = 0; q < 4; ++q) xr[j][q] = make_float2(0.0f, 0.0f);
+            if (last_warp_arrival(arrive) && lane == 0) hand_off(t.sig, ti);
+            ++seq;
             continue;
         }
 
         // ---- GEMV task
+        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
+        const bool fast = (t.flags != kFastNone) && !skip;
         GemvGeom g;
+        gemv_geom(p, t, g, false);
+        // fast-path tiles split every row over all 8 warps (wpg = 8, one group)
         ThreadMap m;
-        bool skip = false;
-        int rows_total = 0;
-        float resid = 0.0f;
-        if (ok) {
-            skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
-            gemv_geom(p, t, g, false);
-            m = thread_map(g.K);
-            rows_total = g.rows * g.nblk;
-            if (!skip) {
-                if (t.op == MK_OP_QKV && t.layer == 0 && tid == 0) {
-                    const int tok = p.tokens[0];
-                    if (tok < 0 || tok >= p.V) set_error(p, kErrInvalid, ti, -5, tok, 0);
-                }
-                if (!(x_key_op == t.op && x_key_layer == t.layer && x_key_b == t.b &&
-                      (x_key_aux == t.aux || t.op != MK_OP_EXP_DOWN))) {
-                    gemv_prologue(p, sm, cph, t, m, g.K, xr);
-                    x_key_op = t.op; x_key_layer = t.layer; x_key_b = t.b; x_key_aux = t.aux;
-                }
-                // residual rows for the epilogue, fetched now so the load overlaps the streaming
-                if (tid < rows_total) {
-                    if (t.op == MK_OP_OPROJ) resid = x_in(p, t.layer, 0, (int)t.r0 + tid);
-                    else if (t.op == MK_OP_DOWN) resid = x_mid_at(p, t.layer, 0, (int)t.r0 + tid);
-                }
+        if (fast) { m.nvec = g.K >> 3; m.wpg = kConsumerWarps; m.G = 1; m.grp = 0; m.lig = tid;
+                    m.gstride = kConsumerThreads; m.vpt = m.nvec / kConsumerThreads; m.active = true; }
+        else m = thread_map(g.K);
+        const int rows_total = g.rows * g.nblk;
+        float resid0 = 0.0f, resid1 = 0.0f;
+        if (!skip) {
+            if (t.op == MK_OP_QKV && t.layer == 0 && tid == 0) {
+                const int tok = p.tokens[0];
+                if (tok < 0 || tok >= p.V) set_error(p, kErrInvalid, ti, -5, tok, 0);
             }
-            const long long c_ch = (p.stats && tid == 0) ? clock64() : 0;
-            const int handled = skip ? 0 : gemv_fast_dispatch(p, sm, ti, g, m, xr, buf, stage, lap);
-            if (handled == 0) (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
-            if (p.stats && tid == 0) stat_add(p, 6, (unsigned long long)(clock64() - c_ch));
+            if (!(x_key_op == t.op && x_key_layer == t.layer && x_key_b == t.b &&
+                  (x_key_aux == t.aux || t.op != MK_OP_EXP_DOWN))) {
+                gemv_prologue(p, sm, cph, t, m, g.K, xr);
+                x_key_op = t.op; x_key_layer = t.layer; x_key_b = t.b; x_key_aux = t.aux;
+            }
+            // residual rows for the epilogue (whichever warp runs it), fetched now so the
+            // loads overlap the streaming
+            if (t.op == MK_OP_OPROJ || t.op == MK_OP_DOWN) {
+                const int r0 = (int)t.r0;
+                if (lane < rows_total)
+                    resid0 = (t.op == MK_OP_OPROJ) ? x_in(p, t.layer, 0, r0 + lane) : x_mid_at(p, t.layer, 0, r0 + lane);
+                if (lane + 32 < rows_total)
+                    resid1 = (t.op == MK_OP_OPROJ) ? x_in(p, t.layer, 0, r0 + lane + 32)
+                                                   : x_mid_at(p, t.layer, 0, r0 + lane + 32);
+            }
         }
-        const long long c_ep = (p.stats && tid == 0) ? clock64() : 0;
-        csync(p, sm, cph);                               // all partial sums are in red[buf]
+        const long long c_ch = (p.stats && tid == 0) ? clock64() : 0;
+        if (fast) (void)gemv_fast_dispatch(p, sm, ti, t.flags, xr, buf, stage, lap);
+        else (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
+        if (p.stats && tid == 0) stat_add(p, 6, (unsigned long long)(clock64() - c_ch));
         if (sm.flag[3]) break;
 
-        // ---- epilogue: reduce the warps' partials in fixed order, apply the op's output rule
+        if (!last_warp_arrival(arrive)) { ++seq; continue; }
+
+        // ---- epilogue (last warp): reduce the warps' partials in fixed order, store
+        const long long c_ep = (p.stats && lane == 0) ? clock64() : 0;
+        uint32_t evt = t.sig;
         if (!skip) {
             const int l = t.layer, b = t.b;
             const int nout = (g.nblk == 2) ? g.rows : rows_total;
-            for (int r = tid; r < nout; r += kConsumerThreads) {
+            for (int r = lane; r < nout; r += 32) {
                 float y = 0.0f;
                 for (int w = 0; w < m.wpg; ++w) y += sm.red[buf][r][w];
                 const int row = (int)t.r0 + r;
+                const float resid = (r < 32) ? resid0 : resid1;
                 switch (t.op) {
                     case MK_OP_QKV:
                         p.qkv[((size_t)l * p.max_batch) * ((p.nq + 2 * p.nkv) * p.hd) + row] = y;
@@ -1622,54 +1650,36 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
                 }
             }
         }
-        buf ^= 1;
-
         if (t.op == MK_OP_ROUTER) {
-            // arrival; the last router tile of the layer selects the experts and signals
-            csync(p, sm, cph);
-            if (tid == 0) {
+            // arrival of this router tile; the layer's last tile selects the experts and
+            // only it signals the router event
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) {
                 __threadfence();
                 const uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
                 __threadfence();
-                sm.flag[0] = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
-                atomicAdd(p.done, 1u);
+                last = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
             }
-            csync(p, sm, cph);
-            const int last = sm.flag[0];
-            csync(p, sm, cph);                           // flag[0] read by everyone
-            if (last) {
-                router_finalize(p, sm, t.layer);
-                csync(p, sm, cph);
-                if (tid == 0) {
-                    __threadfence();
-                    if (t.sig != MK_NO_EVENT) red_release_add(&p.events[t.sig], 1u);
-                }
-            }
-            if (tid == 0 && p.trace) p.trace[(size_t)ti * 4 + 2] = globaltimer();
-            continue;
-        }
-
-        // ---- hand the completion to the signal warp (its fence does not stall the consumers)
-        if (tid == 0) {
-            if (sig_lap > 0 && !mbar_wait_bounded(p, &sm.sig_empty[sig_slot], (sig_lap - 1) & 1, 6))
-                sm.flag[3] = 1;
-            sm.sig_evt[sig_slot] = t.sig;
-            sm.sig_task[sig_slot] = ti;
+            last = __shfl_sync(0xFFFFFFFFu, last, 0);
+            if (last) router_finalize(p, sm, t.layer);
+            else evt = MK_NO_EVENT;
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sig_full[sig_slot]);
-        if (++sig_slot == kSigSlots) { sig_slot = 0; ++sig_lap; }
-        if (p.stats && tid == 0) stat_add(p, 7, (unsigned long long)(clock64() - c_ep));
+        if (lane == 0) hand_off(evt, ti);
+        if (p.stats && lane == 0) stat_add(p, 7, (unsigned long long)(clock64() - c_ep));
+        ++seq;
     }
-    // end of work for the signal warp
+    // end of work for the signal warp: one marker after every warp has left the loop
     csync(p, sm, cph);
     if (tid == 0) {
-        if (sig_lap > 0) (void)mbar_wait_bounded(p, &sm.sig_empty[sig_slot], (sig_lap - 1) & 1, 7);
-        sm.sig_evt[sig_slot] = 0xFFFFFFFEu;
-        sm.sig_task[sig_slot] = -1;
+        const int slot = (int)(seq % kSigSlots);
+        const uint32_t slap = seq / kSigSlots;
+        if (slap > 0) (void)mbar_wait_bounded(p, &sm.sig_empty[slot], (slap - 1) & 1, 7);
+        sm.sig_evt[slot] = 0xFFFFFFFEu;
+        sm.sig_task[slot] = -1;
+        mbar_arrive(&sm.sig_full[slot]);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.sig_full[sig_slot]);
 }
 
 // ----------------------------------------------------------------------------- kernel
@@ -1685,10 +1695,11 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&sm.empty[s], kConsumerWarps);
         }
         for (int s = 0; s < kSigSlots; ++s) {
-            mbar_init(&sm.sig_full[s], kConsumerWarps);
+            mbar_init(&sm.sig_full[s], 1);
             mbar_init(&sm.sig_empty[s], 1);
         }
         mbar_init(&sm.csync, kConsumerWarps);
+        for (int i = 0; i < kRedBufs; ++i) sm.arrive[i] = 0;
         for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
         for (int i = 0; i < 8; ++i) sm.stat[i] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");

@@ -26,10 +26,42 @@ constexpr int kMaxHeadsPerGroup = 8;
 constexpr int kMaxTopK = 16;
 constexpr int kPageSize = 16;
 
+// GEMV fast-path variants (rows whose 16-byte vectors split evenly over the 256
+// consumer threads): vectors per thread, rows per 16 KB stage, rows per task.
+enum FastPath : uint8_t {
+    kFastNone = 0,
+    kFastV2R2N16 = 1,   // K = 4096, 2 rows per stage, 16 rows
+    kFastV2R2N8 = 2,    // K = 4096, 2 rows per stage, 8 rows
+    kFastV1R4N16 = 3,   // K = 2048, 4 rows per stage, 16 rows
+    kFastV1R4N8 = 4,    // K = 2048, 4 rows per stage, 8 rows
+    kFastV7S4N4 = 5,    // K = 14336, rows in 2 segments (4 + 3 vectors per thread), 4 rows
+    kFastV7S4N2 = 6,    // K = 14336, 2 rows
+};
+
+// The variant for a GEMV tile of `rows` rows per weight block, `nblk` blocks, K columns.
+inline uint8_t fast_path_for(int K, int rows, int nblk) {
+    const int nvec = K / 8;
+    if (K % 8 != 0 || nvec % kConsumerThreads != 0) return kFastNone;
+    const int vpt = nvec / kConsumerThreads, total = rows * nblk;
+    const long long rb = 2LL * K;
+    if (rb <= kStageBytes) {
+        const int rps = (int)(kStageBytes / rb);
+        if (rows % rps != 0) return kFastNone;
+        if (vpt == 2 && rps == 2 && total == 16) return kFastV2R2N16;
+        if (vpt == 2 && rps == 2 && total == 8) return kFastV2R2N8;
+        if (vpt == 1 && rps == 4 && total == 16) return kFastV1R4N16;
+        if (vpt == 1 && rps == 4 && total == 8) return kFastV1R4N8;
+        return kFastNone;
+    }
+    if (vpt == 7 && total == 4) return kFastV7S4N4;
+    if (vpt == 7 && total == 2) return kFastV7S4N2;
+    return kFastNone;
+}
+
 // Device task record (32 bytes).
 struct Task {
     uint8_t op;
-    uint8_t flags;
+    uint8_t flags;   // GEMV: fast-path variant chosen by the planner (kFast*), 0 = generic
     uint16_t layer;
     uint16_t b;      // batch row (attention / expert tasks)
     uint16_t aux;    // kv head (attention) or expert slot (expert tasks)
