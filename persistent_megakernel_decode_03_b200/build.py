@@ -29,11 +29,31 @@ def stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+MIN_LAUNCH_REGS = 163   # kMinLaunchRegs in csrc/mk_internal.h (setmaxnreg budget)
+
+
 def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    cmd = nvcc_cmd(ptxas_verbose)
+    cmd = nvcc_cmd(True)
     if verbose:
         print(" ".join(cmd))
-    subprocess.run(cmd, check=True)
+    out = subprocess.run(cmd, check=True, capture_output=True, text=True)
+    log = out.stdout + out.stderr
+    if ptxas_verbose:
+        print(log)
+    # The megakernel re-splits its registers between warpgroups at run time
+    # (setmaxnreg); that split is only valid if every instantiation launches with
+    # at least MIN_LAUNCH_REGS registers per thread.
+    import re
+    cur = None
+    for line in log.splitlines():
+        m = re.search(r"Compiling entry function '(\S+)'", line)
+        if m:
+            cur = m.group(1)
+        m = re.search(r"Used (\d+) registers", line)
+        if m and cur and "megakernel" in cur and int(m.group(1)) < MIN_LAUNCH_REGS:
+            os.remove(LIB)
+            raise RuntimeError(f"{cur} launches with {m.group(1)} registers per thread; the "
+                               f"warpgroup register split needs at least {MIN_LAUNCH_REGS}")
     return LIB
 
 

@@ -164,10 +164,7 @@ struct __align__(128) Smem {
     uint32_t sig_evt[kSigSlots];
     int sig_task[kSigSlots];
     int flag[4];
-    unsigned long long stat[8];              // per-CTA counters (tracing only), flushed at exit
 };
-
-constexpr size_t kStatsOffset = offsetof(Smem, stat);
 
 // ----------------------------------------------------------------------------- geometry
 
@@ -317,9 +314,7 @@ __device__ __forceinline__ bool wait_should_stop(const Params& p, Waiter& w) {
 // free ring slot, [1] consumer thread 0 waits for data, [2] dependency waits,
 // [3] kernel cycles, [4] tasks run, [5] signal-slot waits.
 __device__ __forceinline__ void stat_add(const Params& p, int i, unsigned long long v) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    unsigned long long* acc = reinterpret_cast<unsigned long long*>(smem_raw + kStatsOffset);
-    if (p.stats) atomicAdd(&acc[i], v);
+    if (p.stats) atomicAdd(&p.stats[(size_t)blockIdx.x * 8 + i], v);   // reduction, no return value
 }
 
 __device__ __forceinline__ void wait_stat(const Params& p, int where, long long c0) {
@@ -1077,10 +1072,14 @@ template <int VPT, int RPS, int NROWS>
 __device__ bool gemv_fast_rows(const Params& p, Smem& sm, int ti, const float2 (&xr)[kMaxVecPerThread][4],
                                int buf, int& stage, uint32_t& lap) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // The stage loop stays rolled (small code: the SM's instruction cache is shared
+    // with the producer and signal loops).  Each stage's RPS row sums enter at the
+    // end of `acc` while the older ones shift down, so after NROWS / RPS stages
+    // acc[r] holds row r.
     float acc[NROWS];
 #pragma unroll
     for (int r = 0; r < NROWS; ++r) acc[r] = 0.f;
-#pragma unroll
+#pragma unroll 1
     for (int st = 0; st < NROWS / RPS; ++st) {
         if (st > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) { sm.flag[3] = 1; return false; }
         if (sm.info[stage].task != ti) { set_error(p, kErrFault, ti, -4, sm.info[stage].task, 2); sm.flag[3] = 1; return false; }
@@ -1091,11 +1090,13 @@ __device__ bool gemv_fast_rows(const Params& p, Smem& sm, int ti, const float2 (
 #pragma unroll
             for (int j = 0; j < VPT; ++j) q[rr][j] = sv[(rr * VPT + j) * kConsumerThreads];
 #pragma unroll
+        for (int r = 0; r < NROWS - RPS; ++r) acc[r] = acc[r + RPS];
+#pragma unroll
         for (int rr = 0; rr < RPS; ++rr) {
             float2 a = make_float2(0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < VPT; ++j) dot8(q[rr][j], xr[j], a);
-            acc[st * RPS + rr] += a.x + a.y;
+            acc[NROWS - RPS + rr] = a.x + a.y;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[stage]);
@@ -1107,7 +1108,7 @@ __device__ bool gemv_fast_rows(const Params& p, Smem& sm, int ti, const float2 (
 }
 
 // Rows longer than a stage: each row arrives as segments of SEGJ*256 vectors
-// (the last segment holds the rest); NROWS rows.
+// (the last segment holds the rest); NROWS rows, one rolled iteration per row.
 template <int VPT, int SEGJ, int NROWS>
 __device__ bool gemv_fast_segs(const Params& p, Smem& sm, int ti, const float2 (&xr)[kMaxVecPerThread][4],
                                int buf, int& stage, uint32_t& lap, bool first_seen) {
@@ -1116,8 +1117,9 @@ __device__ bool gemv_fast_segs(const Params& p, Smem& sm, int ti, const float2 (
     float acc[NROWS];
 #pragma unroll
     for (int r = 0; r < NROWS; ++r) acc[r] = 0.f;
-#pragma unroll
+#pragma unroll 1
     for (int r = 0; r < NROWS; ++r) {
+        float2 a = make_float2(0.f, 0.f);
 #pragma unroll
         for (int sg = 0; sg < NSEG; ++sg) {
             if ((r > 0 || sg > 0 || !first_seen) && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) {
@@ -1130,15 +1132,16 @@ __device__ bool gemv_fast_segs(const Params& p, Smem& sm, int ti, const float2 (
 #pragma unroll
             for (int j = 0; j < SEGJ; ++j)
                 if (sg * SEGJ + j < VPT) q[j] = sv[j * kConsumerThreads];
-            float2 a = make_float2(0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < SEGJ; ++j)
                 if (sg * SEGJ + j < VPT) dot8(q[j], xr[sg * SEGJ + j], a);
-            acc[r] += a.x + a.y;
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
             if (++stage == kStages) { stage = 0; ++lap; }
         }
+#pragma unroll
+        for (int i = 0; i < NROWS - 1; ++i) acc[i] = acc[i + 1];
+        acc[NROWS - 1] = a.x + a.y;
     }
     const float tot = warp_reduce_rows<NROWS>(acc);
     if ((lane & (32 / NROWS - 1)) == 0) sm.red[buf][lane / (32 / NROWS)][warp] = tot;
@@ -1701,24 +1704,26 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         mbar_init(&sm.csync, kConsumerWarps);
         for (int i = 0; i < kRedBufs; ++i) sm.arrive[i] = 0;
         for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
-        for (int i = 0; i < 8; ++i) sm.stat[i] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    const long long k0 = clock64();
+    // Hand registers from the support warpgroup to the two consumer warpgroups.
+    // The two branches never meet again (each returns), so the register limit of
+    // one never constrains the code of the other.
     if (warp < kConsumerWarps) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
+        const long long k0 = clock64();
         consumer_loop<HPG, DPL>(p, sm);
         if (threadIdx.x == 0) stat_add(p, 3, (unsigned long long)(clock64() - k0));
-    } else if (warp == kProducerWarp) {
+        return;
+    }
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSupportRegs));
+    if (warp == kProducerWarp) {
         if (lane == 0) producer_loop(p, sm);
     } else if (warp == kSignalWarp) {
         if (lane == 0) signal_loop(p, sm);
-    } else {
+    } else if (warp == kPrefetchWarp) {
         if (lane == 0) prefetch_loop(p);
-    }
-    if (p.stats) {
-        __syncthreads();
-        if (threadIdx.x < 8) p.stats[(size_t)blockIdx.x * 8 + threadIdx.x] += sm.stat[threadIdx.x];
     }
 }
 
