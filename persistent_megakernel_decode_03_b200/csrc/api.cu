@@ -320,6 +320,7 @@ static mk_status build_graph(mk_model* model, int max_batch, int max_ctx, int so
     g->model = model;
     g->device = dev;
     if (solo_op) mk::make_solo(g->plan, solo_op);
+    mk::attach_weights(g->plan, model->w.data());
     const GraphPlan& P = g->plan;
     // RoPE table: cos/sin of pos * theta^(-2i/d), computed in double, stored fp32
     const int half = d.head_dim / 2;

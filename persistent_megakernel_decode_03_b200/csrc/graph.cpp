@@ -341,6 +341,49 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     return true;
 }
 
+void attach_weights(GraphPlan& g, const void* const* w) {
+    const mk_model_desc& d = g.desc;
+    const bool moe = d.n_experts > 0;
+    const int S = moe ? 10 : 9, L = d.n_layers, H = d.hidden, hd = d.head_dim;
+    const int qr = d.n_q_heads * hd, kr = d.n_kv_heads * hd;
+    auto ptr = [&](int layer, int slot) { return reinterpret_cast<uint64_t>(w[1 + layer * S + slot]); };
+    for (Task& t : g.tasks) {
+        int K = 0, nblk = 1;
+        uint64_t a = 0, b = 0;
+        const int l = t.layer;
+        switch (t.op) {
+            case MK_OP_QKV: {
+                K = H;
+                const int r = (int)t.r0;
+                if (r < qr) a = ptr(l, 1) + 2ull * r * H;
+                else if (r < qr + kr) a = ptr(l, 2) + 2ull * (r - qr) * H;
+                else a = ptr(l, 3) + 2ull * (r - qr - kr) * H;
+                break;
+            }
+            case MK_OP_OPROJ: K = qr; a = ptr(l, 4) + 2ull * t.r0 * K; break;
+            case MK_OP_GATEUP:
+                K = H; nblk = 2; a = ptr(l, 6) + 2ull * t.r0 * H; b = ptr(l, 7) + 2ull * t.r0 * H; break;
+            case MK_OP_DOWN: K = d.ffn; a = ptr(l, 8) + 2ull * t.r0 * K; break;
+            case MK_OP_ROUTER: K = H; a = ptr(l, 6) + 2ull * t.r0 * H; break;
+            case MK_OP_LMHEAD:
+                K = H; a = reinterpret_cast<uint64_t>(w[2 + L * S]) + 2ull * t.r0 * H; break;
+            default: continue;   // attention pages and routed experts are resolved on the device
+        }
+        const uint32_t rows = t.r1 - t.r0, rb = 2u * (uint32_t)K;
+        t.src[0] = a;
+        t.src[1] = b;
+        t.row_bytes = rb;
+        t.nblk = (uint16_t)nblk;
+        if (rb <= (uint32_t)kStageBytes) {
+            t.chunk_rows = (uint16_t)(kStageBytes / rb);
+            t.nchunks = (uint32_t)nblk * ((rows + t.chunk_rows - 1) / t.chunk_rows);
+        } else {
+            t.chunk_rows = 0;
+            t.nchunks = (uint32_t)nblk * rows * ((rb + kStageBytes - 1) / kStageBytes);
+        }
+    }
+}
+
 void make_solo(GraphPlan& g, int op) {
     std::vector<Task> kept;
     for (const Task& t : g.tasks)

@@ -32,5 +32,8 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
 // Keeps only the tasks of operator `op` (all layers), without dependencies:
 // a list for timing and profiling one tile type alone.
 void make_solo(GraphPlan& g, int op);
+// Fills each dense GEMV task's streaming plan (weight addresses, chunking) from
+// the model's weight pointers (order of the C ABI's weight list).
+void attach_weights(GraphPlan& g, const void* const* w);
 
 }  // namespace mk

@@ -401,39 +401,30 @@ __device__ bool event_wait(const Params& p, uint32_t e, uint32_t target, int tas
 
 // ----------------------------------------------------------------------------- producer
 
-__device__ void producer_loop(const Params& p, Smem& sm) {
-    const uint64_t pol = l2_evict_first_policy();
-    // Ring position in registers: fill number n goes to stage n % kStages on lap
-    // n / kStages; a slot of lap k > 0 is free once the consumers released lap k-1.
-    int stage = 0;
-    uint32_t lap = 0;
+// Producer ring position: fill number n goes to stage n % kStages on lap
+// n / kStages; a slot of lap k > 0 is free once the consumers released lap k-1.
+struct PRing {
+    int stage;
+    uint32_t lap;
+};
+__device__ __forceinline__ bool pr_acquire(const Params& p, Smem& sm, const PRing& r) {
+    if (r.lap == 0) return true;                       // first lap: slots start empty
+    return mbar_wait_bounded(p, &sm.empty[r.stage], (r.lap - 1) & 1, 1);
+}
+__device__ __forceinline__ void pr_advance(PRing& r) {
+    if (++r.stage == kStages) { r.stage = 0; ++r.lap; }
+}
+
+// Tasks whose streamed data is only known on the device: attention (KV pages of
+// this step's positions) and routed experts (weights of the expert the router
+// picked).  Out of line: it keeps the producer's hot loop small.
+__device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Task& t, int ti, PRing& ring,
+                                             uint32_t& last_router_evt, uint64_t pol) {
+    int& stage = ring.stage;
     bool ok = true;
-
-    auto acquire_slot = [&]() -> bool {
-        if (lap == 0) return true;                       // first lap: slots start empty
-        return mbar_wait_bounded(p, &sm.empty[stage], (lap - 1) & 1, 1);
-    };
-    auto advance = [&]() {
-        if (++stage == kStages) { stage = 0; ++lap; }
-    };
-
-    uint32_t last_router_evt = MK_NO_EVENT;
-    // The next task is claimed while the current one's copies are issued, so the
-    // atomic's round trip overlaps useful work.  Still exactly one failing claim
-    // per CTA, which keeps the queue head at (n_tasks + grid) per step.
-    unsigned long long q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
-    uint32_t n_claimed = 0;
-    while (ok) {
-        // abort checks: the CTA's own flag every task, the grid's status word (an L2
-        // round trip) every 32 tasks; waits below poll it too
-        if (sm.flag[3] != 0 || ((++n_claimed & 31) == 0 && ld_relaxed_int(p.err) != 0)) { ok = false; break; }
-        const long long c_dq = p.stats ? clock64() : 0;
-        const unsigned long long q = q_next;
-        if (q >= p.n_tasks) break;
-        const int ti = (int)q;
-        const Task t = p.tasks[ti];
-        q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
-        if (p.stats) { const uint32_t w0 = t.wait0; stat_add(p, 4, (unsigned long long)(clock64() - c_dq) + (w0 & 0)); }
+    auto acquire_slot = [&]() -> bool { return pr_acquire(p, sm, ring); };
+    auto advance = [&]() { pr_advance(ring); };
+    do {
         if (t.op == MK_OP_ATTN) {
             const int b = t.b;
             int npages = 0, lp0 = 0;
@@ -489,7 +480,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
                 }
                 advance();
             }
-            continue;
+            break;
         }
         // GEMV-type task
         bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
@@ -540,8 +531,76 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
                     }
             }
         }
-        if (!ok) break;
+    } while (false);
+    return ok;
+}
+
+__device__ void producer_loop(const Params& p, Smem& sm) {
+    const uint64_t pol = l2_evict_first_policy();
+    PRing ring{0, 0};
+    bool ok = true;
+    uint32_t last_router_evt = MK_NO_EVENT;
+    // The next task is claimed while the current one's copies are issued, so the
+    // atomic's round trip overlaps useful work.  Still exactly one failing claim
+    // per CTA, which keeps the queue head at (n_tasks + grid) per step.
+    unsigned long long q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
+    uint32_t n_claimed = 0;
+    while (ok) {
+        // abort checks: the CTA's own flag every task, the grid's status word (an L2
+        // round trip) every 32 tasks; waits below poll it too
+        if (sm.flag[3] != 0 || ((++n_claimed & 31) == 0 && ld_relaxed_int(p.err) != 0)) { ok = false; break; }
+        const unsigned long long q = q_next;
+        if (q >= p.n_tasks) break;
+        const int ti = (int)q;
+        const Task t = p.tasks[ti];
+        q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
+        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
+        if (skip) {                                      // nothing to stream: a marker stage
+            if (!pr_acquire(p, sm, ring)) { ok = false; break; }
+            sm.info[ring.stage] = StageInfo{ti, 0, 0, 0, t};
+            mbar_arrive(&sm.full[ring.stage]);
+            pr_advance(ring);
+            continue;
+        }
+        if (t.nchunks == 0 || t.op == MK_OP_ATTN) {
+            ok = produce_special(p, sm, t, ti, ring, last_router_evt, pol);
+            continue;
+        }
+        // dense GEMV tile: the plan the host computed (the consumer walks the same
+        // chunk sequence): per block, chunk_rows whole rows per stage, or each row in
+        // stage-sized segments
+        const uint32_t rb = t.row_bytes, rows = t.r1 - t.r0, nch = t.nchunks;
+        uint32_t c = 0;
+        for (int bi = 0; bi < t.nblk && ok; ++bi) {
+            const uint8_t* base = reinterpret_cast<const uint8_t*>(t.src[bi]);
+            const uint32_t step = t.chunk_rows ? t.chunk_rows * rb : (uint32_t)kStageBytes;
+            const uint32_t total = rows * rb;
+            for (uint32_t off = 0; off < total && ok; ) {
+                uint32_t bytes;
+                if (t.chunk_rows) {
+                    bytes = (total - off < step) ? total - off : step;
+                } else {
+                    const uint32_t in_row = off % rb;          // segments restart at each row
+                    bytes = (rb - in_row < step) ? rb - in_row : step;
+                }
+                if (!pr_acquire(p, sm, ring)) { ok = false; break; }
+                StageInfo& inf = sm.info[ring.stage];
+                inf.task = ti;
+                inf.chunk = (int)c;
+                inf.nchunks = (int)nch;
+                if (c == 0) inf.rec = t;
+                mbar_arrive_expect_tx(&sm.full[ring.stage], bytes);
+                bulk_g2s(sm.ring[ring.stage], base + off, bytes, &sm.full[ring.stage], pol);
+                pr_advance(ring);
+                ++c;
+                off += bytes;
+            }
+        }
     }
+    int& stage = ring.stage;
+    uint32_t& lap = ring.lap;
+    auto acquire_slot = [&]() -> bool { return pr_acquire(p, sm, ring); };
+    auto advance = [&]() { pr_advance(ring); };
     // end-of-work marker (best effort when aborting)
     if (acquire_slot()) {
         sm.info[stage].task = -1;

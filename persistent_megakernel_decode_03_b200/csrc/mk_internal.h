@@ -75,9 +75,19 @@ struct Task {
     uint32_t r0, r1; // output rows; attention: split index, split count
     uint32_t wait0, wait1;
     uint32_t sig;
-    uint32_t pad;
+    uint32_t pad;        // expert tasks: router event to wait on before reading the expert id
+    // Streaming plan of a dense GEMV tile, filled when the graph is built for a
+    // loaded model (zero otherwise): the weight rows of each block start at src[i];
+    // chunks are chunk_rows whole rows, or (chunk_rows == 0) rows in stage-sized
+    // segments.
+    uint64_t src[2];
+    uint32_t row_bytes;
+    uint16_t chunk_rows;
+    uint16_t nblk;
+    uint32_t nchunks;
+    uint32_t pad2;
 };
-static_assert(sizeof(Task) == 32, "task record is 32 bytes");
+static_assert(sizeof(Task) == 64, "task record is 64 bytes");
 
 // Per-layer weight pointers (bf16 bits).
 struct LayerW {
