@@ -758,17 +758,21 @@ __device__ __forceinline__ ThreadMap thread_map(int K) {
 }
 
 // Loads this thread's slice of the (normalised) input into registers.
-// Split partial layout: [L][B][nkv][S][HPG][hd + 2] = (m, l, o[hd]) per head, with
-// m in the log2 domain and o not yet divided by l.
-__device__ __forceinline__ float* attn_part(const Params& p, int l, int b, int g, int s, int h) {
-    const int hpg = hpg_of(p);
-    size_t idx = ((((size_t)l * p.max_batch + b) * p.nkv + g) * p.S + s) * hpg + h;
-    return p.part + idx * (p.hd + 2);
+// Split partials: o[L][B][nkv][S][HPG][hd] (not yet divided by l; 16-byte aligned
+// rows) followed by ml[L][B][nkv][S][HPG][2] = (m in the log2 domain, l).
+__device__ __forceinline__ size_t attn_part_index(const Params& p, int l, int b, int g, int s, int h) {
+    return ((((size_t)l * p.max_batch + b) * p.nkv + g) * p.S + s) * hpg_of(p) + h;
+}
+__device__ __forceinline__ float* attn_part_o(const Params& p, size_t idx) { return p.part + idx * p.hd; }
+__device__ __forceinline__ float* attn_part_ml(const Params& p, size_t idx) {
+    return p.part + (size_t)p.L * p.max_batch * p.nkv * p.S * hpg_of(p) * p.hd + 2 * idx;
 }
 
 // Input of the O-projection: the attention output, merged over the active splits
 // of every (sequence, kv head) in split order.  Eight consecutive columns lie in
-// one q head.
+// one q head.  Up to kMergeFast splits are merged with every load in flight at
+// once; more splits take a second, looped pass.
+constexpr int kMergeFast = 8;
 __device__ __forceinline__ void load8_attn_merge(const Params& p, int l, int b, int col,
                                                  float2 (&x)[4]) {
     const int hd = p.hd, hpg = hpg_of(p);
@@ -777,18 +781,48 @@ __device__ __forceinline__ void load8_attn_merge(const Params& p, int l, int b, 
     int pos = position_of(p, b);
     if (pos < 0 || pos >= p.max_ctx) pos = 0;
     const int sa = attn_active_splits(pos + 1, p.S);
+    const size_t i0 = attn_part_index(p, l, b, g, 0, h);
+    const size_t stride = (size_t)hpg;                  // next split, same head
+    float m[kMergeFast], ls[kMergeFast];
+    float4 oa[kMergeFast], ob[kMergeFast];
+#pragma unroll
+    for (int sp = 0; sp < kMergeFast; ++sp) {
+        if (sp < sa) {
+            const size_t idx = i0 + sp * stride;
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(attn_part_ml(p, idx)));
+            m[sp] = ml.x;
+            ls[sp] = ml.y;
+            oa[sp] = __ldcg(reinterpret_cast<const float4*>(attn_part_o(p, idx) + i));
+            ob[sp] = __ldcg(reinterpret_cast<const float4*>(attn_part_o(p, idx) + i + 4));
+        } else {
+            m[sp] = -INFINITY;
+            ls[sp] = 0.f;
+            oa[sp] = ob[sp] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
     float M = -INFINITY;
-    for (int sp = 0; sp < sa; ++sp) M = fmaxf(M, __ldcg(attn_part(p, l, b, g, sp, h)));
+#pragma unroll
+    for (int sp = 0; sp < kMergeFast; ++sp) M = fmaxf(M, m[sp]);
+    for (int sp = kMergeFast; sp < sa; ++sp) M = fmaxf(M, __ldcg(attn_part_ml(p, i0 + sp * stride)));
     float L = 0.0f;
     float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int sp = 0; sp < sa; ++sp) {
-        const float* pp = attn_part(p, l, b, g, sp, h);
-        const float m = __ldcg(pp);
-        if (m == -INFINITY) continue;
-        const float f = exp2f(m - M);
-        L = fmaf(__ldcg(pp + 1), f, L);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = fmaf(__ldcg(pp + 2 + i + e), f, o[e]);
+    for (int sp = 0; sp < kMergeFast; ++sp) {
+        const float f = (m[sp] == -INFINITY) ? 0.0f : exp2f(m[sp] - M);
+        L = fmaf(ls[sp], f, L);
+        o[0] = fmaf(oa[sp].x, f, o[0]); o[1] = fmaf(oa[sp].y, f, o[1]);
+        o[2] = fmaf(oa[sp].z, f, o[2]); o[3] = fmaf(oa[sp].w, f, o[3]);
+        o[4] = fmaf(ob[sp].x, f, o[4]); o[5] = fmaf(ob[sp].y, f, o[5]);
+        o[6] = fmaf(ob[sp].z, f, o[6]); o[7] = fmaf(ob[sp].w, f, o[7]);
+    }
+    for (int sp = kMergeFast; sp < sa; ++sp) {
+        const size_t idx = i0 + sp * stride;
+        const float mm = __ldcg(attn_part_ml(p, idx));
+        if (mm == -INFINITY) continue;
+        const float f = exp2f(mm - M);
+        L = fmaf(__ldcg(attn_part_ml(p, idx) + 1), f, L);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = fmaf(__ldcg(attn_part_o(p, idx) + i + e), f, o[e]);
     }
     const float inv = 1.0f / L;
 #pragma unroll
@@ -921,6 +955,7 @@ __device__ __forceinline__ void gemv_prologue(const Params& p, Smem& sm, uint32_
         // merged attention output -> shared memory (K <= the scratch size) -> registers
         float* ob = sm.attn;
         csync(p, sm, cph);                       // the scratch is free
+#pragma unroll 2
         for (int v = threadIdx.x; v < K / 8; v += kConsumerThreads) {
             float2 x[4];
             load8_attn_merge(p, t.layer, 0, v * 8, x);
@@ -1487,7 +1522,9 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
                 }
                 val = acc;
             }
-            attn_part(p, l, b, g, s, h)[c] = val;
+            const size_t pidx = attn_part_index(p, l, b, g, s, h);
+            if (c < 2) attn_part_ml(p, pidx)[c] = val;
+            else attn_part_o(p, pidx)[c - 2] = val;
         }
     }
 }

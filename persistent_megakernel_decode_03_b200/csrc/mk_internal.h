@@ -137,7 +137,7 @@ struct Params {
     float* x_out;    // [L][B][H]   residual after the dense FFN
     float* qkv;      // [L][B][(nq+2nkv)*hd]
     float* act;      // dense: [L][B][F]; MoE: [L][B][topk][Fe]
-    float* part;     // [L][B][nkv][S][hpg][hd+2] attention split partials (m, l, o)
+    float* part;     // attention split partials: o [L][B][nkv][S][hpg][hd], then (m, l) pairs
     float* rlogits;  // [L][B][E]
     float* moe_w;    // [L][B][topk]
     int* moe_sel;    // [L][B][topk]
