@@ -238,6 +238,30 @@ mk_status mk_decode_step_host(mk_state* state, const int32_t* token_ids, const i
 mk_status mk_prefill(mk_state* state, const int32_t* tokens, int n_tokens, int pos0,
                      const mk_paged_kv* kv, float* last_logits, mk_stream stream);
 
+/* The decode step of mk_decode_step for callers that cannot allocate device
+ * memory: code running where cudaMalloc is not allowed (inside a host callback,
+ * a signal or real-time path, or a runtime that owns a fixed memory budget and
+ * forbids later allocations).  The pages describe no such entry point; it is a
+ * convenience of this library.
+ *   It allocates no device memory and needs no mk_model / mk_graph / mk_state:
+ * the task list, RoPE table, per-layer pointer table, event counters,
+ * activations and attention partials live in one fixed 32 MiB device array
+ * (file scope, per GPU, held until the process exits).  Arguments are those of
+ * mk_load_model + mk_decode_step for one sequence (batch must be 1) with
+ * contexts up to max_ctx tokens; the caller passes the weights, the paged KV
+ * cache, token and position (device int32 [1]) and logits_out (device fp32
+ * [vocab]).  A model/context whose scratch would exceed 32 MiB is rejected with
+ * MK_ERR_UNSUPPORTED (mk_last_error_string() gives the size needed).
+ *   The first call on a device (and the first after the model, its weight
+ * pointers or max_ctx change) looks up the array's device address, plans the
+ * task list on the host and copies it into the array; later calls only clear
+ * the counters and launch.  Every call shares the array: calls that overlap on
+ * the GPU (other streams, other host threads' work in flight) race.  The call
+ * waits for its step and returns the step's device status. */
+mk_status mk_decode_step_noalloc(const mk_model_desc* desc, const void* const* weight_ptrs, int n_ptrs,
+                                 int max_ctx, const int32_t* token_ids, const int32_t* positions,
+                                 int batch, const mk_paged_kv* kv, float* logits_out, mk_stream stream);
+
 /* Waits for the stream and returns the device status word of the last step
  * (MK_OK, MK_ERR_TIMEOUT, MK_ERR_INVALID_ARG, ...). */
 mk_status mk_sync(mk_state* state, mk_stream stream);

@@ -41,7 +41,8 @@ SYMBOLS = (
     "mk_graph_destroy", "mk_graph_get_info", "mk_graph_export_tasks", "mk_graph_export_thresholds",
     "mk_wave_stats", "mk_state_create", "mk_state_destroy", "mk_state_set_timeout",
     "mk_state_debug_wait_offset", "mk_state_set_prefetch",
-    "mk_decode_step", "mk_decode_step_host", "mk_prefill", "mk_sync", "mk_state_read_counters",
+    "mk_decode_step", "mk_decode_step_host", "mk_prefill", "mk_decode_step_noalloc", "mk_sync",
+    "mk_state_read_counters",
     "mk_state_read_buffer", "mk_state_read_trace", "mk_state_read_stats", "mk_last_error_string",
     "mk_version",
 )
@@ -119,6 +120,8 @@ def lib() -> ctypes.CDLL:
             "mk_decode_step": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_decode_step_host": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_prefill": ([vp, vp, i32, i32, P(mk_paged_kv), vp, vp], st),
+            "mk_decode_step_noalloc": ([P(mk_model_desc), vp, i32, i32, vp, vp, i32, P(mk_paged_kv),
+                                        vp, vp], st),
             "mk_sync": ([vp, vp], st),
             "mk_state_read_counters": ([vp, vp, P(mk_state_counters), vp, i32], st),
             "mk_state_read_buffer": ([vp, i32, i32, vp, ctypes.c_size_t, vp], st),
@@ -248,6 +251,15 @@ def mk_decode_step_host(state: int, token_ids: int, positions: int, batch: int, 
 def mk_prefill(state: int, tokens: int, n_tokens: int, pos0: int, kv: mk_paged_kv,
                last_logits: int, stream: int = 0) -> None:
     _check(lib().mk_prefill(state, tokens, n_tokens, pos0, ctypes.byref(kv), last_logits, stream))
+
+
+def mk_decode_step_noalloc(desc: mk_model_desc, weight_ptrs: Sequence[int], max_ctx: int,
+                           token_ids: int, positions: int, batch: int, kv: mk_paged_kv,
+                           logits_out: int, stream: int = 0) -> None:
+    """The allocation-free decode step (see include/mk.h); waits for the step."""
+    arr = (ctypes.c_void_p * len(weight_ptrs))(*weight_ptrs)
+    _check(lib().mk_decode_step_noalloc(ctypes.byref(desc), arr, len(weight_ptrs), max_ctx, token_ids,
+                                        positions, batch, ctypes.byref(kv), logits_out, stream))
 
 
 def mk_sync(state: int, stream: int = 0) -> int:

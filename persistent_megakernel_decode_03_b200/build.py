@@ -6,7 +6,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["api.cu", "megakernel.cu", "graph.cpp"]
+SOURCES = ["api.cu", "megakernel.cu", "graph.cpp", "noalloc.cu"]
 HEADERS = ["mk_internal.h", "graph.h", "megakernel.h"]
 
 

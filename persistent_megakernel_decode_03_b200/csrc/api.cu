@@ -197,6 +197,10 @@ mk_status launch_step(mk_state* s, mk::Params& p, cudaStream_t st) {
 
 }  // namespace
 
+namespace mk {
+void set_last_error(const char* msg) { g_err = msg; }
+}  // namespace mk
+
 extern "C" {
 
 const char* mk_last_error_string(void) { return g_err.c_str(); }

@@ -156,6 +156,9 @@ struct Params {
     float* logits;
 };
 
+// Sets the text returned by mk_last_error_string() for the calling thread.
+void set_last_error(const char* msg);
+
 // Error status values written by the device (match mk_status).
 constexpr int kErrInvalid = MK_ERR_INVALID_ARG;
 constexpr int kErrTimeout = MK_ERR_TIMEOUT;
