@@ -140,6 +140,22 @@ def workload(name: str):
     raise SystemExit(f"unknown workload {name}")
 
 
+def max_over_ranks(x: float, pg, device) -> float:
+    """Largest value of x over all ranks (identity without a process group)."""
+    if pg is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tokens_per_s(steps: int, world: int, slowest_ms: float, batch: int = 1) -> float:
+    """Whole-job throughput of `world` independent replicas: every rank decodes
+    `steps` steps of `batch` tokens; the job ends with the slowest rank."""
+    return world * steps * batch / (slowest_ms / 1e3)
+
+
 def dist_info():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -301,15 +317,11 @@ def run_gpu(args, W):
     if st != mk.MK_OK:
         raise SystemExit(f"timed steps failed: {mk.mk_last_error_string()}")
     per = [events[k].elapsed_time(events[k + 1]) for k in range(args.steps)]
-    total_ms = events[0].elapsed_time(events[-1])
-    if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(events[0].elapsed_time(events[-1]), pg, dev)
     timed_pos = positions[args.warmup:]
     info = dec.info
     bytes_step = float(info.weight_bytes_per_step) + kv_read_bytes(cfg, timed_pos)
-    tok_s = world * args.steps / (total_ms / 1e3)
+    tok_s = replica_tokens_per_s(args.steps, world, total_ms)
     sol = sol_tokens_per_s(bytes_step, SOL_BW)
     peak, peak_kind = measured_peaks()
     launch_ms = statistics.mean(per)
@@ -334,14 +346,10 @@ def run_gpu(args, W):
                                    logits_h.data_ptr(), stream.cuda_stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
         if dec.sync() != mk.MK_OK:
             raise SystemExit(f"e2e steps failed: {mk.mk_last_error_string()}")
-        e2e = {"value": world * k_e2e / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": replica_tokens_per_s(k_e2e, world, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": 8, "d2h_bytes_per_step": 4 * cfg.vocab, "steps": k_e2e,
                "api": "mk_decode_step_host"}
 
@@ -386,6 +394,72 @@ def run_gpu(args, W):
         pg.destroy_process_group()
 
 
+def run_solo(args, W):
+    """One operator kind's tiles alone (dependencies dropped), on the workload's shapes.
+
+    Prints one JSON line: median launch time and the algorithmic bytes of that
+    operator over all layers divided by it.  Evidence per tile type; not the
+    metric."""
+    import torch
+    import synthetic as syn
+    import persistent_megakernel_decode_03_b200 as mk
+    from persistent_megakernel_decode_03_b200.runner import Decoder
+
+    names = {v: k for k, v in mk.OP_NAMES.items()}
+    if args.solo not in names:
+        raise SystemExit(f"unknown operator {args.solo}")
+    op = names[args.solo]
+    cfg = W["cfg"]
+    if cfg.is_moe:
+        raise SystemExit("solo lists cover the dense operators")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    seed = syn.SEED_WEIGHTS + W["seed"]
+    ts = []
+    for s in syn.tensor_specs(cfg):
+        t = torch.empty(s.shape, dtype=torch.bfloat16, device=dev)
+        syn.dev_fill_tensor(t, s, seed)
+        ts.append(t)
+    ctx = W["prompt"] + W["gen"] // 2
+    max_ctx = W["prompt"] + W["gen"]
+    desc = dict(n_layers=cfg.n_layers, hidden=cfg.hidden, n_q_heads=cfg.n_q_heads,
+                n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, ffn=cfg.ffn, vocab=cfg.vocab,
+                rms_eps=cfg.rms_eps, rope_theta=cfg.rope_theta)
+    dec = Decoder(desc, [t.data_ptr() for t in ts], 1, max_ctx, device="cuda:0")
+    L, H, F, V, d = cfg.n_layers, cfg.hidden, cfg.ffn, cfg.vocab, cfg.head_dim
+    nq, nkv = cfg.n_q_heads, cfg.n_kv_heads
+    nbytes = {"qkv": 2 * (nq + 2 * nkv) * d * H * L, "attn": (ctx + 1) * L * 2 * nkv * d * 2,
+              "oproj": 2 * H * nq * d * L, "gateup": 4 * F * H * L, "down": 2 * H * F * L,
+              "lmhead": 2 * V * H}[args.solo]
+    g = mk.mk_build_taskgraph_solo(dec.model, 1, max_ctx, op)
+    st = mk.mk_state_create(g)
+    info = mk.mk_graph_get_info(g)
+    tok = torch.tensor([7], dtype=torch.int32, device=dev)
+    pos = torch.tensor([ctx], dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for i in range(args.warmup + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        mk.mk_decode_step(st, tok.data_ptr(), pos.data_ptr(), 1, dec.kv, dec.logits.data_ptr(),
+                          stream.cuda_stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    if mk.mk_sync(st, stream.cuda_stream) != mk.MK_OK:
+        raise SystemExit(f"solo run failed: {mk.mk_last_error_string()}")
+    med = statistics.median(times)
+    peak, peak_kind = measured_peaks()
+    gbs = nbytes / (med / 1e3) / 1e9
+    print(json.dumps({"solo": args.solo, "workload": W["desc"], "tasks": info.n_tasks,
+                      "bytes_per_launch": nbytes, "median_us": med * 1e3, "achieved_gbs": gbs,
+                      "peak_gbs": peak, "frac": gbs / peak, "peak_kind": peak_kind}), flush=True)
+    mk.mk_state_destroy(st)
+    mk.mk_graph_destroy(g)
+    dec.close()
+
+
 def kernel_source_sha() -> str:
     import hashlib
     h = hashlib.sha256()
@@ -404,13 +478,24 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama8b", choices=["llama8b", "tiny", "moe30b", "long131k"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: run the workload with its first N layers (not a bench line)")
+    ap.add_argument("--solo", default="",
+                    help="profiling only: time one operator kind's task list alone "
+                         "(qkv, attn, oproj, gateup, down, lmhead) and print its GB/s")
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds of CPU time the reference arm may spend on timed steps")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "mk":
         raise SystemExit("at least 3 warm-up steps")
     W = workload(args.workload)
-    if args.impl == "reference":
+    if args.layers:
+        import dataclasses
+        W["cfg"] = dataclasses.replace(W["cfg"], n_layers=min(args.layers, W["cfg"].n_layers))
+        W["desc"] += f" [first {W['cfg'].n_layers} layers only: profiling case]"
+    if args.solo:
+        run_solo(args, W)
+    elif args.impl == "reference":
         run_reference(args, W)
     else:
         run_gpu(args, W)

@@ -160,6 +160,7 @@ struct __align__(128) Smem {
     uint64_t sig_full[kSigSlots], sig_empty[kSigSlots];
     uint64_t csync;                          // all-consumer-warp sync (arrival count 8)
     uint32_t arrive[kRedBufs];               // per-task warp arrivals (monotone, 8 per use)
+    uint64_t red_free[kRedBufs];             // completes when a task's last warp has read red[buf]
     StageInfo info[kStages];
     uint32_t sig_evt[kSigSlots];
     int sig_task[kSigSlots];
@@ -1645,6 +1646,14 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
         }
         uint32_t* arrive = &sm.arrive[seq % kRedBufs];
         const int buf = (int)(seq % kRedBufs);
+        // Warps drift apart by as many tasks as the ring holds stages, which is more
+        // than kRedBufs when tasks are one stage long; a warp may reuse red[buf] and
+        // arrive[buf] only once the task that used them kRedBufs tasks ago is finished.
+        if (seq >= (uint32_t)kRedBufs &&
+            !mbar_wait_bounded(p, &sm.red_free[buf], ((seq / kRedBufs) - 1) & 1, 9)) {
+            sm.flag[3] = 1;
+            break;
+        }
 
         if (t.op == MK_OP_ATTN) {
             bool abort_all = false;
@@ -1656,7 +1665,10 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             for (int j = 0; j < kMaxVecPerThread; ++j)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) xr[j][q] = make_float2(0.0f, 0.0f);
-            if (last_warp_arrival(arrive) && lane == 0) hand_off(t.sig, ti);
+            if (last_warp_arrival(arrive) && lane == 0) {
+                mbar_arrive(&sm.red_free[buf]);
+                hand_off(t.sig, ti);
+            }
             ++seq;
             continue;
         }
@@ -1765,7 +1777,10 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             else evt = MK_NO_EVENT;
         }
         __syncwarp();
-        if (lane == 0) hand_off(evt, ti);
+        if (lane == 0) {
+            mbar_arrive(&sm.red_free[buf]);     // red[buf] is read; it may be reused
+            hand_off(evt, ti);
+        }
         if (p.stats && lane == 0) stat_add(p, 7, (unsigned long long)(clock64() - c_ep));
         ++seq;
     }
@@ -1798,7 +1813,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&sm.sig_empty[s], 1);
         }
         mbar_init(&sm.csync, kConsumerWarps);
-        for (int i = 0; i < kRedBufs; ++i) sm.arrive[i] = 0;
+        for (int i = 0; i < kRedBufs; ++i) {
+            sm.arrive[i] = 0;
+            mbar_init(&sm.red_free[i], 1);
+        }
         for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }

@@ -273,3 +273,26 @@ def test_8b_full_size_synthetic_context(n_ctx):
         assert ok, (p, d, cos)
         check_counters(dec)
     dec.close()
+
+
+def test_prefill_with_many_one_stage_tiles_per_cta():
+    """Prefill at 8B shapes (two layers, full 128256-row LM head): the prompt's
+    non-final steps skip the LM head, so every CTA runs ~54 tiles of one ring
+    stage each in a row, and its warps drift apart by more tasks than there
+    are per-task reduction slots.  Last logits, KV contents and counters must
+    still match."""
+    cfg = dataclasses.replace(syn.LLAMA8B, n_layers=2)
+    seed = syn.SEED_WEIGHTS + 2
+    specs, ts = device_weights(cfg, seed)
+    n = 6
+    prompt = syn.host_tokens(n, syn.SEED_PROMPT + 2, cfg.vocab)
+    dec = make_decoder(cfg, ts, 1, 64)
+    last = dec.prefill(torch.tensor(prompt, dtype=torch.int32, device="cuda")).cpu().numpy()
+    dec.check()
+    check_counters(dec)
+    orc = oracle.Model(cfg, syn.host_weights(cfg, seed), 64, names(cfg))
+    for p, t in enumerate(prompt):
+        ref = orc.decode_step(int(t), p)["logits"]
+    d, cos, ok = compare_logits(last, ref)
+    assert ok, (d, cos)
+    dec.close()
