@@ -10,8 +10,10 @@
 // worker loop fetch -> execute -> notify; event fires at its threshold).
 //
 // Warp roles inside a CTA:
-//   warps 0-7  consumers: dependency wait, prologue (RMSNorm / RoPE), dot
-//              products out of shared memory, epilogue, reductions
+//   warps 0-7  consumers: dependency wait, input stage (embedding, RMSNorm,
+//              split merge), attention, dot products out of shared memory and
+//              warp reductions; each warp leaves its partial row sums in a
+//              rotating buffer and moves straight on to the next task
 //   warp 8     producer: dequeues the next tasks and streams their weight rows
 //              and KV pages into an 11-stage shared-memory ring with bulk
 //              asynchronous copies (cp.async.bulk, mbarrier completion).
@@ -20,13 +22,16 @@
 //              layer's weights are in flight while this layer's tail finishes
 //              (Cohere page, "Honnan jön a gyorsulás?": weight tiles are
 //              prefetched before the activation dependency is met).
-//   warp 9     signal: publishes completions (fence + release add) so that the
-//              consumers do not stall on the gpu-scope fence.
+//   warp 9     epilogue: reduces the consumers' partials in a fixed order,
+//              applies each operator's tail (residual add, SiLU gate, expert
+//              selection), stores, and publishes the completion (fence +
+//              release add), so no consumer stalls on a task's tail or on the
+//              gpu-scope fence.
 //
 // Deadlock freedom: tasks are dequeued in list order, the list is topological
 // and each CTA runs its tasks in dequeue order, so the lowest unfinished task
 // always has its producers finished and its CTA free to run it.
-// Every wait (event counter, ring slot, signal slot) gives up after
+// Every wait (event counter, ring slot, buffer set) gives up after
 // Params::timeout_ns, records MK_ERR_TIMEOUT and the kernel drains its own
 // copies in flight and returns.
 #include <cuda_runtime.h>
@@ -48,6 +53,9 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t n) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t tx) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(tx)
@@ -142,8 +150,8 @@ struct StageInfo {
 };
 
 constexpr int kAttnScratch = kConsumerWarps * kMaxHeadsPerGroup * (128 + 2);   // >= n_q * head_dim floats too
-// Rotating buffers of per-warp row sums.  A consumer warp runs at most one ring's
-// worth of stages (< 2 tasks) ahead of the slowest, so 4 buffers never collide.
+// Rotating buffer sets (row sums, task record, residual rows) between the consumer
+// warps and the epilogue warp: consumers may run kRedBufs - 1 tasks ahead of it.
 constexpr int kRedBufs = 4;
 
 struct __align__(128) Smem {
@@ -157,13 +165,13 @@ struct __align__(128) Smem {
     float kn[128], vn[128];                   // the new token's k, v (bf16-rounded)
     float bcast[kConsumerWarps + 8];
     uint64_t full[kStages], empty[kStages];
-    uint64_t sig_full[kSigSlots], sig_empty[kSigSlots];
     uint64_t csync;                          // all-consumer-warp sync (arrival count 8)
-    uint32_t arrive[kRedBufs];               // per-task warp arrivals (monotone, 8 per use)
-    uint64_t red_free[kRedBufs];             // completes when a task's last warp has read red[buf]
+    uint64_t red_full[kRedBufs];             // 8 consumer-warp arrivals: the task's partials are in red[buf]
+    uint64_t red_free[kRedBufs];             // the epilogue warp has finished with buffer set buf
     StageInfo info[kStages];
-    uint32_t sig_evt[kSigSlots];
-    int sig_task[kSigSlots];
+    Task ep_task[kRedBufs];                  // task record for the epilogue warp
+    int ep_ti[kRedBufs];                     // its index (-1: end of work)
+    float ep_resid[kRedBufs][kMaxTaskRows];  // residual rows (O-proj, down), loaded early by warp 0
     int flag[4];
 };
 
@@ -323,7 +331,6 @@ __device__ __forceinline__ void wait_stat(const Params& p, int where, long long 
     const unsigned long long d = (unsigned long long)(clock64() - c0);
     if (where == 1) stat_add(p, 0, d);                                   // producer: ring full
     else if ((where == 3 || where == 4 || where == 5) && threadIdx.x == 0) stat_add(p, 1, d);
-    else if (where == 6) stat_add(p, 5, d);
 }
 
 __device__ bool mbar_wait_slow(const Params& p, uint64_t* bar, uint32_t parity, int where) {
@@ -357,19 +364,6 @@ __device__ __forceinline__ void csync(const Params& p, Smem& sm, uint32_t& phase
     phase ^= 1;
 }
 
-// Every consumer warp calls this once per task after depositing its share;
-// returns true in the warp that arrives last (acquire: it sees every other
-// warp's shared-memory writes), which then finishes the task alone.
-__device__ __forceinline__ bool last_warp_arrival(uint32_t* cnt) {
-    __syncwarp();
-    uint32_t old = 0;
-    if ((threadIdx.x & 31) == 0)
-        asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
-                     : "=r"(old) : "r"(smem_u32(cnt)) : "memory");
-    old = __shfl_sync(0xFFFFFFFFu, old, 0);
-    __syncwarp();
-    return (old % kConsumerWarps) == kConsumerWarps - 1;
-}
 
 // Wait on a phase that another thread of this CTA has already seen complete
 // (so it returns at once); bounded anyway: on failure it records a fault and
@@ -671,25 +665,6 @@ __device__ void prefetch_loop(const Params& p) {
                 const int64_t n = bytes - off < 32768 ? bytes - off : 32768;
                 prefetch_l2(reinterpret_cast<const uint8_t*>(g.w[bi]) + off, (uint32_t)n);
             }
-    }
-}
-
-// ----------------------------------------------------------------------------- signal warp
-
-__device__ void signal_loop(const Params& p, Smem& sm) {
-    int slot = 0;
-    uint32_t lap = 0;
-    while (true) {
-        if (!mbar_wait_bounded(p, &sm.sig_full[slot], lap & 1, 2)) return;
-        uint32_t e = sm.sig_evt[slot];
-        int task = sm.sig_task[slot];
-        if (e == 0xFFFFFFFEu) return;   // end of work
-        __threadfence();
-        if (e != MK_NO_EVENT) red_release_add(&p.events[e], 1u);
-        atomicAdd(p.done, 1u);
-        if (p.trace && task >= 0) p.trace[(size_t)task * 4 + 2] = globaltimer();
-        mbar_arrive(&sm.sig_empty[slot]);
-        if (++slot == kSigSlots) { slot = 0; ++lap; }
     }
 }
 
@@ -1592,31 +1567,21 @@ __device__ void router_finalize(const Params& p, Smem& sm, int l) {
 
 template <int HPG, int DPL>
 __device__ void consumer_loop(const Params& p, Smem& sm) {
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int stage = 0;
     uint32_t lap = 0;
-    uint32_t seq = 0;                                   // tasks finished by this CTA (same in every warp)
+    uint32_t seq = 0;                                   // tasks started by this CTA (same in every warp)
     uint32_t cph = 0;                                   // phase of sm.csync
     float2 xr[kMaxVecPerThread][4];
     int x_key_op = -1, x_key_layer = -1, x_key_b = -1, x_key_aux = -1;
     uint32_t ok_evt[4] = {MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT};   // per warp
 
-    // Hands task `ti` to the signal warp: called by one lane-0 thread (the warp that
-    // finished the task last) after its warp's stores; slots are used in task order.
-    auto hand_off = [&](uint32_t evt, int ti) {
-        const int slot = (int)(seq % kSigSlots);
-        const uint32_t slap = seq / kSigSlots;
-        if (slap > 0 && !mbar_wait_bounded(p, &sm.sig_empty[slot], (slap - 1) & 1, 6)) sm.flag[3] = 1;
-        sm.sig_evt[slot] = evt;
-        sm.sig_task[slot] = ti;
-        mbar_arrive(&sm.sig_full[slot]);
-    };
-
-    // Each warp waits for its own data and dependencies and runs its share of the
-    // task; the last warp to finish a task reduces the shares, stores the output
-    // and hands the completion to the signal warp.  Warps meet only inside
-    // prologues and attention tasks (bounded mbarrier syncs).  A failure raises
-    // sm.flag[3]; every warp checks it before its next task.
+    // Each warp waits for its own data and dependencies, runs its share of the task,
+    // leaves its partial row sums in red[buf] and arrives on red_full[buf]; the
+    // epilogue warp reduces, stores and signals, so no consumer warp ever waits for
+    // a task's tail.  Warps meet only inside prologues and attention tasks (bounded
+    // mbarrier syncs).  A failure raises sm.flag[3]; every warp checks it before
+    // its next task.
     while (true) {
         if (sm.flag[3]) break;
         bool ok = mbar_wait_bounded(p, &sm.full[stage], lap & 1, 4);
@@ -1644,15 +1609,17 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             p.trace[(size_t)ti * 4 + 1] = globaltimer();
             p.trace[(size_t)ti * 4 + 3] = (uint64_t)blockIdx.x;
         }
-        uint32_t* arrive = &sm.arrive[seq % kRedBufs];
         const int buf = (int)(seq % kRedBufs);
-        // Warps drift apart by as many tasks as the ring holds stages, which is more
-        // than kRedBufs when tasks are one stage long; a warp may reuse red[buf] and
-        // arrive[buf] only once the task that used them kRedBufs tasks ago is finished.
+        // buffer set `buf` is reused once the epilogue warp has finished the task that
+        // used it kRedBufs tasks ago
         if (seq >= (uint32_t)kRedBufs &&
             !mbar_wait_bounded(p, &sm.red_free[buf], ((seq / kRedBufs) - 1) & 1, 9)) {
             sm.flag[3] = 1;
             break;
+        }
+        if (tid == 0) {
+            sm.ep_task[buf] = t;
+            sm.ep_ti[buf] = ti;
         }
 
         if (t.op == MK_OP_ATTN) {
@@ -1665,10 +1632,8 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             for (int j = 0; j < kMaxVecPerThread; ++j)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) xr[j][q] = make_float2(0.0f, 0.0f);
-            if (last_warp_arrival(arrive) && lane == 0) {
-                mbar_arrive(&sm.red_free[buf]);
-                hand_off(t.sig, ti);
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.red_full[buf]);
             ++seq;
             continue;
         }
@@ -1684,6 +1649,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
                     m.gstride = kConsumerThreads; m.vpt = m.nvec / kConsumerThreads; m.active = true; }
         else m = thread_map(g.K);
         const int rows_total = g.rows * g.nblk;
+        const bool resid = !skip && warp == 0 && (t.op == MK_OP_OPROJ || t.op == MK_OP_DOWN);
         float resid0 = 0.0f, resid1 = 0.0f;
         if (!skip) {
             if (t.op == MK_OP_QKV && t.layer == 0 && tid == 0) {
@@ -1695,9 +1661,9 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
                 gemv_prologue(p, sm, cph, t, m, g.K, xr);
                 x_key_op = t.op; x_key_layer = t.layer; x_key_b = t.b; x_key_aux = t.aux;
             }
-            // residual rows for the epilogue (whichever warp runs it), fetched now so the
-            // loads overlap the streaming
-            if (t.op == MK_OP_OPROJ || t.op == MK_OP_DOWN) {
+            // residual rows for the epilogue warp, fetched by warp 0 now so the loads
+            // overlap the streaming
+            if (resid) {
                 const int r0 = (int)t.r0;
                 if (lane < rows_total)
                     resid0 = (t.op == MK_OP_OPROJ) ? x_in(p, t.layer, 0, r0 + lane) : x_mid_at(p, t.layer, 0, r0 + lane);
@@ -1711,88 +1677,129 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
         else (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
         if (p.stats && tid == 0) stat_add(p, 6, (unsigned long long)(clock64() - c_ch));
         if (sm.flag[3]) break;
-
-        if (!last_warp_arrival(arrive)) { ++seq; continue; }
-
-        // ---- epilogue (last warp): reduce the warps' partials in fixed order, store
-        const long long c_ep = (p.stats && lane == 0) ? clock64() : 0;
-        uint32_t evt = t.sig;
-        if (!skip) {
-            const int l = t.layer, b = t.b;
-            const int nout = (g.nblk == 2) ? g.rows : rows_total;
-            for (int r = lane; r < nout; r += 32) {
-                float y = 0.0f;
-                for (int w = 0; w < m.wpg; ++w) y += sm.red[buf][r][w];
-                const int row = (int)t.r0 + r;
-                const float resid = (r < 32) ? resid0 : resid1;
-                switch (t.op) {
-                    case MK_OP_QKV:
-                        p.qkv[((size_t)l * p.max_batch) * ((p.nq + 2 * p.nkv) * p.hd) + row] = y;
-                        break;
-                    case MK_OP_OPROJ:
-                        p.x_mid[((size_t)l * p.max_batch) * p.H + row] = resid + y;
-                        break;
-                    case MK_OP_GATEUP: {
-                        float u = 0.0f;
-                        for (int w = 0; w < m.wpg; ++w) u += sm.red[buf][g.rows + r][w];
-                        p.act[((size_t)l * p.max_batch) * p.F + row] = silu_f(y) * u;
-                        break;
-                    }
-                    case MK_OP_DOWN:
-                        p.x_out[((size_t)l * p.max_batch) * p.H + row] = resid + y;
-                        break;
-                    case MK_OP_LMHEAD:
-                        p.logits[row] = y;
-                        break;
-                    case MK_OP_ROUTER:
-                        p.rlogits[((size_t)l * p.max_batch) * p.E + row] = y;
-                        break;
-                    case MK_OP_EXP_GATEUP: {
-                        float u = 0.0f;
-                        for (int w = 0; w < m.wpg; ++w) u += sm.red[buf][g.rows + r][w];
-                        p.act[(((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.Fe + row] = silu_f(y) * u;
-                        break;
-                    }
-                    case MK_OP_EXP_DOWN:
-                        p.ypart[(((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.H + row] = y;
-                        break;
-                    default:
-                        break;
-                }
-            }
-        }
-        if (t.op == MK_OP_ROUTER) {
-            // arrival of this router tile; the layer's last tile selects the experts and
-            // only it signals the router event
-            __syncwarp();
-            int last = 0;
-            if (lane == 0) {
-                __threadfence();
-                const uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
-                __threadfence();
-                last = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
-            }
-            last = __shfl_sync(0xFFFFFFFFu, last, 0);
-            if (last) router_finalize(p, sm, t.layer);
-            else evt = MK_NO_EVENT;
+        if (resid) {
+            if (lane < rows_total) sm.ep_resid[buf][lane] = resid0;
+            if (lane + 32 < rows_total) sm.ep_resid[buf][lane + 32] = resid1;
         }
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&sm.red_free[buf]);     // red[buf] is read; it may be reused
-            hand_off(evt, ti);
-        }
-        if (p.stats && lane == 0) stat_add(p, 7, (unsigned long long)(clock64() - c_ep));
+        if (lane == 0) mbar_arrive(&sm.red_full[buf]);
         ++seq;
     }
-    // end of work for the signal warp: one marker after every warp has left the loop
+    // end of work for the epilogue warp: a marker once every consumer warp has left
+    // the loop (a full set of arrivals on the next buffer set)
     csync(p, sm, cph);
     if (tid == 0) {
-        const int slot = (int)(seq % kSigSlots);
-        const uint32_t slap = seq / kSigSlots;
-        if (slap > 0) (void)mbar_wait_bounded(p, &sm.sig_empty[slot], (slap - 1) & 1, 7);
-        sm.sig_evt[slot] = 0xFFFFFFFEu;
-        sm.sig_task[slot] = -1;
-        mbar_arrive(&sm.sig_full[slot]);
+        const int buf = (int)(seq % kRedBufs);
+        if (seq < (uint32_t)kRedBufs || mbar_wait_bounded(p, &sm.red_free[buf], ((seq / kRedBufs) - 1) & 1, 7)) {
+            sm.ep_ti[buf] = -1;
+            mbar_arrive_cnt(&sm.red_full[buf], kConsumerWarps);
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- epilogue warp
+
+// Output rows of a finished GEMV task: the consumer warps' partial sums reduced in
+// a fixed order (bit-identical from run to run), then the operator's tail.
+__device__ __forceinline__ void gemv_store(const Params& p, const Smem& sm, const Task& t, const GemvGeom& g,
+                                           int wpg, int buf, int lane) {
+    const int l = t.layer, b = t.b;
+    const int rows_total = g.rows * g.nblk;
+    const int nout = (g.nblk == 2) ? g.rows : rows_total;
+    auto row_sum = [&](int r) -> float {
+        float y = 0.0f;
+        if (wpg == kConsumerWarps) {
+            const float4 a = *reinterpret_cast<const float4*>(&sm.red[buf][r][0]);
+            const float4 c = *reinterpret_cast<const float4*>(&sm.red[buf][r][4]);
+            y = a.x; y += a.y; y += a.z; y += a.w; y += c.x; y += c.y; y += c.z; y += c.w;
+        } else {
+            for (int w = 0; w < wpg; ++w) y += sm.red[buf][r][w];
+        }
+        return y;
+    };
+    for (int r = lane; r < nout; r += 32) {
+        const float y = row_sum(r);
+        const int row = (int)t.r0 + r;
+        switch (t.op) {
+            case MK_OP_QKV:
+                p.qkv[((size_t)l * p.max_batch) * ((p.nq + 2 * p.nkv) * p.hd) + row] = y;
+                break;
+            case MK_OP_OPROJ:
+                p.x_mid[((size_t)l * p.max_batch) * p.H + row] = sm.ep_resid[buf][r] + y;
+                break;
+            case MK_OP_GATEUP:
+                p.act[((size_t)l * p.max_batch) * p.F + row] = silu_f(y) * row_sum(g.rows + r);
+                break;
+            case MK_OP_DOWN:
+                p.x_out[((size_t)l * p.max_batch) * p.H + row] = sm.ep_resid[buf][r] + y;
+                break;
+            case MK_OP_LMHEAD:
+                p.logits[row] = y;
+                break;
+            case MK_OP_ROUTER:
+                p.rlogits[((size_t)l * p.max_batch) * p.E + row] = y;
+                break;
+            case MK_OP_EXP_GATEUP:
+                p.act[(((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.Fe + row] =
+                    silu_f(y) * row_sum(g.rows + r);
+                break;
+            case MK_OP_EXP_DOWN:
+                p.ypart[(((size_t)l * p.max_batch + b) * p.topk + t.aux) * p.H + row] = y;
+                break;
+            default:
+                break;
+        }
+    }
+}
+
+// One warp of the support warpgroup finishes every task of its CTA, in order: it
+// stores the GEMV outputs, selects the experts after a layer's last router tile,
+// makes the task's writes visible (fence) and adds to the task's event counter
+// with release semantics (MPK digest, "Part 2. Runtime": a finished task
+// increments its event).  Router finalisation uses the scratch that attention
+// and O-projection input stages also use; no consumer can reach one of those
+// before the router event it precedes is signalled, since every later attention
+// and O-projection depends on it.
+__device__ void epilogue_loop(const Params& p, Smem& sm) {
+    const int lane = threadIdx.x & 31;
+    for (uint32_t seq = 0;; ++seq) {
+        const int buf = (int)(seq % kRedBufs);
+        if (!mbar_wait_bounded(p, &sm.red_full[buf], (seq / kRedBufs) & 1, 2)) return;
+        const int ti = sm.ep_ti[buf];
+        if (ti < 0) return;                              // end of work
+        const Task t = sm.ep_task[buf];
+        uint32_t evt = t.sig;
+        if (t.op != MK_OP_ATTN && !(t.op == MK_OP_LMHEAD && p.skip_lm)) {
+            GemvGeom g;
+            gemv_geom(p, t, g, false);
+            const int wpg = (t.flags != kFastNone) ? kConsumerWarps : thread_map(g.K).wpg;
+            gemv_store(p, sm, t, g, wpg, buf, lane);
+            if (t.op == MK_OP_ROUTER) {
+                // arrival of this router tile; the layer's last tile selects the experts
+                // and only it signals the router event
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) {
+                    const uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
+                    __threadfence();
+                    last = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
+                }
+                last = __shfl_sync(0xFFFFFFFFu, last, 0);
+                if (last) router_finalize(p, sm, t.layer);
+                else evt = MK_NO_EVENT;
+            }
+        }
+        // every lane orders its own stores (and, through the consumers' arrivals, theirs)
+        // before lane 0's release of the event
+        if (evt != MK_NO_EVENT) __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+            if (evt != MK_NO_EVENT) red_release_add(&p.events[evt], 1u);
+            atomicAdd(p.done, 1u);
+            if (p.trace) p.trace[(size_t)ti * 4 + 2] = globaltimer();
+            mbar_arrive(&sm.red_free[buf]);
+        }
     }
 }
 
@@ -1808,13 +1815,9 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kConsumerWarps);
         }
-        for (int s = 0; s < kSigSlots; ++s) {
-            mbar_init(&sm.sig_full[s], 1);
-            mbar_init(&sm.sig_empty[s], 1);
-        }
         mbar_init(&sm.csync, kConsumerWarps);
         for (int i = 0; i < kRedBufs; ++i) {
-            sm.arrive[i] = 0;
+            mbar_init(&sm.red_full[i], kConsumerWarps);
             mbar_init(&sm.red_free[i], 1);
         }
         for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
@@ -1834,8 +1837,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSupportRegs));
     if (warp == kProducerWarp) {
         if (lane == 0) producer_loop(p, sm);
-    } else if (warp == kSignalWarp) {
-        if (lane == 0) signal_loop(p, sm);
+    } else if (warp == kEpilogueWarp) {
+        epilogue_loop(p, sm);
     } else if (warp == kPrefetchWarp) {
         if (lane == 0) prefetch_loop(p);
     }

@@ -10,11 +10,11 @@ namespace mk {
 
 // Kernel geometry.  One CTA per SM: 8 consumer warps compute, 1 producer warp
 // streams weights and KV pages into a shared-memory ring with bulk async copies,
-// 1 signal warp publishes task completions.
+// 1 epilogue warp finishes tasks (reduction, stores) and publishes completions.
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kProducerWarp = kConsumerWarps;        // warp 8
-constexpr int kSignalWarp = kConsumerWarps + 1;      // warp 9
+constexpr int kEpilogueWarp = kConsumerWarps + 1;    // warp 9: task epilogues and event signals
 constexpr int kPrefetchWarp = kConsumerWarps + 2;    // warp 10 (warp 11 idles)
 constexpr int kThreads = 384;                        // 3 warpgroups: 2 consumer + 1 support
 // Register split between the warpgroups (setmaxnreg): the support warpgroup gives
@@ -28,7 +28,6 @@ constexpr int kStageBytes = 16 * 1024;
 constexpr int kStages = 11;
 constexpr int kMaxTaskRows = 64;        // rows (all weight blocks) of one GEMV task
 constexpr int kMaxVecPerThread = 8;     // 16-byte vectors of x per consumer thread (K <= 16384)
-constexpr int kSigSlots = 8;            // signal queue depth
 constexpr int kMaxHeadsPerGroup = 8;
 constexpr int kMaxTopK = 16;
 constexpr int kPageSize = 16;
