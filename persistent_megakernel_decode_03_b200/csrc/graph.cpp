@@ -191,31 +191,53 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     };
     auto gemv_op = [&](int op, int layer, int64_t rows, int R, int out_kind, int out_layer,
                        std::vector<Region> in) {
-        for (int64_t r0 = 0; r0 < rows; r0 += R) {
+        for (int64_t r0 = 0; r0 < rows;) {
             int64_t r1 = std::min<int64_t>(rows, r0 + R);
             int t = new_task(op, layer, 0, 0, (uint32_t)r0, (uint32_t)r1);
             task_in[t] = in;
             own_entity(t, {Region{tensor_key(out_kind, out_layer, 0), 0, B, r0, r1}});
+            r0 = r1;
         }
     };
 
-    for (int l = 0; l < L; ++l) {
-        // QKV: primary input is the residual stream entering the layer.
-        gemv_op(MK_OP_QKV, l, qkv_rows, R_qkv, T_QKV, l, {all_rows(T_XIN, l, 0, H)});
-        // attention: per (sequence, kv head, split); each split writes its softmax partial,
-        // and the O-projection's input stage merges the splits.
+    // QKV rows of one KV group: its q heads, then its k and v rows
+    auto qkv_group = [&](int l, int kh) {
+        const std::vector<Region> in = {all_rows(T_XIN, l, 0, H)};
+        const int64_t spans[3][2] = {{(int64_t)kh * hpg * hd, (int64_t)(kh + 1) * hpg * hd},
+                                     {(int64_t)nq * hd + kh * hd, (int64_t)nq * hd + (kh + 1) * hd},
+                                     {(int64_t)(nq + nkv) * hd + kh * hd, (int64_t)(nq + nkv) * hd + (kh + 1) * hd}};
+        for (const auto& sp : spans)
+            for (int64_t r0 = sp[0]; r0 < sp[1];) {
+                int64_t r1 = std::min<int64_t>(sp[1], r0 + R_qkv);
+                int t = new_task(MK_OP_QKV, l, 0, 0, (uint32_t)r0, (uint32_t)r1);
+                task_in[t] = in;
+                own_entity(t, {Region{tensor_key(T_QKV, l, 0), 0, B, r0, r1}});
+                r0 = r1;
+            }
+    };
+    // attention of one KV group: per (sequence, split); each split writes its softmax
+    // partial, and the O-projection's input stage merges the splits
+    auto attn_group = [&](int l, int kh) {
         for (int b = 0; b < B; ++b)
-            for (int kh = 0; kh < nkv; ++kh)
-                for (int s = 0; s < S; ++s) {
-                    int t = new_task(MK_OP_ATTN, l, b, kh, (uint32_t)s, (uint32_t)S);
-                    int key = tensor_key(T_QKV, l, 0);
-                    task_in[t] = {Region{key, 0, B, (int64_t)kh * hpg * hd, (int64_t)(kh + 1) * hpg * hd},
-                                  Region{key, 0, B, (int64_t)nq * hd + kh * hd, (int64_t)nq * hd + (kh + 1) * hd},
-                                  Region{key, 0, B, (int64_t)(nq + nkv) * hd + kh * hd,
-                                         (int64_t)(nq + nkv) * hd + (kh + 1) * hd}};
-                    own_entity(t, {Region{tensor_key(T_O, l, 0), b, b + 1, (int64_t)kh * hpg * hd,
-                                          (int64_t)(kh + 1) * hpg * hd}});
-                }
+            for (int s = 0; s < S; ++s) {
+                int t = new_task(MK_OP_ATTN, l, b, kh, (uint32_t)s, (uint32_t)S);
+                int key = tensor_key(T_QKV, l, 0);
+                task_in[t] = {Region{key, 0, B, (int64_t)kh * hpg * hd, (int64_t)(kh + 1) * hpg * hd},
+                              Region{key, 0, B, (int64_t)nq * hd + kh * hd, (int64_t)nq * hd + (kh + 1) * hd},
+                              Region{key, 0, B, (int64_t)(nq + nkv) * hd + kh * hd,
+                                     (int64_t)(nq + nkv) * hd + (kh + 1) * hd}};
+                own_entity(t, {Region{tensor_key(T_O, l, 0), b, b + 1, (int64_t)kh * hpg * hd,
+                                      (int64_t)(kh + 1) * hpg * hd}});
+            }
+    };
+
+    for (int l = 0; l < L; ++l) {
+        // QKV (input: the residual stream entering the layer), one KV group at a time,
+        // so that the first groups' attention can start while the last QKV tiles
+        // stream.  Attention follows all QKV tiles: a CTA that claimed a task still
+        // waiting on its inputs streams nothing meanwhile.
+        for (int kh = 0; kh < nkv; ++kh) qkv_group(l, kh);
+        for (int kh = 0; kh < nkv; ++kh) attn_group(l, kh);
         gemv_op(MK_OP_OPROJ, l, H, R_o, T_XMID, l, {all_rows(T_O, l, 0, (int64_t)nq * hd)});
         if (!moe) {
             gemv_op(MK_OP_GATEUP, l, d.ffn, R_gu, T_ACT, l, {all_rows(T_XMID, l, 0, H)});

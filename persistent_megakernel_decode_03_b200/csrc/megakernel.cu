@@ -1227,7 +1227,10 @@ __device__ __forceinline__ bool gemv_fast_dispatch(const Params& p, Smem& sm, in
         case kFastV2R2N8: return gemv_fast_rows<2, 2, 8>(p, sm, ti, xr, buf, stage, lap);
         case kFastV1R4N16: return gemv_fast_rows<1, 4, 16>(p, sm, ti, xr, buf, stage, lap);
         case kFastV1R4N8: return gemv_fast_rows<1, 4, 8>(p, sm, ti, xr, buf, stage, lap);
+        case kFastV2R2N4: return gemv_fast_rows<2, 2, 4>(p, sm, ti, xr, buf, stage, lap);
+        case kFastV1R4N4: return gemv_fast_rows<1, 4, 4>(p, sm, ti, xr, buf, stage, lap);
         case kFastV7S4N4: return gemv_fast_segs<7, 4, 4>(p, sm, ti, xr, buf, stage, lap, true);
+        case kFastV7S4N1: return gemv_fast_segs<7, 4, 1>(p, sm, ti, xr, buf, stage, lap, true);
         default: return gemv_fast_segs<7, 4, 2>(p, sm, ti, xr, buf, stage, lap, true);
     }
 }

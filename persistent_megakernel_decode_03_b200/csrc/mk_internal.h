@@ -42,6 +42,9 @@ enum FastPath : uint8_t {
     kFastV1R4N8 = 4,    // K = 2048, 4 rows per stage, 8 rows
     kFastV7S4N4 = 5,    // K = 14336, rows in 2 segments (4 + 3 vectors per thread), 4 rows
     kFastV7S4N2 = 6,    // K = 14336, 2 rows
+    kFastV2R2N4 = 7,    // K = 4096, 4 rows (tail tiles)
+    kFastV1R4N4 = 8,    // K = 2048, 4 rows (tail tiles)
+    kFastV7S4N1 = 9,    // K = 14336, 1 row (tail tiles)
 };
 
 // The variant for a GEMV tile of `rows` rows per weight block, `nblk` blocks, K columns.
@@ -57,10 +60,13 @@ inline uint8_t fast_path_for(int K, int rows, int nblk) {
         if (vpt == 2 && rps == 2 && total == 8) return kFastV2R2N8;
         if (vpt == 1 && rps == 4 && total == 16) return kFastV1R4N16;
         if (vpt == 1 && rps == 4 && total == 8) return kFastV1R4N8;
+        if (vpt == 2 && rps == 2 && total == 4) return kFastV2R2N4;
+        if (vpt == 1 && rps == 4 && total == 4) return kFastV1R4N4;
         return kFastNone;
     }
     if (vpt == 7 && total == 4) return kFastV7S4N4;
     if (vpt == 7 && total == 2) return kFastV7S4N2;
+    if (vpt == 7 && total == 1) return kFastV7S4N1;
     return kFastNone;
 }
 

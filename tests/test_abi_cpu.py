@@ -95,9 +95,22 @@ def test_plan_dependency_granularity_8b():
     # each kv head waits on its own event (only its QKV tiles), not on the whole projection
     assert len({t.wait[0] for t in attn}) == syn.LLAMA8B.n_kv_heads
     qkv_tiles = [t for t in tasks if t.op == mk.MK_OP_QKV and t.layer == 3]
-    per_head = [thr[t.wait[0]] for t in attn]
-    rows = qkv_tiles[0].r1 - qkv_tiles[0].r0
-    assert all(p == (4 * 128 + 2 * 128) // rows for p in per_head)
+    # the threshold of a kv head's event counts exactly the QKV tiles over its
+    # q, k and v rows
+    nq, nkv, hd = syn.LLAMA8B.n_q_heads, syn.LLAMA8B.n_kv_heads, syn.LLAMA8B.head_dim
+    hpg = nq // nkv
+    for t in attn:
+        g = t.aux
+        spans = [(g * hpg * hd, (g + 1) * hpg * hd), (nq * hd + g * hd, nq * hd + (g + 1) * hd),
+                 ((nq + nkv) * hd + g * hd, (nq + nkv) * hd + (g + 1) * hd)]
+        mine = [q for q in qkv_tiles if any(a <= q.r0 and q.r1 <= b for a, b in spans)]
+        assert sum(q.r1 - q.r0 for q in mine) == (hpg + 2) * hd
+        assert thr[t.wait[0]] == len(mine)
+        assert {q.signal for q in mine} == {t.wait[0]}
+    # QKV tiles are listed one KV group at a time (q heads, then k, then v rows)
+    first_row = [t.r0 for t in qkv_tiles]
+    group_of = [r // (hpg * hd) if r < nq * hd else (r - nq * hd) // hd % nkv for r in first_row]
+    assert group_of == sorted(group_of)
     # the dense GEMV operators cover the SMs at least once
     for op in (mk.MK_OP_QKV, mk.MK_OP_OPROJ, mk.MK_OP_GATEUP, mk.MK_OP_DOWN, mk.MK_OP_LMHEAD):
         n = sum(1 for t in tasks if t.op == op and t.layer in (0, 32))
