@@ -46,8 +46,9 @@ struct mk_state {
     uint32_t* done = nullptr;
     int* err = nullptr;
     uint32_t* router_cnt = nullptr;
+    uint32_t* attn_cnt = nullptr;
     float *x_mid = nullptr, *x_out = nullptr, *qkv = nullptr, *act = nullptr;
-    float *part = nullptr, *rlogits = nullptr, *moe_w = nullptr, *ypart = nullptr;
+    float *part = nullptr, *attn_o = nullptr, *rlogits = nullptr, *moe_w = nullptr, *ypart = nullptr;
     int* moe_sel = nullptr;
     int32_t* tokpos = nullptr;     // host-input variant: [2][max_batch]
     float* logits = nullptr;       // host-output variant: [max_batch][vocab]
@@ -106,6 +107,9 @@ mk_status reset_counters(mk_state* s, cudaStream_t st) {
     if (e == cudaSuccess) e = cudaMemsetAsync(s->done, 0, sizeof(uint32_t), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(s->err, 0, sizeof(int) * 8, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(s->router_cnt, 0, sizeof(uint32_t) * d.n_layers, st);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(s->attn_cnt, 0,
+                            sizeof(uint32_t) * d.n_layers * s->g->plan.max_batch * d.n_kv_heads, st);
     if (e != cudaSuccess) return cuda_fail(e, "reset");
     s->epoch = 0;
     s->needs_reset = false;
@@ -140,6 +144,7 @@ mk::Params base_params(mk_state* s) {
     p.done = s->done;
     p.err = s->err;
     p.router_cnt = s->router_cnt;
+    p.attn_cnt = s->attn_cnt;
     p.timeout_ns = s->timeout_ns;
     p.wait_offset = s->wait_offset;
     p.trace = s->trace;
@@ -171,6 +176,7 @@ mk::Params base_params(mk_state* s) {
     p.qkv = s->qkv;
     p.act = s->act;
     p.part = s->part;
+    p.attn_o = s->attn_o;
     p.rlogits = s->rlogits;
     p.moe_w = s->moe_w;
     p.moe_sel = s->moe_sel;
@@ -424,6 +430,7 @@ mk_status mk_state_create(mk_graph* g, mk_state** out) {
     ALLOC(done, 1);
     ALLOC(err, 8);
     ALLOC(router_cnt, L);
+    ALLOC(attn_cnt, L * B * d.n_kv_heads);
     ALLOC(x_mid, L * B * H);
     ALLOC(x_out, L * B * H);
     ALLOC(qkv, L * B * qkvw);
@@ -437,6 +444,7 @@ mk_status mk_state_create(mk_graph* g, mk_state** out) {
         ALLOC(act, L * B * d.ffn);
     }
     ALLOC(part, L * B * d.n_kv_heads * P.S * hpg * (d.head_dim + 2));
+    ALLOC(attn_o, L * B * d.n_q_heads * d.head_dim);
     ALLOC(tokpos, 2 * B);
     ALLOC(logits, B * (size_t)d.vocab);
     if (d.flags & MK_FLAG_TRACE) ALLOC(trace, P.tasks.size() * 4);

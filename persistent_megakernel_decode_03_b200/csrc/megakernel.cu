@@ -172,6 +172,7 @@ struct __align__(128) Smem {
     Task ep_task[kRedBufs];                  // task record for the epilogue warp
     int ep_ti[kRedBufs];                     // its index (-1: end of work)
     float ep_resid[kRedBufs][kMaxTaskRows];  // residual rows (O-proj, down), loaded early by warp 0
+    int attn_last;                           // this CTA's attention split arrived last
     int flag[4];
 };
 
@@ -744,65 +745,47 @@ __device__ __forceinline__ float* attn_part_ml(const Params& p, size_t idx) {
     return p.part + (size_t)p.L * p.max_batch * p.nkv * p.S * hpg_of(p) * p.hd + 2 * idx;
 }
 
-// Input of the O-projection: the attention output, merged over the active splits
-// of every (sequence, kv head) in split order.  Eight consecutive columns lie in
-// one q head.  Up to kMergeFast splits are merged with every load in flight at
-// once; more splits take a second, looped pass.
-constexpr int kMergeFast = 8;
-__device__ __forceinline__ void load8_attn_merge(const Params& p, int l, int b, int col,
-                                                 float2 (&x)[4]) {
-    const int hd = p.hd, hpg = hpg_of(p);
-    const int head = col / hd, i = col % hd;
-    const int g = head / hpg, h = head % hpg;
+// The attention output of one (sequence, kv group): the active splits' partials
+// merged in split order (m* = max m_s; o = sum 2^(m_s - m*) o_s / sum 2^(m_s - m*) l_s,
+// the split-K merge of flash-decoding), normalised, for the group's q heads.  Run
+// once, by all consumer threads of the CTA whose split arrived last: the (m, l)
+// pairs go through shared memory in one parallel pass, then every thread merges
+// four consecutive columns of one head with all of its loads in flight.
+__device__ void attn_merge_group(const Params& p, Smem& sm, uint32_t& cph, int l, int b, int g) {
+    const int hd = p.hd, hpg = hpg_of(p), tid = threadIdx.x;
     int pos = position_of(p, b);
     if (pos < 0 || pos >= p.max_ctx) pos = 0;
-    const int sa = attn_active_splits(pos + 1, p.S);
-    const size_t i0 = attn_part_index(p, l, b, g, 0, h);
-    const size_t stride = (size_t)hpg;                  // next split, same head
-    float m[kMergeFast], ls[kMergeFast];
-    float4 oa[kMergeFast], ob[kMergeFast];
-#pragma unroll
-    for (int sp = 0; sp < kMergeFast; ++sp) {
-        if (sp < sa) {
-            const size_t idx = i0 + sp * stride;
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(attn_part_ml(p, idx)));
-            m[sp] = ml.x;
-            ls[sp] = ml.y;
-            oa[sp] = __ldcg(reinterpret_cast<const float4*>(attn_part_o(p, idx) + i));
-            ob[sp] = __ldcg(reinterpret_cast<const float4*>(attn_part_o(p, idx) + i + 4));
-        } else {
-            m[sp] = -INFINITY;
-            ls[sp] = 0.f;
-            oa[sp] = ob[sp] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int sa = attn_active_splits(pos + 1, p.S);      // (S + 1) * hpg floats fit the scratch
+    float* f = sm.attn;                                     // [sa][hpg] weights, then [hpg] 1/L
+    const size_t i0 = attn_part_index(p, l, b, g, 0, 0);   // split s, head h at i0 + s*hpg + h
+    for (int k = tid; k < sa * hpg; k += kConsumerThreads) f[k] = __ldcg(attn_part_ml(p, i0 + k));
+    csync(p, sm, cph);
+    if (tid < hpg) {
+        float M = -INFINITY;
+        for (int sp = 0; sp < sa; ++sp) M = fmaxf(M, f[sp * hpg + tid]);
+        float L = 0.0f;
+        for (int sp = 0; sp < sa; ++sp) {
+            const float mm = f[sp * hpg + tid];
+            const float w = (mm == -INFINITY) ? 0.0f : exp2f(mm - M);
+            L = fmaf(__ldcg(attn_part_ml(p, i0 + (size_t)sp * hpg + tid) + 1), w, L);
+            f[sp * hpg + tid] = w;
         }
+        f[sa * hpg + tid] = (L > 0.0f) ? 1.0f / L : 0.0f;
     }
-    float M = -INFINITY;
-#pragma unroll
-    for (int sp = 0; sp < kMergeFast; ++sp) M = fmaxf(M, m[sp]);
-    for (int sp = kMergeFast; sp < sa; ++sp) M = fmaxf(M, __ldcg(attn_part_ml(p, i0 + sp * stride)));
-    float L = 0.0f;
-    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int sp = 0; sp < kMergeFast; ++sp) {
-        const float f = (m[sp] == -INFINITY) ? 0.0f : exp2f(m[sp] - M);
-        L = fmaf(ls[sp], f, L);
-        o[0] = fmaf(oa[sp].x, f, o[0]); o[1] = fmaf(oa[sp].y, f, o[1]);
-        o[2] = fmaf(oa[sp].z, f, o[2]); o[3] = fmaf(oa[sp].w, f, o[3]);
-        o[4] = fmaf(ob[sp].x, f, o[4]); o[5] = fmaf(ob[sp].y, f, o[5]);
-        o[6] = fmaf(ob[sp].z, f, o[6]); o[7] = fmaf(ob[sp].w, f, o[7]);
+    csync(p, sm, cph);
+    float* out = p.attn_o + ((size_t)l * p.max_batch + b) * p.nq * hd + (size_t)g * hpg * hd;
+    for (int q = tid; q < hpg * hd / 4; q += kConsumerThreads) {
+        const int h = (q * 4) / hd, i = (q * 4) % hd;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int sp = 0; sp < sa; ++sp) {
+            const float w = f[sp * hpg + h];
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(attn_part_o(p, i0 + (size_t)sp * hpg + h) + i));
+            o.x = fmaf(v.x, w, o.x); o.y = fmaf(v.y, w, o.y); o.z = fmaf(v.z, w, o.z); o.w = fmaf(v.w, w, o.w);
+        }
+        const float inv = f[sa * hpg + h];
+        *reinterpret_cast<float4*>(out + (size_t)h * hd + i) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
     }
-    for (int sp = kMergeFast; sp < sa; ++sp) {
-        const size_t idx = i0 + sp * stride;
-        const float mm = __ldcg(attn_part_ml(p, idx));
-        if (mm == -INFINITY) continue;
-        const float f = exp2f(mm - M);
-        L = fmaf(__ldcg(attn_part_ml(p, idx) + 1), f, L);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = fmaf(__ldcg(attn_part_o(p, idx) + i + e), f, o[e]);
-    }
-    const float inv = 1.0f / L;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] = make_float2(o[2 * e] * inv, o[2 * e + 1] * inv);
 }
 
 // Where a GEMV task's input vector lives: an fp32 row, a bf16 embedding row, and
@@ -840,7 +823,7 @@ __device__ __forceinline__ InSrc gemv_src(const Params& p, const Task& t) {
     switch (t.op) {
         case MK_OP_QKV: return xin_src(p, l, 0);
         case MK_OP_LMHEAD: return xin_src(p, p.L, 0);
-        case MK_OP_OPROJ: break;   // merged from the attention partials (load8_attn_merge)
+        case MK_OP_OPROJ: s.base = p.attn_o + ((size_t)l * p.max_batch) * p.nq * p.hd; break;
         case MK_OP_GATEUP:
         case MK_OP_ROUTER: s.base = p.x_mid + ((size_t)l * p.max_batch) * p.H; break;
         case MK_OP_EXP_GATEUP: s.base = p.x_mid + ((size_t)l * p.max_batch + b) * p.H; break;
@@ -927,35 +910,6 @@ __device__ void gemv_prologue_t(const Params& p, Smem& sm, uint32_t& cph, const 
 __device__ __forceinline__ void gemv_prologue(const Params& p, Smem& sm, uint32_t& cph, const Task& t,
                                               const ThreadMap& m, int K,
                                               float2 (&xr)[kMaxVecPerThread][4]) {
-    if (t.op == MK_OP_OPROJ) {
-        // merged attention output -> shared memory (K <= the scratch size) -> registers
-        float* ob = sm.attn;
-        csync(p, sm, cph);                       // the scratch is free
-#pragma unroll 2
-        for (int v = threadIdx.x; v < K / 8; v += kConsumerThreads) {
-            float2 x[4];
-            load8_attn_merge(p, t.layer, 0, v * 8, x);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                ob[v * 8 + 2 * e] = x[e].x;
-                ob[v * 8 + 2 * e + 1] = x[e].y;
-            }
-        }
-        csync(p, sm, cph);
-#pragma unroll
-        for (int j = 0; j < kMaxVecPerThread; ++j) {
-            const int v = m.lig + j * m.gstride;
-            if (j < m.vpt && v < m.nvec && m.active) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) xr[j][e] = make_float2(ob[v * 8 + 2 * e], ob[v * 8 + 2 * e + 1]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) xr[j][e] = make_float2(0.0f, 0.0f);
-            }
-        }
-        csync(p, sm, cph);                       // everyone has its slice
-        return;
-    }
     const InSrc src = gemv_src(p, t);
     if (src.nparts > 0) gemv_prologue_t<true>(p, sm, cph, t, m, K, src, xr);
     else gemv_prologue_t<false>(p, sm, cph, t, m, K, src, xr);
@@ -1506,6 +1460,18 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
             else attn_part_o(p, pidx)[c - 2] = val;
         }
     }
+    // arrival of this split (active or not); the split that arrives last for its
+    // (sequence, kv group) merges the partials once, before its completion is signalled
+    __threadfence();
+    csync(p, sm, cph);
+    if (tid == 0) {
+        const uint32_t old = atomicAdd(p.attn_cnt + ((size_t)l * p.max_batch + b) * p.nkv + g, 1u);
+        __threadfence();
+        sm.attn_last = (old == (uint32_t)S * p.epoch - 1u) ? 1 : 0;
+    }
+    csync(p, sm, cph);
+    if (sm.flag[3]) { abort_all = true; return; }
+    if (sm.attn_last && active_row) attn_merge_group(p, sm, cph, l, b, g);
 }
 
 // ----------------------------------------------------------------------------- consumer: router top-k

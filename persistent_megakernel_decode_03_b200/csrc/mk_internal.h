@@ -122,6 +122,7 @@ struct Params {
     uint32_t* done;              // completed-task counter
     int* err;                    // [0] status, [1..4] info
     uint32_t* router_cnt;        // [L] router tile arrivals
+    uint32_t* attn_cnt;          // [L][B][nkv] attention split arrivals (the last one merges)
     long long timeout_ns;
     uint32_t wait_offset;        // added to every wait target (0; tests set 1 to force a timeout)
     unsigned long long* trace;   // [n_tasks][4] or null
@@ -143,6 +144,7 @@ struct Params {
     float* qkv;      // [L][B][(nq+2nkv)*hd]
     float* act;      // dense: [L][B][F]; MoE: [L][B][topk][Fe]
     float* part;     // attention split partials: o [L][B][nkv][S][hpg][hd], then (m, l) pairs
+    float* attn_o;   // [L][B][nq*hd] attention output, the splits merged and normalised
     float* rlogits;  // [L][B][E]
     float* moe_w;    // [L][B][topk]
     int* moe_sel;    // [L][B][topk]

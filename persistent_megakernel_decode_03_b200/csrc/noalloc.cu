@@ -24,9 +24,9 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 struct Layout {
-    size_t tasks, thr, rope, layers, events, queue, done, err, router_cnt;
-    size_t x_mid, x_out, qkv, act, part, rlogits, moe_w, moe_sel, ypart, end;
-    size_t counters_begin, counters_end;   // [events .. router_cnt] is cleared every call
+    size_t tasks, thr, rope, layers, events, queue, done, err, router_cnt, attn_cnt;
+    size_t x_mid, x_out, qkv, act, part, attn_o, rlogits, moe_w, moe_sel, ypart, end;
+    size_t counters_begin, counters_end;   // [events .. attn_cnt] is cleared every call
 };
 
 struct DeviceCache {
@@ -61,6 +61,7 @@ Layout make_layout(const mk::GraphPlan& P) {
     o.done = take(sizeof(uint32_t));
     o.err = take(8 * sizeof(int));
     o.router_cnt = take(sizeof(uint32_t) * L);
+    o.attn_cnt = take(sizeof(uint32_t) * L * B * d.n_kv_heads);
     o.counters_end = at;
     o.x_mid = take(sizeof(float) * L * B * H);
     o.x_out = take(sizeof(float) * L * B * H);
@@ -76,6 +77,7 @@ Layout make_layout(const mk::GraphPlan& P) {
         o.rlogits = o.moe_w = o.moe_sel = o.ypart = 0;
     }
     o.part = take(sizeof(float) * L * B * d.n_kv_heads * P.S * hpg * (d.head_dim + 2));
+    o.attn_o = take(sizeof(float) * L * B * d.n_q_heads * d.head_dim);
     o.end = at;
     return o;
 }
@@ -212,6 +214,7 @@ extern "C" mk_status mk_decode_step_noalloc(const mk_model_desc* desc, const voi
     p.done = reinterpret_cast<uint32_t*>(b + lay.done);
     p.err = reinterpret_cast<int*>(b + lay.err);
     p.router_cnt = reinterpret_cast<uint32_t*>(b + lay.router_cnt);
+    p.attn_cnt = reinterpret_cast<uint32_t*>(b + lay.attn_cnt);
     p.timeout_ns = 2000000000LL;
     p.layers = reinterpret_cast<const mk::LayerW*>(b + lay.layers);
     p.tok_emb = static_cast<const uint16_t*>(weight_ptrs[0]);
@@ -227,6 +230,7 @@ extern "C" mk_status mk_decode_step_noalloc(const mk_model_desc* desc, const voi
     p.qkv = reinterpret_cast<float*>(b + lay.qkv);
     p.act = reinterpret_cast<float*>(b + lay.act);
     p.part = reinterpret_cast<float*>(b + lay.part);
+    p.attn_o = reinterpret_cast<float*>(b + lay.attn_o);
     if (d.n_experts > 0) {
         p.rlogits = reinterpret_cast<float*>(b + lay.rlogits);
         p.moe_w = reinterpret_cast<float*>(b + lay.moe_w);
