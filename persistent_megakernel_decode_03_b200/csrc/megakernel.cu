@@ -153,6 +153,12 @@ constexpr int kAttnScratch = kConsumerWarps * kMaxHeadsPerGroup * (128 + 2);   /
 // Rotating buffer sets (row sums, task record, residual rows) between the consumer
 // warps and the epilogue warp: consumers may run kRedBufs - 1 tasks ahead of it.
 constexpr int kRedBufs = 4;
+// Page ids the producer reads ahead for an attention split: batches of 16, loaded
+// when fewer than 16 ids beyond the current stage remain; the ring keeps up to 31
+// ids ahead plus the current stage's (<= 4), so 64 entries never overwrite an id
+// still in use.
+constexpr int kPidBatch = 16;
+constexpr int kPidRing = 4 * kPidBatch;
 
 struct __align__(128) Smem {
     uint8_t ring[kStages][kStageBytes];
@@ -173,6 +179,7 @@ struct __align__(128) Smem {
     int ep_ti[kRedBufs];                     // its index (-1: end of work)
     float ep_resid[kRedBufs][kMaxTaskRows];  // residual rows (O-proj, down), loaded early by warp 0
     int attn_last;                           // this CTA's attention split arrived last
+    int pid[kPidRing];                       // producer: physical page ids read ahead
     int flag[4];
 };
 
@@ -446,18 +453,35 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                 mbar_arrive(&sm.full[stage]);
                 advance();
             }
+            // physical page ids, read kPidBatch at a time (independent loads, one round
+            // trip per batch) into a small ring in shared memory, a batch ahead of use
+            const int* prow = p.page_table + (size_t)b * p.max_pages;
+            int pid_have = 0;                              // ids [0, pid_have) of the split loaded
+            auto pid_ensure = [&](int upto) {
+                while (pid_have < upto) {
+                    int v[kPidBatch];
+#pragma unroll
+                    for (int i = 0; i < kPidBatch; ++i) {
+                        const int k = pid_have + i;
+                        v[i] = (k < npages) ? __ldg(prow + lp0 + k) : 0;
+                    }
+#pragma unroll
+                    for (int i = 0; i < kPidBatch; ++i) sm.pid[(pid_have + i) % kPidRing] = v[i];
+                    pid_have += kPidBatch;
+                }
+            };
             for (int c = 0; c < nch && ok; ++c) {
-                if (!acquire_slot()) { ok = false; break; }
                 int first = lp0 + c * pps;
                 int n = min(pps, lp0 + npages - first);
+                pid_ensure(min(npages, c * pps + n + kPidBatch));
+                if (!acquire_slot()) { ok = false; break; }
                 sm.info[stage].task = ti; sm.info[stage].chunk = c; sm.info[stage].nchunks = nch;
                 sm.info[stage].aux = first;
                 if (c == 0) sm.info[stage].rec = t;
                 // validate page indices before issuing any copy
-                const int* prow = p.page_table + (size_t)b * p.max_pages;
                 bool bad = false;
                 for (int i = 0; i < n; ++i) {
-                    int ph = prow[first + i];
+                    int ph = sm.pid[(c * pps + i) % kPidRing];
                     if (ph < 0 || ph >= p.n_pages) bad = true;
                 }
                 if (bad) {
@@ -468,7 +492,7 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                 }
                 mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)n * 2u * blk);
                 for (int i = 0; i < n; ++i) {
-                    int ph = prow[first + i];
+                    int ph = sm.pid[(c * pps + i) % kPidRing];
                     size_t off = (((size_t)t.layer * p.n_pages + ph) * p.nkv + t.aux) * (size_t)kPageSize * p.hd;
                     uint8_t* dst = sm.ring[stage] + (size_t)i * 2 * blk;
                     bulk_g2s(dst, p.k_pages + off, blk, &sm.full[stage], pol);
@@ -1214,55 +1238,6 @@ struct AttnState {
     float m[HPG], l[HPG];
 };
 
-// T tokens at once: the T*HPG partial dot products are summed over the warp
-// together (independent shuffle chains), then one online-softmax update per head.
-// ok[t] masks tokens beyond the range.
-template <int HPG, int DPL, int T>
-__device__ __forceinline__ void attn_tokens(AttnState<HPG, DPL>& st, const float (&k)[T][DPL],
-                                            const float (&v)[T][DPL], const bool (&ok)[T]) {
-    float sc[T][HPG];
-#pragma unroll
-    for (int t = 0; t < T; ++t)
-#pragma unroll
-        for (int h = 0; h < HPG; ++h) {
-            float a = 0.0f;
-#pragma unroll
-            for (int d = 0; d < DPL; ++d) a = fmaf(st.q[h][d], k[t][d], a);
-            sc[t][h] = a;
-        }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int t = 0; t < T; ++t)
-#pragma unroll
-            for (int h = 0; h < HPG; ++h) sc[t][h] += __shfl_xor_sync(0xFFFFFFFFu, sc[t][h], o);
-#pragma unroll
-    for (int h = 0; h < HPG; ++h) {
-        float mx = st.m[h];
-#pragma unroll
-        for (int t = 0; t < T; ++t)
-            if (ok[t]) mx = fmaxf(mx, sc[t][h]);
-        if (mx == -INFINITY) continue;                   // no token yet
-        const float corr = exp2f(st.m[h] - mx);          // 0 when m was -inf
-        float pw[T];
-        float ps = 0.0f;
-#pragma unroll
-        for (int t = 0; t < T; ++t) {
-            pw[t] = ok[t] ? exp2f(sc[t][h] - mx) : 0.0f;
-            ps += pw[t];
-        }
-        st.l[h] = fmaf(st.l[h], corr, ps);
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) {
-            float acc = st.o[h][d] * corr;
-#pragma unroll
-            for (int t = 0; t < T; ++t) acc = fmaf(pw[t], v[t][d], acc);
-            st.o[h][d] = acc;
-        }
-        st.m[h] = mx;
-    }
-}
-
 template <int DPL>
 __device__ __forceinline__ void load_bf16_dpl(const uint16_t* src, float (&out)[DPL]) {
     if (DPL == 4) {
@@ -1275,6 +1250,104 @@ __device__ __forceinline__ void load_bf16_dpl(const uint16_t* src, float (&out)[
     }
 }
 
+// One page (16 tokens) of one kv head.  Every lane forms the partial dot products
+// of its DPL dims with all 16 keys; one reduce-scatter per head sums them over the
+// warp (lanes 2t and 2t+1 end up with token t's score: 15 shuffles per 16 tokens
+// instead of 5 per token).  Block-wise online softmax (one rescale per page), then
+// the probabilities go through shared memory to every lane for P.V over its dims.
+// Tokens outside [k_lo, k_hi) are masked (their scores, and their values, which
+// may be stale cache contents).  st.l holds per-lane partial sums (summed over the
+// warp at the end).
+template <int HPG, int DPL>
+__device__ __forceinline__ void attn_page(AttnState<HPG, DPL>& st, const uint16_t* kblk, const uint16_t* vblk,
+                                          int k_lo, int k_hi, float* pbuf) {
+    constexpr int HD = DPL * 32;
+    const int lane = threadIdx.x & 31;
+    const int my_t = lane >> 1;                            // the token whose score this lane receives
+    const bool my_ok = my_t >= k_lo && my_t < k_hi;
+    float kf[kPageSize][DPL];
+#pragma unroll
+    for (int t = 0; t < kPageSize; ++t) load_bf16_dpl<DPL>(kblk + t * HD + lane * DPL, kf[t]);
+    float pm[HPG];
+#pragma unroll
+    for (int h = 0; h < HPG; ++h) {
+        float part[kPageSize];
+#pragma unroll
+        for (int t = 0; t < kPageSize; ++t) {
+            float a = 0.0f;
+#pragma unroll
+            for (int d = 0; d < DPL; ++d) a = fmaf(st.q[h][d], kf[t][d], a);
+            part[t] = a;
+        }
+        // every lane takes part in the full-warp shuffles; masking comes after
+        float sc = warp_reduce_rows<kPageSize>(part);
+        sc = my_ok ? sc : -INFINITY;
+        float mb = sc;
+#pragma unroll
+        for (int o = 16; o > 1; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+        const float m_new = fmaxf(st.m[h], mb);            // warp-uniform
+        float pv = 0.0f;
+        if (m_new != -INFINITY) {
+            const float corr = exp2f(st.m[h] - m_new);      // 0 while m was -inf
+            pv = my_ok ? exp2f(sc - m_new) : 0.0f;
+            st.l[h] = fmaf(st.l[h], corr, (lane & 1) ? 0.0f : pv);
+#pragma unroll
+            for (int d = 0; d < DPL; ++d) st.o[h][d] *= corr;
+            st.m[h] = m_new;
+        }
+        pm[h] = pv;
+    }
+    if ((lane & 1) == 0) {
+#pragma unroll
+        for (int h = 0; h < HPG; ++h) pbuf[h * kPageSize + my_t] = pm[h];
+    }
+    __syncwarp();
+    float vf[kPageSize][DPL];
+#pragma unroll
+    for (int t = 0; t < kPageSize; ++t) {
+        load_bf16_dpl<DPL>(vblk + t * HD + lane * DPL, vf[t]);
+        const bool ok = t >= k_lo && t < k_hi;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) vf[t][d] = ok ? vf[t][d] : 0.0f;
+    }
+#pragma unroll
+    for (int h = 0; h < HPG; ++h) {
+        const float4* pb = reinterpret_cast<const float4*>(pbuf + h * kPageSize);
+#pragma unroll
+        for (int q4 = 0; q4 < kPageSize / 4; ++q4) {
+            const float4 pq = pb[q4];
+            const float pr[4] = {pq.x, pq.y, pq.z, pq.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int d = 0; d < DPL; ++d) st.o[h][d] = fmaf(pr[u], vf[q4 * 4 + u][d], st.o[h][d]);
+        }
+    }
+    __syncwarp();                                          // pbuf is reused by the next page
+}
+
+// The new token (not yet in the streamed pages), by one warp: full-warp dot
+// products and one online-softmax update per head (per-lane partial l as above).
+template <int HPG, int DPL>
+__device__ __forceinline__ void attn_new_token(AttnState<HPG, DPL>& st, const float (&kf)[DPL],
+                                               const float (&vf)[DPL]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int h = 0; h < HPG; ++h) {
+        float a = 0.0f;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) a = fmaf(st.q[h][d], kf[d], a);
+        const float sc = warp_sum(a);
+        const float m_new = fmaxf(st.m[h], sc);
+        const float corr = exp2f(st.m[h] - m_new);
+        const float pv = exp2f(sc - m_new);
+        st.l[h] = fmaf(st.l[h], corr, lane == 0 ? pv : 0.0f);
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) st.o[h][d] = fmaf(pv, vf[d], st.o[h][d] * corr);
+        st.m[h] = m_new;
+    }
+}
+
 // One split of decode attention for (layer, sequence b, kv head g): RoPE on the
 // group's q heads and the new k, KV-cache append (the split that owns the new
 // position), softmax partial over the split's positions streamed from the paged
@@ -1284,7 +1357,6 @@ template <int HPG, int DPL>
 __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti, int& stage,
                                uint32_t& lap, bool& abort_all) {
     constexpr int HD = DPL * 32;
-    constexpr int TB = (HPG >= 8) ? 2 : 4;               // tokens per warp step
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = t.b, g = t.aux, s = (int)t.r0, S = (int)t.r1, l = t.layer;
     const bool active_row = b < p.batch;
@@ -1373,6 +1445,7 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
     const int jc = min(j1, pos);
     const int pps = pages_per_stage(p);
     const int blk_elems = kPageSize * HD;
+    float* pbuf = sm.attn + warp * HPG * kPageSize;      // this warp's page probabilities
     for (int c = 0;; ++c) {
         if (c == 0) {
             seen_complete_wait(p, &sm.full[stage], lap & 1, &sm.flag[3]);
@@ -1391,20 +1464,15 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
             const int first_page = inf.aux;
             const int tok_lo = max(j0, first_page * kPageSize);
             const int tok_hi = min(jc, (first_page + pps) * kPageSize);
-            for (int t0 = tok_lo + warp * TB; t0 < tok_hi; t0 += kConsumerWarps * TB) {
-                float kf[TB][DPL], vf[TB][DPL];
-                bool ok[TB];
-#pragma unroll
-                for (int u = 0; u < TB; ++u) {
-                    const int pt = t0 + u;
-                    ok[u] = pt < tok_hi;
-                    const int ptc = ok[u] ? pt : t0;
-                    const int pi = ptc / kPageSize - first_page, slot = ptc % kPageSize;
-                    const uint16_t* kb = base + (size_t)pi * 2 * blk_elems + slot * HD + lane * DPL;
-                    load_bf16_dpl<DPL>(kb, kf[u]);
-                    load_bf16_dpl<DPL>(kb + blk_elems, vf[u]);
-                }
-                attn_tokens<HPG, DPL, TB>(st, kf, vf, ok);
+            // pages are dealt to the warps round-robin over the whole stream
+#pragma unroll 1
+            for (int pi = 0; pi < pps; ++pi) {
+                if (((inf.chunk * pps + pi) & (kConsumerWarps - 1)) != warp) continue;
+                const int pf = (first_page + pi) * kPageSize;
+                const int k_lo = max(tok_lo - pf, 0), k_hi = min(tok_hi - pf, kPageSize);
+                if (k_hi <= k_lo) continue;
+                const uint16_t* kb = base + (size_t)pi * 2 * blk_elems;
+                attn_page<HPG, DPL>(st, kb, kb + blk_elems, k_lo, k_hi, pbuf);
             }
         }
         __syncwarp();
@@ -1414,15 +1482,17 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
         if (last) break;
     }
     if (has_new && warp == 0) {
-        float kf[1][DPL], vf[1][DPL];
-        const bool ok[1] = {true};
+        float kf[DPL], vf[DPL];
 #pragma unroll
         for (int d = 0; d < DPL; ++d) {
-            kf[0][d] = sm.kn[lane * DPL + d];
-            vf[0][d] = sm.vn[lane * DPL + d];
+            kf[d] = sm.kn[lane * DPL + d];
+            vf[d] = sm.vn[lane * DPL + d];
         }
-        attn_tokens<HPG, DPL, 1>(st, kf, vf, ok);
+        attn_new_token<HPG, DPL>(st, kf, vf);
     }
+#pragma unroll
+    for (int h = 0; h < HPG; ++h) st.l[h] = warp_sum(st.l[h]);
+    csync(p, sm, cph);                                   // every warp is done with its pbuf
     // combine the warps' partials (fixed order) into this split's partial
     float* sc = sm.attn;
 #pragma unroll
