@@ -134,9 +134,10 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     const int64_t qkv_rows = (int64_t)(nq + 2 * nkv) * hd;
     const int64_t target = 128 * 1024;
 
-    // attention split-K: enough (sequence, kv head, split) tasks to cover the SMs,
-    // but at most one split per 64 positions of context.
-    int S = (int)ceil_div(n_sm, (int64_t)B * nkv);
+    // attention split-K: as many (sequence, kv head, split) tasks as fit in one wave
+    // over the SMs (one more would make every layer's attention phase take two
+    // task durations), but at most one split per 64 positions of context.
+    int S = n_sm / (B * nkv);
     S = std::max(1, std::min<int>(S, (int)ceil_div(max_ctx, 64)));
     g.S = S;
 

@@ -153,11 +153,11 @@ constexpr int kAttnScratch = kConsumerWarps * kMaxHeadsPerGroup * (128 + 2);   /
 // Rotating buffer sets (row sums, task record, residual rows) between the consumer
 // warps and the epilogue warp: consumers may run kRedBufs - 1 tasks ahead of it.
 constexpr int kRedBufs = 4;
-// Page ids the producer reads ahead for an attention split: batches of 16, loaded
-// when fewer than 16 ids beyond the current stage remain; the ring keeps up to 31
-// ids ahead plus the current stage's (<= 4), so 64 entries never overwrite an id
+// Page ids the producer reads ahead for an attention split: batches of 8, loaded
+// when fewer than 8 ids beyond the current stage remain; the ring keeps up to 15
+// ids ahead plus the current stage's (<= 4), so 32 entries never overwrite an id
 // still in use.
-constexpr int kPidBatch = 16;
+constexpr int kPidBatch = 8;
 constexpr int kPidRing = 4 * kPidBatch;
 
 struct __align__(128) Smem {
@@ -1231,121 +1231,203 @@ __device__ __forceinline__ bool gemv_task_dispatch(const Params& p, Smem& sm, in
 
 // ----------------------------------------------------------------------------- consumer: attention
 
+
+// ---- attention on the tensor cores (mma.sync m16n8k16, bf16 inputs, fp32 accumulators)
+//
+// Scores S = Q K^T and the output O = P V of one kv group, 16 tokens (one page) at a
+// time.  The A operand has 16 rows: rows 0..7 carry the bf16 value of q (or of the
+// probabilities p) of head h = row, rows 8..15 the bf16 rounding residual of the
+// same values, so one MMA yields hi and lo products whose sum is the fp32
+// product to about 2^-16 relative; each result row h is then the sum of rows h
+// and h + 8.  Rows of heads >= HPG are zero.  Keys and values are bf16 already.
+// A page is first copied by its warp into a per-warp staging buffer with its
+// 16-byte chunks XOR-swizzled by row, so that the ldmatrix loads that gather MMA
+// operands across 8 tokens hit 8 different bank groups.
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    return (uint32_t)f32_to_bf16_rne(lo) | ((uint32_t)f32_to_bf16_rne(hi) << 16);
+}
+// hi and lo parts of a pair of fp32 values as two bf16x2 words
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const uint16_t ha = f32_to_bf16_rne(a), hb = f32_to_bf16_rne(b);
+    hi = (uint32_t)ha | ((uint32_t)hb << 16);
+    lo = pack_bf16x2(a - bf16_to_f32(ha), b - bf16_to_f32(hb));
+}
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+
 template <int HPG, int DPL>
-struct AttnState {
-    float q[HPG][DPL];
-    float o[HPG][DPL];
-    float m[HPG], l[HPG];
+struct AttnMma {
+    static constexpr int HD = DPL * 32, KS = HD / 16, NT = HD / 8;
+    uint32_t qa[KS][4];   // A fragments of q (rows 0..7 hi, 8..15 lo)
+    float o[NT][4];       // accumulator fragments of P V
+    float m, l;           // running max (log2 domain) and partial sum of this thread's row
 };
 
-template <int DPL>
-__device__ __forceinline__ void load_bf16_dpl(const uint16_t* src, float (&out)[DPL]) {
-    if (DPL == 4) {
-        uint2 u = *reinterpret_cast<const uint2*>(src);
-        out[0] = bf_lo(u.x); out[1] = bf_hi(u.x);
-        out[2 % DPL] = bf_lo(u.y); out[3 % DPL] = bf_hi(u.y);
-    } else {
-        uint32_t u = *reinterpret_cast<const uint32_t*>(src);
-        out[0] = bf_lo(u); out[1 % DPL] = bf_hi(u);
+// Byte offset of 16-byte chunk c of token row r in a swizzled staging page.
+template <int HD>
+__device__ __forceinline__ uint32_t stg_off(int r, int c) {
+    return (uint32_t)(r * HD * 2 + 16 * (c ^ (r & 7)));
+}
+
+// Copies one 16 x HD bf16 page block from the ring into the warp's staging buffer,
+// swizzled; with `zero_out` the rows outside [k_lo, k_hi) become zeros (values of
+// masked tokens must not reach P V, whatever the cache holds there).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// (shared-memory addresses throughout: the ring and the staging page are both in
+// this CTA's shared memory)
+template <int HD>
+__device__ __forceinline__ void stage_page(const uint16_t* src, uint8_t* stg, int k_lo, int k_hi, bool zero_out) {
+    constexpr int CPR = HD / 8;                         // 16-byte chunks per row
+    const int lane = threadIdx.x & 31;
+    const uint32_t s0 = smem_u32(src), d0 = smem_u32(stg);
+    uint4 v[kPageSize * CPR / 32];
+#pragma unroll
+    for (int i = 0; i < kPageSize * CPR / 32; ++i) v[i] = lds128(s0 + 16u * (lane + 32 * i));
+#pragma unroll
+    for (int i = 0; i < kPageSize * CPR / 32; ++i) {
+        const int q = lane + 32 * i, r = q / CPR, c = q % CPR;
+        if (zero_out && (r < k_lo || r >= k_hi)) v[i] = make_uint4(0u, 0u, 0u, 0u);
+        sts128(d0 + stg_off<HD>(r, c), v[i]);
     }
 }
 
-// One page (16 tokens) of one kv head.  Every lane forms the partial dot products
-// of its DPL dims with all 16 keys; one reduce-scatter per head sums them over the
-// warp (lanes 2t and 2t+1 end up with token t's score: 15 shuffles per 16 tokens
-// instead of 5 per token).  Block-wise online softmax (one rescale per page), then
-// the probabilities go through shared memory to every lane for P.V over its dims.
-// Tokens outside [k_lo, k_hi) are masked (their scores, and their values, which
-// may be stale cache contents).  st.l holds per-lane partial sums (summed over the
-// warp at the end).
+// S (two n-tiles of 8 tokens) = Q K^T for the staged page.
 template <int HPG, int DPL>
-__device__ __forceinline__ void attn_page(AttnState<HPG, DPL>& st, const uint16_t* kblk, const uint16_t* vblk,
-                                          int k_lo, int k_hi, float* pbuf) {
+__device__ __forceinline__ void attn_qk(const AttnMma<HPG, DPL>& st, const uint8_t* stg, float (&s0)[4],
+                                        float (&s1)[4]) {
+    constexpr int HD = DPL * 32, KS = HD / 16;
+    const int lane = threadIdx.x & 31, mi = lane >> 3, rr = lane & 7;
+    const int tok = rr + ((mi & 2) ? 8 : 0);
+    const uint32_t base = smem_u32(stg);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s0[e] = s1[e] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        uint32_t b[4];
+        ldsm_x4(b, base + stg_off<HD>(tok, 2 * ks + (mi & 1)));
+        mma_16816(s0, st.qa[ks], b[0], b[1]);
+        mma_16816(s1, st.qa[ks], b[2], b[3]);
+    }
+}
+
+// Online softmax over the page's 16 scores of this thread's row, then the
+// hi/lo A fragments of the probabilities.
+template <int HPG, int DPL>
+__device__ __forceinline__ void attn_softmax(AttnMma<HPG, DPL>& st, const float (&s0)[4], const float (&s1)[4],
+                                             int k_lo, int k_hi, uint32_t (&pa)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    float sc[4] = {s0[0] + s0[2], s0[1] + s0[3], s1[0] + s1[2], s1[1] + s1[3]};
+    const int tk[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (g >= HPG || tk[i] < k_lo || tk[i] >= k_hi) sc[i] = -INFINITY;
+    float mb = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
+    mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 2));
+    const float m_new = fmaxf(st.m, mb);
+    float pr[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (m_new != -INFINITY) {
+        const float corr = exp2f(st.m - m_new);         // 0 while m was -inf
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pr[i] = exp2f(sc[i] - m_new);
+        st.l = fmaf(st.l, corr, (pr[0] + pr[1]) + (pr[2] + pr[3]));
+#pragma unroll
+        for (int j = 0; j < AttnMma<HPG, DPL>::NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) st.o[j][e] *= corr;
+        st.m = m_new;
+    }
+    split_bf16x2(pr[0], pr[1], pa[0], pa[1]);
+    split_bf16x2(pr[2], pr[3], pa[2], pa[3]);
+}
+
+// O += P V for the staged page (values of masked tokens already zero).
+template <int HPG, int DPL>
+__device__ __forceinline__ void attn_pv(AttnMma<HPG, DPL>& st, const uint8_t* stg, const uint32_t (&pa)[4]) {
+    constexpr int HD = DPL * 32, NT = HD / 8;
+    const int lane = threadIdx.x & 31, mi = lane >> 3, rr = lane & 7;
+    const int tok = rr + ((mi & 1) ? 8 : 0);
+    const uint32_t base = smem_u32(stg);
+#pragma unroll
+    for (int jj = 0; jj < NT / 2; ++jj) {
+        uint32_t b[4];
+        ldsm_x4_trans(b, base + stg_off<HD>(tok, 2 * jj + ((mi & 2) ? 1 : 0)));
+        mma_16816(st.o[2 * jj], pa, b[0], b[1]);
+        mma_16816(st.o[2 * jj + 1], pa, b[2], b[3]);
+    }
+}
+
+// One cached page of the split (tokens [k_lo, k_hi) of it valid).
+template <int HPG, int DPL>
+__device__ __forceinline__ void attn_page(AttnMma<HPG, DPL>& st, const uint16_t* kblk, const uint16_t* vblk,
+                                          int k_lo, int k_hi, uint8_t* stg) {
     constexpr int HD = DPL * 32;
-    const int lane = threadIdx.x & 31;
-    const int my_t = lane >> 1;                            // the token whose score this lane receives
-    const bool my_ok = my_t >= k_lo && my_t < k_hi;
-    float kf[kPageSize][DPL];
-#pragma unroll
-    for (int t = 0; t < kPageSize; ++t) load_bf16_dpl<DPL>(kblk + t * HD + lane * DPL, kf[t]);
-    float pm[HPG];
-#pragma unroll
-    for (int h = 0; h < HPG; ++h) {
-        float part[kPageSize];
-#pragma unroll
-        for (int t = 0; t < kPageSize; ++t) {
-            float a = 0.0f;
-#pragma unroll
-            for (int d = 0; d < DPL; ++d) a = fmaf(st.q[h][d], kf[t][d], a);
-            part[t] = a;
-        }
-        // every lane takes part in the full-warp shuffles; masking comes after
-        float sc = warp_reduce_rows<kPageSize>(part);
-        sc = my_ok ? sc : -INFINITY;
-        float mb = sc;
-#pragma unroll
-        for (int o = 16; o > 1; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
-        const float m_new = fmaxf(st.m[h], mb);            // warp-uniform
-        float pv = 0.0f;
-        if (m_new != -INFINITY) {
-            const float corr = exp2f(st.m[h] - m_new);      // 0 while m was -inf
-            pv = my_ok ? exp2f(sc - m_new) : 0.0f;
-            st.l[h] = fmaf(st.l[h], corr, (lane & 1) ? 0.0f : pv);
-#pragma unroll
-            for (int d = 0; d < DPL; ++d) st.o[h][d] *= corr;
-            st.m[h] = m_new;
-        }
-        pm[h] = pv;
-    }
-    if ((lane & 1) == 0) {
-#pragma unroll
-        for (int h = 0; h < HPG; ++h) pbuf[h * kPageSize + my_t] = pm[h];
-    }
+    stage_page<HD>(kblk, stg, k_lo, k_hi, false);
     __syncwarp();
-    float vf[kPageSize][DPL];
-#pragma unroll
-    for (int t = 0; t < kPageSize; ++t) {
-        load_bf16_dpl<DPL>(vblk + t * HD + lane * DPL, vf[t]);
-        const bool ok = t >= k_lo && t < k_hi;
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) vf[t][d] = ok ? vf[t][d] : 0.0f;
-    }
-#pragma unroll
-    for (int h = 0; h < HPG; ++h) {
-        const float4* pb = reinterpret_cast<const float4*>(pbuf + h * kPageSize);
-#pragma unroll
-        for (int q4 = 0; q4 < kPageSize / 4; ++q4) {
-            const float4 pq = pb[q4];
-            const float pr[4] = {pq.x, pq.y, pq.z, pq.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int d = 0; d < DPL; ++d) st.o[h][d] = fmaf(pr[u], vf[q4 * 4 + u][d], st.o[h][d]);
-        }
-    }
-    __syncwarp();                                          // pbuf is reused by the next page
+    float s0[4], s1[4];
+    attn_qk<HPG, DPL>(st, stg, s0, s1);
+    uint32_t pa[4];
+    attn_softmax<HPG, DPL>(st, s0, s1, k_lo, k_hi, pa);
+    __syncwarp();                                        // every lane is done with the keys
+    stage_page<HD>(vblk, stg, k_lo, k_hi, true);
+    __syncwarp();
+    attn_pv<HPG, DPL>(st, stg, pa);
+    __syncwarp();                                        // staging is reused by the next page
 }
 
-// The new token (not yet in the streamed pages), by one warp: full-warp dot
-// products and one online-softmax update per head (per-lane partial l as above).
+// The new token (its k and v, bf16-rounded, in shared memory) as a one-token page.
 template <int HPG, int DPL>
-__device__ __forceinline__ void attn_new_token(AttnState<HPG, DPL>& st, const float (&kf)[DPL],
-                                               const float (&vf)[DPL]) {
+__device__ __forceinline__ void attn_new_token(AttnMma<HPG, DPL>& st, const float* kn, const float* vn,
+                                               uint8_t* stg) {
+    constexpr int HD = DPL * 32, CPR = HD / 8;
     const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int h = 0; h < HPG; ++h) {
-        float a = 0.0f;
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) a = fmaf(st.q[h][d], kf[d], a);
-        const float sc = warp_sum(a);
-        const float m_new = fmaxf(st.m[h], sc);
-        const float corr = exp2f(st.m[h] - m_new);
-        const float pv = exp2f(sc - m_new);
-        st.l[h] = fmaf(st.l[h], corr, lane == 0 ? pv : 0.0f);
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) st.o[h][d] = fmaf(pv, vf[d], st.o[h][d] * corr);
-        st.m[h] = m_new;
-    }
+    auto stage_row0 = [&](const float* x) {             // row 0 = x, rows 1..15 = 0
+        for (int q = lane; q < kPageSize * CPR; q += 32) {
+            const int r = q / CPR, c = q % CPR;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (r == 0) {
+                const float* e = x + 8 * c;
+                v = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
+                               pack_bf16x2(e[6], e[7]));
+            }
+            sts128(smem_u32(stg) + stg_off<HD>(r, c), v);
+        }
+    };
+    stage_row0(kn);
+    __syncwarp();
+    float s0[4], s1[4];
+    attn_qk<HPG, DPL>(st, stg, s0, s1);
+    uint32_t pa[4];
+    attn_softmax<HPG, DPL>(st, s0, s1, 0, 1, pa);
+    __syncwarp();
+    stage_row0(vn);
+    __syncwarp();
+    attn_pv<HPG, DPL>(st, stg, pa);
+    __syncwarp();
 }
 
 // One split of decode attention for (layer, sequence b, kv head g): RoPE on the
@@ -1371,14 +1453,17 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
     const bool has_new = valid && pos >= j0 && pos < j1;
     const float qscale = 1.4426950408889634f / sqrtf((float)HD);   // log2(e) / sqrt(d)
 
-    AttnState<HPG, DPL> st;
+    AttnMma<HPG, DPL> st;
+    st.m = -INFINITY;
+    st.l = 0.0f;
 #pragma unroll
-    for (int h = 0; h < HPG; ++h) {
-        st.m[h] = -INFINITY;
-        st.l[h] = 0.0f;
+    for (int j = 0; j < AttnMma<HPG, DPL>::NT; ++j)
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) st.o[h][d] = 0.0f;
-    }
+        for (int e = 0; e < 4; ++e) st.o[j][e] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < AttnMma<HPG, DPL>::KS; ++ks)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.qa[ks][e] = 0u;
     const bool work = valid && j1 > j0;
     csync(p, sm, cph);                                   // shared scratch of the previous task is free
     if (work) {
@@ -1435,17 +1520,24 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
                 set_error(p, kErrInvalid, ti, -2, pos / kPageSize, b);
             }
         }
+        // q as hi/lo bf16 A fragments: thread (g, t) holds head g's columns
+        // 16ks + 2t, +1, +8, +9 (rows of heads >= HPG stay zero)
+        const int g4 = lane >> 2, t4 = lane & 3;
+        if (g4 < HPG) {
 #pragma unroll
-        for (int h = 0; h < HPG; ++h)
-#pragma unroll
-            for (int d = 0; d < DPL; ++d) st.q[h][d] = sm.qs[h * HD + lane * DPL + d];
+            for (int ks = 0; ks < AttnMma<HPG, DPL>::KS; ++ks) {
+                const float* qh = sm.qs + g4 * HD + 16 * ks + 2 * t4;
+                split_bf16x2(qh[0], qh[1], st.qa[ks][0], st.qa[ks][1]);
+                split_bf16x2(qh[8], qh[9], st.qa[ks][2], st.qa[ks][3]);
+            }
+        }
     }
 
     // streamed chunks of cached pages (the first stage was seen complete by thread 0)
     const int jc = min(j1, pos);
     const int pps = pages_per_stage(p);
     const int blk_elems = kPageSize * HD;
-    float* pbuf = sm.attn + warp * HPG * kPageSize;      // this warp's page probabilities
+    uint8_t* stg = reinterpret_cast<uint8_t*>(sm.attn) + warp * (kPageSize * HD * 2);   // staging page
     for (int c = 0;; ++c) {
         if (c == 0) {
             seen_complete_wait(p, &sm.full[stage], lap & 1, &sm.flag[3]);
@@ -1472,7 +1564,7 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
                 const int k_lo = max(tok_lo - pf, 0), k_hi = min(tok_hi - pf, kPageSize);
                 if (k_hi <= k_lo) continue;
                 const uint16_t* kb = base + (size_t)pi * 2 * blk_elems;
-                attn_page<HPG, DPL>(st, kb, kb + blk_elems, k_lo, k_hi, pbuf);
+                attn_page<HPG, DPL>(st, kb, kb + blk_elems, k_lo, k_hi, stg);
             }
         }
         __syncwarp();
@@ -1481,26 +1573,24 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
         if (++stage == kStages) { stage = 0; ++lap; }
         if (last) break;
     }
-    if (has_new && warp == 0) {
-        float kf[DPL], vf[DPL];
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) {
-            kf[d] = sm.kn[lane * DPL + d];
-            vf[d] = sm.vn[lane * DPL + d];
-        }
-        attn_new_token<HPG, DPL>(st, kf, vf);
-    }
-#pragma unroll
-    for (int h = 0; h < HPG; ++h) st.l[h] = warp_sum(st.l[h]);
-    csync(p, sm, cph);                                   // every warp is done with its pbuf
+    if (has_new && warp == 0) attn_new_token<HPG, DPL>(st, sm.kn, sm.vn, stg);
+    // this thread's row sum over its quad (the four threads of head lane / 4)
+    st.l += __shfl_xor_sync(0xFFFFFFFFu, st.l, 1);
+    st.l += __shfl_xor_sync(0xFFFFFFFFu, st.l, 2);
+    csync(p, sm, cph);                                   // every warp is done with its staging page
     // combine the warps' partials (fixed order) into this split's partial
     float* sc = sm.attn;
+    {
+        const int g4 = lane >> 2, t4 = lane & 3;
+        if (g4 < HPG) {
+            float* w = sc + ((size_t)warp * HPG + g4) * (HD + 2);
+            if (t4 == 0) { w[0] = st.m; w[1] = st.l; }
 #pragma unroll
-    for (int h = 0; h < HPG; ++h) {
-        float* w = sc + ((size_t)warp * HPG + h) * (HD + 2);
-        if (lane == 0) { w[0] = st.m[h]; w[1] = st.l[h]; }
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) w[2 + lane * DPL + d] = st.o[h][d];
+            for (int j = 0; j < AttnMma<HPG, DPL>::NT; ++j) {
+                w[2 + 8 * j + 2 * t4] = st.o[j][0] + st.o[j][2];
+                w[2 + 8 * j + 2 * t4 + 1] = st.o[j][1] + st.o[j][3];
+            }
+        }
     }
     csync(p, sm, cph);
     if (sm.flag[3]) { abort_all = true; return; }
