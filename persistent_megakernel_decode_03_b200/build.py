@@ -29,7 +29,7 @@ def stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-MIN_LAUNCH_REGS = 163   # kMinLaunchRegs in csrc/mk_internal.h (setmaxnreg budget)
+MIN_LAUNCH_REGS = 168   # kMinLaunchRegs in csrc/mk_internal.h (setmaxnreg budget)
 
 
 def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:

@@ -444,6 +444,12 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                     }
                 }
             }
+            // (this function is out of line: the parameters the loop needs are read once
+            // into registers rather than through the parameter block's address per stage)
+            const int nkv = p.nkv, n_pages = p.n_pages;
+            const uint16_t* const kpool = p.k_pages;
+            const uint16_t* const vpool = p.v_pages;
+            const size_t blk_elems = (size_t)kPageSize * p.hd;
             const int pps = pages_per_stage(p);
             const int nch = (npages + pps - 1) / pps;
             const uint32_t blk = (uint32_t)(kPageSize * p.hd * 2);
@@ -482,7 +488,7 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                 bool bad = false;
                 for (int i = 0; i < n; ++i) {
                     int ph = sm.pid[(c * pps + i) % kPidRing];
-                    if (ph < 0 || ph >= p.n_pages) bad = true;
+                    if (ph < 0 || ph >= n_pages) bad = true;
                 }
                 if (bad) {
                     set_error(p, kErrInvalid, ti, -2, first, b);
@@ -493,10 +499,10 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                 mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)n * 2u * blk);
                 for (int i = 0; i < n; ++i) {
                     int ph = sm.pid[(c * pps + i) % kPidRing];
-                    size_t off = (((size_t)t.layer * p.n_pages + ph) * p.nkv + t.aux) * (size_t)kPageSize * p.hd;
+                    size_t off = (((size_t)t.layer * n_pages + ph) * nkv + t.aux) * blk_elems;
                     uint8_t* dst = sm.ring[stage] + (size_t)i * 2 * blk;
-                    bulk_g2s(dst, p.k_pages + off, blk, &sm.full[stage], pol);
-                    bulk_g2s(dst + blk, p.v_pages + off, blk, &sm.full[stage], pol);
+                    bulk_g2s(dst, kpool + off, blk, &sm.full[stage], pol);
+                    bulk_g2s(dst + blk, vpool + off, blk, &sm.full[stage], pol);
                 }
                 advance();
             }

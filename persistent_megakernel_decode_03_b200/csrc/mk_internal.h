@@ -18,12 +18,12 @@ constexpr int kEpilogueWarp = kConsumerWarps + 1;    // warp 9: task epilogues a
 constexpr int kPrefetchWarp = kConsumerWarps + 2;    // warp 10 (warp 11 idles)
 constexpr int kThreads = 384;                        // 3 warpgroups: 2 consumer + 1 support
 // Register split between the warpgroups (setmaxnreg): the support warpgroup gives
-// registers to the consumers.  256*216 + 128*56 = 62464 must not exceed the
+// registers to the consumers.  256*216 + 128*72 = 64512 must not exceed the
 // launch's 384 * (registers per thread at launch); the build checks the launch
 // count is at least kMinLaunchRegs.
 constexpr int kConsumerRegs = 216;
-constexpr int kSupportRegs = 56;
-constexpr int kMinLaunchRegs = (256 * kConsumerRegs + 128 * kSupportRegs + 383) / 384;   // 163
+constexpr int kSupportRegs = 72;
+constexpr int kMinLaunchRegs = (256 * kConsumerRegs + 128 * kSupportRegs + 383) / 384;   // 168
 constexpr int kStageBytes = 16 * 1024;
 constexpr int kStages = 11;
 constexpr int kMaxTaskRows = 64;        // rows (all weight blocks) of one GEMV task
