@@ -291,7 +291,7 @@ __device__ __forceinline__ int gemv_chunks(const GemvGeom& g) {
 
 // Splits of one (sequence, kv head) actually used this step: about one per
 // kAttnSplitTokens positions of context, at most the graph's split count S.
-constexpr int kAttnSplitTokens = 128;
+constexpr int kAttnSplitTokens = 64;
 __device__ __forceinline__ int attn_active_splits(int n_ctx, int S) {
     int a = (n_ctx + kAttnSplitTokens - 1) / kAttnSplitTokens;
     return a < 1 ? 1 : (a > S ? S : a);
