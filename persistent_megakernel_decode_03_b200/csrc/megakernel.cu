@@ -54,6 +54,17 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t n) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
 }
@@ -1897,44 +1908,62 @@ __device__ __forceinline__ void gemv_store(const Params& p, const Smem& sm, cons
 // and O-projection depends on it.
 __device__ void epilogue_loop(const Params& p, Smem& sm) {
     const int lane = threadIdx.x & 31;
-    for (uint32_t seq = 0;; ++seq) {
-        const int buf = (int)(seq % kRedBufs);
-        if (!mbar_wait_bounded(p, &sm.red_full[buf], (seq / kRedBufs) & 1, 2)) return;
-        const int ti = sm.ep_ti[buf];
-        if (ti < 0) return;                              // end of work
-        const Task t = sm.ep_task[buf];
-        uint32_t evt = t.sig;
-        if (t.op != MK_OP_ATTN && !(t.op == MK_OP_LMHEAD && p.skip_lm)) {
-            GemvGeom g;
-            gemv_geom(p, t, g, false);
-            const int wpg = (t.flags != kFastNone) ? kConsumerWarps : thread_map(g.K).wpg;
-            gemv_store(p, sm, t, g, wpg, buf, lane);
-            if (t.op == MK_OP_ROUTER) {
-                // arrival of this router tile; the layer's last tile selects the experts
-                // and only it signals the router event
-                __threadfence();
-                __syncwarp();
-                int last = 0;
-                if (lane == 0) {
-                    const uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
+    uint32_t seq = 0;
+    while (true) {
+        if (!mbar_wait_bounded(p, &sm.red_full[seq % kRedBufs], (seq / kRedBufs) & 1, 2)) return;
+        // finish every task whose partials are already in (up to all buffer sets), then
+        // one fence for all of them, then their signals in task order
+        uint32_t evts[kRedBufs];
+        int tis[kRedBufs];
+        int nb = 0;
+        bool end = false;
+        do {
+            const int buf = (int)(seq % kRedBufs);
+            const int ti = sm.ep_ti[buf];
+            if (ti < 0) { end = true; break; }          // end of work
+            const Task t = sm.ep_task[buf];
+            uint32_t evt = t.sig;
+            if (t.op != MK_OP_ATTN && !(t.op == MK_OP_LMHEAD && p.skip_lm)) {
+                GemvGeom g;
+                gemv_geom(p, t, g, false);
+                const int wpg = (t.flags != kFastNone) ? kConsumerWarps : thread_map(g.K).wpg;
+                gemv_store(p, sm, t, g, wpg, buf, lane);
+                if (t.op == MK_OP_ROUTER) {
+                    // arrival of this router tile; the layer's last tile selects the experts
+                    // and only it signals the router event
                     __threadfence();
-                    last = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
+                    __syncwarp();
+                    int last = 0;
+                    if (lane == 0) {
+                        const uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
+                        __threadfence();
+                        last = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
+                    }
+                    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+                    if (last) router_finalize(p, sm, t.layer);
+                    else evt = MK_NO_EVENT;
                 }
-                last = __shfl_sync(0xFFFFFFFFu, last, 0);
-                if (last) router_finalize(p, sm, t.layer);
-                else evt = MK_NO_EVENT;
             }
-        }
+            evts[nb] = evt;
+            tis[nb] = ti;
+            ++nb;
+            ++seq;
+        } while (nb < kRedBufs && mbar_test_wait(&sm.red_full[seq % kRedBufs], (seq / kRedBufs) & 1));
         // every lane orders its own stores (and, through the consumers' arrivals, theirs)
-        // before lane 0's release of the event
-        if (evt != MK_NO_EVENT) __threadfence();
+        // before lane 0's releases of the events
+        bool any = false;
+        for (int k = 0; k < nb; ++k) any |= (evts[k] != MK_NO_EVENT);
+        if (any) __threadfence();
         __syncwarp();
         if (lane == 0) {
-            if (evt != MK_NO_EVENT) red_release_add(&p.events[evt], 1u);
-            atomicAdd(p.done, 1u);
-            if (p.trace) p.trace[(size_t)ti * 4 + 2] = globaltimer();
-            mbar_arrive(&sm.red_free[buf]);
+            for (int k = 0; k < nb; ++k) {
+                if (evts[k] != MK_NO_EVENT) red_release_add(&p.events[evts[k]], 1u);
+                atomicAdd(p.done, 1u);
+                if (p.trace) p.trace[(size_t)tis[k] * 4 + 2] = globaltimer();
+                mbar_arrive(&sm.red_free[(seq - nb + k) % kRedBufs]);
+            }
         }
+        if (end) return;
     }
 }
 
