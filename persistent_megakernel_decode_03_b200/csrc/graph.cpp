@@ -74,7 +74,9 @@ void wave_stats(int n_tiles, int n_sm, int* waves, int* idle) {
 // divides it (QKV tiles never straddle two heads, so each feeds one KV head).
 int choose_tile_rows(int64_t rows, int64_t row_bytes, int n_blocks, int n_sm, int64_t target,
                      int divide) {
-    int cap = 16 / n_blocks;   // <= 16 rows per task: the fast GEMV path keeps row sums in registers
+    // <= 16 rows per task where the fast GEMV path keeps row sums in registers; short
+    // rows (<= 2 KB, no fast path) take up to 64 rows so a task still moves ~100 KB
+    int cap = (row_bytes <= 2048) ? kMaxTaskRows / n_blocks : 16 / n_blocks;
     int R = (int)std::max<int64_t>(1, std::min<int64_t>(cap, target / (row_bytes * n_blocks)));
     if (divide > 0) R = largest_divisor_at_most(divide, R);
     const int64_t min_bytes = 16 * 1024;

@@ -296,3 +296,28 @@ def test_prefill_with_many_one_stage_tiles_per_cta():
     d, cos, ok = compare_logits(last, ref)
     assert ok, (d, cos)
     dec.close()
+
+
+@pytest.mark.parametrize("nq,nkv,hd", [(4, 4, 64), (8, 1, 64), (8, 2, 64), (4, 2, 128), (8, 8, 128), (8, 1, 128)],
+                         ids=lambda v: str(v))
+def test_head_layouts_every_kernel_variant(nq, nkv, hd):
+    """MHA, GQA and MQA with head_dim 64 and 128: every (q heads per kv head,
+    head_dim) variant of the kernel, small shapes, 20 steps against the oracle,
+    with an odd vocabulary (a ragged last LM-head tile) and a 1-layer model."""
+    cfg = dataclasses.replace(syn.TINY, name=f"heads-{nq}-{nkv}-{hd}", n_layers=1, hidden=256,
+                              n_q_heads=nq, n_kv_heads=nkv, head_dim=hd, ffn=512, vocab=1000)
+    seed = 7700 + nq * 100 + nkv * 10 + hd
+    specs, ts = device_weights(cfg, seed, 0.1)
+    host_w = syn.host_weights(cfg, seed, 0.1)
+    dec = make_decoder(cfg, ts, 1, 64)
+    orc = oracle.Model(cfg, host_w, 64, names(cfg))
+    toks = syn.host_tokens(20, seed, cfg.vocab)
+    for p, t in enumerate(toks):
+        g = dec.step(torch.tensor([int(t)], dtype=torch.int32, device="cuda"),
+                     torch.tensor([p], dtype=torch.int32, device="cuda")).cpu().numpy()[0]
+        dec.check()
+        ref = orc.decode_step(int(t), p)["logits"]
+        d, cos, ok = compare_logits(g, ref)
+        assert ok, (p, d, cos)
+    check_counters(dec)
+    dec.close()
