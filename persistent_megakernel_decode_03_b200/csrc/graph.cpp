@@ -400,7 +400,7 @@ void attach_weights(GraphPlan& g, const void* const* w) {
         t.row_bytes = rb;
         t.nblk = (uint16_t)nblk;
         if (rb <= (uint32_t)kStageBytes) {
-            t.chunk_rows = (uint16_t)(kStageBytes / rb);
+            t.chunk_rows = (uint16_t)(is_warp_row(t.flags) ? kWarpRows : kStageBytes / rb);
             t.nchunks = (uint32_t)nblk * ((rows + t.chunk_rows - 1) / t.chunk_rows);
         } else {
             t.chunk_rows = 0;

@@ -288,11 +288,11 @@ __device__ __forceinline__ bool is_gemv(int op) { return op != MK_OP_ATTN; }
 
 // Chunks of a GEMV task: per weight block, groups of whole rows that fit one
 // stage, or (rows longer than a stage) each row in stage-sized segments.
-__device__ __forceinline__ int gemv_chunks(const GemvGeom& g) {
+__device__ __forceinline__ int gemv_chunks(const GemvGeom& g, uint8_t flags) {
     const int64_t RB = (int64_t)g.K * 2;
     int per_blk;
     if (RB <= kStageBytes) {
-        const int rps = (int)(kStageBytes / RB);
+        const int rps = is_warp_row(flags) ? kWarpRows : (int)(kStageBytes / RB);
         per_blk = (g.rows + rps - 1) / rps;
     } else {
         per_blk = g.rows * (int)((RB + kStageBytes - 1) / kStageBytes);
@@ -529,7 +529,7 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
         }
         GemvGeom g;
         gemv_geom(p, t, g, !skip);
-        const int nch = skip ? 0 : gemv_chunks(g);
+        const int nch = skip ? 0 : gemv_chunks(g, t.flags);
         if (nch == 0) {
             if (!acquire_slot()) { ok = false; break; }
             sm.info[stage] = StageInfo{ti, 0, 0, 0, t};
@@ -554,7 +554,7 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
         for (int bi = 0; bi < g.nblk && ok; ++bi) {
             const uint8_t* base = reinterpret_cast<const uint8_t*>(g.w[bi]);
             if (RB <= kStageBytes) {
-                const int rps = (int)(kStageBytes / RB);
+                const int rps = is_warp_row(t.flags) ? kWarpRows : (int)(kStageBytes / RB);
                 for (int r0 = 0; r0 < g.rows && ok; r0 += rps) {
                     const int n = min(rps, g.rows - r0);
                     ok = issue(base + (int64_t)r0 * RB, (uint32_t)(n * RB));
@@ -1213,11 +1213,40 @@ __device__ bool gemv_fast_segs(const Params& p, Smem& sm, int ti, const float2 (
     return true;
 }
 
+// Short rows (VPL 16-byte vectors per lane): each stage holds kWarpRows rows, warp w
+// takes row w, sums it with a warp reduction and leaves the total in red[buf][row][0].
+template <int VPL>
+__device__ bool gemv_fast_warprow(const Params& p, Smem& sm, int ti, int rows,
+                                  const float2 (&xr)[kMaxVecPerThread][4], int buf, int& stage, uint32_t& lap) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int rb = VPL * 32 * 16;                        // bytes per row
+#pragma unroll 1
+    for (int r0 = 0; r0 < rows; r0 += kWarpRows) {
+        if (r0 > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 5)) { sm.flag[3] = 1; return false; }
+        if (sm.info[stage].task != ti) { set_error(p, kErrFault, ti, -4, sm.info[stage].task, 4); sm.flag[3] = 1; return false; }
+        if (r0 + warp < rows) {
+            const uint4* sv = reinterpret_cast<const uint4*>(sm.ring[stage] + warp * rb) + lane;
+            float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < VPL; ++j) dot8(sv[32 * j], xr[j], a);
+            const float tot = warp_sum(a.x + a.y);
+            if (lane == 0) sm.red[buf][r0 + warp][0] = tot;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        if (++stage == kStages) { stage = 0; ++lap; }
+    }
+    return true;
+}
+
 // Runs the task's fast path (variant chosen by the planner); false on abort.
-__device__ __forceinline__ bool gemv_fast_dispatch(const Params& p, Smem& sm, int ti, int variant,
+__device__ __forceinline__ bool gemv_fast_dispatch(const Params& p, Smem& sm, int ti, int variant, int rows,
                                                    const float2 (&xr)[kMaxVecPerThread][4], int buf,
                                                    int& stage, uint32_t& lap) {
     switch (variant) {
+        case kFastW2: return gemv_fast_warprow<2>(p, sm, ti, rows, xr, buf, stage, lap);
+        case kFastW3: return gemv_fast_warprow<3>(p, sm, ti, rows, xr, buf, stage, lap);
+        case kFastW4: return gemv_fast_warprow<4>(p, sm, ti, rows, xr, buf, stage, lap);
         case kFastV2R2N16: return gemv_fast_rows<2, 2, 16>(p, sm, ti, xr, buf, stage, lap);
         case kFastV2R2N8: return gemv_fast_rows<2, 2, 8>(p, sm, ti, xr, buf, stage, lap);
         case kFastV1R4N16: return gemv_fast_rows<1, 4, 16>(p, sm, ti, xr, buf, stage, lap);
@@ -1791,9 +1820,15 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
         gemv_geom(p, t, g, false);
         // fast-path tiles split every row over all 8 warps (wpg = 8, one group)
         ThreadMap m;
-        if (fast) { m.nvec = g.K >> 3; m.wpg = kConsumerWarps; m.G = 1; m.grp = 0; m.lig = tid;
-                    m.gstride = kConsumerThreads; m.vpt = m.nvec / kConsumerThreads; m.active = true; }
-        else m = thread_map(g.K);
+        if (fast && is_warp_row(t.flags)) {      // one row per warp: every warp holds the whole input
+            m.nvec = g.K >> 3; m.wpg = 1; m.G = kConsumerWarps; m.grp = warp; m.lig = lane;
+            m.gstride = 32; m.vpt = m.nvec / 32; m.active = true;
+        } else if (fast) {
+            m.nvec = g.K >> 3; m.wpg = kConsumerWarps; m.G = 1; m.grp = 0; m.lig = tid;
+            m.gstride = kConsumerThreads; m.vpt = m.nvec / kConsumerThreads; m.active = true;
+        } else {
+            m = thread_map(g.K);
+        }
         const int rows_total = g.rows * g.nblk;
         const bool resid = !skip && warp == 0 && (t.op == MK_OP_OPROJ || t.op == MK_OP_DOWN);
         float resid0 = 0.0f, resid1 = 0.0f;
@@ -1819,7 +1854,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             }
         }
         const long long c_ch = (p.stats && tid == 0) ? clock64() : 0;
-        if (fast) (void)gemv_fast_dispatch(p, sm, ti, t.flags, xr, buf, stage, lap);
+        if (fast) (void)gemv_fast_dispatch(p, sm, ti, t.flags, g.rows, xr, buf, stage, lap);
         else (void)gemv_task_dispatch(p, sm, ti, g, m, xr, buf, stage, lap, skip);
         if (p.stats && tid == 0) stat_add(p, 6, (unsigned long long)(clock64() - c_ch));
         if (sm.flag[3]) break;
@@ -1926,7 +1961,8 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
             if (t.op != MK_OP_ATTN && !(t.op == MK_OP_LMHEAD && p.skip_lm)) {
                 GemvGeom g;
                 gemv_geom(p, t, g, false);
-                const int wpg = (t.flags != kFastNone) ? kConsumerWarps : thread_map(g.K).wpg;
+                const int wpg = is_warp_row(t.flags) ? 1
+                                : (t.flags != kFastNone) ? kConsumerWarps : thread_map(g.K).wpg;
                 gemv_store(p, sm, t, g, wpg, buf, lane);
                 if (t.op == MK_OP_ROUTER) {
                     // arrival of this router tile; the layer's last tile selects the experts

@@ -45,11 +45,26 @@ enum FastPath : uint8_t {
     kFastV2R2N4 = 7,    // K = 4096, 4 rows (tail tiles)
     kFastV1R4N4 = 8,    // K = 2048, 4 rows (tail tiles)
     kFastV7S4N1 = 9,    // K = 14336, 1 row (tail tiles)
+    kFastW2 = 10,       // K = 512: one row per warp per stage (8 rows per stage)
+    kFastW3 = 11,       // K = 768
+    kFastW4 = 12,       // K = 1024
 };
+
+// Short rows are given one warp each: a stage holds 8 rows, one per consumer warp.
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+inline bool is_warp_row(uint8_t f) { return f >= kFastW2 && f <= kFastW4; }
+constexpr int kWarpRows = 8;
 
 // The variant for a GEMV tile of `rows` rows per weight block, `nblk` blocks, K columns.
 inline uint8_t fast_path_for(int K, int rows, int nblk) {
     const int nvec = K / 8;
+    if (nblk == 1 && rows <= kMaxTaskRows) {
+        if (K == 512) return kFastW2;
+        if (K == 768) return kFastW3;
+        if (K == 1024) return kFastW4;
+    }
     if (K % 8 != 0 || nvec % kConsumerThreads != 0) return kFastNone;
     const int vpt = nvec / kConsumerThreads, total = rows * nblk;
     const long long rb = 2LL * K;
