@@ -916,10 +916,15 @@ __device__ void gemv_prologue_t(const Params& p, Smem& sm, uint32_t& cph, const 
                                 int K, const InSrc& src, float2 (&xr)[kMaxVecPerThread][4]) {
     const uint16_t* gain = gemv_norm_gain(p, t);
     float ss = 0.0f;
+    // the norm gains of this thread's columns are loaded together with the input, so
+    // their latency overlaps the input loads and the block-wide sum
+    uint4 gv[kMaxVecPerThread];
 #pragma unroll
     for (int j = 0; j < kMaxVecPerThread; ++j) {
         const int v = m.lig + j * m.gstride;
-        if (j < m.vpt && v < m.nvec && m.active) {
+        const bool mine = j < m.vpt && v < m.nvec && m.active;
+        gv[j] = (gain && mine) ? __ldg(reinterpret_cast<const uint4*>(gain + v * 8)) : make_uint4(0u, 0u, 0u, 0u);
+        if (mine) {
             load8<PARTS>(src, v * 8, xr[j]);
         } else {
 #pragma unroll
@@ -937,7 +942,7 @@ __device__ void gemv_prologue_t(const Params& p, Smem& sm, uint32_t& cph, const 
         for (int j = 0; j < kMaxVecPerThread; ++j) {
             const int v = m.lig + j * m.gstride;
             if (j < m.vpt && v < m.nvec && m.active) {
-                const uint4 u = __ldg(reinterpret_cast<const uint4*>(gain + v * 8));
+                const uint4 u = gv[j];
                 const float g[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
                                     bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
 #pragma unroll
