@@ -120,7 +120,10 @@ void mk_model_destroy(mk_model* model);
 
 /* Builds the task list for batches up to max_batch and contexts up to max_ctx
  * tokens (positions 0..max_ctx-1) on the current device (its SM count sets
- * the tile sizes and the grid) and uploads it.  Operator graph -> per-tile
+ * the tile sizes and the grid) and uploads it.  max_batch 1 streams every
+ * weight row through CUDA-core GEMV tiles; max_batch 2..64 (dense models
+ * only) uses tcgen05 tensor-core tiles for the projections, with the batch as
+ * the MMA's N dimension (padded to 16, 32 or 64).  Operator graph -> per-tile
  * tasks; a task depends on the tasks whose output rows overlap its input
  * rows (MPK digest, "Part 1. Compiler"; HN thread answer on task granularity
  * and dependency analysis). */
@@ -156,7 +159,18 @@ enum {
     MK_OP_LMHEAD = 6,     /* rows of Wlm . rmsnorm(x)                   */
     MK_OP_ROUTER = 7,     /* rows of Wr . rmsnorm(x); last tile: top-k  */
     MK_OP_EXP_GATEUP = 8, /* expert slot k: rows of silu(Wg_e h)*(Wu_e h) */
-    MK_OP_EXP_DOWN = 9    /* expert slot k: rows of Wd_e . a_e          */
+    MK_OP_EXP_DOWN = 9,   /* expert slot k: rows of Wd_e . a_e          */
+    /* Batched graphs (max_batch > 1, dense models) replace the GEMV tiles with
+     * tensor-core tiles: 128 weight rows times all batch rows, over one K-split.
+     * The last split of a tile to finish reduces the splits' partial sums in
+     * split order and applies the operator's epilogue. */
+    MK_OP_NORM = 10,      /* rmsnorm of batch rows [r0, r1) into the bf16 hi/lo operand
+                             of the next projection (aux: 0 attention, 1 FFN, 2 final) */
+    MK_OP_MM_QKV = 11,    /* rows [r0, r1) of [Wq;Wk;Wv] . h for every batch row */
+    MK_OP_MM_OPROJ = 12,  /* rows of Wo . o plus the residual */
+    MK_OP_MM_GATEUP = 13, /* FFN rows [r0, r1) (<= 64): silu(Wg h) * (Wu h) */
+    MK_OP_MM_DOWN = 14,   /* rows of Wd . a plus the residual */
+    MK_OP_MM_LMHEAD = 15  /* rows of Wlm . rmsnorm(x) */
 };
 
 #define MK_NO_EVENT 0xFFFFFFFFu
@@ -169,7 +183,9 @@ enum {
  * (b, kv head) signals, after merging the partial results; router tiles: only
  * the last tile of a layer, after selecting the experts).  Expert tasks also
  * wait on pointer_wait (the router's event) before the weight address of the
- * routed expert is read; MK_NO_EVENT elsewhere. */
+ * routed expert is read; MK_NO_EVENT elsewhere.  Tensor-core tiles
+ * (MK_OP_MM_*) export b = their split index and aux = the tile's split count;
+ * all splits of a tile name its event, and only the last to finish signals it. */
 typedef struct {
     int op, layer, b, aux;
     uint32_t r0, r1;

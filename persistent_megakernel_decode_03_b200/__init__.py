@@ -31,6 +31,9 @@ MK_NO_EVENT = 0xFFFFFFFF
 
 MK_OP_QKV, MK_OP_ATTN, MK_OP_OPROJ, MK_OP_GATEUP, MK_OP_DOWN, MK_OP_LMHEAD = 1, 2, 3, 4, 5, 6
 MK_OP_ROUTER, MK_OP_EXP_GATEUP, MK_OP_EXP_DOWN = 7, 8, 9
+MK_OP_NORM, MK_OP_MM_QKV, MK_OP_MM_OPROJ, MK_OP_MM_GATEUP, MK_OP_MM_DOWN, MK_OP_MM_LMHEAD = (
+    10, 11, 12, 13, 14, 15)
+MM_OPS = (MK_OP_MM_QKV, MK_OP_MM_OPROJ, MK_OP_MM_GATEUP, MK_OP_MM_DOWN, MK_OP_MM_LMHEAD)
 OP_NAMES = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
             8: "exp_gateup", 9: "exp_down"}
 

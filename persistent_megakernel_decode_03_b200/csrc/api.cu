@@ -1,5 +1,6 @@
 // C ABI of the decode megakernel (declared in include/mk.h): model
 // registration, task-graph build and upload, per-stream state, decode steps.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -31,6 +32,7 @@ struct mk_graph {
     mk::Task* d_tasks = nullptr;
     uint32_t* d_thr = nullptr;
     float* d_rope = nullptr;
+    std::vector<CUtensorMap> wmaps;   // batched graphs: operand slots (filled per state), then weights
 };
 
 struct mk_state {
@@ -50,6 +52,10 @@ struct mk_state {
     float *x_mid = nullptr, *x_out = nullptr, *qkv = nullptr, *act = nullptr;
     float *part = nullptr, *attn_o = nullptr, *rlogits = nullptr, *moe_w = nullptr, *ypart = nullptr;
     int* moe_sel = nullptr;
+    uint16_t* opnd[mk::kNumOperands] = {};   // batched graphs: bf16 hi/lo operands
+    float* mm_part = nullptr;
+    uint32_t* mm_cnt = nullptr;
+    void* tmaps = nullptr;         // device copy of the tensor maps (operands, then weights)
     int32_t* tokpos = nullptr;     // host-input variant: [2][max_batch]
     float* logits = nullptr;       // host-output variant: [max_batch][vocab]
     unsigned long long* trace = nullptr;
@@ -77,6 +83,39 @@ mk_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 int slots_per_layer(const mk_model_desc& d) { return d.n_experts > 0 ? 10 : 9; }
+
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point (no
+// link against the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// A 2-D bf16 matrix [rows][cols] (row pitch cols * 2 bytes) loaded in boxes of
+// box_rows x 64 columns (128 bytes) with the 128-byte swizzle; rows or columns
+// past the matrix read as zeros.
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn || ((uintptr_t)base & 15) || (cols * 2) % 16 != 0) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)mk::kMmK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 template <typename T>
 mk_status dev_alloc(mk_state* s, T** p, size_t count) {
@@ -110,6 +149,8 @@ mk_status reset_counters(mk_state* s, cudaStream_t st) {
     if (e == cudaSuccess)
         e = cudaMemsetAsync(s->attn_cnt, 0,
                             sizeof(uint32_t) * d.n_layers * s->g->plan.max_batch * d.n_kv_heads, st);
+    if (e == cudaSuccess && s->mm_cnt)
+        e = cudaMemsetAsync(s->mm_cnt, 0, sizeof(uint32_t) * std::max(1, s->g->plan.mm_counters), st);
     if (e != cudaSuccess) return cuda_fail(e, "reset");
     s->epoch = 0;
     s->needs_reset = false;
@@ -181,6 +222,12 @@ mk::Params base_params(mk_state* s) {
     p.moe_w = s->moe_w;
     p.moe_sel = s->moe_sel;
     p.ypart = s->ypart;
+    p.mm = P.bp > 0 ? 1 : 0;
+    p.bp = P.bp;
+    p.tmaps = s->tmaps;
+    for (int i = 0; i < mk::kNumOperands; ++i) p.opnd[i] = s->opnd[i];
+    p.mm_part = s->mm_part;
+    p.mm_cnt = s->mm_cnt;
     return p;
 }
 
@@ -329,9 +376,36 @@ static mk_status build_graph(mk_model* model, int max_batch, int max_ctx, int so
     if (st != MK_OK) return st;
     g->model = model;
     g->device = dev;
+    if (solo_op && g->plan.bp > 0) {
+        mk_graph_destroy(g);
+        return fail(MK_ERR_UNSUPPORTED, "mk_build_taskgraph_solo: batch-1 graphs only");
+    }
     if (solo_op) mk::make_solo(g->plan, solo_op);
     mk::attach_weights(g->plan, model->w.data());
     const GraphPlan& P = g->plan;
+    if (P.bp > 0) {
+        // tensor maps of the weights for the tensor-core tiles (the operand slots in
+        // front are filled by each state, which owns the operand buffers)
+        const int L = d.n_layers, H = d.hidden, S = slots_per_layer(d);
+        const uint64_t qr = (uint64_t)d.n_q_heads * d.head_dim, kr = (uint64_t)d.n_kv_heads * d.head_dim;
+        g->wmaps.assign((size_t)mk::lm_map_index(L) + 1, CUtensorMap{});
+        bool ok = true;
+        for (int l = 0; l < L && ok; ++l) {
+            const void* const* q = model->w.data() + 1 + l * S;
+            ok = encode_bf16_2d(&g->wmaps[mk::weight_map_index(l, 0)], q[1], qr, H, mk::kMmRows) &&
+                 encode_bf16_2d(&g->wmaps[mk::weight_map_index(l, 1)], q[2], kr, H, mk::kMmRows) &&
+                 encode_bf16_2d(&g->wmaps[mk::weight_map_index(l, 2)], q[3], kr, H, mk::kMmRows) &&
+                 encode_bf16_2d(&g->wmaps[mk::weight_map_index(l, 3)], q[4], H, qr, mk::kMmRows) &&
+                 encode_bf16_2d(&g->wmaps[mk::weight_map_index(l, 4)], q[6], d.ffn, H, mk::kMmRows / 2) &&
+                 encode_bf16_2d(&g->wmaps[mk::weight_map_index(l, 5)], q[7], d.ffn, H, mk::kMmRows / 2) &&
+                 encode_bf16_2d(&g->wmaps[mk::weight_map_index(l, 6)], q[8], H, d.ffn, mk::kMmRows);
+        }
+        if (ok) ok = encode_bf16_2d(&g->wmaps[mk::lm_map_index(L)], model->w[2 + L * S], d.vocab, H, mk::kMmRows);
+        if (!ok) {
+            mk_graph_destroy(g);
+            return fail(MK_ERR_CUDA, "mk_build_taskgraph: tensor map encoding failed");
+        }
+    }
     // RoPE table: cos/sin of pos * theta^(-2i/d), computed in double, stored fp32
     const int half = d.head_dim / 2;
     std::vector<float> rope((size_t)max_ctx * half * 2);
@@ -376,7 +450,7 @@ mk_status mk_graph_get_info(const mk_graph* g, mk_graph_info* info) {
     info->max_batch = P.max_batch;
     info->max_ctx = P.max_ctx;
     info->attn_splits = P.S;
-    info->n_ops = P.desc.n_experts > 0 ? 7 : 6;
+    info->n_ops = P.bp > 0 ? 7 : (P.desc.n_experts > 0 ? 7 : 6);   // batched: norm, 5 tiles, attention
     info->weight_bytes_per_step = P.weight_bytes;
     return MK_OK;
 }
@@ -396,6 +470,11 @@ mk_status mk_graph_export_tasks(const mk_graph* g, mk_task_info* out, int cap, i
         out[i].wait[1] = T[i].wait1;
         out[i].signal = T[i].sig;
         out[i].pointer_wait = T[i].pad;
+        if (mk::is_mm_op(T[i].op)) {          // split s of a tile with nblk splits
+            out[i].b = T[i].chunk_rows;
+            out[i].aux = T[i].nblk;
+            out[i].pointer_wait = MK_NO_EVENT;
+        }
     }
     *n = k;
     return MK_OK;
@@ -445,6 +524,34 @@ mk_status mk_state_create(mk_graph* g, mk_state** out) {
     }
     ALLOC(part, L * B * d.n_kv_heads * P.S * hpg * (d.head_dim + 2));
     ALLOC(attn_o, L * B * d.n_q_heads * d.head_dim);
+    if (P.bp > 0) {
+        const size_t BP = P.bp, qr = (size_t)d.n_q_heads * d.head_dim;
+        ALLOC(opnd[mk::kOpXq], L * 2 * BP * H);
+        ALLOC(opnd[mk::kOpXf], L * 2 * BP * H);
+        ALLOC(opnd[mk::kOpAo], L * 2 * BP * qr);
+        ALLOC(opnd[mk::kOpAct], L * 2 * BP * d.ffn);
+        ALLOC(opnd[mk::kOpXl], 2 * BP * H);
+        ALLOC(mm_part, (size_t)std::max(1, P.mm_slots) * BP * mk::kMmRows);
+        ALLOC(mm_cnt, (size_t)std::max(1, P.mm_counters));
+        if (st == MK_OK) {
+            std::vector<CUtensorMap> maps = g->wmaps;
+            const uint64_t rows = (uint64_t)L * 2 * BP;
+            const uint32_t box = (uint32_t)(2 * BP);
+            bool ok = encode_bf16_2d(&maps[mk::kOpXq], s->opnd[mk::kOpXq], rows, H, box) &&
+                      encode_bf16_2d(&maps[mk::kOpXf], s->opnd[mk::kOpXf], rows, H, box) &&
+                      encode_bf16_2d(&maps[mk::kOpAo], s->opnd[mk::kOpAo], rows, qr, box) &&
+                      encode_bf16_2d(&maps[mk::kOpAct], s->opnd[mk::kOpAct], rows, d.ffn, box) &&
+                      encode_bf16_2d(&maps[mk::kOpXl], s->opnd[mk::kOpXl], 2 * BP, H, box);
+            if (!ok) st = fail(MK_ERR_CUDA, "mk_state_create: tensor map encoding failed");
+            unsigned char* dm = nullptr;
+            if (st == MK_OK) st = dev_alloc(s, &dm, maps.size() * sizeof(CUtensorMap));
+            if (st == MK_OK) {
+                cudaError_t e = cudaMemcpy(dm, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice);
+                if (e != cudaSuccess) st = cuda_fail(e, "mk_state_create: tensor maps");
+                s->tmaps = dm;
+            }
+        }
+    }
     ALLOC(tokpos, 2 * B);
     ALLOC(logits, B * (size_t)d.vocab);
     if (d.flags & MK_FLAG_TRACE) ALLOC(trace, P.tasks.size() * 4);

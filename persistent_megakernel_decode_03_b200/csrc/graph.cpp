@@ -27,7 +27,8 @@ namespace mk {
 namespace {
 
 // Tensor kinds for the region-overlap analysis.
-enum TensorKind { T_XIN = 1, T_QKV, T_O, T_XMID, T_ACT, T_ACTE, T_SEL, T_LOGITS };
+enum TensorKind { T_XIN = 1, T_QKV, T_O, T_XMID, T_ACT, T_ACTE, T_SEL, T_LOGITS,
+                  T_XQOP, T_XFOP, T_XLOP };   // the last three: bf16 hi/lo operands of batched tiles
 
 struct Region {
     int tensor;         // encoded (kind, layer, slot)
@@ -122,7 +123,8 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     const int L = d.n_layers, H = d.hidden, nq = d.n_q_heads, nkv = d.n_kv_heads, hd = d.head_dim;
     const bool moe = d.n_experts > 0;
     if (max_batch < 1) return fail("max_batch must be >= 1");
-    if (max_batch > 1) return fail("max_batch > 1 is not supported by this build");
+    if (max_batch > kMaxMmBatch) return fail("max_batch must be <= 64");
+    if (max_batch > 1 && moe) return fail("max_batch > 1 needs a dense model (MoE decode is batch 1)");
     if (max_ctx < 1 || max_ctx > (1 << 22)) return fail("max_ctx must be in 1..4194304");
     if (n_sm < 1) return fail("n_sm must be >= 1");
 
@@ -139,7 +141,9 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     // attention split-K: as many (sequence, kv head, split) tasks as fit in one wave
     // over the SMs (one more would make every layer's attention phase take two
     // task durations), but at most one split per 64 positions of context.
-    int S = n_sm / (B * nkv);
+    // Batched graphs aim at about two tasks per SM instead: ragged context lengths
+    // make the splits unequal, and the dynamic queue evens them out.
+    int S = (B == 1) ? n_sm / (B * nkv) : (int)std::lround(2.0 * n_sm / (double)(B * nkv));
     S = std::max(1, std::min<int>(S, (int)ceil_div(max_ctx, 64)));
     g.S = S;
 
@@ -234,7 +238,95 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
             }
     };
 
-    for (int l = 0; l < L; ++l) {
+    if (B > 1) {
+        // ---- batched step: tensor-core tiles of 128 weight rows x all batch rows.
+        // A tile's K range is cut into splits so that (tiles x splits) fills the SMs;
+        // every split of a tile belongs to one producer entity, and the last split to
+        // arrive reduces the partial sums and signals.
+        g.bp = (B <= 16) ? 16 : (B <= 32) ? 32 : 64;
+        auto choose_splits = [&](int64_t tiles, int64_t kblocks) {
+            int best = 1;
+            double best_eff = 0.0;
+            const int cap = (int)std::max<int64_t>(1, std::min<int64_t>(16, kblocks / 2));
+            for (int sp = 1; sp <= cap; ++sp) {
+                const int64_t n = tiles * sp, w = ceil_div(n, n_sm);
+                const double eff = (double)n / (double)(w * n_sm);
+                if (eff >= 0.9) return sp;
+                if (eff > best_eff + 1e-9) { best_eff = eff; best = sp; }
+            }
+            return best;
+        };
+        int slot = 0;   // partial-sum slots, numbered per layer (layers reuse them in turn)
+        // one operator: blocks of (rows, weight map(s)); tiles of `tile_rows` output rows
+        struct WBlock { int64_t out0, n; int map0, map1; };
+        auto mm_op = [&](int op, int l, const std::vector<WBlock>& blocks, int tile_rows, int64_t K,
+                         std::vector<Region> in, int out_kind, int out_layer) {
+            int64_t tiles = 0;
+            for (const WBlock& wb : blocks) tiles += ceil_div(wb.n, tile_rows);
+            const int64_t kblocks = ceil_div(K, kMmK);
+            const int Sk = choose_splits(tiles, kblocks);
+            for (const WBlock& wb : blocks)
+                for (int64_t y = 0; y < wb.n; y += tile_rows) {
+                    const int64_t r0 = wb.out0 + y, r1 = wb.out0 + std::min<int64_t>(wb.n, y + tile_rows);
+                    Entity e;
+                    e.outs = {Region{tensor_key(out_kind, out_layer, 0), 0, B, r0, r1}};
+                    const int eid = (int)ent.size();
+                    ent.push_back(e);
+                    const int counter = g.mm_counters++;
+                    for (int sp = 0; sp < Sk; ++sp) {
+                        const int64_t kb0 = kblocks * sp / Sk, kb1 = kblocks * (sp + 1) / Sk;
+                        int t = new_task(op, l, 0, slot, (uint32_t)r0, (uint32_t)r1);
+                        Task& tk = T[t];
+                        tk.src[0] = (uint64_t)(uint32_t)wb.map0 | ((uint64_t)y << 32);
+                        tk.src[1] = (wb.map1 >= 0) ? ((uint64_t)(uint32_t)wb.map1 | ((uint64_t)y << 32)) : 0;
+                        tk.row_bytes = (uint32_t)kb0;
+                        tk.pad2 = (uint32_t)kb1;
+                        tk.chunk_rows = (uint16_t)sp;
+                        tk.nblk = (uint16_t)Sk;
+                        tk.nchunks = (uint32_t)(2 * (kb1 - kb0));
+                        tk.pad = (uint32_t)counter;
+                        task_in[t] = in;
+                        task_entity[t] = eid;
+                        ent[eid].tasks.push_back(t);
+                    }
+                    slot += Sk;
+                }
+        };
+        // rmsnorm of the batch rows into an operand, kNormRowsPerTask rows per task
+        auto norm_op = [&](int l, int kind, int in_kind, int in_layer, int out_kind) {
+            for (int b0 = 0; b0 < B; b0 += kNormRowsPerTask) {
+                const int b1 = std::min(B, b0 + kNormRowsPerTask);
+                int t = new_task(MK_OP_NORM, l, 0, kind, (uint32_t)b0, (uint32_t)b1);
+                task_in[t] = {Region{tensor_key(in_kind, in_layer, 0), b0, b1, 0, H}};
+                own_entity(t, {Region{tensor_key(out_kind, l, 0), b0, b1, 0, H}});
+            }
+        };
+        const int64_t qr = (int64_t)nq * hd, kr = (int64_t)nkv * hd;
+        for (int l = 0; l < L; ++l) {
+            slot = 0;
+            norm_op(l, 0, T_XIN, l, T_XQOP);
+            mm_op(MK_OP_MM_QKV, l,
+                  {{0, qr, weight_map_index(l, 0), -1}, {qr, kr, weight_map_index(l, 1), -1},
+                   {qr + kr, kr, weight_map_index(l, 2), -1}},
+                  kMmRows, H, {all_rows(T_XQOP, l, 0, H)}, T_QKV, l);
+            for (int kh = 0; kh < nkv; ++kh) attn_group(l, kh);
+            mm_op(MK_OP_MM_OPROJ, l, {{0, H, weight_map_index(l, 3), -1}}, kMmRows, qr,
+                  {all_rows(T_O, l, 0, qr)}, T_XMID, l);
+            norm_op(l, 1, T_XMID, l, T_XFOP);
+            mm_op(MK_OP_MM_GATEUP, l, {{0, d.ffn, weight_map_index(l, 4), weight_map_index(l, 5)}},
+                  kMmRows / 2, H, {all_rows(T_XFOP, l, 0, H)}, T_ACT, l);
+            mm_op(MK_OP_MM_DOWN, l, {{0, H, weight_map_index(l, 6), -1}}, kMmRows, d.ffn,
+                  {all_rows(T_ACT, l, 0, d.ffn)}, T_XIN, l + 1);
+            g.mm_slots = std::max(g.mm_slots, slot);
+        }
+        slot = 0;
+        norm_op(L, 2, T_XIN, L, T_XLOP);
+        mm_op(MK_OP_MM_LMHEAD, L, {{0, d.vocab, lm_map_index(L), -1}}, kMmRows, H,
+              {all_rows(T_XLOP, L, 0, H)}, T_LOGITS, 0);
+        g.mm_slots = std::max(g.mm_slots, slot);
+        if (g.mm_slots > 65535) return fail("too many tensor-core tiles per layer");
+    }
+    for (int l = 0; l < L && B == 1; ++l) {
         // QKV (input: the residual stream entering the layer), one KV group at a time,
         // so that the first groups' attention can start while the last QKV tiles
         // stream.  Attention follows all QKV tiles: a CTA that claimed a task still
@@ -276,7 +368,7 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
                     }
         }
     }
-    gemv_op(MK_OP_LMHEAD, L, d.vocab, R_lm, T_LOGITS, 0, {all_rows(T_XIN, L, 0, H)});
+    if (B == 1) gemv_op(MK_OP_LMHEAD, L, d.vocab, R_lm, T_LOGITS, 0, {all_rows(T_XIN, L, 0, H)});
 
     // ---- dependency analysis: producers overlapping each task's primary input
     std::map<int, std::vector<int>> by_tensor;   // tensor -> entities writing it

@@ -20,6 +20,10 @@ struct GraphPlan {
     std::vector<int> tile_rows;  // qkv, o, gate/up, down, lm, router, expert gate/up, expert down
     std::vector<Task> tasks;     // topological order
     std::vector<uint32_t> thr;   // per-event threshold per step
+    // batched graphs (max_batch > 1): tensor-core projection tiles
+    int bp = 0;                  // padded batch (the MMA's N); 0 for batch-1 graphs
+    int mm_slots = 0;            // split partial-sum slots per layer (each bp x 128 floats)
+    int mm_counters = 0;         // per-tile split arrival counters
 };
 
 int64_t ceil_div(int64_t a, int64_t b);

@@ -96,6 +96,80 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
+// Tiled TMA load of one 2-D box (tensor map in global memory) into shared memory;
+// x is the inner (column) coordinate, a multiple of 64 bf16 elements here.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, int x, int y, uint64_t* bar,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+// ---- tcgen05: tensor memory and the fifth-generation MMA (one CTA, no cluster)
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {      // whole warp
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {                               // whole warp
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {    // whole warp
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Arrives (once) on `bar` when every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+// D[tmem] (+)= A[smem] . B[smem]^T, bf16 inputs, fp32 accumulator; accumulate = 0 overwrites D.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 32 TMEM lanes (one per thread of the warp) x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Shared-memory matrix descriptor: K-major operand in the 128-byte swizzle layout
+// that a TMA box of 128-byte rows writes (8-row atoms of 1 KB; the leading
+// offset is unused in this layout, the stride offset steps from one 8-row atom
+// to the next).  Fields: start address >> 4, leading offset >> 4 at bit 16,
+// stride offset >> 4 at bit 32, descriptor version 1 at bit 46, swizzle mode 2
+// (128 B) at bit 61.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator (bit 4), bf16 A (bit 7)
+// and B (bit 10), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t mm_idesc(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kMmRows >> 4) << 24);
+}
+
 // Hint: bring [src, src+bytes) into L2 (16-byte aligned, multiple of 16 bytes).
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
@@ -190,6 +264,11 @@ struct __align__(128) Smem {
     int ep_ti[kRedBufs];                     // its index (-1: end of work)
     float ep_resid[kRedBufs][kMaxTaskRows];  // residual rows (O-proj, down), loaded early by warp 0
     int attn_last;                           // this CTA's attention split arrived last
+    uint64_t mm_acc;                         // tensor-core tile: the accumulator is complete
+    uint64_t mm_drain;                       // tensor-core work drained before TMEM is freed
+    uint64_t mm_sync;                        // consumer warps 0-3 (arrival count 4)
+    uint32_t tmem_base;                      // TMEM address of the accumulator (batched graphs)
+    int mm_last;                             // this CTA's split of a tile arrived last
     int pid[kPidRing];                       // producer: physical page ids read ahead
     int flag[4];
 };
@@ -284,7 +363,7 @@ __device__ __forceinline__ void gemv_geom(const Params& p, const Task& t, GemvGe
     }
 }
 
-__device__ __forceinline__ bool is_gemv(int op) { return op != MK_OP_ATTN; }
+__device__ __forceinline__ bool is_gemv(int op) { return op != MK_OP_ATTN && op <= MK_OP_EXP_DOWN; }
 
 // Chunks of a GEMV task: per weight block, groups of whole rows that fit one
 // stage, or (rows longer than a stage) each row in stage-sized segments.
@@ -381,6 +460,16 @@ __device__ __forceinline__ void csync(const Params& p, Smem& sm, uint32_t& phase
     if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.csync);
     if (!mbar_wait_bounded(p, &sm.csync, phase, 8)) sm.flag[3] = 1;
     phase ^= 1;
+}
+// The same among consumer warps 0-3 (the warps that own the TMEM lane quarters);
+// false when the wait gave up (the CTA is aborting).
+__device__ __forceinline__ bool msync4(const Params& p, Smem& sm, uint32_t& phase) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.mm_sync);
+    const bool ok = mbar_wait_bounded(p, &sm.mm_sync, phase, 13);
+    if (!ok) sm.flag[3] = 1;
+    phase ^= 1;
+    return ok;
 }
 
 
@@ -572,6 +661,67 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
     return ok;
 }
 
+// Tensor-core tile: per K-block one weight box (128 rows, or the matching 64 gate
+// and 64 up rows) and one activation box (hi rows then lo rows), each in its own
+// stage.  The activations are written by earlier tasks, so the first weight box
+// goes out before the wait for them and every other load after it.
+__device__ __forceinline__ const void* tmap_at(const Params& p, uint32_t idx) {
+    return reinterpret_cast<const uint8_t*>(p.tmaps) + (size_t)idx * 128;
+}
+__device__ __noinline__ bool produce_mm(const Params& p, Smem& sm, const Task& t, int ti, PRing& ring,
+                                        uint64_t pol) {
+    const bool two = (t.op == MK_OP_MM_GATEUP);
+    const void* w0 = tmap_at(p, (uint32_t)t.src[0]);
+    const void* w1 = two ? tmap_at(p, (uint32_t)t.src[1]) : nullptr;
+    const int wy = (int)(t.src[0] >> 32);
+    int xop = kOpXq;
+    switch (t.op) {
+        case MK_OP_MM_OPROJ: xop = kOpAo; break;
+        case MK_OP_MM_GATEUP: xop = kOpXf; break;
+        case MK_OP_MM_DOWN: xop = kOpAct; break;
+        case MK_OP_MM_LMHEAD: xop = kOpXl; break;
+        default: break;
+    }
+    const void* xm = tmap_at(p, (uint32_t)xop);
+    const int xy = (t.op == MK_OP_MM_LMHEAD) ? 0 : (int)t.layer * 2 * p.bp;
+    const uint32_t xbytes = 2u * (uint32_t)p.bp * 128u;
+    const int kb0 = (int)t.row_bytes, kb1 = (int)t.pad2, nch = (int)t.nchunks;
+    int c = 0;
+    auto open_stage = [&](uint32_t bytes) -> bool {
+        if (!pr_acquire(p, sm, ring)) return false;
+        StageInfo& inf = sm.info[ring.stage];
+        inf.task = ti;
+        inf.chunk = c;
+        inf.nchunks = nch;
+        if (c == 0) inf.rec = t;
+        mbar_arrive_expect_tx(&sm.full[ring.stage], bytes);
+        return true;
+    };
+    for (int kb = kb0; kb < kb1; ++kb) {
+        if (!open_stage((uint32_t)kStageBytes)) return false;
+        uint8_t* dst = sm.ring[ring.stage];
+        if (two) {
+            tma_load_2d_hint(dst, w0, kb * kMmK, wy, &sm.full[ring.stage], pol);
+            tma_load_2d_hint(dst + kStageBytes / 2, w1, kb * kMmK, wy, &sm.full[ring.stage], pol);
+        } else {
+            tma_load_2d_hint(dst, w0, kb * kMmK, wy, &sm.full[ring.stage], pol);
+        }
+        pr_advance(ring);
+        ++c;
+        if (kb == kb0 && t.wait0 != MK_NO_EVENT) {
+            if (!event_wait(p, t.wait0, p.thr[t.wait0] * p.epoch + p.wait_offset, ti)) return false;
+            // the operand was written through the generic proxy by other CTAs; order
+            // those writes before this CTA's tensor loads
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        if (!open_stage(xbytes)) return false;
+        tma_load_2d(sm.ring[ring.stage], xm, kb * kMmK, xy, &sm.full[ring.stage]);
+        pr_advance(ring);
+        ++c;
+    }
+    return true;
+}
+
 __device__ void producer_loop(const Params& p, Smem& sm) {
     const uint64_t pol = l2_evict_first_policy();
     PRing ring{0, 0};
@@ -591,7 +741,11 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         const int ti = (int)q;
         const Task t = p.tasks[ti];
         q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
-        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
+        if (is_mm_op(t.op)) {
+            ok = produce_mm(p, sm, t, ti, ring, pol);
+            continue;
+        }
+        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm) || t.op == MK_OP_NORM;
         if (skip) {                                      // nothing to stream: a marker stage
             if (!pr_acquire(p, sm, ring)) { ok = false; break; }
             sm.info[ring.stage] = StageInfo{ti, 0, 0, 0, t};
@@ -697,7 +851,7 @@ __device__ void prefetch_loop(const Params& p) {
             }
             continue;
         }
-        if (t.op == MK_OP_EXP_GATEUP || t.op == MK_OP_EXP_DOWN) continue;
+        if (t.op == MK_OP_EXP_GATEUP || t.op == MK_OP_EXP_DOWN || t.op >= MK_OP_NORM) continue;
         if (t.op == MK_OP_LMHEAD && p.skip_lm) continue;
         GemvGeom g;
         gemv_geom(p, t, g, true);
@@ -711,6 +865,33 @@ __device__ void prefetch_loop(const Params& p) {
 }
 
 // ----------------------------------------------------------------------------- consumer helpers
+
+// bf16 split of an fp32 value: hi = bf16(v), lo = bf16(v - hi); hi + lo carries
+// about 16 significant bits, so a bf16 x bf16 product of the weight and the pair
+// keeps the activation's fp32 precision to within ~2^-17 relative.
+__device__ __forceinline__ void split_hilo(float v, uint16_t& hi, uint16_t& lo) {
+    hi = f32_to_bf16_rne(v);
+    lo = f32_to_bf16_rne(v - bf16_to_f32(hi));
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Operand rows of batch row b: hi at row (base + b), lo at row (base + bp + b).
+__device__ __forceinline__ void put_operand4(const Params& p, int op, int layer, int b, int K, int col,
+                                             float4 v) {
+    const size_t base = (size_t)layer * 2 * p.bp;
+    uint16_t h[4], l[4];
+    split_hilo(v.x, h[0], l[0]);
+    split_hilo(v.y, h[1], l[1]);
+    split_hilo(v.z, h[2], l[2]);
+    split_hilo(v.w, h[3], l[3]);
+    uint16_t* hi = p.opnd[op] + (base + b) * K + col;
+    uint16_t* lo = p.opnd[op] + (base + p.bp + b) * K + col;
+    *reinterpret_cast<uint2*>(hi) = make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
+    *reinterpret_cast<uint2*>(lo) = make_uint2(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16));
+}
+
 
 // Residual stream entering layer l (l == L: after the last layer), element i of batch row b.
 __device__ __forceinline__ float x_in(const Params& p, int l, int b, int i) {
@@ -825,8 +1006,11 @@ __device__ void attn_merge_group(const Params& p, Smem& sm, uint32_t& cph, int l
             o.x = fmaf(v.x, w, o.x); o.y = fmaf(v.y, w, o.y); o.z = fmaf(v.z, w, o.z); o.w = fmaf(v.w, w, o.w);
         }
         const float inv = f[sa * hpg + h];
-        *reinterpret_cast<float4*>(out + (size_t)h * hd + i) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+        const float4 r = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+        *reinterpret_cast<float4*>(out + (size_t)h * hd + i) = r;
+        if (p.mm) put_operand4(p, kOpAo, l, b, p.nq * hd, g * hpg * hd + h * hd + i, r);
     }
+    if (p.mm) fence_proxy_async_global();
 }
 
 // Where a GEMV task's input vector lives: an fp32 row, a bf16 embedding row, and
@@ -1745,6 +1929,194 @@ __device__ void router_finalize(const Params& p, Smem& sm, int l) {
 
 // ----------------------------------------------------------------------------- consumer loop
 
+// ----------------------------------------------------------------------------- batched tiles
+
+// RMSNorm of one batch row per warp into the operand of the next projection:
+// h = x / sqrt(mean(x^2) + eps) * g (kind 0: attention norm of the residual
+// entering layer l, the token embedding at l = 0; kind 1: FFN norm of the
+// residual after attention; kind 2: final norm).  Rows past the step's batch
+// are written as zeros.
+__device__ void norm_task(const Params& p, const Task& t, int ti, int warp, int lane) {
+    const int b = (int)t.r0 + warp;
+    if (b >= (int)t.r1) return;
+    const int kind = t.aux, l = t.layer, H = p.H;
+    const int op = (kind == 0) ? kOpXq : (kind == 1) ? kOpXf : kOpXl;
+    const int olayer = (kind == 2) ? 0 : l;
+    if (b >= p.batch) {
+        for (int i = lane * 4; i < H; i += 128) put_operand4(p, op, olayer, b, H, i, make_float4(0.f, 0.f, 0.f, 0.f));
+        return;
+    }
+    const uint16_t* gain = (kind == 0) ? p.layers[l].attn_norm : (kind == 1) ? p.layers[l].ffn_norm : p.final_norm;
+    const uint16_t* emb = nullptr;
+    const float* src = nullptr;
+    if (kind == 0 && l == 0) {
+        int tok = p.tokens[b];
+        if (tok < 0 || tok >= p.V) {
+            if (lane == 0) set_error(p, kErrInvalid, ti, -5, tok, b);
+            tok = 0;
+        }
+        emb = p.tok_emb + (size_t)tok * H;
+    } else if (kind == 1) {
+        src = p.x_mid + ((size_t)l * p.max_batch + b) * H;
+    } else {
+        src = p.x_out + ((size_t)(l - 1) * p.max_batch + b) * H;   // kind 2 runs at l = L
+    }
+    auto load4 = [&](int i) -> float4 {
+        if (emb) {
+            const uint2 u = __ldg(reinterpret_cast<const uint2*>(emb + i));
+            return make_float4(bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y));
+        }
+        return __ldcg(reinterpret_cast<const float4*>(src + i));
+    };
+    float ss = 0.0f;
+    for (int i = lane * 4; i < H; i += 128) {
+        const float4 x = load4(i);
+        ss = fmaf(x.x, x.x, ss);
+        ss = fmaf(x.y, x.y, ss);
+        ss = fmaf(x.z, x.z, ss);
+        ss = fmaf(x.w, x.w, ss);
+    }
+    ss = warp_sum(ss);
+    const float rstd = 1.0f / sqrtf(ss / (float)H + p.eps);
+    for (int i = lane * 4; i < H; i += 128) {
+        const float4 x = load4(i);
+        const uint2 g = __ldg(reinterpret_cast<const uint2*>(gain + i));
+        put_operand4(p, op, olayer, b, H, i,
+                     make_float4((x.x * rstd) * bf_lo(g.x), (x.y * rstd) * bf_hi(g.x),
+                                 (x.z * rstd) * bf_lo(g.y), (x.w * rstd) * bf_hi(g.y)));
+    }
+}
+
+// The last split of a tile: the splits' partial sums added in split order (the
+// same order on every run), then the operator's epilogue for every batch row of
+// the step.  128 threads (consumer warps 0-3).
+__device__ void mm_epilogue(const Params& p, const Task& t, int tid) {
+    const int Sk = t.nblk, l = t.layer, nrows = (int)(t.r1 - t.r0);
+    const size_t sstride = (size_t)p.bp * kMmRows;
+    const float* part0 = p.mm_part + (size_t)t.aux * sstride;
+    if (t.op == MK_OP_MM_GATEUP) {            // rows 0..63 gate, 64..127 up, of FFN rows r0..r0+63
+        const int i = tid & 63;
+        if (i >= nrows) return;
+        const int f = (int)t.r0 + i;
+        for (int b = tid >> 6; b < p.batch; b += 2) {
+            float g = 0.0f, u = 0.0f;
+            for (int sp = 0; sp < Sk; ++sp) {
+                g += __ldcg(part0 + sp * sstride + (size_t)b * kMmRows + i);
+                u += __ldcg(part0 + sp * sstride + (size_t)b * kMmRows + 64 + i);
+            }
+            const float a = silu_f(g) * u;
+            p.act[((size_t)l * p.max_batch + b) * p.F + f] = a;
+            uint16_t hi, lo;
+            split_hilo(a, hi, lo);
+            const size_t base = (size_t)l * 2 * p.bp;
+            p.opnd[kOpAct][(base + b) * p.F + f] = hi;
+            p.opnd[kOpAct][(base + p.bp + b) * p.F + f] = lo;
+        }
+        return;
+    }
+    const int i = tid;
+    if (i >= nrows) return;
+    const int r = (int)t.r0 + i;
+    const size_t qkvw = (size_t)(p.nq + 2 * p.nkv) * p.hd;
+    for (int b = 0; b < p.batch; ++b) {
+        float v = 0.0f;
+        for (int sp = 0; sp < Sk; ++sp) v += __ldcg(part0 + sp * sstride + (size_t)b * kMmRows + i);
+        const size_t lb = (size_t)l * p.max_batch + b;
+        switch (t.op) {
+            case MK_OP_MM_QKV: p.qkv[lb * qkvw + r] = v; break;
+            case MK_OP_MM_OPROJ: p.x_mid[lb * p.H + r] = x_in(p, l, b, r) + v; break;
+            case MK_OP_MM_DOWN: p.x_out[lb * p.H + r] = x_mid_at(p, l, b, r) + v; break;
+            case MK_OP_MM_LMHEAD: p.logits[(size_t)b * p.V + r] = v; break;
+            default: break;
+        }
+    }
+}
+
+// Tensor-core tile (one K-split of 128 weight rows x bp batch columns).  Warp 0
+// issues the MMAs from one lane as each K-block's weight and activation boxes
+// land; the commit after each K-block releases both stages once the MMAs have
+// read them (it is the eighth arrival on their empty barriers, warps 1-7 give
+// the other seven).  Then warps 0-3 read the accumulator (warp q owns TMEM lanes
+// 32q..32q+31, which are tile rows), store this split's partial sums, and the
+// last split of the tile to arrive reduces and finishes it.
+__device__ bool mm_task(const Params& p, Smem& sm, const Task& t, int ti, int& stage, uint32_t& lap,
+                        uint32_t& mm_seq, uint32_t& mph, int buf) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nch = (int)t.nchunks;
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t idesc = mm_idesc(p.bp);
+    const uint32_t lo_off = (uint32_t)p.bp * 128u;
+    int wst = stage;
+    for (int c = 0; c < nch; ++c) {
+        if (c > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 10)) {
+            sm.flag[3] = 1;
+            return false;
+        }
+        if (sm.info[stage].task != ti) {
+            set_error(p, kErrFault, ti, -4, sm.info[stage].task, 3);
+            sm.flag[3] = 1;
+            return false;
+        }
+        if (warp == 0) {
+            if (c & 1) {
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(sm.ring[wst]), x = smem_u32(sm.ring[stage]);
+#pragma unroll
+                    for (int kk = 0; kk < kMmK / 16; ++kk) {
+                        const uint64_t ad = sw128_desc(a + kk * 32);
+                        tc_mma_bf16(tmem, ad, sw128_desc(x + kk * 32), idesc, (c > 1 || kk > 0) ? 1u : 0u);
+                        tc_mma_bf16(tmem, ad, sw128_desc(x + lo_off + kk * 32), idesc, 1u);
+                    }
+                    tc_commit(&sm.empty[wst]);
+                    tc_commit(&sm.empty[stage]);
+                    if (c == nch - 1) tc_commit(&sm.mm_acc);
+                }
+                __syncwarp();
+            } else {
+                wst = stage;
+            }
+        } else {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        }
+        if (++stage == kStages) { stage = 0; ++lap; }
+    }
+    ++mm_seq;
+    if (warp >= 4) return true;
+    if (!mbar_wait_bounded(p, &sm.mm_acc, (mm_seq - 1) & 1, 11)) {
+        sm.flag[3] = 1;
+        return false;
+    }
+    tc_fence_after();
+    const int row = warp * 32 + lane;
+    float* part = p.mm_part + ((size_t)t.aux + t.chunk_rows) * p.bp * kMmRows;
+    for (int c0 = 0; c0 < p.bp; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) part[(size_t)(c0 + j) * kMmRows + row] = __uint_as_float(r[j]);
+    }
+    tc_fence_before();
+    __threadfence();
+    if (!msync4(p, sm, mph)) return false;   // every partial stored; the accumulator is free again
+    if (tid == 0) {
+        const uint32_t old = atomicAdd(p.mm_cnt + t.pad, 1u);
+        sm.mm_last = (old + 1u == (uint32_t)t.nblk * p.epoch) ? 1 : 0;
+    }
+    if (!msync4(p, sm, mph)) return false;
+    const bool last = sm.mm_last != 0;
+    if (last) {
+        __threadfence();
+        mm_epilogue(p, t, tid);
+        fence_proxy_async_global();
+        __threadfence();
+    }
+    if (tid == 0) sm.ep_task[buf].sig = last ? t.sig : MK_NO_EVENT;
+    return true;
+}
+
 template <int HPG, int DPL>
 __device__ void consumer_loop(const Params& p, Smem& sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1755,6 +2127,19 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
     float2 xr[kMaxVecPerThread][4];
     int x_key_op = -1, x_key_layer = -1, x_key_b = -1, x_key_aux = -1;
     uint32_t ok_evt[4] = {MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT};   // per warp
+    uint32_t mm_seq = 0;                                // tensor-core tiles started by this CTA
+    uint32_t mph = 0;                                   // phase of sm.mm_sync (warps 0-3)
+    const uint32_t tmem_cols = (p.bp <= 32) ? 32u : (uint32_t)p.bp;
+    if (p.mm) {
+        // the accumulator of the batched tiles: 128 lanes x bp fp32 columns of TMEM
+        if (warp == 0) {
+            tmem_alloc(&sm.tmem_base, tmem_cols);
+            tmem_relinquish();
+        }
+        tc_fence_before();
+        csync(p, sm, cph);
+        tc_fence_after();
+    }
 
     // Each warp waits for its own data and dependencies, runs its share of the task,
     // leaves its partial row sums in red[buf] and arrives on red_full[buf]; the
@@ -1802,6 +2187,25 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             sm.ep_ti[buf] = ti;
         }
 
+        if (t.op == MK_OP_NORM) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);     // the marker stage
+            if (++stage == kStages) { stage = 0; ++lap; }
+            norm_task(p, t, ti, warp, lane);
+            fence_proxy_async_global();
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.red_full[buf]);
+            ++seq;
+            continue;
+        }
+        if (is_mm_op(t.op)) {
+            if (!mm_task(p, sm, t, ti, stage, lap, mm_seq, mph, buf)) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.red_full[buf]);
+            ++seq;
+            continue;
+        }
         if (t.op == MK_OP_ATTN) {
             bool abort_all = false;
             attention_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
@@ -1880,6 +2284,17 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             sm.ep_ti[buf] = -1;
             mbar_arrive_cnt(&sm.red_full[buf], kConsumerWarps);
         }
+    }
+    if (p.mm && warp == 0) {
+        // every MMA this CTA issued has completed (also after an abort) before the
+        // tensor memory is released
+        if (lane == 0) {
+            tc_commit(&sm.mm_drain);
+            (void)mbar_wait_bounded(p, &sm.mm_drain, 0, 12);
+        }
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(sm.tmem_base, tmem_cols);
     }
 }
 
@@ -1963,7 +2378,7 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
             if (ti < 0) { end = true; break; }          // end of work
             const Task t = sm.ep_task[buf];
             uint32_t evt = t.sig;
-            if (t.op != MK_OP_ATTN && !(t.op == MK_OP_LMHEAD && p.skip_lm)) {
+            if (is_gemv(t.op) && !(t.op == MK_OP_LMHEAD && p.skip_lm)) {
                 GemvGeom g;
                 gemv_geom(p, t, g, false);
                 const int wpg = is_warp_row(t.flags) ? 1
@@ -2021,11 +2436,19 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&sm.empty[s], kConsumerWarps);
         }
         mbar_init(&sm.csync, kConsumerWarps);
+        mbar_init(&sm.mm_acc, 1);
+        mbar_init(&sm.mm_drain, 1);
+        mbar_init(&sm.mm_sync, 4);
         for (int i = 0; i < kRedBufs; ++i) {
             mbar_init(&sm.red_full[i], kConsumerWarps);
             mbar_init(&sm.red_free[i], 1);
         }
         for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
+        // the 128-byte-swizzled tensor-core operands need 1 KB-aligned stages
+        if (p.mm && (smem_u32(sm.ring) & 1023u) != 0) {
+            set_error(p, kErrFault, -1, -9, (int)(smem_u32(sm.ring) & 1023u), 0);
+            sm.flag[3] = 1;
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();

@@ -85,6 +85,25 @@ inline uint8_t fast_path_for(int K, int rows, int nblk) {
     return kFastNone;
 }
 
+// Batched projection tiles (tcgen05): 128 weight rows (the MMA's M) by the
+// padded batch (its N: 16, 32 or 64) per tile, streamed in K-blocks of 64
+// columns.  Each K-block takes two ring stages: the weight box (128 rows x 128
+// bytes, 128-byte swizzle, 16 KB) and the activation box (the N hi rows then
+// the N lo rows of the bf16 split of the fp32 input, 128-byte swizzle).
+constexpr int kMmRows = 128;
+constexpr int kMmK = 64;
+constexpr int kMaxMmBatch = 64;
+constexpr int kNormRowsPerTask = 8;     // one batch row per consumer warp
+// Tensor maps: the five activation operands first, then the weights.
+enum MmOperand { kOpXq = 0, kOpXf = 1, kOpAo = 2, kOpAct = 3, kOpXl = 4, kNumOperands = 5 };
+constexpr int kMapsPerLayer = 7;        // wq, wk, wv, wo, w_gate, w_up, w_down
+inline int weight_map_index(int layer, int which) { return kNumOperands + layer * kMapsPerLayer + which; }
+inline int lm_map_index(int n_layers) { return kNumOperands + n_layers * kMapsPerLayer; }
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+inline bool is_mm_op(int op) { return op >= MK_OP_MM_QKV && op <= MK_OP_MM_LMHEAD; }
+
 // Device task record (32 bytes).
 struct Task {
     uint8_t op;
@@ -100,6 +119,12 @@ struct Task {
     // loaded model (zero otherwise): the weight rows of each block start at src[i];
     // chunks are chunk_rows whole rows, or (chunk_rows == 0) rows in stage-sized
     // segments.
+    //
+    // Tensor-core tiles (MK_OP_MM_*) use the same fields differently:
+    //   src[i]     weight box i: tensor-map index (low 32 bits), first row (high 32)
+    //   row_bytes  first K-block of this split; pad2: one past its last K-block
+    //   chunk_rows split index s; nblk: the tile's split count; nchunks: 2 per K-block
+    //   pad        the tile's arrival counter; aux: partial-sum slot of split 0
     uint64_t src[2];
     uint32_t row_bytes;
     uint16_t chunk_rows;
@@ -176,6 +201,14 @@ struct Params {
     const int* page_table;
     int n_pages, max_pages;
     float* logits;
+
+    // batched projection tiles (max_batch > 1)
+    int mm;                      // 1: the graph uses tensor-core tiles
+    int bp;                      // padded batch: the MMA's N (16, 32 or 64)
+    const void* tmaps;           // CUtensorMap array (operands, then weights), 64-byte aligned
+    uint16_t* opnd[kNumOperands];   // bf16 [rows][K]: per layer 2 * bp rows (hi, then lo)
+    float* mm_part;              // split partial sums: [slot][bp][128]
+    uint32_t* mm_cnt;            // per-tile split arrivals
 };
 
 // Sets the text returned by mk_last_error_string() for the calling thread.

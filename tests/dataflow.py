@@ -20,6 +20,17 @@ Read/write sets per operator mirror the megakernel's tiles:
   lmhead   reads x_in[L] (all)                 writes logits[rows]
 For MoE models x_in[l+1][i] is x_mid[l][i] combined with ypart[l][k][i] for all k
 and the routing weights sel[l].
+
+Batched graphs (tensor-core tiles; x_in, x_mid hold B rows of H):
+  norm     reads its batch rows [r0, r1) of x_in[l] (aux 0), x_mid[l] (aux 1)
+           or x_in[L] (aux 2)              writes those rows of opq[l] / opf[l] / opl
+  mm_*     split b of aux splits writes its partial; the last split to run reads
+           every partial and the tile's inputs, writes the rows, and signals:
+  mm_qkv   reads opq[l] (all)                  writes qkv[l][rows]
+  mm_oproj reads part[l] (all), x_in[l][b, rows] for every b   writes x_mid[l][b, rows]
+  mm_gu    reads opf[l] (all)                  writes act[l][rows]
+  mm_down  reads act[l] (all), x_mid[l][b, rows]   writes x_in[l+1][b, rows]
+  mm_lm    reads opl (all)                     writes logits[rows]
 """
 from __future__ import annotations
 
@@ -30,7 +41,8 @@ from typing import Dict, List
 import numpy as np
 
 OP = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
-      8: "exp_gu", 9: "exp_dn"}
+      8: "exp_gu", 9: "exp_dn", 10: "norm", 11: "mm_qkv", 12: "mm_oproj", 13: "mm_gu", 14: "mm_down",
+      15: "mm_lm"}
 NO_EVENT = 0xFFFFFFFF
 M64 = (1 << 64) - 1
 
@@ -91,7 +103,11 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
         else:
             T[("act", l)] = Tensor(F)
             T[("x_in", l + 1)] = Tensor(B * H)
+        T[("opq", l)] = Tensor(B * H)
+        T[("opf", l)] = Tensor(B * H)
+    T[("opl",)] = Tensor(B * H)
     T[("logits",)] = Tensor(V)
+    mm_arrivals = defaultdict(int)
     tasks_split = {tk.layer: tk.r1 for tk in tasks if tk.op == 2}
     router_arr = defaultdict(int)
     n_router = defaultdict(int)
@@ -194,6 +210,43 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
             d = read_xin(L, 0, H, who)
             t("logits").write(r0, r1, _mix(base ^ d), who)
             signal(tk.signal)
+        elif op == "norm":
+            src = {0: ("x_in", l), 1: ("x_mid", l), 2: ("x_in", L)}[tk.aux]
+            dst = {0: ("opq", l), 1: ("opf", l), 2: ("opl",)}[tk.aux]
+            d = T[src].read(r0 * H, r1 * H, who)
+            T[dst].write(r0 * H, r1 * H, _mix(base ^ d), who)
+            signal(tk.signal)
+        elif op.startswith("mm_"):
+            key = (op, l, r0)
+            if ("mmp",) + key not in T:
+                T[("mmp",) + key] = Tensor(tk.aux)
+            T[("mmp",) + key].write(tk.b, tk.b + 1, _mix(base), who)
+            mm_arrivals[key] += 1
+            if mm_arrivals[key] == tk.aux:               # the last split finishes the tile
+                d = T[("mmp",) + key].read(0, tk.aux, who)
+                if op == "mm_qkv":
+                    d += t("opq", l).read(0, B * H, who)
+                    t("qkv", l).write(r0, r1, _mix(d & M64), who)
+                elif op == "mm_oproj":
+                    for bb in range(B):
+                        for gg in range(nkv):
+                            lo = (bb * nkv + gg) * 4096
+                            d += t("part", l).read(lo, lo + tasks_split[l], who)
+                    for bb in range(B):
+                        dd = (d + t("x_in", l).read(bb * H + r0, bb * H + r1, who)) & M64
+                        t("x_mid", l).write(bb * H + r0, bb * H + r1, _mix(dd), who)
+                elif op == "mm_gu":
+                    d += t("opf", l).read(0, B * H, who)
+                    t("act", l).write(r0, r1, _mix(d & M64), who)
+                elif op == "mm_down":
+                    d += t("act", l).read(0, F, who)
+                    for bb in range(B):
+                        dd = (d + t("x_mid", l).read(bb * H + r0, bb * H + r1, who)) & M64
+                        t("x_in", l + 1).write(bb * H + r0, bb * H + r1, _mix(dd), who)
+                else:
+                    d += t("opl").read(0, B * H, who)
+                    t("logits").write(r0, r1, _mix(d & M64), who)
+                signal(tk.signal)
         else:
             raise Violation(f"unknown op {tk.op}")
         done += 1

@@ -176,3 +176,101 @@ def test_invalid_shapes_are_rejected_on_the_host():
         mk.mk_plan_taskgraph(desc_of(syn.TINY), 0, 64, 148)
     with pytest.raises(mk.MkError):
         mk.mk_plan_taskgraph(desc_of(syn.TINY), 1, 0, 148)
+
+
+# ---------------------------------------------------------------- batched graphs
+
+def _tile_groups(tasks):
+    """Tensor-core tiles grouped by (op, layer, first row): one producer each."""
+    groups = {}
+    for i, t in enumerate(tasks):
+        if t.op in mk.MM_OPS:
+            groups.setdefault((t.op, t.layer, t.r0), []).append(i)
+    return groups
+
+
+@pytest.mark.parametrize("B", [2, 4, 16, 64])
+@pytest.mark.parametrize("cfg", [syn.TINY, syn.LLAMA8B], ids=lambda c: c.name)
+def test_batched_plan_is_topological_and_thresholds_match_signals(cfg, B):
+    info, tasks, thr = plan(cfg, max_batch=B, max_ctx=8192 + 200)
+    assert info.max_batch == B
+    ops = {t.op for t in tasks}
+    assert ops == {mk.MK_OP_NORM, mk.MK_OP_ATTN, *mk.MM_OPS}, "batched graphs use only tensor-core tiles"
+    groups = _tile_groups(tasks)
+    signalled = [0] * len(thr)
+    for i, t in enumerate(tasks):
+        if t.op not in mk.MM_OPS and t.signal != mk.MK_NO_EVENT:
+            signalled[t.signal] += 1
+        assert t.pointer_wait == mk.MK_NO_EVENT
+    for key, idx in groups.items():
+        splits = sorted(tasks[i].b for i in idx)
+        assert splits == list(range(tasks[idx[0]].aux)), f"tile {key}: splits {splits}"
+        sigs = {tasks[i].signal for i in idx}
+        assert len(sigs) == 1
+        sig = sigs.pop()
+        if sig != mk.MK_NO_EVENT:
+            signalled[sig] += 1                 # the last split signals once per tile
+    assert signalled == thr
+    last_signal = {}
+    for i, t in enumerate(tasks):
+        if t.signal != mk.MK_NO_EVENT:
+            last_signal[t.signal] = i
+    for i, t in enumerate(tasks):
+        if t.wait[0] != mk.MK_NO_EVENT:
+            assert last_signal[t.wait[0]] < i, "a wait on a later task"
+    # tiles: 128 output rows (64 FFN rows for gate/up: their 64 gate and 64 up rows)
+    for t in tasks:
+        if t.op in mk.MM_OPS:
+            assert t.r1 - t.r0 <= (64 if t.op == mk.MK_OP_MM_GATEUP else 128)
+    # every output row of every projection is covered exactly once per layer
+    qkv_rows = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+    for op, n in ((mk.MK_OP_MM_QKV, qkv_rows), (mk.MK_OP_MM_OPROJ, cfg.hidden),
+                  (mk.MK_OP_MM_GATEUP, cfg.ffn), (mk.MK_OP_MM_DOWN, cfg.hidden)):
+        rows = sorted((k[2], tasks[v[0]].r1) for k, v in groups.items() if k[0] == op and k[1] == 0)
+        assert rows[0][0] == 0 and rows[-1][1] == n
+        assert all(a[1] == b[0] for a, b in zip(rows, rows[1:]))
+    norms = [t for t in tasks if t.op == mk.MK_OP_NORM and t.layer == 0 and t.aux == 0]
+    assert sorted((t.r0, t.r1) for t in norms)[-1][1] == B
+
+
+def test_batched_splits_fill_the_sms_8b():
+    """Tiles x splits per projection keep >= 90% of the slots of their waves busy
+    (8B shapes, 148 SMs), so no projection runs a mostly idle last wave."""
+    info, tasks, thr = plan(syn.LLAMA8B, max_batch=16, max_ctx=8192 + 200)
+    for op in mk.MM_OPS:
+        n = sum(1 for t in tasks if t.op == op and t.layer == (syn.LLAMA8B.n_layers if op == mk.MK_OP_MM_LMHEAD else 0))
+        waves = -(-n // 148)
+        assert n / (waves * 148) >= 0.85, f"op {op}: {n} tasks"
+
+
+@pytest.mark.parametrize("B", [4, 16])
+def test_batched_random_topological_orders_give_identical_bits(B):
+    info, tasks, thr = plan(syn.TINY, max_batch=B, max_ctx=128, n_sm=16)
+    ref = dataflow.run(tasks, thr, shape_of(syn.TINY, B), seed=0)
+    for s in range(1, 40):
+        out = dataflow.run(tasks, thr, shape_of(syn.TINY, B), seed=s)
+        assert (out["logits"] == ref["logits"]).all()
+
+
+def test_batched_executor_detects_a_missing_dependency():
+    """Dropping the waits of one O-projection tile must be caught in some order."""
+    info, tasks, thr = plan(syn.TINY, max_batch=4, max_ctx=128, n_sm=16)
+    victim = next(t for t in tasks if t.op == mk.MK_OP_MM_OPROJ)
+    for t in tasks:
+        if t.op == victim.op and t.layer == victim.layer and t.r0 == victim.r0:
+            t.wait[0] = mk.MK_NO_EVENT
+    caught = 0
+    for s in range(40):
+        try:
+            dataflow.run(tasks, thr, shape_of(syn.TINY, 4), seed=s)
+        except dataflow.Violation:
+            caught += 1
+    assert caught > 0
+
+
+def test_batched_plan_rejections():
+    with pytest.raises(mk.MkError) as e:
+        mk.mk_plan_taskgraph(desc_of(syn.TINY), 65, 64, 148)
+    assert e.value.status == mk.MK_ERR_UNSUPPORTED
+    with pytest.raises(mk.MkError):
+        mk.mk_plan_taskgraph(desc_of(syn.TINY_MOE), 4, 64, 148)
