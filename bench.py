@@ -44,10 +44,11 @@ def sol_tokens_per_s(bytes_per_step: float, bandwidth: float, batch: int = 1) ->
     return batch * bandwidth / bytes_per_step
 
 
-def kv_read_bytes(cfg, positions) -> float:
-    """Mean KV bytes read per step: (p+1) cached tokens x layers x (K,V) x heads x dim x 2 B."""
+def kv_read_bytes(cfg, positions, batch: int = 1) -> float:
+    """Mean KV bytes read per step: (p+1) cached tokens x layers x (K,V) x heads x dim x 2 B,
+    summed over the batch (`positions` lists every sequence's position of every step)."""
     per_tok = cfg.n_layers * 2 * cfg.n_kv_heads * cfg.head_dim * 2
-    return sum((p + 1) * per_tok for p in positions) / len(positions)
+    return batch * sum((p + 1) * per_tok for p in positions) / len(positions)
 
 
 def measured_peaks():
@@ -137,7 +138,23 @@ def workload(name: str):
         return dict(cfg=syn.LLAMA8B, seed=5, prompt=131072, gen=64, ctx0=131072,
                     desc="llama-8b-class decode, batch 1, 131072-token synthetic paged KV "
                          "(shuffled 16-token pages), 64 steps")
+    if name in BATCH_WORKLOADS:
+        B = int(name[len("batch"):])
+        lens = ragged_lengths(B, 512, 8192, 4700 + B)
+        return dict(cfg=syn.LLAMA8B, seed=6, batch=B, lens=lens, prompt=lens[0], gen=128,
+                    ctx0=max(lens),
+                    desc=f"llama-8b-class continuous batching, batch {B}, ragged contexts "
+                         f"U(512, 8192) in shuffled 16-token pages, 128 steps")
     raise SystemExit(f"unknown workload {name}")
+
+
+BATCH_WORKLOADS = ("batch1", "batch4", "batch16", "batch64")
+
+
+def ragged_lengths(B: int, lo: int, hi: int, seed: int):
+    """Cached tokens per sequence, uniform on [lo, hi] (seeded)."""
+    import numpy as np
+    return [int(x) for x in np.random.default_rng(seed).integers(lo, hi + 1, size=B)]
 
 
 def max_over_ranks(x: float, pg, device) -> float:
@@ -219,7 +236,7 @@ def run_reference(args, W):
             "n_gpus": world, "steps": n, "warmup": min(args.warmup, 1),
             "ms_per_step": 1000.0 / rate, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": W["desc"], "batch": 1},
+            "config": {"workload": W["desc"], "batch": W.get("batch", 1)},
             "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -261,34 +278,41 @@ def run_gpu(args, W):
                 n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, ffn=cfg.ffn, vocab=cfg.vocab,
                 rms_eps=cfg.rms_eps, rope_theta=cfg.rope_theta, n_experts=cfg.n_experts,
                 top_k=cfg.top_k, expert_ffn=cfg.expert_ffn, moe_renorm=cfg.moe_renorm)
+    B = W.get("batch", 1)
+    lens = W.get("lens", [W["prompt"]])
+    if "lens" in W:
+        max_ctx = max(lens) + span
     page_table = None
     n_pages = None
-    if args.workload == "long131k":
-        pages = (max_ctx + 15) // 16
+    if args.workload == "long131k" or "lens" in W:
+        per_seq = (max_ctx + 15) // 16
+        pages = B * per_seq
         perm = syn.page_permutation(pages, syn.SEED_KV + W["seed"])
-        page_table = torch.tensor(perm, dtype=torch.int32, device=dev).view(1, pages)
+        page_table = torch.tensor(perm, dtype=torch.int32, device=dev).view(B, per_seq)
         n_pages = pages
-    dec = Decoder(desc, [t.data_ptr() for t in ts], 1, max_ctx, page_table=page_table,
+    dec = Decoder(desc, [t.data_ptr() for t in ts], B, max_ctx, page_table=page_table,
                   n_pages=n_pages, device=f"cuda:{local}")
     stream = torch.cuda.current_stream(dev)
     prompt_toks = torch.tensor(syn.host_tokens(W["prompt"], syn.SEED_PROMPT + W["seed"], cfg.vocab),
                                dtype=torch.int32, device=dev)
     if ctx0 > 0:
-        for l in range(cfg.n_layers):
-            syn.dev_fill_kv_paged(dec.k_pages[l], dec.page_table[0], 0, 0, ctx0, cfg, 16,
-                                  syn.SEED_KV + W["seed"], syn.TID_K_BASE + l)
-            syn.dev_fill_kv_paged(dec.v_pages[l], dec.page_table[0], 0, 0, ctx0, cfg, 16,
-                                  syn.SEED_KV + W["seed"], syn.TID_V_BASE + l)
+        for b in range(B):
+            for l in range(cfg.n_layers):
+                syn.dev_fill_kv_paged(dec.k_pages[l], dec.page_table[b], b, 0, lens[b], cfg, 16,
+                                      syn.SEED_KV + W["seed"], syn.TID_K_BASE + l)
+                syn.dev_fill_kv_paged(dec.v_pages[l], dec.page_table[b], b, 0, lens[b], cfg, 16,
+                                      syn.SEED_KV + W["seed"], syn.TID_V_BASE + l)
     else:
         dec.prefill(prompt_toks)          # the 39-token prompt through the same megakernel
     dec.check()
-    gen_toks = syn.host_tokens(n_steps_total, syn.SEED_PROMPT + 100 + W["seed"], cfg.vocab)
-    positions = [W["prompt"] + (i % span) for i in range(n_steps_total)]
+    # step i feeds B tokens; sequence b is at position lens[b] + (i % span)
+    gen_toks = syn.host_tokens(n_steps_total * B, syn.SEED_PROMPT + 100 + W["seed"], cfg.vocab)
+    positions = [lens[b] + (i % span) for i in range(n_steps_total) for b in range(B)]
     toks_d = torch.tensor(gen_toks, dtype=torch.int32, device=dev)
     pos_d = torch.tensor(positions, dtype=torch.int32, device=dev)
 
     def launch(i):
-        mk.mk_decode_step(dec.state, toks_d[i:].data_ptr(), pos_d[i:].data_ptr(), 1, dec.kv,
+        mk.mk_decode_step(dec.state, toks_d[i * B:].data_ptr(), pos_d[i * B:].data_ptr(), B, dec.kv,
                           dec.logits.data_ptr(), stream.cuda_stream)
 
     for i in range(args.warmup):
@@ -318,11 +342,11 @@ def run_gpu(args, W):
         raise SystemExit(f"timed steps failed: {mk.mk_last_error_string()}")
     per = [events[k].elapsed_time(events[k + 1]) for k in range(args.steps)]
     total_ms = max_over_ranks(events[0].elapsed_time(events[-1]), pg, dev)
-    timed_pos = positions[args.warmup:]
+    timed_pos = positions[args.warmup * B:]
     info = dec.info
-    bytes_step = float(info.weight_bytes_per_step) + kv_read_bytes(cfg, timed_pos)
-    tok_s = replica_tokens_per_s(args.steps, world, total_ms)
-    sol = sol_tokens_per_s(bytes_step, SOL_BW)
+    bytes_step = float(info.weight_bytes_per_step) + kv_read_bytes(cfg, timed_pos, B)
+    tok_s = replica_tokens_per_s(args.steps, world, total_ms, B)
+    sol = sol_tokens_per_s(bytes_step, SOL_BW, B)
     peak, peak_kind = measured_peaks()
     launch_ms = statistics.mean(per)
     achieved = bytes_step / (launch_ms / 1e3) / 1e9
@@ -333,7 +357,7 @@ def run_gpu(args, W):
         k_e2e = min(args.steps, 100)
         tok_h = torch.tensor(gen_toks, dtype=torch.int32).pin_memory()
         pos_h = torch.tensor(positions, dtype=torch.int32).pin_memory()
-        logits_h = torch.empty((1, cfg.vocab), dtype=torch.float32).pin_memory()
+        logits_h = torch.empty((B, cfg.vocab), dtype=torch.float32).pin_memory()
         torch.cuda.synchronize(dev)
         if pg:
             pg.barrier()
@@ -342,15 +366,15 @@ def run_gpu(args, W):
         e0.record(stream)
         for k in range(k_e2e):
             i = args.warmup + k
-            mk.mk_decode_step_host(dec.state, tok_h[i:].data_ptr(), pos_h[i:].data_ptr(), 1, dec.kv,
-                                   logits_h.data_ptr(), stream.cuda_stream)
+            mk.mk_decode_step_host(dec.state, tok_h[i * B:].data_ptr(), pos_h[i * B:].data_ptr(), B,
+                                   dec.kv, logits_h.data_ptr(), stream.cuda_stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
         if dec.sync() != mk.MK_OK:
             raise SystemExit(f"e2e steps failed: {mk.mk_last_error_string()}")
-        e2e = {"value": replica_tokens_per_s(k_e2e, world, e2e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": 8, "d2h_bytes_per_step": 4 * cfg.vocab, "steps": k_e2e,
+        e2e = {"value": replica_tokens_per_s(k_e2e, world, e2e_ms, B), "unit": "tokens/s",
+               "h2d_bytes_per_step": 8 * B, "d2h_bytes_per_step": 4 * cfg.vocab * B, "steps": k_e2e,
                "api": "mk_decode_step_host"}
 
     traffic = None
@@ -366,13 +390,14 @@ def run_gpu(args, W):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": W["desc"], "batch": 1, "weights": "bf16", "activations": "f32",
-                   "kv_cache": "bf16", "positions": [timed_pos[0], max(timed_pos)],
+        "config": {"workload": W["desc"], "batch": B, "weights": "bf16", "activations": "f32",
+                   "kv_cache": "bf16", "positions": [min(timed_pos), max(timed_pos)],
                    "l2": "inputs larger than L2 (every step streams all weights)",
                    "parallelism": "replicas" if world > 1 else "single-gpu"},
         "sol_pct": 100.0 * tok_s / world / sol,
         "sol_tokens_per_s": sol,
         "bytes_per_step": bytes_step,
+        "tiles": "tcgen05 projection tiles" if B > 1 else "CUDA-core GEMV tiles",
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_kind": f"{peak_kind} hbm_gbs (copy)",
@@ -475,7 +500,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=507)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mk", "reference"], default="mk")
-    ap.add_argument("--workload", default="llama8b", choices=["llama8b", "tiny", "moe30b", "long131k"])
+    ap.add_argument("--workload", default="llama8b",
+                    choices=["llama8b", "tiny", "moe30b", "long131k", *BATCH_WORKLOADS])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,

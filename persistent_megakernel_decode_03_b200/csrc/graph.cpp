@@ -141,9 +141,12 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     // attention split-K: as many (sequence, kv head, split) tasks as fit in one wave
     // over the SMs (one more would make every layer's attention phase take two
     // task durations), but at most one split per 64 positions of context.
-    // Batched graphs aim at about two tasks per SM instead: ragged context lengths
-    // make the splits unequal, and the dynamic queue evens them out.
-    int S = (B == 1) ? n_sm / (B * nkv) : (int)std::lround(2.0 * n_sm / (double)(B * nkv));
+    // Batched graphs aim at about four tasks per SM instead (ragged context lengths
+    // make the splits unequal; the dynamic queue evens them out), with splits of at
+    // least ~512 positions of a half-full context (shorter ones cost more in fixed
+    // per-task work than they gain in balance).
+    int S = (B == 1) ? n_sm / (B * nkv)
+                     : (int)std::min<int64_t>(std::lround(4.0 * n_sm / (double)(B * nkv)), ceil_div(max_ctx, 1024));
     S = std::max(1, std::min<int>(S, (int)ceil_div(max_ctx, 64)));
     g.S = S;
 
@@ -283,7 +286,9 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
                         tk.pad2 = (uint32_t)kb1;
                         tk.chunk_rows = (uint16_t)sp;
                         tk.nblk = (uint16_t)Sk;
-                        tk.nchunks = (uint32_t)(2 * (kb1 - kb0));
+                        // a stage per weight box, plus one per group of kx activation boxes
+                        const int64_t kx = std::max(1, kStageBytes / (2 * g.bp * 128));
+                        tk.nchunks = (uint32_t)((kb1 - kb0) + ceil_div(kb1 - kb0, kx));
                         tk.pad = (uint32_t)counter;
                         task_in[t] = in;
                         task_entity[t] = eid;

@@ -264,9 +264,10 @@ struct __align__(128) Smem {
     int ep_ti[kRedBufs];                     // its index (-1: end of work)
     float ep_resid[kRedBufs][kMaxTaskRows];  // residual rows (O-proj, down), loaded early by warp 0
     int attn_last;                           // this CTA's attention split arrived last
-    uint64_t mm_acc;                         // tensor-core tile: the accumulator is complete
+    uint64_t mm_acc[2];                      // tensor-core tiles: accumulator buffer a is complete
+    uint64_t mm_free[2];                     // ... and has been read (4 arrivals: warps 4-7)
     uint64_t mm_drain;                       // tensor-core work drained before TMEM is freed
-    uint64_t mm_sync;                        // consumer warps 0-3 (arrival count 4)
+    uint64_t mm_sync;                        // consumer warps 4-7 (arrival count 4)
     uint32_t tmem_base;                      // TMEM address of the accumulator (batched graphs)
     int mm_last;                             // this CTA's split of a tile arrived last
     int pid[kPidRing];                       // producer: physical page ids read ahead
@@ -461,8 +462,8 @@ __device__ __forceinline__ void csync(const Params& p, Smem& sm, uint32_t& phase
     if (!mbar_wait_bounded(p, &sm.csync, phase, 8)) sm.flag[3] = 1;
     phase ^= 1;
 }
-// The same among consumer warps 0-3 (the warps that own the TMEM lane quarters);
-// false when the wait gave up (the CTA is aborting).
+// The same among consumer warps 4-7 (the warps that read the accumulators: warp
+// w owns TMEM lane quarter w - 4); false when the wait gave up (the CTA is aborting).
 __device__ __forceinline__ bool msync4(const Params& p, Smem& sm, uint32_t& phase) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.mm_sync);
@@ -662,9 +663,14 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
 }
 
 // Tensor-core tile: per K-block one weight box (128 rows, or the matching 64 gate
-// and 64 up rows) and one activation box (hi rows then lo rows), each in its own
-// stage.  The activations are written by earlier tasks, so the first weight box
-// goes out before the wait for them and every other load after it.
+// and 64 up rows) in its own stage; the activation boxes (hi rows then lo rows)
+// of up to mm_kblocks_per_xstage consecutive K-blocks share one stage ahead of
+// their weight boxes, so most of the ring holds weights in flight.  The
+// activations are written by earlier tasks: the loads wait for their event.
+__device__ __forceinline__ int mm_kblocks_per_xstage(int bp) {
+    const int k = kStageBytes / (2 * bp * 128);
+    return k < 1 ? 1 : k;
+}
 __device__ __forceinline__ const void* tmap_at(const Params& p, uint32_t idx) {
     return reinterpret_cast<const uint8_t*>(p.tmaps) + (size_t)idx * 128;
 }
@@ -686,6 +692,7 @@ __device__ __noinline__ bool produce_mm(const Params& p, Smem& sm, const Task& t
     const int xy = (t.op == MK_OP_MM_LMHEAD) ? 0 : (int)t.layer * 2 * p.bp;
     const uint32_t xbytes = 2u * (uint32_t)p.bp * 128u;
     const int kb0 = (int)t.row_bytes, kb1 = (int)t.pad2, nch = (int)t.nchunks;
+    const int kx = mm_kblocks_per_xstage(p.bp);
     int c = 0;
     auto open_stage = [&](uint32_t bytes) -> bool {
         if (!pr_acquire(p, sm, ring)) return false;
@@ -697,27 +704,33 @@ __device__ __noinline__ bool produce_mm(const Params& p, Smem& sm, const Task& t
         mbar_arrive_expect_tx(&sm.full[ring.stage], bytes);
         return true;
     };
-    for (int kb = kb0; kb < kb1; ++kb) {
-        if (!open_stage((uint32_t)kStageBytes)) return false;
-        uint8_t* dst = sm.ring[ring.stage];
-        if (two) {
-            tma_load_2d_hint(dst, w0, kb * kMmK, wy, &sm.full[ring.stage], pol);
-            tma_load_2d_hint(dst + kStageBytes / 2, w1, kb * kMmK, wy, &sm.full[ring.stage], pol);
-        } else {
-            tma_load_2d_hint(dst, w0, kb * kMmK, wy, &sm.full[ring.stage], pol);
-        }
+    if (t.wait0 != MK_NO_EVENT) {
+        if (!event_wait(p, t.wait0, p.thr[t.wait0] * p.epoch + p.wait_offset, ti)) return false;
+        // the operand was written through the generic proxy by other CTAs; order those
+        // writes before this CTA's tensor loads
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    for (int g0 = kb0; g0 < kb1; g0 += kx) {
+        const int g1 = min(kb1, g0 + kx);
+        // the activation boxes of the group's K-blocks, side by side in one stage, ahead
+        // of the weight boxes: each weight box is multiplied as soon as it lands
+        if (!open_stage(xbytes * (uint32_t)(g1 - g0))) return false;
+        for (int kb = g0; kb < g1; ++kb)
+            tma_load_2d(sm.ring[ring.stage] + (size_t)(kb - g0) * xbytes, xm, kb * kMmK, xy, &sm.full[ring.stage]);
         pr_advance(ring);
         ++c;
-        if (kb == kb0 && t.wait0 != MK_NO_EVENT) {
-            if (!event_wait(p, t.wait0, p.thr[t.wait0] * p.epoch + p.wait_offset, ti)) return false;
-            // the operand was written through the generic proxy by other CTAs; order
-            // those writes before this CTA's tensor loads
-            asm volatile("fence.proxy.async.global;" ::: "memory");
+        for (int kb = g0; kb < g1; ++kb) {
+            if (!open_stage((uint32_t)kStageBytes)) return false;
+            uint8_t* dst = sm.ring[ring.stage];
+            if (two) {
+                tma_load_2d_hint(dst, w0, kb * kMmK, wy, &sm.full[ring.stage], pol);
+                tma_load_2d_hint(dst + kStageBytes / 2, w1, kb * kMmK, wy, &sm.full[ring.stage], pol);
+            } else {
+                tma_load_2d_hint(dst, w0, kb * kMmK, wy, &sm.full[ring.stage], pol);
+            }
+            pr_advance(ring);
+            ++c;
         }
-        if (!open_stage(xbytes)) return false;
-        tma_load_2d(sm.ring[ring.stage], xm, kb * kMmK, xy, &sm.full[ring.stage]);
-        pr_advance(ring);
-        ++c;
     }
     return true;
 }
@@ -1931,59 +1944,75 @@ __device__ void router_finalize(const Params& p, Smem& sm, int l) {
 
 // ----------------------------------------------------------------------------- batched tiles
 
-// RMSNorm of one batch row per warp into the operand of the next projection:
-// h = x / sqrt(mean(x^2) + eps) * g (kind 0: attention norm of the residual
-// entering layer l, the token embedding at l = 0; kind 1: FFN norm of the
-// residual after attention; kind 2: final norm).  Rows past the step's batch
-// are written as zeros.
-__device__ void norm_task(const Params& p, const Task& t, int ti, int warp, int lane) {
-    const int b = (int)t.r0 + warp;
-    if (b >= (int)t.r1) return;
-    const int kind = t.aux, l = t.layer, H = p.H;
+// RMSNorm of one batch row into the operand of the next projection, by all 256
+// consumer threads: h = x / sqrt(mean(x^2) + eps) * g (kind 0: attention norm of
+// the residual entering layer l, the token embedding at l = 0; kind 1: FFN norm
+// of the residual after attention; kind 2: final norm).  Every thread loads its
+// 4-column groups (and their gains) at once, so the row costs one round trip, a
+// block-wide sum and the stores.  Rows past the step's batch are written as zeros.
+constexpr int kNormVec = 16;   // 4-column groups per thread: hidden <= 16384
+template <bool EMB>
+__device__ __forceinline__ float4 norm_load4(const float* src, const uint16_t* emb, int i) {
+    if constexpr (EMB) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(emb + i));
+        return make_float4(bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y));
+    } else {
+        return __ldcg(reinterpret_cast<const float4*>(src + i));
+    }
+}
+template <bool EMB>
+__device__ void norm_row(const Params& p, Smem& sm, uint32_t& cph, const float* src, const uint16_t* emb,
+                         const uint16_t* gain, int op, int olayer, int b) {
+    const int H = p.H, tid = threadIdx.x;
+    float4 v[kNormVec];
+    uint2 g[kNormVec];
+    float ss = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kNormVec; ++u) {
+        const int i = (tid + u * kConsumerThreads) * 4;
+        if (i < H) {
+            v[u] = norm_load4<EMB>(src, emb, i);
+            g[u] = __ldg(reinterpret_cast<const uint2*>(gain + i));
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kNormVec; ++u) {
+        const int i = (tid + u * kConsumerThreads) * 4;
+        if (i < H) ss = fmaf(v[u].w, v[u].w, fmaf(v[u].z, v[u].z, fmaf(v[u].y, v[u].y, fmaf(v[u].x, v[u].x, ss))));
+    }
+    const float tot = block_sum(p, sm, cph, ss);
+    const float rstd = 1.0f / sqrtf(tot / (float)H + p.eps);
+#pragma unroll
+    for (int u = 0; u < kNormVec; ++u) {
+        const int i = (tid + u * kConsumerThreads) * 4;
+        if (i < H)
+            put_operand4(p, op, olayer, b, H, i,
+                         make_float4((v[u].x * rstd) * bf_lo(g[u].x), (v[u].y * rstd) * bf_hi(g[u].x),
+                                     (v[u].z * rstd) * bf_lo(g[u].y), (v[u].w * rstd) * bf_hi(g[u].y)));
+    }
+}
+__device__ void norm_task(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti) {
+    const int kind = t.aux, l = t.layer, H = p.H, tid = threadIdx.x;
     const int op = (kind == 0) ? kOpXq : (kind == 1) ? kOpXf : kOpXl;
     const int olayer = (kind == 2) ? 0 : l;
-    if (b >= p.batch) {
-        for (int i = lane * 4; i < H; i += 128) put_operand4(p, op, olayer, b, H, i, make_float4(0.f, 0.f, 0.f, 0.f));
-        return;
-    }
     const uint16_t* gain = (kind == 0) ? p.layers[l].attn_norm : (kind == 1) ? p.layers[l].ffn_norm : p.final_norm;
-    const uint16_t* emb = nullptr;
-    const float* src = nullptr;
-    if (kind == 0 && l == 0) {
-        int tok = p.tokens[b];
-        if (tok < 0 || tok >= p.V) {
-            if (lane == 0) set_error(p, kErrInvalid, ti, -5, tok, b);
-            tok = 0;
+    for (int b = (int)t.r0; b < (int)t.r1; ++b) {
+        if (b >= p.batch) {
+            for (int i = tid * 4; i < H; i += kConsumerThreads * 4)
+                put_operand4(p, op, olayer, b, H, i, make_float4(0.f, 0.f, 0.f, 0.f));
+        } else if (kind == 0 && l == 0) {
+            int tok = p.tokens[b];
+            if (tok < 0 || tok >= p.V) {
+                if (tid == 0) set_error(p, kErrInvalid, ti, -5, tok, b);
+                tok = 0;
+            }
+            norm_row<true>(p, sm, cph, nullptr, p.tok_emb + (size_t)tok * H, gain, op, olayer, b);
+        } else if (kind == 1) {
+            norm_row<false>(p, sm, cph, p.x_mid + ((size_t)l * p.max_batch + b) * H, nullptr, gain, op, olayer, b);
+        } else {   // kind 0 at l > 0, or kind 2 (l = L): the residual after layer l - 1
+            norm_row<false>(p, sm, cph, p.x_out + ((size_t)(l - 1) * p.max_batch + b) * H, nullptr, gain, op,
+                            olayer, b);
         }
-        emb = p.tok_emb + (size_t)tok * H;
-    } else if (kind == 1) {
-        src = p.x_mid + ((size_t)l * p.max_batch + b) * H;
-    } else {
-        src = p.x_out + ((size_t)(l - 1) * p.max_batch + b) * H;   // kind 2 runs at l = L
-    }
-    auto load4 = [&](int i) -> float4 {
-        if (emb) {
-            const uint2 u = __ldg(reinterpret_cast<const uint2*>(emb + i));
-            return make_float4(bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y));
-        }
-        return __ldcg(reinterpret_cast<const float4*>(src + i));
-    };
-    float ss = 0.0f;
-    for (int i = lane * 4; i < H; i += 128) {
-        const float4 x = load4(i);
-        ss = fmaf(x.x, x.x, ss);
-        ss = fmaf(x.y, x.y, ss);
-        ss = fmaf(x.z, x.z, ss);
-        ss = fmaf(x.w, x.w, ss);
-    }
-    ss = warp_sum(ss);
-    const float rstd = 1.0f / sqrtf(ss / (float)H + p.eps);
-    for (int i = lane * 4; i < H; i += 128) {
-        const float4 x = load4(i);
-        const uint2 g = __ldg(reinterpret_cast<const uint2*>(gain + i));
-        put_operand4(p, op, olayer, b, H, i,
-                     make_float4((x.x * rstd) * bf_lo(g.x), (x.y * rstd) * bf_hi(g.x),
-                                 (x.z * rstd) * bf_lo(g.y), (x.w * rstd) * bf_hi(g.y)));
     }
 }
 
@@ -2032,76 +2061,111 @@ __device__ void mm_epilogue(const Params& p, const Task& t, int tid) {
     }
 }
 
-// Tensor-core tile (one K-split of 128 weight rows x bp batch columns).  Warp 0
-// issues the MMAs from one lane as each K-block's weight and activation boxes
-// land; the commit after each K-block releases both stages once the MMAs have
-// read them (it is the eighth arrival on their empty barriers, warps 1-7 give
-// the other seven).  Then warps 0-3 read the accumulator (warp q owns TMEM lanes
-// 32q..32q+31, which are tile rows), store this split's partial sums, and the
-// last split of the tile to arrive reduces and finishes it.
+// Tensor-core tile (one K-split of 128 weight rows x bp batch columns).
+//  * Every consumer warp waits for every stage of the tile and warps 1-7 release
+//    it at once; one lane of warp 0 issues the MMAs of each weight box as it lands
+//    (the group's activation stage came first) and adds the eighth arrival with a
+//    tcgen05.commit, once the MMAs have read the stage.  (Every warp walks every
+//    stage so that no warp can run a lap ahead of the producer on a stage's
+//    barrier, where a parity wait could not tell two phases apart.)
+//  * The accumulator is double-buffered in TMEM: tile k of this CTA uses buffer
+//    k & 1, so warp 0 multiplies tile k + 1 while warps 4-7 (warp w owns TMEM lane
+//    quarter w - 4, i.e. tile rows 32 (w - 4) ..) read tile k, store this split's
+//    partial sums, and the last split of the tile to arrive reduces and finishes it.
 __device__ bool mm_task(const Params& p, Smem& sm, const Task& t, int ti, int& stage, uint32_t& lap,
                         uint32_t& mm_seq, uint32_t& mph, int buf) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nch = (int)t.nchunks;
-    const uint32_t tmem = sm.tmem_base;
-    const uint32_t idesc = mm_idesc(p.bp);
-    const uint32_t lo_off = (uint32_t)p.bp * 128u;
-    int wst = stage;
-    for (int c = 0; c < nch; ++c) {
-        if (c > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 10)) {
-            sm.flag[3] = 1;
-            return false;
-        }
-        if (sm.info[stage].task != ti) {
-            set_error(p, kErrFault, ti, -4, sm.info[stage].task, 3);
-            sm.flag[3] = 1;
-            return false;
-        }
-        if (warp == 0) {
-            if (c & 1) {
-                if (lane == 0) {
-                    tc_fence_after();
-                    const uint32_t a = smem_u32(sm.ring[wst]), x = smem_u32(sm.ring[stage]);
-#pragma unroll
-                    for (int kk = 0; kk < kMmK / 16; ++kk) {
-                        const uint64_t ad = sw128_desc(a + kk * 32);
-                        tc_mma_bf16(tmem, ad, sw128_desc(x + kk * 32), idesc, (c > 1 || kk > 0) ? 1u : 0u);
-                        tc_mma_bf16(tmem, ad, sw128_desc(x + lo_off + kk * 32), idesc, 1u);
-                    }
-                    tc_commit(&sm.empty[wst]);
-                    tc_commit(&sm.empty[stage]);
-                    if (c == nch - 1) tc_commit(&sm.mm_acc);
-                }
-                __syncwarp();
-            } else {
-                wst = stage;
+    const uint32_t abuf = mm_seq & 1u, use = mm_seq >> 1;   // accumulator buffer and its use count
+    ++mm_seq;
+    const uint32_t acc = sm.tmem_base + abuf * (uint32_t)(2 * p.bp);
+    if (warp != 0) {
+        for (int c = 0; c < nch; ++c) {
+            if (c > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 10)) {
+                sm.flag[3] = 1;
+                return false;
             }
-        } else {
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
+            if (++stage == kStages) { stage = 0; ++lap; }
         }
-        if (++stage == kStages) { stage = 0; ++lap; }
+    } else {
+        // one MMA per 16 columns of K multiplies the weight rows by the hi AND lo rows
+        // of the activations (N = 2 bp: its cost does not depend on N); the two halves
+        // of the accumulator are added when it is read
+        const uint32_t idesc = mm_idesc(2 * p.bp);
+        const uint32_t xbytes = 2u * (uint32_t)p.bp * 128u;
+        const int kx = mm_kblocks_per_xstage(p.bp);
+        int kb_left = (int)t.pad2 - (int)t.row_bytes;   // K-blocks not yet multiplied
+        int gs = min(kx, kb_left), gk = -1;              // group size; -1: its activation stage is next
+        int xst = stage;
+        bool first_mma = true;
+        for (int c = 0; c < nch; ++c) {
+            if (c > 0 && !mbar_wait_bounded(p, &sm.full[stage], lap & 1, 10)) {
+                sm.flag[3] = 1;
+                return false;
+            }
+            if (sm.info[stage].task != ti) {
+                set_error(p, kErrFault, ti, -4, sm.info[stage].task, 3);
+                sm.flag[3] = 1;
+                return false;
+            }
+            if (gk < 0) {
+                xst = stage;
+                gk = 0;
+            } else {
+                if (lane == 0) {
+                    if (first_mma && use > 0 && !mbar_wait_bounded(p, &sm.mm_free[abuf], (use - 1) & 1, 14))
+                        sm.flag[3] = 1;
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(sm.ring[stage]);
+                    const uint32_t x = smem_u32(sm.ring[xst]) + (uint32_t)gk * xbytes;
+#pragma unroll
+                    for (int kk = 0; kk < kMmK / 16; ++kk) {
+                        tc_mma_bf16(acc, sw128_desc(a + kk * 32), sw128_desc(x + kk * 32), idesc,
+                                    first_mma ? 0u : 1u);
+                        first_mma = false;
+                    }
+                    tc_commit(&sm.empty[stage]);
+                    if (gk == gs - 1) tc_commit(&sm.empty[xst]);
+                    if (c == nch - 1) tc_commit(&sm.mm_acc[abuf]);
+                }
+                __syncwarp();
+                if (sm.flag[3]) return false;
+                if (++gk == gs) {
+                    kb_left -= gs;
+                    gs = min(kx, kb_left);
+                    gk = -1;
+                }
+            }
+            if (++stage == kStages) { stage = 0; ++lap; }
+        }
     }
-    ++mm_seq;
-    if (warp >= 4) return true;
-    if (!mbar_wait_bounded(p, &sm.mm_acc, (mm_seq - 1) & 1, 11)) {
+    if (warp < 4) return true;
+    // ---- warps 4-7: read the accumulator, store this split's partial sums
+    const int q = warp - 4, row = q * 32 + lane, etid = tid - 4 * 32;
+    if (!mbar_wait_bounded(p, &sm.mm_acc[abuf], use & 1, 11)) {
         sm.flag[3] = 1;
         return false;
     }
     tc_fence_after();
-    const int row = warp * 32 + lane;
     float* part = p.mm_part + ((size_t)t.aux + t.chunk_rows) * p.bp * kMmRows;
+    const uint32_t lane_base = acc + ((uint32_t)(q * 32) << 16);
     for (int c0 = 0; c0 < p.bp; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, r);
+        uint32_t h[16], lo[16];
+        tmem_ld16(lane_base + (uint32_t)c0, h);                 // W . x_hi
+        tmem_ld16(lane_base + (uint32_t)(p.bp + c0), lo);       // W . x_lo
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) part[(size_t)(c0 + j) * kMmRows + row] = __uint_as_float(r[j]);
+        for (int j = 0; j < 16; ++j)
+            part[(size_t)(c0 + j) * kMmRows + row] = __uint_as_float(h[j]) + __uint_as_float(lo[j]);
     }
     tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.mm_free[abuf]);        // the buffer may take the next tile
     __threadfence();
-    if (!msync4(p, sm, mph)) return false;   // every partial stored; the accumulator is free again
-    if (tid == 0) {
+    if (!msync4(p, sm, mph)) return false;                // every partial of this split stored
+    if (etid == 0) {
         const uint32_t old = atomicAdd(p.mm_cnt + t.pad, 1u);
         sm.mm_last = (old + 1u == (uint32_t)t.nblk * p.epoch) ? 1 : 0;
     }
@@ -2109,11 +2173,11 @@ __device__ bool mm_task(const Params& p, Smem& sm, const Task& t, int ti, int& s
     const bool last = sm.mm_last != 0;
     if (last) {
         __threadfence();
-        mm_epilogue(p, t, tid);
+        mm_epilogue(p, t, etid);
         fence_proxy_async_global();
         __threadfence();
     }
-    if (tid == 0) sm.ep_task[buf].sig = last ? t.sig : MK_NO_EVENT;
+    if (etid == 0) sm.ep_task[buf].sig = last ? t.sig : MK_NO_EVENT;
     return true;
 }
 
@@ -2128,10 +2192,10 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
     int x_key_op = -1, x_key_layer = -1, x_key_b = -1, x_key_aux = -1;
     uint32_t ok_evt[4] = {MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT, MK_NO_EVENT};   // per warp
     uint32_t mm_seq = 0;                                // tensor-core tiles started by this CTA
-    uint32_t mph = 0;                                   // phase of sm.mm_sync (warps 0-3)
-    const uint32_t tmem_cols = (p.bp <= 32) ? 32u : (uint32_t)p.bp;
+    uint32_t mph = 0;                                   // phase of sm.mm_sync (warps 4-7)
+    const uint32_t tmem_cols = (uint32_t)(4 * p.bp);     // 64, 128 or 256: two buffers of hi and lo halves
     if (p.mm) {
-        // the accumulator of the batched tiles: 128 lanes x bp fp32 columns of TMEM
+        // the accumulators of the batched tiles: 128 lanes x 2 x 2 bp fp32 columns of TMEM
         if (warp == 0) {
             tmem_alloc(&sm.tmem_base, tmem_cols);
             tmem_relinquish();
@@ -2191,7 +2255,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);     // the marker stage
             if (++stage == kStages) { stage = 0; ++lap; }
-            norm_task(p, t, ti, warp, lane);
+            norm_task(p, sm, cph, t, ti);
             fence_proxy_async_global();
             __threadfence();
             __syncwarp();
@@ -2436,7 +2500,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&sm.empty[s], kConsumerWarps);
         }
         mbar_init(&sm.csync, kConsumerWarps);
-        mbar_init(&sm.mm_acc, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.mm_acc[i], 1);
+            mbar_init(&sm.mm_free[i], 4);
+        }
         mbar_init(&sm.mm_drain, 1);
         mbar_init(&sm.mm_sync, 4);
         for (int i = 0; i < kRedBufs; ++i) {

@@ -87,13 +87,14 @@ inline uint8_t fast_path_for(int K, int rows, int nblk) {
 
 // Batched projection tiles (tcgen05): 128 weight rows (the MMA's M) by the
 // padded batch (its N: 16, 32 or 64) per tile, streamed in K-blocks of 64
-// columns.  Each K-block takes two ring stages: the weight box (128 rows x 128
-// bytes, 128-byte swizzle, 16 KB) and the activation box (the N hi rows then
-// the N lo rows of the bf16 split of the fp32 input, 128-byte swizzle).
+// columns.  Each K-block's weight box (128 rows x 128 bytes, 128-byte swizzle,
+// 16 KB) takes a ring stage; the activation boxes (the N hi rows then the N lo
+// rows of the bf16 split of the fp32 input, 128-byte swizzle) of up to 4
+// consecutive K-blocks share one more stage.
 constexpr int kMmRows = 128;
 constexpr int kMmK = 64;
 constexpr int kMaxMmBatch = 64;
-constexpr int kNormRowsPerTask = 8;     // one batch row per consumer warp
+constexpr int kNormRowsPerTask = 1;     // a norm task: one batch row, all consumer threads
 // Tensor maps: the five activation operands first, then the weights.
 enum MmOperand { kOpXq = 0, kOpXf = 1, kOpAo = 2, kOpAct = 3, kOpXl = 4, kNumOperands = 5 };
 constexpr int kMapsPerLayer = 7;        // wq, wk, wv, wo, w_gate, w_up, w_down
@@ -123,7 +124,9 @@ struct Task {
     // Tensor-core tiles (MK_OP_MM_*) use the same fields differently:
     //   src[i]     weight box i: tensor-map index (low 32 bits), first row (high 32)
     //   row_bytes  first K-block of this split; pad2: one past its last K-block
-    //   chunk_rows split index s; nblk: the tile's split count; nchunks: 2 per K-block
+    //   chunk_rows split index s; nblk: the tile's split count
+    //   nchunks    stages: one per K-block's weight box, plus one per group of
+    //              16 KB / (2 * bp * 128 B) K-blocks' activation boxes
     //   pad        the tile's arrival counter; aux: partial-sum slot of split 0
     uint64_t src[2];
     uint32_t row_bytes;
