@@ -384,7 +384,9 @@ def run_gpu(args, W):
             tr = json.load(f)
         ent = tr.get(args.workload)
         if ent and ent.get("kernel_source_sha") == kernel_source_sha():
-            traffic = ent["bytes_per_launch"]
+            # DRAM bytes of a smaller capture of the same kernel, as a ratio to its
+            # algorithmic bytes (traffic grows with the weight and KV bytes streamed)
+            traffic = ent["ratio_to_algorithmic"] * bytes_step
     line = {
         "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,

@@ -1950,7 +1950,7 @@ __device__ void router_finalize(const Params& p, Smem& sm, int l) {
 // of the residual after attention; kind 2: final norm).  Every thread loads its
 // 4-column groups (and their gains) at once, so the row costs one round trip, a
 // block-wide sum and the stores.  Rows past the step's batch are written as zeros.
-constexpr int kNormVec = 16;   // 4-column groups per thread: hidden <= 16384
+constexpr int kNormCols = 4 * kConsumerThreads;   // columns per pass chunk: 4 per thread
 template <bool EMB>
 __device__ __forceinline__ float4 norm_load4(const float* src, const uint16_t* emb, int i) {
     if constexpr (EMB) {
@@ -1960,38 +1960,30 @@ __device__ __forceinline__ float4 norm_load4(const float* src, const uint16_t* e
         return __ldcg(reinterpret_cast<const float4*>(src + i));
     }
 }
+// Each thread owns 4 consecutive columns of every 1024-column chunk; the sum of
+// squares pass, a block-wide sum, then the scaling pass re-reads x with the gains.
 template <bool EMB>
 __device__ void norm_row(const Params& p, Smem& sm, uint32_t& cph, const float* src, const uint16_t* emb,
                          const uint16_t* gain, int op, int olayer, int b) {
-    const int H = p.H, tid = threadIdx.x;
-    float4 v[kNormVec];
-    uint2 g[kNormVec];
+    const int H = p.H, c0 = threadIdx.x * 4;
     float ss = 0.0f;
-#pragma unroll
-    for (int u = 0; u < kNormVec; ++u) {
-        const int i = (tid + u * kConsumerThreads) * 4;
-        if (i < H) {
-            v[u] = norm_load4<EMB>(src, emb, i);
-            g[u] = __ldg(reinterpret_cast<const uint2*>(gain + i));
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < kNormVec; ++u) {
-        const int i = (tid + u * kConsumerThreads) * 4;
-        if (i < H) ss = fmaf(v[u].w, v[u].w, fmaf(v[u].z, v[u].z, fmaf(v[u].y, v[u].y, fmaf(v[u].x, v[u].x, ss))));
+    for (int i = c0; i < H; i += kNormCols) {
+        const float4 v = norm_load4<EMB>(src, emb, i);
+        ss = fmaf(v.w, v.w, fmaf(v.z, v.z, fmaf(v.y, v.y, fmaf(v.x, v.x, ss))));
     }
     const float tot = block_sum(p, sm, cph, ss);
     const float rstd = 1.0f / sqrtf(tot / (float)H + p.eps);
-#pragma unroll
-    for (int u = 0; u < kNormVec; ++u) {
-        const int i = (tid + u * kConsumerThreads) * 4;
-        if (i < H)
-            put_operand4(p, op, olayer, b, H, i,
-                         make_float4((v[u].x * rstd) * bf_lo(g[u].x), (v[u].y * rstd) * bf_hi(g[u].x),
-                                     (v[u].z * rstd) * bf_lo(g[u].y), (v[u].w * rstd) * bf_hi(g[u].y)));
+    for (int i = c0; i < H; i += kNormCols) {
+        const float4 v = norm_load4<EMB>(src, emb, i);
+        const uint2 g = __ldg(reinterpret_cast<const uint2*>(gain + i));
+        put_operand4(p, op, olayer, b, H, i,
+                     make_float4((v.x * rstd) * bf_lo(g.x), (v.y * rstd) * bf_hi(g.x),
+                                 (v.z * rstd) * bf_lo(g.y), (v.w * rstd) * bf_hi(g.y)));
     }
 }
-__device__ void norm_task(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti) {
+// (Out of line, like the tensor-core tile below: the batched tasks keep their
+// registers out of the batch-1 consumer loop's allocation.)
+__device__ __noinline__ void norm_task(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti) {
     const int kind = t.aux, l = t.layer, H = p.H, tid = threadIdx.x;
     const int op = (kind == 0) ? kOpXq : (kind == 1) ? kOpXf : kOpXl;
     const int olayer = (kind == 2) ? 0 : l;
@@ -2072,7 +2064,7 @@ __device__ void mm_epilogue(const Params& p, const Task& t, int tid) {
 //    k & 1, so warp 0 multiplies tile k + 1 while warps 4-7 (warp w owns TMEM lane
 //    quarter w - 4, i.e. tile rows 32 (w - 4) ..) read tile k, store this split's
 //    partial sums, and the last split of the tile to arrive reduces and finishes it.
-__device__ bool mm_task(const Params& p, Smem& sm, const Task& t, int ti, int& stage, uint32_t& lap,
+__device__ __noinline__ bool mm_task(const Params& p, Smem& sm, const Task& t, int ti, int& stage, uint32_t& lap,
                         uint32_t& mm_seq, uint32_t& mph, int buf) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nch = (int)t.nchunks;
@@ -2181,8 +2173,10 @@ __device__ bool mm_task(const Params& p, Smem& sm, const Task& t, int ti, int& s
     return true;
 }
 
-template <int HPG, int DPL>
-__device__ void consumer_loop(const Params& p, Smem& sm) {
+// MM: the instantiation for batched graphs (norm tasks, tensor-core tiles,
+// attention); the batch-1 instantiation holds the GEMV tiles and none of that.
+template <int HPG, int DPL, bool MM>
+__device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int stage = 0;
     uint32_t lap = 0;
@@ -2194,7 +2188,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
     uint32_t mm_seq = 0;                                // tensor-core tiles started by this CTA
     uint32_t mph = 0;                                   // phase of sm.mm_sync (warps 4-7)
     const uint32_t tmem_cols = (uint32_t)(4 * p.bp);     // 64, 128 or 256: two buffers of hi and lo halves
-    if (p.mm) {
+    if constexpr (MM) {
         // the accumulators of the batched tiles: 128 lanes x 2 x 2 bp fp32 columns of TMEM
         if (warp == 0) {
             tmem_alloc(&sm.tmem_base, tmem_cols);
@@ -2251,6 +2245,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             sm.ep_ti[buf] = ti;
         }
 
+        if constexpr (MM) {
         if (t.op == MK_OP_NORM) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);     // the marker stage
@@ -2270,6 +2265,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             ++seq;
             continue;
         }
+        }
         if (t.op == MK_OP_ATTN) {
             bool abort_all = false;
             attention_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
@@ -2286,6 +2282,12 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             continue;
         }
 
+        if constexpr (MM) {
+            // a batched graph holds no GEMV tiles
+            set_error(p, kErrFault, ti, -10, t.op, 0);
+            sm.flag[3] = 1;
+            break;
+        } else {
         // ---- GEMV task
         const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm);
         const bool fast = (t.flags != kFastNone) && !skip;
@@ -2338,6 +2340,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.red_full[buf]);
         ++seq;
+        }
     }
     // end of work for the epilogue warp: a marker once every consumer warp has left
     // the loop (a full set of arrivals on the next buffer set)
@@ -2349,7 +2352,7 @@ __device__ void consumer_loop(const Params& p, Smem& sm) {
             mbar_arrive_cnt(&sm.red_full[buf], kConsumerWarps);
         }
     }
-    if (p.mm && warp == 0) {
+    if (MM && warp == 0) {
         // every MMA this CTA issued has completed (also after an abort) before the
         // tensor memory is released
         if (lane == 0) {
@@ -2489,7 +2492,7 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
 
 // ----------------------------------------------------------------------------- kernel
 
-template <int HPG, int DPL>
+template <int HPG, int DPL, bool MM>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
@@ -2525,7 +2528,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     if (warp < kConsumerWarps) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
         const long long k0 = clock64();
-        consumer_loop<HPG, DPL>(p, sm);
+        consumer_loop<HPG, DPL, MM>(p, sm);
         if (threadIdx.x == 0) stat_add(p, 3, (unsigned long long)(clock64() - k0));
         return;
     }
@@ -2543,7 +2546,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 
 template <int HPG, int DPL>
 static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream) {
-    auto kern = megakernel<HPG, DPL>;
+    auto kern = p.mm ? megakernel<HPG, DPL, true> : megakernel<HPG, DPL, false>;
     static bool attr_set = false;   // per instantiation; set before first launch on each device use
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(Smem));
@@ -2586,15 +2589,15 @@ cudaError_t megakernel_occupancy(int hpg, int hd, int* blocks_per_sm) {
     const int dpl = hd / 32;
     const void* f = nullptr;
     if (dpl == 4) {
-        if (hpg == 1) f = (const void*)megakernel<1, 4>;
-        if (hpg == 2) f = (const void*)megakernel<2, 4>;
-        if (hpg == 4) f = (const void*)megakernel<4, 4>;
-        if (hpg == 8) f = (const void*)megakernel<8, 4>;
+        if (hpg == 1) f = (const void*)megakernel<1, 4, false>;
+        if (hpg == 2) f = (const void*)megakernel<2, 4, false>;
+        if (hpg == 4) f = (const void*)megakernel<4, 4, false>;
+        if (hpg == 8) f = (const void*)megakernel<8, 4, false>;
     } else {
-        if (hpg == 1) f = (const void*)megakernel<1, 2>;
-        if (hpg == 2) f = (const void*)megakernel<2, 2>;
-        if (hpg == 4) f = (const void*)megakernel<4, 2>;
-        if (hpg == 8) f = (const void*)megakernel<8, 2>;
+        if (hpg == 1) f = (const void*)megakernel<1, 2, false>;
+        if (hpg == 2) f = (const void*)megakernel<2, 2, false>;
+        if (hpg == 4) f = (const void*)megakernel<4, 2, false>;
+        if (hpg == 8) f = (const void*)megakernel<8, 2, false>;
     }
     if (!f) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
