@@ -170,7 +170,9 @@ enum {
     MK_OP_MM_OPROJ = 12,  /* rows of Wo . o plus the residual */
     MK_OP_MM_GATEUP = 13, /* FFN rows [r0, r1) (<= 64): silu(Wg h) * (Wu h) */
     MK_OP_MM_DOWN = 14,   /* rows of Wd . a plus the residual */
-    MK_OP_MM_LMHEAD = 15  /* rows of Wlm . rmsnorm(x) */
+    MK_OP_MM_LMHEAD = 15, /* rows of Wlm . rmsnorm(x) */
+    MK_OP_KVAPPEND = 16   /* batched graphs: K (rotated) and V of batch rows [r0, r1) into
+                             their pages; the attention tasks of the layer wait for them */
 };
 
 #define MK_NO_EVENT 0xFFFFFFFFu
@@ -246,13 +248,23 @@ mk_status mk_decode_step_host(mk_state* state, const int32_t* token_ids, const i
                               int batch, const mk_paged_kv* kv, float* logits_host,
                               mk_stream stream);
 
-/* Runs a prompt through the same graph, one token per step, for ONE sequence
- * whose page-table row is kv->page_table[0]: tokens (device int32
- * [n_tokens]) at positions pos0 .. pos0+n_tokens-1.  Writes the logits of
- * the last prompt token to last_logits (device fp32 [vocab]); the LM head is
- * skipped for the other tokens. */
+/* Runs a prompt through the same graph for ONE sequence whose page-table row
+ * is kv->page_table[0]: tokens (device int32 [n_tokens]) at positions
+ * pos0 .. pos0+n_tokens-1.  Writes the logits of the last prompt token to
+ * last_logits (device fp32 [vocab]).
+ *  - batch-1 graph: one token per step; the LM head is skipped for all but the
+ *    last token;
+ *  - batched graph (max_batch > 1): up to max_batch prompt tokens per step, as
+ *    the batch rows of the tensor-core tiles (row i at position pos0 + i), with
+ *    causal attention over the cache: each row's K/V is appended before any row
+ *    attends (MPK digest, Part 1: a prompt's tokens are one batched operator). */
 mk_status mk_prefill(mk_state* state, const int32_t* tokens, int n_tokens, int pos0,
                      const mk_paged_kv* kv, float* last_logits, mk_stream stream);
+
+/* mk_prefill for the sequence whose page-table row is kv->page_table[seq_slot]
+ * (0 <= seq_slot < max_batch; batch-1 graphs: 0). */
+mk_status mk_prefill_seq(mk_state* state, const int32_t* tokens, int n_tokens, int pos0, int seq_slot,
+                         const mk_paged_kv* kv, float* last_logits, mk_stream stream);
 
 /* The decode step of mk_decode_step for callers that cannot allocate device
  * memory: code running where cudaMalloc is not allowed (inside a host callback,

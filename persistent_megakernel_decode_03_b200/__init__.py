@@ -34,9 +34,10 @@ MK_OP_ROUTER, MK_OP_EXP_GATEUP, MK_OP_EXP_DOWN = 7, 8, 9
 MK_OP_NORM, MK_OP_MM_QKV, MK_OP_MM_OPROJ, MK_OP_MM_GATEUP, MK_OP_MM_DOWN, MK_OP_MM_LMHEAD = (
     10, 11, 12, 13, 14, 15)
 MM_OPS = (MK_OP_MM_QKV, MK_OP_MM_OPROJ, MK_OP_MM_GATEUP, MK_OP_MM_DOWN, MK_OP_MM_LMHEAD)
+MK_OP_KVAPPEND = 16
 OP_NAMES = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
             8: "exp_gateup", 9: "exp_down", 10: "norm", 11: "mm_qkv", 12: "mm_oproj", 13: "mm_gateup",
-            14: "mm_down", 15: "mm_lmhead"}
+            14: "mm_down", 15: "mm_lmhead", 16: "kvappend"}
 
 # Exported symbols (declared in include/mk.h).
 SYMBOLS = (
@@ -45,7 +46,7 @@ SYMBOLS = (
     "mk_graph_destroy", "mk_graph_get_info", "mk_graph_export_tasks", "mk_graph_export_thresholds",
     "mk_wave_stats", "mk_state_create", "mk_state_destroy", "mk_state_set_timeout",
     "mk_state_debug_wait_offset", "mk_state_set_prefetch",
-    "mk_decode_step", "mk_decode_step_host", "mk_prefill", "mk_decode_step_noalloc", "mk_sync",
+    "mk_decode_step", "mk_decode_step_host", "mk_prefill", "mk_prefill_seq", "mk_decode_step_noalloc", "mk_sync",
     "mk_state_read_counters",
     "mk_state_read_buffer", "mk_state_read_trace", "mk_state_read_stats", "mk_last_error_string",
     "mk_version",
@@ -124,6 +125,7 @@ def lib() -> ctypes.CDLL:
             "mk_decode_step": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_decode_step_host": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_prefill": ([vp, vp, i32, i32, P(mk_paged_kv), vp, vp], st),
+            "mk_prefill_seq": ([vp, vp, i32, i32, i32, P(mk_paged_kv), vp, vp], st),
             "mk_decode_step_noalloc": ([P(mk_model_desc), vp, i32, i32, vp, vp, i32, P(mk_paged_kv),
                                         vp, vp], st),
             "mk_sync": ([vp, vp], st),
@@ -255,6 +257,12 @@ def mk_decode_step_host(state: int, token_ids: int, positions: int, batch: int, 
 def mk_prefill(state: int, tokens: int, n_tokens: int, pos0: int, kv: mk_paged_kv,
                last_logits: int, stream: int = 0) -> None:
     _check(lib().mk_prefill(state, tokens, n_tokens, pos0, ctypes.byref(kv), last_logits, stream))
+
+
+def mk_prefill_seq(state: int, tokens: int, n_tokens: int, pos0: int, seq_slot: int, kv: mk_paged_kv,
+                   last_logits: int, stream: int = 0) -> None:
+    _check(lib().mk_prefill_seq(state, tokens, n_tokens, pos0, seq_slot, ctypes.byref(kv), last_logits,
+                                stream))
 
 
 def mk_decode_step_noalloc(desc: mk_model_desc, weight_ptrs: Sequence[int], max_ctx: int,

@@ -222,6 +222,8 @@ mk::Params base_params(mk_state* s) {
     p.moe_w = s->moe_w;
     p.moe_sel = s->moe_sel;
     p.ypart = s->ypart;
+    p.seq_row = -1;
+    p.pos_stride = 0;
     p.mm = P.bp > 0 ? 1 : 0;
     p.bp = P.bp;
     p.tmaps = s->tmaps;
@@ -632,30 +634,67 @@ mk_status mk_decode_step_host(mk_state* s, const int32_t* token_ids, const int32
     return MK_OK;
 }
 
-mk_status mk_prefill(mk_state* s, const int32_t* tokens, int n_tokens, int pos0, const mk_paged_kv* kv,
-                     float* last_logits, mk_stream stream) {
+mk_status mk_prefill_seq(mk_state* s, const int32_t* tokens, int n_tokens, int pos0, int seq_slot,
+                         const mk_paged_kv* kv, float* last_logits, mk_stream stream) {
     if (!s || !tokens || !last_logits) return fail(MK_ERR_INVALID_ARG, "mk_prefill: null argument");
-    if (n_tokens < 1 || pos0 < 0 || pos0 + n_tokens > s->g->plan.max_ctx)
+    const GraphPlan& P = s->g->plan;
+    if (n_tokens < 1 || pos0 < 0 || pos0 + n_tokens > P.max_ctx)
         return fail(MK_ERR_INVALID_ARG, "mk_prefill: positions %d..%d outside the graph's context", pos0, pos0 + n_tokens - 1);
+    if (seq_slot < 0 || seq_slot >= P.max_batch)
+        return fail(MK_ERR_INVALID_ARG, "mk_prefill: sequence slot %d outside 0..%d", seq_slot, P.max_batch - 1);
     mk_status r = check_kv(s, kv);
     if (r != MK_OK) return r;
-    for (int i = 0; i < n_tokens; ++i) {
-        mk::Params p = base_params(s);
-        p.tokens = tokens + i;
+    auto common = [&](mk::Params& p) {
         p.positions = nullptr;
-        p.pos_offset = pos0 + i;
-        p.batch = 1;
-        p.skip_lm = (i + 1 < n_tokens) ? 1 : 0;
+        p.seq_row = seq_slot;
         p.k_pages = static_cast<uint16_t*>(kv->k_pages);
         p.v_pages = static_cast<uint16_t*>(kv->v_pages);
         p.page_table = kv->page_table;
         p.n_pages = kv->n_pages;
         p.max_pages = kv->max_pages_per_seq;
+    };
+    if (P.bp > 0) {
+        // batched graph: up to max_batch prompt tokens per launch, as the batch rows
+        // (row i at position pos0 + start + i of the one sequence)
+        const int B = P.max_batch;
+        for (int start = 0; start < n_tokens; start += B) {
+            const int chunk = std::min(B, n_tokens - start);
+            mk::Params p = base_params(s);
+            common(p);
+            p.tokens = tokens + start;
+            p.pos_offset = pos0 + start;
+            p.pos_stride = 1;
+            p.batch = chunk;
+            p.skip_lm = 0;
+            p.logits = s->logits;
+            r = launch_step(s, p, (cudaStream_t)stream);
+            if (r != MK_OK) return r;
+            if (start + chunk == n_tokens) {
+                cudaError_t e = cudaMemcpyAsync(last_logits, s->logits + (size_t)(chunk - 1) * P.desc.vocab,
+                                                sizeof(float) * P.desc.vocab, cudaMemcpyDeviceToDevice,
+                                                (cudaStream_t)stream);
+                if (e != cudaSuccess) return cuda_fail(e, "mk_prefill: logits");
+            }
+        }
+        return MK_OK;
+    }
+    for (int i = 0; i < n_tokens; ++i) {
+        mk::Params p = base_params(s);
+        common(p);
+        p.tokens = tokens + i;
+        p.pos_offset = pos0 + i;
+        p.batch = 1;
+        p.skip_lm = (i + 1 < n_tokens) ? 1 : 0;
         p.logits = last_logits;
         r = launch_step(s, p, (cudaStream_t)stream);
         if (r != MK_OK) return r;
     }
     return MK_OK;
+}
+
+mk_status mk_prefill(mk_state* s, const int32_t* tokens, int n_tokens, int pos0, const mk_paged_kv* kv,
+                     float* last_logits, mk_stream stream) {
+    return mk_prefill_seq(s, tokens, n_tokens, pos0, 0, kv, last_logits, stream);
 }
 
 mk_status mk_sync(mk_state* s, mk_stream stream) {

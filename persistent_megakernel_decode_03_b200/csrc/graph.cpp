@@ -28,7 +28,8 @@ namespace {
 
 // Tensor kinds for the region-overlap analysis.
 enum TensorKind { T_XIN = 1, T_QKV, T_O, T_XMID, T_ACT, T_ACTE, T_SEL, T_LOGITS,
-                  T_XQOP, T_XFOP, T_XLOP };   // the last three: bf16 hi/lo operands of batched tiles
+                  T_XQOP, T_XFOP, T_XLOP,     // bf16 hi/lo operands of batched tiles
+                  T_KV };                     // batched graphs: this step's K/V rows in the cache
 
 struct Region {
     int tensor;         // encoded (kind, layer, slot)
@@ -236,6 +237,9 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
                               Region{key, 0, B, (int64_t)nq * hd + kh * hd, (int64_t)nq * hd + (kh + 1) * hd},
                               Region{key, 0, B, (int64_t)(nq + nkv) * hd + kh * hd,
                                      (int64_t)(nq + nkv) * hd + (kh + 1) * hd}};
+                // batched graphs: the appended K/V of every row (whose tasks wait on all of
+                // QKV) is the one input, so the event is theirs alone
+                if (B > 1) task_in[t] = {Region{tensor_key(T_KV, l, 0), 0, B, 0, 1}};
                 own_entity(t, {Region{tensor_key(T_O, l, 0), b, b + 1, (int64_t)kh * hpg * hd,
                                       (int64_t)(kh + 1) * hpg * hd}});
             }
@@ -314,6 +318,13 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
                   {{0, qr, weight_map_index(l, 0), -1}, {qr, kr, weight_map_index(l, 1), -1},
                    {qr + kr, kr, weight_map_index(l, 2), -1}},
                   kMmRows, H, {all_rows(T_XQOP, l, 0, H)}, T_QKV, l);
+            // each sequence's new K/V into its pages; every attention task of the layer
+            // waits for all of them (under batched prefill, the rows are one sequence)
+            for (int b = 0; b < B; ++b) {
+                int t = new_task(MK_OP_KVAPPEND, l, 0, 0, (uint32_t)b, (uint32_t)(b + 1));
+                task_in[t] = {all_rows(T_QKV, l, 0, qr + 2 * kr)};
+                own_entity(t, {Region{tensor_key(T_KV, l, 0), b, b + 1, 0, 1}});
+            }
             for (int kh = 0; kh < nkv; ++kh) attn_group(l, kh);
             mm_op(MK_OP_MM_OPROJ, l, {{0, H, weight_map_index(l, 3), -1}}, kMmRows, qr,
                   {all_rows(T_O, l, 0, qr)}, T_XMID, l);
@@ -430,8 +441,14 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
         if (T[t].sig != MK_NO_EVENT) last_signaler[T[t].sig] = t;
     for (int t = 0; t < (int)T.size(); ++t) {
         uint32_t w = T[t].wait0;
-        if (w != MK_NO_EVENT && last_signaler[w] >= t)
-            return fail("internal: task list is not topologically ordered");
+        if (w != MK_NO_EVENT && last_signaler[w] >= t) {
+            const Task& a = T[t];
+            const Task& z = T[last_signaler[w]];
+            return fail("internal: task list is not topologically ordered (task " + std::to_string(t) + " op " +
+                        std::to_string(a.op) + " layer " + std::to_string(a.layer) + " waits on event " +
+                        std::to_string(w) + ", signalled by task " + std::to_string(last_signaler[w]) +
+                        " op " + std::to_string(z.op) + " layer " + std::to_string(z.layer) + ")");
+        }
     }
     g.n_events = (int)thr.size();
 

@@ -35,6 +35,7 @@
 // Params::timeout_ns, records MK_ERR_TIMEOUT and the kernel drains its own
 // copies in flight and returns.
 #include <cuda_runtime.h>
+#include <limits.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -280,7 +281,11 @@ __device__ __forceinline__ int hpg_of(const Params& p) { return p.nq / p.nkv; }
 
 // Token position of batch row b this step (validated by the caller).
 __device__ __forceinline__ int position_of(const Params& p, int b) {
-    return (p.positions ? p.positions[b] : 0) + p.pos_offset;
+    return (p.positions ? p.positions[b] : 0) + p.pos_offset + b * p.pos_stride;
+}
+// Page-table row of batch row b: its own, or (batched prefill) the one sequence's.
+__device__ __forceinline__ const int* page_row(const Params& p, int b) {
+    return p.page_table + (size_t)(p.seq_row >= 0 ? p.seq_row : b) * p.max_pages;
 }
 
 struct GemvGeom {
@@ -538,7 +543,9 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                     int j0 = 0, j1 = 0;
                     const int sa = attn_active_splits(pos + 1, (int)t.r1);
                     if ((int)t.r0 < sa) attn_range(pos + 1, sa, (int)t.r0, j0, j1);
-                    int jc = min(j1, pos);          // cached positions only; the new token is fresh
+                    // batch-1 graphs: cached positions only (the new token is fresh);
+                    // batched graphs: the new positions are in the cache too
+                    int jc = p.mm ? j1 : min(j1, pos);
                     if (jc > j0) {
                         lp0 = j0 / kPageSize;
                         npages = (jc - 1) / kPageSize - lp0 + 1;
@@ -562,8 +569,13 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
             }
             // physical page ids, read kPidBatch at a time (independent loads, one round
             // trip per batch) into a small ring in shared memory, a batch ahead of use
-            const int* prow = p.page_table + (size_t)b * p.max_pages;
+            const int* prow = page_row(p, b);
             int pid_have = 0;                              // ids [0, pid_have) of the split loaded
+            // batched graphs append this step's K/V in tasks of their own: pages holding a
+            // new position are loaded only after the attention task's event (which
+            // counts those appends); older pages stream at once
+            const int first_new = p.mm ? (p.seq_row >= 0 ? position_of(p, 0) : position_of(p, b)) : INT_MAX;
+            bool appended = !p.mm || t.wait0 == MK_NO_EVENT;
             auto pid_ensure = [&](int upto) {
                 while (pid_have < upto) {
                     int v[kPidBatch];
@@ -581,6 +593,11 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                 int first = lp0 + c * pps;
                 int n = min(pps, lp0 + npages - first);
                 pid_ensure(min(npages, c * pps + n + kPidBatch));
+                if (!appended && (first + n) * kPageSize > first_new) {
+                    if (!event_wait(p, t.wait0, p.thr[t.wait0] * p.epoch + p.wait_offset, ti)) { ok = false; break; }
+                    asm volatile("fence.proxy.async.global;" ::: "memory");   // generic-proxy writes first
+                    appended = true;
+                }
                 if (!acquire_slot()) { ok = false; break; }
                 sm.info[stage].task = ti; sm.info[stage].chunk = c; sm.info[stage].nchunks = nch;
                 sm.info[stage].aux = first;
@@ -758,7 +775,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
             ok = produce_mm(p, sm, t, ti, ring, pol);
             continue;
         }
-        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm) || t.op == MK_OP_NORM;
+        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm) || t.op == MK_OP_NORM || t.op == MK_OP_KVAPPEND;
         if (skip) {                                      // nothing to stream: a marker stage
             if (!pr_acquire(p, sm, ring)) { ok = false; break; }
             sm.info[ring.stage] = StageInfo{ti, 0, 0, 0, t};
@@ -853,7 +870,7 @@ __device__ void prefetch_loop(const Params& p) {
             attn_range(pos + 1, sa, (int)t.r0, j0, j1);
             const int jc = min(j1, pos);
             if (jc <= j0) continue;
-            const int* prow = p.page_table + (size_t)b * p.max_pages;
+            const int* prow = page_row(p, b);
             const uint32_t blk = (uint32_t)(kPageSize * p.hd * 2);
             for (int lp = j0 / kPageSize; lp <= (jc - 1) / kPageSize; ++lp) {
                 const int ph = prow[lp];
@@ -1683,7 +1700,9 @@ __device__ __forceinline__ void attn_new_token(AttnMma<HPG, DPL>& st, const floa
 // position), softmax partial over the split's positions streamed from the paged
 // cache.  Writes the partial and hands the completion to the signal warp; the
 // O-projection's input stage merges the splits in a fixed order.
-template <int HPG, int DPL>
+// MM: batched graphs, whose KV append runs in tasks of its own before attention;
+// every position, the new one included, then comes from the cache.
+template <int HPG, int DPL, bool MM>
 __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti, int& stage,
                                uint32_t& lap, bool& abort_all) {
     constexpr int HD = DPL * 32;
@@ -1698,7 +1717,7 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
         const int sa = attn_active_splits(pos + 1, S);
         if (s < sa) attn_range(pos + 1, sa, s, j0, j1);
     }
-    const bool has_new = valid && pos >= j0 && pos < j1;
+    const bool has_new = !MM && valid && pos >= j0 && pos < j1;
     const float qscale = 1.4426950408889634f / sqrtf((float)HD);   // log2(e) / sqrt(d)
 
     AttnMma<HPG, DPL> st;
@@ -1756,7 +1775,7 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
         csync(p, sm, cph);
         // KV append: the split that owns the new position writes it
         if (has_new) {
-            const int* prow = p.page_table + (size_t)b * p.max_pages;
+            const int* prow = page_row(p, b);
             const int ph = prow[pos / kPageSize];
             if (ph >= 0 && ph < p.n_pages) {
                 size_t off = ((((size_t)l * p.n_pages + ph) * p.nkv + g) * kPageSize + pos % kPageSize) * HD;
@@ -1782,7 +1801,7 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
     }
 
     // streamed chunks of cached pages (the first stage was seen complete by thread 0)
-    const int jc = min(j1, pos);
+    const int jc = MM ? j1 : min(j1, pos);
     const int pps = pages_per_stage(p);
     const int blk_elems = kPageSize * HD;
     uint8_t* stg = reinterpret_cast<uint8_t*>(sm.attn) + warp * (kPageSize * HD * 2);   // staging page
@@ -1943,6 +1962,45 @@ __device__ void router_finalize(const Params& p, Smem& sm, int l) {
 // ----------------------------------------------------------------------------- consumer loop
 
 // ----------------------------------------------------------------------------- batched tiles
+
+// K (rotated at the row's position with the RoPE table, as the attention tile
+// rotates it) and V of batch rows [r0, r1) of layer l, rounded to bf16 (RNE),
+// into their pages.  Batched graphs run this before the layer's attention, which
+// then reads every position from the cache: under batched prefill, a prompt row
+// attends to the rows before it.
+__device__ __noinline__ void kvappend_task(const Params& p, const Task& t, int ti) {
+    const int HD = p.hd, half = HD / 2, tid = threadIdx.x, l = t.layer;
+    for (int b = (int)t.r0; b < (int)t.r1; ++b) {
+        if (b >= p.batch) continue;
+        const int pos = position_of(p, b);
+        if (pos < 0 || pos >= p.max_ctx || pos / kPageSize >= p.max_pages) {
+            if (tid == 0) set_error(p, kErrInvalid, ti, -3, pos, b);
+            continue;
+        }
+        const int ph = page_row(p, b)[pos / kPageSize];
+        if (ph < 0 || ph >= p.n_pages) {
+            if (tid == 0) set_error(p, kErrInvalid, ti, -2, pos / kPageSize, b);
+            continue;
+        }
+        const float* qkv = p.qkv + ((size_t)l * p.max_batch + b) * ((p.nq + 2 * p.nkv) * HD);
+        const float2* rope = reinterpret_cast<const float2*>(p.rope + (size_t)pos * HD);   // [HD/2] (cos, sin)
+        const size_t base = (((size_t)l * p.n_pages + ph) * p.nkv) * kPageSize;
+        for (int idx = tid; idx < p.nkv * half; idx += kConsumerThreads) {
+            const int g = idx / half, i = idx % half;
+            const float* k = qkv + (size_t)(p.nq + g) * HD;
+            const float x0 = __ldcg(k + i), x1 = __ldcg(k + i + half);
+            const float2 r = __ldg(rope + i);
+            const size_t off = ((base + (size_t)g * kPageSize) + pos % kPageSize) * HD;
+            p.k_pages[off + i] = f32_to_bf16_rne(x0 * r.x - x1 * r.y);
+            p.k_pages[off + i + half] = f32_to_bf16_rne(x1 * r.x + x0 * r.y);
+        }
+        for (int idx = tid; idx < p.nkv * HD; idx += kConsumerThreads) {
+            const int g = idx / HD, i = idx % HD;
+            const size_t off = ((base + (size_t)g * kPageSize) + pos % kPageSize) * HD;
+            p.v_pages[off + i] = f32_to_bf16_rne(__ldcg(qkv + (size_t)(p.nq + p.nkv + g) * HD + i));
+        }
+    }
+}
 
 // RMSNorm of one batch row into the operand of the next projection, by all 256
 // consumer threads: h = x / sqrt(mean(x^2) + eps) * g (kind 0: attention norm of
@@ -2246,11 +2304,12 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
         }
 
         if constexpr (MM) {
-        if (t.op == MK_OP_NORM) {
+        if (t.op == MK_OP_NORM || t.op == MK_OP_KVAPPEND) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);     // the marker stage
             if (++stage == kStages) { stage = 0; ++lap; }
-            norm_task(p, sm, cph, t, ti);
+            if (t.op == MK_OP_NORM) norm_task(p, sm, cph, t, ti);
+            else kvappend_task(p, t, ti);
             fence_proxy_async_global();
             __threadfence();
             __syncwarp();
@@ -2268,7 +2327,7 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
         }
         if (t.op == MK_OP_ATTN) {
             bool abort_all = false;
-            attention_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
+            attention_task<HPG, DPL, MM>(p, sm, cph, t, ti, stage, lap, abort_all);
             if (abort_all) break;
             x_key_op = -1;
             // the input slice in registers is dead across an attention task (saves registers)

@@ -197,6 +197,8 @@ struct Params {
     const int* tokens;
     const int* positions;        // may be null (then position = pos_offset)
     int pos_offset;
+    int pos_stride;              // position of row b = positions[b] + pos_offset + b * pos_stride
+    int seq_row;                 // >= 0: every batch row uses this page-table row (batched prefill)
     int batch;
     int skip_lm;                 // 1: LM-head tasks do nothing
     uint16_t* k_pages;

@@ -239,6 +239,8 @@ extern "C" mk_status mk_decode_step_noalloc(const mk_model_desc* desc, const voi
     }
     p.tokens = token_ids;
     p.positions = positions;
+    p.seq_row = -1;
+    p.pos_stride = 0;
     p.batch = 1;
     p.k_pages = static_cast<uint16_t*>(kv->k_pages);
     p.v_pages = static_cast<uint16_t*>(kv->v_pages);

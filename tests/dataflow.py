@@ -31,6 +31,8 @@ Batched graphs (tensor-core tiles; x_in, x_mid hold B rows of H):
   mm_gu    reads opf[l] (all)                  writes act[l][rows]
   mm_down  reads act[l] (all), x_mid[l][b, rows]   writes x_in[l+1][b, rows]
   mm_lm    reads opl (all)                     writes logits[rows]
+  kvappend reads qkv[l] (all)                  writes kv[l][its batch rows]; the layer's
+           attention tasks then also read kv[l] (all rows)
 """
 from __future__ import annotations
 
@@ -42,7 +44,7 @@ import numpy as np
 
 OP = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
       8: "exp_gu", 9: "exp_dn", 10: "norm", 11: "mm_qkv", 12: "mm_oproj", 13: "mm_gu", 14: "mm_down",
-      15: "mm_lm"}
+      15: "mm_lm", 16: "kvappend"}
 NO_EVENT = 0xFFFFFFFF
 M64 = (1 << 64) - 1
 
@@ -106,6 +108,9 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
         T[("opq", l)] = Tensor(B * H)
         T[("opf", l)] = Tensor(B * H)
     T[("opl",)] = Tensor(B * H)
+    has_append = any(tk.op == 16 for tk in tasks)
+    for l in range(L):
+        T[("kv", l)] = Tensor(B)
     T[("logits",)] = Tensor(V)
     mm_arrivals = defaultdict(int)
     tasks_split = {tk.layer: tk.r1 for tk in tasks if tk.op == 2}
@@ -168,6 +173,8 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
             d = qkv.read(g * hpg * hd, (g + 1) * hpg * hd, who)
             d += qkv.read(nq * hd + g * hd, nq * hd + (g + 1) * hd, who)
             d += qkv.read((nq + nkv) * hd + g * hd, (nq + nkv) * hd + (g + 1) * hd, who)
+            if has_append:
+                d += t("kv", l).read(0, B, who)
             idx = (b * nkv + g) * 4096 + r0            # r0 = split index
             t("part", l).write(idx, idx + 1, _mix(base ^ (d & M64)), who)
             signal(tk.signal)
@@ -209,6 +216,10 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
         elif op == "lmhead":
             d = read_xin(L, 0, H, who)
             t("logits").write(r0, r1, _mix(base ^ d), who)
+            signal(tk.signal)
+        elif op == "kvappend":
+            d = t("qkv", l).read(0, qkv_rows, who)
+            t("kv", l).write(r0, r1, _mix(base ^ d), who)
             signal(tk.signal)
         elif op == "norm":
             src = {0: ("x_in", l), 1: ("x_mid", l), 2: ("x_in", L)}[tk.aux]

@@ -195,7 +195,8 @@ def test_batched_plan_is_topological_and_thresholds_match_signals(cfg, B):
     info, tasks, thr = plan(cfg, max_batch=B, max_ctx=8192 + 200)
     assert info.max_batch == B
     ops = {t.op for t in tasks}
-    assert ops == {mk.MK_OP_NORM, mk.MK_OP_ATTN, *mk.MM_OPS}, "batched graphs use only tensor-core tiles"
+    assert ops == {mk.MK_OP_NORM, mk.MK_OP_KVAPPEND, mk.MK_OP_ATTN, *mk.MM_OPS}, \
+        "batched graphs use only tensor-core tiles"
     groups = _tile_groups(tasks)
     signalled = [0] * len(thr)
     for i, t in enumerate(tasks):

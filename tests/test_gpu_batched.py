@@ -15,6 +15,7 @@ import pytest
 import torch
 
 import oracle
+import persistent_megakernel_decode_03_b200 as mk
 import synthetic as syn
 from tests.gpu_util import compare_logits, device_weights, fill_kv_context, fill_oracle_kv, make_decoder
 from tests.test_gpu_parity import check_counters, names
@@ -138,3 +139,102 @@ def test_batched_head_layouts(nq, nkv, hd):
     lens = _ragged_lengths(4, 1, 90, 4600 + nq + nkv + hd)
     _run_batched(cfg, 8800 + nq * 100 + nkv * 10 + hd, 4, lens, 5, 90 + nkv, greedy=True,
                  label=f"heads {nq}/{nkv}/{hd}")
+
+
+# ---------------------------------------------------------------- batched prefill
+
+def _prefill_case(cfg, seed, max_batch, n_prompt, n_decode, seed_off, label, greedy=True):
+    """Prompt through a batched graph (up to max_batch tokens per launch), then
+    decode steps of that sequence alone; every logit against the oracle run
+    token by token, and the cached K bits of the prompt against the oracle's."""
+    max_ctx = n_prompt + n_decode + 8
+    specs, ts = device_weights(cfg, seed)
+    dec = make_decoder(cfg, ts, max_batch, max_ctx)
+    prompt = [int(t) for t in syn.host_tokens(n_prompt, syn.SEED_PROMPT + seed_off, cfg.vocab)]
+    last = dec.prefill(torch.tensor(prompt, dtype=torch.int32, device="cuda")).cpu().numpy()
+    dec.check()
+    check_counters(dec)
+    orc = oracle.Model(cfg, syn.host_weights(cfg, seed), max_ctx, names(cfg))
+    for p, t in enumerate(prompt):
+        ref = orc.decode_step(t, p)["logits"]
+    d, cos, ok = compare_logits(last, ref)
+    print(f"{label}: prefill of {n_prompt} tokens in launches of {max_batch}: max|diff| {d:.3g} cos {cos:.8f}")
+    assert ok, (d, cos)
+    # K of every prompt position in layer 0, sequence 0's pages: each element within one
+    # bf16 step of its own value (2^-7 relative), plus 2^-10 of the row's scale for
+    # elements near zero (the projection accumulates in another order than the
+    # oracle's double, so a value may round to its neighbour); a misplaced row would be
+    # off by the scale itself
+    k = dec.k_pages[0].float().cpu().numpy()
+    rows = dec.page_table[0].cpu().numpy()
+    worst = 0.0
+    for p in range(n_prompt):
+        got = k[rows[p // 16], :, p % 16, :]
+        ref_k = oracle.bf16_to_f64(orc.k[0][p])
+        scale = float(np.sqrt(np.mean(ref_k ** 2)))
+        bound = 2.0 ** -7 * np.abs(ref_k) + 2.0 ** -10 * scale
+        ratio = float(np.max(np.abs(got - ref_k) / bound))
+        worst = max(worst, ratio)
+        assert ratio <= 1.0, (p, ratio)
+    print(f"{label}: cached K of the prompt within {worst:.3g} of the bound")
+    tok = int(np.argmax(ref))
+    for i in range(n_decode):
+        p = n_prompt + i
+        g = dec.step(torch.tensor([tok], dtype=torch.int32, device="cuda"),
+                     torch.tensor([p], dtype=torch.int32, device="cuda")).cpu().numpy()[0]
+        dec.check()
+        ref = orc.decode_step(tok, p)["logits"]
+        d, cos, ok = compare_logits(g, ref)
+        assert ok, (label, p, d, cos)
+        if greedy:
+            assert int(np.argmax(g)) == int(np.argmax(ref)), (label, p)
+        tok = int(np.argmax(ref))
+    check_counters(dec)
+    dec.close()
+
+
+@pytest.mark.parametrize("max_batch", [4, 16, 64], ids=lambda v: f"B{v}")
+def test_tiny_batched_prefill_then_decode(max_batch):
+    """The 39-token prompt of the tiny config as batch rows (launches of 4, 16 or
+    64 tokens: 10, 3 or 1 launches), then 16 greedy decode steps."""
+    _prefill_case(syn.TINY, syn.SEED_WEIGHTS + 90, max_batch, 39, 16, 90, f"tiny B{max_batch}")
+
+
+def test_8b_shapes_batched_prefill():
+    """8B-class shapes (2 layers): a 100-token prompt in launches of 64 and 36
+    rows, then 2 decode steps."""
+    cfg = dataclasses.replace(syn.LLAMA8B, n_layers=2)
+    _prefill_case(cfg, syn.SEED_WEIGHTS + 91, 64, 100, 2, 91, "8b-2layer", greedy=False)
+
+
+def test_prefill_into_one_slot_then_mixed_batch():
+    """mk_prefill_seq into sequence slot 2 of a 4-row graph, then one batched step in
+    which slot 2 continues its prompt and slots 0, 1, 3 start at position 0."""
+    cfg = syn.TINY
+    seed = syn.SEED_WEIGHTS + 92
+    specs, ts = device_weights(cfg, seed)
+    dec = make_decoder(cfg, ts, 4, 64)
+    prompt = [int(t) for t in syn.host_tokens(20, syn.SEED_PROMPT + 92, cfg.vocab)]
+    kv = mk.make_kv(dec.k_pages.data_ptr(), dec.v_pages.data_ptr(), dec.page_table.data_ptr(), dec.n_pages,
+                    dec.max_pages)
+    out = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    toks_d = torch.tensor(prompt, dtype=torch.int32, device="cuda")
+    mk.mk_prefill_seq(dec.state, toks_d.data_ptr(), len(prompt), 0, 2, kv, out.data_ptr(), dec.stream())
+    dec.check()
+    host_w = syn.host_weights(cfg, seed)
+    orcs = [oracle.Model(cfg, host_w, 64, names(cfg)) for _ in range(4)]
+    for p, t in enumerate(prompt):
+        ref = orcs[2].decode_step(t, p)["logits"]
+    d, cos, ok = compare_logits(out.cpu().numpy(), ref)
+    assert ok, (d, cos)
+    step_toks = [3, 5, int(np.argmax(ref)), 7]
+    pos = [0, 0, len(prompt), 0]
+    g = dec.step(torch.tensor(step_toks, dtype=torch.int32, device="cuda"),
+                 torch.tensor(pos, dtype=torch.int32, device="cuda")).cpu().numpy()
+    dec.check()
+    for b in range(4):
+        ref = orcs[b].decode_step(step_toks[b], pos[b])["logits"]
+        d, cos, ok = compare_logits(g[b], ref)
+        assert ok, (b, d, cos)
+    check_counters(dec)
+    dec.close()
