@@ -421,6 +421,53 @@ def run_gpu(args, W):
         pg.destroy_process_group()
 
 
+def run_prefill(args, W):
+    """Prompt processing (the step before the decode loop): the workload's 39-token
+    prompt through mk_prefill on a batch-64 graph (tensor-core tiles, the prompt's
+    tokens as batch rows: one launch), timed beside the batch-1 graph's
+    token-by-token prefill (39 launches).  Prints one JSON line; not a decode line."""
+    import torch
+    import synthetic as syn
+    from persistent_megakernel_decode_03_b200.runner import Decoder
+
+    cfg = W["cfg"]
+    seed = syn.SEED_WEIGHTS + W["seed"]
+    ts = []
+    for s in syn.tensor_specs(cfg):
+        t = torch.empty(s.shape, dtype=torch.bfloat16, device="cuda")
+        syn.dev_fill_tensor(t, s, seed)
+        ts.append(t)
+    desc = dict(n_layers=cfg.n_layers, hidden=cfg.hidden, n_q_heads=cfg.n_q_heads,
+                n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, ffn=cfg.ffn, vocab=cfg.vocab,
+                rms_eps=cfg.rms_eps, rope_theta=cfg.rope_theta)
+    n = PROMPT
+    prompt = torch.tensor(syn.host_tokens(n, syn.SEED_PROMPT + W["seed"], cfg.vocab), dtype=torch.int32,
+                          device="cuda")
+    res = {}
+    for name, mb in (("batched", 64), ("token_by_token", 1)):
+        dec = Decoder(desc, [t.data_ptr() for t in ts], mb, n + 16)
+        for _ in range(args.warmup):
+            dec.prefill(prompt)
+        torch.cuda.synchronize()
+        dec.check()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            dec.prefill(prompt)
+        e1.record()
+        torch.cuda.synchronize()
+        dec.check()
+        res[name] = e0.elapsed_time(e1) / args.steps
+        dec.close()
+    line = {"metric": "prompt tokens/s (prefill)", "value": n / (res["batched"] / 1e3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_prefill": res["batched"],
+            "token_by_token_ms_per_prefill": res["token_by_token"],
+            "speedup_vs_token_by_token": res["token_by_token"] / res["batched"],
+            "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": W["desc"] + f"; {n}-token prompt", "prefill": "batched (one launch, batch-64 graph)"}}
+    print(json.dumps(line), flush=True)
+
+
 def run_solo(args, W):
     """One operator kind's tiles alone (dependencies dropped), on the workload's shapes.
 
@@ -511,6 +558,8 @@ def main(argv=None):
     ap.add_argument("--solo", default="",
                     help="profiling only: time one operator kind's task list alone "
                          "(qkv, attn, oproj, gateup, down, lmhead) and print its GB/s")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the 39-token prompt's prefill (batched vs token by token) instead")
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds of CPU time the reference arm may spend on timed steps")
     args = ap.parse_args(argv)
@@ -523,6 +572,8 @@ def main(argv=None):
         W["desc"] += f" [first {W['cfg'].n_layers} layers only: profiling case]"
     if args.solo:
         run_solo(args, W)
+    elif args.prefill:
+        run_prefill(args, W)
     elif args.impl == "reference":
         run_reference(args, W)
     else:

@@ -2068,28 +2068,46 @@ __device__ __noinline__ void norm_task(const Params& p, Smem& sm, uint32_t& cph,
 
 // The last split of a tile: the splits' partial sums added in split order (the
 // same order on every run), then the operator's epilogue for every batch row of
-// the step.  128 threads (consumer warps 0-3).
-__device__ void mm_epilogue(const Params& p, const Task& t, int tid) {
-    const int Sk = t.nblk, l = t.layer, nrows = (int)(t.r1 - t.r0);
+// the step.  128 threads (consumer warps 4-7), each owning one tile row (gate/up:
+// one FFN row and half of the batch rows).  The loads of 8 batch rows are issued
+// before any of their stores, so a tile costs batch / 8 round trips to L2, not one
+// per batch row.
+constexpr int kEpiRows = 8;
+__device__ __noinline__ void mm_epilogue(const Params& p, const Task& t, int tid) {
+    const int Sk = t.nblk, l = t.layer, nrows = (int)(t.r1 - t.r0), batch = p.batch;
     const size_t sstride = (size_t)p.bp * kMmRows;
-    const float* part0 = p.mm_part + (size_t)t.aux * sstride;
+    const float* __restrict__ part0 = p.mm_part + (size_t)t.aux * sstride;
     if (t.op == MK_OP_MM_GATEUP) {            // rows 0..63 gate, 64..127 up, of FFN rows r0..r0+63
         const int i = tid & 63;
         if (i >= nrows) return;
         const int f = (int)t.r0 + i;
-        for (int b = tid >> 6; b < p.batch; b += 2) {
-            float g = 0.0f, u = 0.0f;
+        const size_t base = (size_t)l * 2 * p.bp;
+        for (int b0 = tid >> 6; b0 < batch; b0 += 2 * kEpiRows) {
+            float g[kEpiRows], u[kEpiRows];
+#pragma unroll
+            for (int k = 0; k < kEpiRows; ++k) { g[k] = 0.0f; u[k] = 0.0f; }
             for (int sp = 0; sp < Sk; ++sp) {
-                g += __ldcg(part0 + sp * sstride + (size_t)b * kMmRows + i);
-                u += __ldcg(part0 + sp * sstride + (size_t)b * kMmRows + 64 + i);
+                const float* ps = part0 + sp * sstride;
+#pragma unroll
+                for (int k = 0; k < kEpiRows; ++k) {
+                    const int b = b0 + 2 * k;
+                    if (b < batch) {
+                        g[k] += __ldcg(ps + (size_t)b * kMmRows + i);
+                        u[k] += __ldcg(ps + (size_t)b * kMmRows + 64 + i);
+                    }
+                }
             }
-            const float a = silu_f(g) * u;
-            p.act[((size_t)l * p.max_batch + b) * p.F + f] = a;
-            uint16_t hi, lo;
-            split_hilo(a, hi, lo);
-            const size_t base = (size_t)l * 2 * p.bp;
-            p.opnd[kOpAct][(base + b) * p.F + f] = hi;
-            p.opnd[kOpAct][(base + p.bp + b) * p.F + f] = lo;
+#pragma unroll
+            for (int k = 0; k < kEpiRows; ++k) {
+                const int b = b0 + 2 * k;
+                if (b >= batch) continue;
+                const float a = silu_f(g[k]) * u[k];
+                p.act[((size_t)l * p.max_batch + b) * p.F + f] = a;
+                uint16_t hi, lo;
+                split_hilo(a, hi, lo);
+                p.opnd[kOpAct][(base + b) * p.F + f] = hi;
+                p.opnd[kOpAct][(base + p.bp + b) * p.F + f] = lo;
+            }
         }
         return;
     }
@@ -2097,16 +2115,34 @@ __device__ void mm_epilogue(const Params& p, const Task& t, int tid) {
     if (i >= nrows) return;
     const int r = (int)t.r0 + i;
     const size_t qkvw = (size_t)(p.nq + 2 * p.nkv) * p.hd;
-    for (int b = 0; b < p.batch; ++b) {
-        float v = 0.0f;
-        for (int sp = 0; sp < Sk; ++sp) v += __ldcg(part0 + sp * sstride + (size_t)b * kMmRows + i);
-        const size_t lb = (size_t)l * p.max_batch + b;
-        switch (t.op) {
-            case MK_OP_MM_QKV: p.qkv[lb * qkvw + r] = v; break;
-            case MK_OP_MM_OPROJ: p.x_mid[lb * p.H + r] = x_in(p, l, b, r) + v; break;
-            case MK_OP_MM_DOWN: p.x_out[lb * p.H + r] = x_mid_at(p, l, b, r) + v; break;
-            case MK_OP_MM_LMHEAD: p.logits[(size_t)b * p.V + r] = v; break;
-            default: break;
+    for (int b0 = 0; b0 < batch; b0 += kEpiRows) {
+        float v[kEpiRows], res[kEpiRows];
+#pragma unroll
+        for (int k = 0; k < kEpiRows; ++k) { v[k] = 0.0f; res[k] = 0.0f; }
+        for (int sp = 0; sp < Sk; ++sp) {
+            const float* ps = part0 + sp * sstride;
+#pragma unroll
+            for (int k = 0; k < kEpiRows; ++k)
+                if (b0 + k < batch) v[k] += __ldcg(ps + (size_t)(b0 + k) * kMmRows + i);
+        }
+        if (t.op == MK_OP_MM_OPROJ || t.op == MK_OP_MM_DOWN) {
+#pragma unroll
+            for (int k = 0; k < kEpiRows; ++k)
+                if (b0 + k < batch)
+                    res[k] = (t.op == MK_OP_MM_OPROJ) ? x_in(p, l, b0 + k, r) : x_mid_at(p, l, b0 + k, r);
+        }
+#pragma unroll
+        for (int k = 0; k < kEpiRows; ++k) {
+            const int b = b0 + k;
+            if (b >= batch) continue;
+            const size_t lb = (size_t)l * p.max_batch + b;
+            switch (t.op) {
+                case MK_OP_MM_QKV: p.qkv[lb * qkvw + r] = v[k]; break;
+                case MK_OP_MM_OPROJ: p.x_mid[lb * p.H + r] = res[k] + v[k]; break;
+                case MK_OP_MM_DOWN: p.x_out[lb * p.H + r] = res[k] + v[k]; break;
+                case MK_OP_MM_LMHEAD: p.logits[(size_t)b * p.V + r] = v[k]; break;
+                default: break;
+            }
         }
     }
 }
