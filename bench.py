@@ -468,6 +468,80 @@ def run_prefill(args, W):
     print(json.dumps(line), flush=True)
 
 
+def run_per_op(args, W):
+    """The same decode step as a kernel-per-operator baseline: one launch per
+    (operator, layer) run of the task list, replayed as a CUDA graph, timed beside
+    the megakernel on the same workload.  Prints one JSON line; not a decode line."""
+    import torch
+    import synthetic as syn
+    import persistent_megakernel_decode_03_b200 as mk
+    from persistent_megakernel_decode_03_b200.runner import Decoder
+
+    cfg = W["cfg"]
+    seed = syn.SEED_WEIGHTS + W["seed"]
+    ts = []
+    for s in syn.tensor_specs(cfg):
+        t = torch.empty(s.shape, dtype=torch.bfloat16, device="cuda")
+        syn.dev_fill_tensor(t, s, seed)
+        ts.append(t)
+    desc = dict(n_layers=cfg.n_layers, hidden=cfg.hidden, n_q_heads=cfg.n_q_heads,
+                n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, ffn=cfg.ffn, vocab=cfg.vocab,
+                rms_eps=cfg.rms_eps, rope_theta=cfg.rope_theta)
+    ctx = 300
+    dec = Decoder(desc, [t.data_ptr() for t in ts], 1, ctx + 8)
+    for l in range(cfg.n_layers):
+        syn.dev_fill_kv_paged(dec.k_pages[l], dec.page_table[0], 0, 0, ctx, cfg, 16, syn.SEED_KV + 2,
+                              syn.TID_K_BASE + l)
+        syn.dev_fill_kv_paged(dec.v_pages[l], dec.page_table[0], 0, 0, ctx, cfg, 16, syn.SEED_KV + 2,
+                              syn.TID_V_BASE + l)
+    tok = torch.tensor([7], dtype=torch.int32, device="cuda")
+    pos = torch.tensor([ctx], dtype=torch.int32, device="cuda")
+    out = torch.empty((1, cfg.vocab), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    n_launch = [0]
+
+    def per_op():
+        n_launch[0] = mk.mk_decode_step_per_op(dec.state, tok.data_ptr(), pos.data_ptr(), 1, dec.kv,
+                                               out.data_ptr(), stream.cuda_stream)
+
+    def mega():
+        mk.mk_decode_step(dec.state, tok.data_ptr(), pos.data_ptr(), 1, dec.kv, out.data_ptr(),
+                          stream.cuda_stream)
+
+    ms_direct = timed(per_op, args.steps)
+    dec.check()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
+        per_op()
+    ms_graph = timed(graph.replay, args.steps)
+    dec.check()
+    del graph
+    ms_mega = timed(mega, args.steps)
+    dec.check()
+    dec.close()
+    line = {"metric": "decode step time: megakernel vs kernel-per-operator baseline (same tiles)",
+            "unit": "ms", "higher_is_better": False, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "megakernel_ms": ms_mega, "per_op_graph_ms": ms_graph, "per_op_direct_ms": ms_direct,
+            "launches_per_step": n_launch[0], "speedup_vs_per_op_graph": ms_graph / ms_mega,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": W["desc"] + f"; batch 1 at position {ctx}"}}
+    print(json.dumps(line), flush=True)
+
+
 def run_solo(args, W):
     """One operator kind's tiles alone (dependencies dropped), on the workload's shapes.
 
@@ -558,6 +632,8 @@ def main(argv=None):
     ap.add_argument("--solo", default="",
                     help="profiling only: time one operator kind's task list alone "
                          "(qkv, attn, oproj, gateup, down, lmhead) and print its GB/s")
+    ap.add_argument("--per-op", action="store_true",
+                    help="time the kernel-per-operator baseline of the step beside the megakernel instead")
     ap.add_argument("--prefill", action="store_true",
                     help="time the 39-token prompt's prefill (batched vs token by token) instead")
     ap.add_argument("--ref-budget", type=float, default=120.0,
@@ -574,6 +650,8 @@ def main(argv=None):
         run_solo(args, W)
     elif args.prefill:
         run_prefill(args, W)
+    elif args.per_op:
+        run_per_op(args, W)
     elif args.impl == "reference":
         run_reference(args, W)
     else:

@@ -241,6 +241,17 @@ mk_status mk_state_debug_wait_offset(mk_state* state, uint32_t offset);
 mk_status mk_decode_step(mk_state* state, const int32_t* token_ids, const int32_t* positions,
                          int batch, const mk_paged_kv* kv, float* logits_out, mk_stream stream);
 
+/* The same step as a kernel-per-operator baseline (the pages' comparison point:
+ * kernels with boundaries between operators, MPK digest "Part 1"): one launch per
+ * maximal run of tasks of one (operator, layer) in the task list, in order on
+ * `stream`, each running the same tiles without the events that let the
+ * megakernel overlap them.  Counters are zeroed first, so the whole call can be
+ * captured into a CUDA graph and replayed.  Results equal mk_decode_step's.
+ * n_launches (optional) receives the number of launches. */
+mk_status mk_decode_step_per_op(mk_state* state, const int32_t* token_ids, const int32_t* positions,
+                                int batch, const mk_paged_kv* kv, float* logits_out, mk_stream stream,
+                                int* n_launches);
+
 /* Same step with HOST inputs and outputs: copies token_ids and positions
  * (host int32 [batch]) to the device, runs the step, copies the logits back
  * to logits_host (host fp32 [batch][vocab]) and waits for the stream. */

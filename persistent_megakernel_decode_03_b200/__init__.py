@@ -46,7 +46,7 @@ SYMBOLS = (
     "mk_graph_destroy", "mk_graph_get_info", "mk_graph_export_tasks", "mk_graph_export_thresholds",
     "mk_wave_stats", "mk_state_create", "mk_state_destroy", "mk_state_set_timeout",
     "mk_state_debug_wait_offset", "mk_state_set_prefetch",
-    "mk_decode_step", "mk_decode_step_host", "mk_prefill", "mk_prefill_seq", "mk_decode_step_noalloc", "mk_sync",
+    "mk_decode_step", "mk_decode_step_host", "mk_decode_step_per_op", "mk_prefill", "mk_prefill_seq", "mk_decode_step_noalloc", "mk_sync",
     "mk_state_read_counters",
     "mk_state_read_buffer", "mk_state_read_trace", "mk_state_read_stats", "mk_last_error_string",
     "mk_version",
@@ -125,6 +125,7 @@ def lib() -> ctypes.CDLL:
             "mk_decode_step": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_decode_step_host": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_prefill": ([vp, vp, i32, i32, P(mk_paged_kv), vp, vp], st),
+            "mk_decode_step_per_op": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp, P(ctypes.c_int)], st),
             "mk_prefill_seq": ([vp, vp, i32, i32, i32, P(mk_paged_kv), vp, vp], st),
             "mk_decode_step_noalloc": ([P(mk_model_desc), vp, i32, i32, vp, vp, i32, P(mk_paged_kv),
                                         vp, vp], st),
@@ -257,6 +258,15 @@ def mk_decode_step_host(state: int, token_ids: int, positions: int, batch: int, 
 def mk_prefill(state: int, tokens: int, n_tokens: int, pos0: int, kv: mk_paged_kv,
                last_logits: int, stream: int = 0) -> None:
     _check(lib().mk_prefill(state, tokens, n_tokens, pos0, ctypes.byref(kv), last_logits, stream))
+
+
+def mk_decode_step_per_op(state: int, token_ids: int, positions: int, batch: int, kv: mk_paged_kv,
+                          logits_out: int, stream: int = 0) -> int:
+    """Kernel-per-operator baseline of one step; returns the number of launches."""
+    n = ctypes.c_int(0)
+    _check(lib().mk_decode_step_per_op(state, token_ids, positions, batch, ctypes.byref(kv), logits_out,
+                                       stream, ctypes.byref(n)))
+    return n.value
 
 
 def mk_prefill_seq(state: int, tokens: int, n_tokens: int, pos0: int, seq_slot: int, kv: mk_paged_kv,

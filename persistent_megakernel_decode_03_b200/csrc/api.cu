@@ -33,6 +33,7 @@ struct mk_graph {
     uint32_t* d_thr = nullptr;
     float* d_rope = nullptr;
     std::vector<CUtensorMap> wmaps;   // batched graphs: operand slots (filled per state), then weights
+    std::vector<std::pair<int, int>> phases;   // (first task, task count) of each (operator, layer) run
 };
 
 struct mk_state {
@@ -418,6 +419,13 @@ static mk_status build_graph(mk_model* model, int max_batch, int max_ctx, int so
             rope[((size_t)pos * half + i) * 2 + 0] = (float)std::cos(a);
             rope[((size_t)pos * half + i) * 2 + 1] = (float)std::sin(a);
         }
+    // the kernel-per-op baseline launches each maximal run of one (operator, layer)
+    for (size_t i = 0; i < P.tasks.size();) {
+        size_t j = i + 1;
+        while (j < P.tasks.size() && P.tasks[j].op == P.tasks[i].op && P.tasks[j].layer == P.tasks[i].layer) ++j;
+        g->phases.emplace_back((int)i, (int)(j - i));
+        i = j;
+    }
     e = cudaMalloc(&g->d_tasks, sizeof(mk::Task) * P.tasks.size());
     if (e == cudaSuccess) e = cudaMalloc(&g->d_thr, sizeof(uint32_t) * std::max<size_t>(1, P.thr.size()));
     if (e == cudaSuccess) e = cudaMalloc(&g->d_rope, sizeof(float) * rope.size());
@@ -612,6 +620,54 @@ mk_status mk_decode_step(mk_state* s, const int32_t* token_ids, const int32_t* p
     p.max_pages = kv->max_pages_per_seq;
     p.logits = logits_out;
     return launch_step(s, p, (cudaStream_t)stream);
+}
+
+mk_status mk_decode_step_per_op(mk_state* s, const int32_t* token_ids, const int32_t* positions, int batch,
+                                const mk_paged_kv* kv, float* logits_out, mk_stream stream, int* n_launches) {
+    if (!s || !token_ids || !positions || !logits_out)
+        return fail(MK_ERR_INVALID_ARG, "mk_decode_step_per_op: null argument");
+    if (batch < 1 || batch > s->g->plan.max_batch)
+        return fail(MK_ERR_INVALID_ARG, "mk_decode_step_per_op: batch %d outside 1..%d", batch, s->g->plan.max_batch);
+    mk_status r = check_kv(s, kv);
+    if (r != MK_OK) return r;
+    cudaStream_t st = (cudaStream_t)stream;
+    // counters from zero, epoch 1 in every launch: each launch's waits are met by the
+    // launches before it on the stream, and the next megakernel step starts afresh
+    r = reset_counters(s, st);
+    if (r != MK_OK) return r;
+    const GraphPlan& P = s->g->plan;
+    unsigned long long base = 0;
+    for (const auto& ph : s->g->phases) {
+        mk::Params p = base_params(s);
+        p.tasks = s->g->d_tasks + ph.first;
+        p.n_tasks = (uint32_t)ph.second;
+        p.trace = nullptr;
+        p.stats = nullptr;
+        p.pf_dist = 0;
+        p.tokens = token_ids;
+        p.positions = positions;
+        p.pos_offset = 0;
+        p.batch = batch;
+        p.skip_lm = 0;
+        p.k_pages = static_cast<uint16_t*>(kv->k_pages);
+        p.v_pages = static_cast<uint16_t*>(kv->v_pages);
+        p.page_table = kv->page_table;
+        p.n_pages = kv->n_pages;
+        p.max_pages = kv->max_pages_per_seq;
+        p.logits = logits_out;
+        p.epoch = 1;
+        p.queue_base = base;                       // each launch claims its tasks + one per CTA
+        base += (unsigned long long)ph.second + (unsigned long long)P.n_sm;
+        cudaError_t e = mk::megakernel_launch(p, P.n_sm, st, /*cooperative=*/false);
+        if (e != cudaSuccess) {
+            s->needs_reset = true;
+            return cuda_fail(e, "per-op launch");
+        }
+    }
+    s->epoch = 1;
+    s->needs_reset = true;    // the queue head is not (n_tasks + grid) x epoch: reset before a megakernel step
+    if (n_launches) *n_launches = (int)s->g->phases.size();
+    return MK_OK;
 }
 
 mk_status mk_decode_step_host(mk_state* s, const int32_t* token_ids, const int32_t* positions, int batch,

@@ -2640,37 +2640,43 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 // ----------------------------------------------------------------------------- host launch
 
 template <int HPG, int DPL>
-static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream) {
+static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream, bool cooperative) {
     auto kern = p.mm ? megakernel<HPG, DPL, true> : megakernel<HPG, DPL, false>;
-    static bool attr_set = false;   // per instantiation; set before first launch on each device use
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(Smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-    (void)attr_set;
+    // the shared-memory attribute, once per instantiation and device (so that a step
+    // can be captured into a CUDA graph without host-side calls in between)
+    static unsigned attr_set[2] = {0u, 0u};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned bit = 1u << (dev & 31);
+    if (!(attr_set[p.mm ? 1 : 0] & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
+        if (e != cudaSuccess) return e;
+        attr_set[p.mm ? 1 : 0] |= bit;
+    }
     void* args[] = {const_cast<Params*>(&p)};
-    return cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kThreads), args,
-                                       sizeof(Smem), stream);
+    if (cooperative)
+        return cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kThreads), args, sizeof(Smem), stream);
+    return cudaLaunchKernel((const void*)kern, dim3(grid), dim3(kThreads), args, sizeof(Smem), stream);
 }
 
 size_t megakernel_smem_bytes() { return sizeof(Smem); }
 
-cudaError_t megakernel_launch(const Params& p, int grid, cudaStream_t stream) {
+cudaError_t megakernel_launch(const Params& p, int grid, cudaStream_t stream, bool cooperative) {
     const int hpg = p.nq / p.nkv;
     const int dpl = p.hd / 32;
     if (dpl == 4) {
         switch (hpg) {
-            case 1: return launch_t<1, 4>(p, grid, stream);
-            case 2: return launch_t<2, 4>(p, grid, stream);
-            case 4: return launch_t<4, 4>(p, grid, stream);
-            case 8: return launch_t<8, 4>(p, grid, stream);
+            case 1: return launch_t<1, 4>(p, grid, stream, cooperative);
+            case 2: return launch_t<2, 4>(p, grid, stream, cooperative);
+            case 4: return launch_t<4, 4>(p, grid, stream, cooperative);
+            case 8: return launch_t<8, 4>(p, grid, stream, cooperative);
         }
     } else if (dpl == 2) {
         switch (hpg) {
-            case 1: return launch_t<1, 2>(p, grid, stream);
-            case 2: return launch_t<2, 2>(p, grid, stream);
-            case 4: return launch_t<4, 2>(p, grid, stream);
-            case 8: return launch_t<8, 2>(p, grid, stream);
+            case 1: return launch_t<1, 2>(p, grid, stream, cooperative);
+            case 2: return launch_t<2, 2>(p, grid, stream, cooperative);
+            case 4: return launch_t<4, 2>(p, grid, stream, cooperative);
+            case 8: return launch_t<8, 2>(p, grid, stream, cooperative);
         }
     }
     return cudaErrorInvalidValue;

@@ -8,8 +8,10 @@
 namespace mk {
 
 size_t megakernel_smem_bytes();
-// One cooperative launch of `grid` CTAs (one per SM) on `stream`.
-cudaError_t megakernel_launch(const Params& p, int grid, cudaStream_t stream);
+// One launch of `grid` CTAs (one per SM) on `stream`: cooperative (the CTAs of a
+// step wait on one another), or plain for a task list without waits inside the
+// launch (one phase of the kernel-per-op baseline).
+cudaError_t megakernel_launch(const Params& p, int grid, cudaStream_t stream, bool cooperative = true);
 bool megakernel_supports(int heads_per_group, int head_dim);
 cudaError_t megakernel_occupancy(int heads_per_group, int head_dim, int* blocks_per_sm);
 
