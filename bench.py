@@ -542,6 +542,75 @@ def run_per_op(args, W):
     print(json.dumps(line), flush=True)
 
 
+def run_generate(args, W):
+    """Greedy generation (the loop after the hot path): 128 new tokens of the 8B
+    model after its 39-token prompt, with mk_generate (each step's argmax chosen on
+    the device, all steps enqueued at once) beside a host loop that copies each
+    step's logits to the host, takes the argmax there and sends the token back.
+    Prints one JSON line; not a decode line."""
+    import numpy as np
+    import torch
+    import synthetic as syn
+    import persistent_megakernel_decode_03_b200 as mk
+    from persistent_megakernel_decode_03_b200.runner import Decoder
+
+    cfg = W["cfg"]
+    seed = syn.SEED_WEIGHTS + W["seed"]
+    ts = []
+    for s in syn.tensor_specs(cfg):
+        t = torch.empty(s.shape, dtype=torch.bfloat16, device="cuda")
+        syn.dev_fill_tensor(t, s, seed)
+        ts.append(t)
+    desc = dict(n_layers=cfg.n_layers, hidden=cfg.hidden, n_q_heads=cfg.n_q_heads,
+                n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, ffn=cfg.ffn, vocab=cfg.vocab,
+                rms_eps=cfg.rms_eps, rope_theta=cfg.rope_theta)
+    n = 128
+    dec = Decoder(desc, [t.data_ptr() for t in ts], 1, PROMPT + n + 8)
+    prompt = torch.tensor(syn.host_tokens(PROMPT, syn.SEED_PROMPT + W["seed"], cfg.vocab), dtype=torch.int32,
+                          device="cuda")
+    last = dec.prefill(prompt)
+    first = int(torch.argmax(last).item())
+    dec.check()
+    stream = torch.cuda.current_stream().cuda_stream
+    out = torch.zeros((n, 1), dtype=torch.int32, device="cuda")
+    logits = torch.empty((1, cfg.vocab), dtype=torch.float32, device="cuda")
+    first_d = torch.tensor([first], dtype=torch.int32, device="cuda")
+    pos_d = torch.tensor([PROMPT], dtype=torch.int32, device="cuda")
+    for _ in range(2):   # warm-up (the same positions are rewritten each time)
+        mk.mk_generate(dec.state, first_d.data_ptr(), pos_d.data_ptr(), 1, n, dec.kv, out.data_ptr(),
+                       logits.data_ptr(), stream)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    mk.mk_generate(dec.state, first_d.data_ptr(), pos_d.data_ptr(), 1, n, dec.kv, out.data_ptr(),
+                   logits.data_ptr(), stream)
+    torch.cuda.synchronize()
+    t_dev = time.perf_counter() - t0
+    dec.check()
+    dev_tokens = out[:, 0].cpu().tolist()
+    # host loop: step, logits to the host, argmax there, token back
+    tok_h = torch.zeros(1, dtype=torch.int32).pin_memory()
+    pos_h = torch.zeros(1, dtype=torch.int32).pin_memory()
+    lg_h = torch.empty((1, cfg.vocab), dtype=torch.float32).pin_memory()
+    host_tokens = []
+    t0 = time.perf_counter()
+    tok = first
+    for i in range(n):
+        tok_h[0] = tok
+        pos_h[0] = PROMPT + i
+        mk.mk_decode_step_host(dec.state, tok_h.data_ptr(), pos_h.data_ptr(), 1, dec.kv, lg_h.data_ptr(), stream)
+        tok = int(np.argmax(lg_h.numpy()[0]))
+        host_tokens.append(tok)
+    t_host = time.perf_counter() - t0
+    dec.check()
+    dec.close()
+    line = {"metric": "greedy generation tokens/s (wall clock, batch 1)", "value": n / t_dev, "unit": "tokens/s",
+            "n_gpus": 1, "tokens": n, "device_loop_ms_per_token": 1e3 * t_dev / n,
+            "host_loop_tokens_per_s": n / t_host, "host_loop_ms_per_token": 1e3 * t_host / n,
+            "same_tokens": dev_tokens == host_tokens, "higher_is_better": True, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": W["desc"] + f"; greedy, {n} new tokens"}}
+    print(json.dumps(line), flush=True)
+
+
 def run_solo(args, W):
     """One operator kind's tiles alone (dependencies dropped), on the workload's shapes.
 
@@ -632,6 +701,8 @@ def main(argv=None):
     ap.add_argument("--solo", default="",
                     help="profiling only: time one operator kind's task list alone "
                          "(qkv, attn, oproj, gateup, down, lmhead) and print its GB/s")
+    ap.add_argument("--generate", action="store_true",
+                    help="time greedy generation with the device-side loop beside a host loop instead")
     ap.add_argument("--per-op", action="store_true",
                     help="time the kernel-per-operator baseline of the step beside the megakernel instead")
     ap.add_argument("--prefill", action="store_true",
@@ -652,6 +723,8 @@ def main(argv=None):
         run_prefill(args, W)
     elif args.per_op:
         run_per_op(args, W)
+    elif args.generate:
+        run_generate(args, W)
     elif args.impl == "reference":
         run_reference(args, W)
     else:

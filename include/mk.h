@@ -241,6 +241,17 @@ mk_status mk_state_debug_wait_offset(mk_state* state, uint32_t offset);
 mk_status mk_decode_step(mk_state* state, const int32_t* token_ids, const int32_t* positions,
                          int batch, const mk_paged_kv* kv, float* logits_out, mk_stream stream);
 
+/* Greedy generation without a host round trip per token: n_steps decode steps
+ * for `batch` sequences, enqueued at once on `stream`.  Step k feeds each
+ * sequence the token chosen at step k - 1 (step 0: first_tokens, device int32
+ * [batch]) at position positions[b] + k (positions: device int32 [batch]), and
+ * after it a small kernel writes the argmax of each logits row (ties to the
+ * lowest index) to tokens_out[k][b] (device int32 [n_steps][batch]).
+ * logits_out (device fp32 [batch][vocab]) holds each step's logits in turn. */
+mk_status mk_generate(mk_state* state, const int32_t* first_tokens, const int32_t* positions, int batch,
+                      int n_steps, const mk_paged_kv* kv, int32_t* tokens_out, float* logits_out,
+                      mk_stream stream);
+
 /* The same step as a kernel-per-operator baseline (the pages' comparison point:
  * kernels with boundaries between operators, MPK digest "Part 1"): one launch per
  * maximal run of tasks of one (operator, layer) in the task list, in order on

@@ -46,7 +46,7 @@ SYMBOLS = (
     "mk_graph_destroy", "mk_graph_get_info", "mk_graph_export_tasks", "mk_graph_export_thresholds",
     "mk_wave_stats", "mk_state_create", "mk_state_destroy", "mk_state_set_timeout",
     "mk_state_debug_wait_offset", "mk_state_set_prefetch",
-    "mk_decode_step", "mk_decode_step_host", "mk_decode_step_per_op", "mk_prefill", "mk_prefill_seq", "mk_decode_step_noalloc", "mk_sync",
+    "mk_decode_step", "mk_decode_step_host", "mk_decode_step_per_op", "mk_generate", "mk_prefill", "mk_prefill_seq", "mk_decode_step_noalloc", "mk_sync",
     "mk_state_read_counters",
     "mk_state_read_buffer", "mk_state_read_trace", "mk_state_read_stats", "mk_last_error_string",
     "mk_version",
@@ -126,6 +126,7 @@ def lib() -> ctypes.CDLL:
             "mk_decode_step_host": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp], st),
             "mk_prefill": ([vp, vp, i32, i32, P(mk_paged_kv), vp, vp], st),
             "mk_decode_step_per_op": ([vp, vp, vp, i32, P(mk_paged_kv), vp, vp, P(ctypes.c_int)], st),
+            "mk_generate": ([vp, vp, vp, i32, i32, P(mk_paged_kv), vp, vp, vp], st),
             "mk_prefill_seq": ([vp, vp, i32, i32, i32, P(mk_paged_kv), vp, vp], st),
             "mk_decode_step_noalloc": ([P(mk_model_desc), vp, i32, i32, vp, vp, i32, P(mk_paged_kv),
                                         vp, vp], st),
@@ -267,6 +268,12 @@ def mk_decode_step_per_op(state: int, token_ids: int, positions: int, batch: int
     _check(lib().mk_decode_step_per_op(state, token_ids, positions, batch, ctypes.byref(kv), logits_out,
                                        stream, ctypes.byref(n)))
     return n.value
+
+
+def mk_generate(state: int, first_tokens: int, positions: int, batch: int, n_steps: int, kv: mk_paged_kv,
+                tokens_out: int, logits_out: int, stream: int = 0) -> None:
+    _check(lib().mk_generate(state, first_tokens, positions, batch, n_steps, ctypes.byref(kv), tokens_out,
+                             logits_out, stream))
 
 
 def mk_prefill_seq(state: int, tokens: int, n_tokens: int, pos0: int, seq_slot: int, kv: mk_paged_kv,
