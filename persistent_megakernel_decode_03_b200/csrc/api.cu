@@ -427,10 +427,13 @@ static mk_status build_graph(mk_model* model, int max_batch, int max_ctx, int so
             rope[((size_t)pos * half + i) * 2 + 0] = (float)std::cos(a);
             rope[((size_t)pos * half + i) * 2 + 1] = (float)std::sin(a);
         }
-    // the kernel-per-op baseline launches each maximal run of one (operator, layer)
+    // the kernel-per-op baseline launches each maximal run of one (operator, layer,
+    // and for norm tasks their kind)
     for (size_t i = 0; i < P.tasks.size();) {
         size_t j = i + 1;
-        while (j < P.tasks.size() && P.tasks[j].op == P.tasks[i].op && P.tasks[j].layer == P.tasks[i].layer) ++j;
+        while (j < P.tasks.size() && P.tasks[j].op == P.tasks[i].op && P.tasks[j].layer == P.tasks[i].layer &&
+               (P.tasks[i].op != MK_OP_NORM || P.tasks[j].aux == P.tasks[i].aux))
+            ++j;
         g->phases.emplace_back((int)i, (int)(j - i));
         i = j;
     }
@@ -468,7 +471,7 @@ mk_status mk_graph_get_info(const mk_graph* g, mk_graph_info* info) {
     info->max_batch = P.max_batch;
     info->max_ctx = P.max_ctx;
     info->attn_splits = P.S;
-    info->n_ops = P.bp > 0 ? 7 : (P.desc.n_experts > 0 ? 7 : 6);   // batched: norm, 5 tiles, attention
+    info->n_ops = P.bp > 0 ? 8 : (P.desc.n_experts > 0 ? 7 : 6);   // batched: norm, append, attention, 5 tiles
     info->weight_bytes_per_step = P.weight_bytes;
     return MK_OK;
 }

@@ -275,3 +275,34 @@ def test_batched_plan_rejections():
     assert e.value.status == mk.MK_ERR_UNSUPPORTED
     with pytest.raises(mk.MkError):
         mk.mk_plan_taskgraph(desc_of(syn.TINY_MOE), 4, 64, 148)
+
+
+@pytest.mark.parametrize("cfg,B", [(syn.TINY, 1), (syn.LLAMA8B, 1), (syn.TINY_MOE, 1), (syn.MOE30B, 1),
+                                   (syn.TINY, 4), (syn.LLAMA8B, 64)], ids=lambda v: str(v))
+def test_each_operator_and_layer_is_one_contiguous_run(cfg, B):
+    """The kernel-per-operator baseline launches each maximal run of one (operator,
+    layer); that is one launch per operator and layer (per norm kind) only if no
+    such key appears in two runs, and every wait must point into an earlier run."""
+    info, tasks, thr = plan(cfg, max_batch=B, max_ctx=2048)
+    runs, seen = [], set()
+    for i, t in enumerate(tasks):
+        key = (t.op, t.layer, t.aux if t.op == mk.MK_OP_NORM else 0)   # a layer's two norms differ in kind
+        if not runs or runs[-1][0] != key:
+            assert key not in seen, f"{key} appears in two runs"
+            seen.add(key)
+            runs.append((key, i))
+    run_of = {}
+    for r, (key, start) in enumerate(runs):
+        end = runs[r + 1][1] if r + 1 < len(runs) else len(tasks)
+        for i in range(start, end):
+            run_of[i] = r
+    signal_runs = {}
+    for i, t in enumerate(tasks):
+        if t.signal != mk.MK_NO_EVENT:
+            signal_runs.setdefault(t.signal, set()).add(run_of[i])
+    for i, t in enumerate(tasks):
+        for e in (t.wait[0], t.pointer_wait):
+            if e != mk.MK_NO_EVENT:
+                assert max(signal_runs[e]) < run_of[i], (i, e)
+    if B > 1:
+        assert info.n_ops == 8
