@@ -2005,9 +2005,9 @@ __device__ __noinline__ void kvappend_task(const Params& p, const Task& t, int t
 // RMSNorm of one batch row into the operand of the next projection, by all 256
 // consumer threads: h = x / sqrt(mean(x^2) + eps) * g (kind 0: attention norm of
 // the residual entering layer l, the token embedding at l = 0; kind 1: FFN norm
-// of the residual after attention; kind 2: final norm).  Every thread loads its
-// 4-column groups (and their gains) at once, so the row costs one round trip, a
-// block-wide sum and the stores.  Rows past the step's batch are written as zeros.
+// of the residual after attention; kind 2: final norm).  Two passes over the row
+// (sum of squares, then scale and store, re-reading x with the gains) around one
+// block-wide sum.  Rows past the step's batch are written as zeros.
 constexpr int kNormCols = 4 * kConsumerThreads;   // columns per pass chunk: 4 per thread
 template <bool EMB>
 __device__ __forceinline__ float4 norm_load4(const float* src, const uint16_t* emb, int i) {
