@@ -527,6 +527,8 @@ __device__ __forceinline__ void pr_advance(PRing& r) {
 // Tasks whose streamed data is only known on the device: attention (KV pages of
 // this step's positions) and routed experts (weights of the expert the router
 // picked).  Out of line: it keeps the producer's hot loop small.
+// MM: the instantiation for batched graphs (their KV appends run in tasks of their own).
+template <bool MM>
 __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Task& t, int ti, PRing& ring,
                                              uint32_t& last_router_evt, uint64_t pol) {
     int& stage = ring.stage;
@@ -545,7 +547,7 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                     if ((int)t.r0 < sa) attn_range(pos + 1, sa, (int)t.r0, j0, j1);
                     // batch-1 graphs: cached positions only (the new token is fresh);
                     // batched graphs: the new positions are in the cache too
-                    int jc = p.mm ? j1 : min(j1, pos);
+                    int jc = MM ? j1 : min(j1, pos);
                     if (jc > j0) {
                         lp0 = j0 / kPageSize;
                         npages = (jc - 1) / kPageSize - lp0 + 1;
@@ -574,8 +576,8 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
             // batched graphs append this step's K/V in tasks of their own: pages holding a
             // new position are loaded only after the attention task's event (which
             // counts those appends); older pages stream at once
-            const int first_new = p.mm ? (p.seq_row >= 0 ? position_of(p, 0) : position_of(p, b)) : INT_MAX;
-            bool appended = !p.mm || t.wait0 == MK_NO_EVENT;
+            const int first_new = MM ? (p.seq_row >= 0 ? position_of(p, 0) : position_of(p, b)) : INT_MAX;
+            bool appended = !MM || t.wait0 == MK_NO_EVENT;
             auto pid_ensure = [&](int upto) {
                 while (pid_have < upto) {
                     int v[kPidBatch];
@@ -593,7 +595,7 @@ __device__ __noinline__ bool produce_special(const Params& p, Smem& sm, const Ta
                 int first = lp0 + c * pps;
                 int n = min(pps, lp0 + npages - first);
                 pid_ensure(min(npages, c * pps + n + kPidBatch));
-                if (!appended && (first + n) * kPageSize > first_new) {
+                if (MM && !appended && (first + n) * kPageSize > first_new) {
                     if (!event_wait(p, t.wait0, p.thr[t.wait0] * p.epoch + p.wait_offset, ti)) { ok = false; break; }
                     asm volatile("fence.proxy.async.global;" ::: "memory");   // generic-proxy writes first
                     appended = true;
@@ -752,6 +754,7 @@ __device__ __noinline__ bool produce_mm(const Params& p, Smem& sm, const Task& t
     return true;
 }
 
+template <bool MM>
 __device__ void producer_loop(const Params& p, Smem& sm) {
     const uint64_t pol = l2_evict_first_policy();
     PRing ring{0, 0};
@@ -771,9 +774,11 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         const int ti = (int)q;
         const Task t = p.tasks[ti];
         q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
-        if (is_mm_op(t.op)) {
-            ok = produce_mm(p, sm, t, ti, ring, pol);
-            continue;
+        if constexpr (MM) {
+            if (is_mm_op(t.op)) {
+                ok = produce_mm(p, sm, t, ti, ring, pol);
+                continue;
+            }
         }
         const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm) || t.op == MK_OP_NORM || t.op == MK_OP_KVAPPEND;
         if (skip) {                                      // nothing to stream: a marker stage
@@ -784,7 +789,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
             continue;
         }
         if (t.nchunks == 0 || t.op == MK_OP_ATTN) {
-            ok = produce_special(p, sm, t, ti, ring, last_router_evt, pol);
+            ok = produce_special<MM>(p, sm, t, ti, ring, last_router_evt, pol);
             continue;
         }
         // dense GEMV tile: the plan the host computed (the consumer walks the same
@@ -2629,7 +2634,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     }
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSupportRegs));
     if (warp == kProducerWarp) {
-        if (lane == 0) producer_loop(p, sm);
+        if (lane == 0) producer_loop<MM>(p, sm);
     } else if (warp == kEpilogueWarp) {
         epilogue_loop(p, sm);
     } else if (warp == kPrefetchWarp) {
