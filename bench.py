@@ -199,11 +199,12 @@ def oracle_rate(W: dict, max_steps: int, budget_s: float, warmup: int = 1):
         experts = ("w_gate", "w_up", "w_down")
         host_w = {s.name: syn.host_tensor(s, seed) for s in specs
                   if not any(s.name.endswith(e) for e in experts)}
-        n = cfg.expert_ffn * cfg.hidden
+        expert_elems = cfg.expert_ffn * cfg.hidden
 
         def prov(l, e, which):
             s = by_name[f"layers.{l}.{experts[which]}"]
-            return syn.host_bf16(n, seed, s.tensor_id, s.sigma, s.mean, offset=e * n)
+            return syn.host_bf16(expert_elems, seed, s.tensor_id, s.sigma, s.mean,
+                                 offset=e * expert_elems)
         model = oracle.Model(cfg, host_w, cap, names, expert_provider=prov)
     else:
         model = oracle.Model(cfg, syn.host_weights(cfg, seed), cap, names)
@@ -214,13 +215,14 @@ def oracle_rate(W: dict, max_steps: int, budget_s: float, warmup: int = 1):
     for i in range(warmup):
         model.decode_step(int(toks[i]), ctx + i)
     t0 = time.perf_counter()
-    n = 0
-    while n < max_steps:
-        model.decode_step(int(toks[warmup + n]), ctx + warmup + n)
-        n += 1
+    n_done = 0
+    while n_done < max_steps:
+        model.decode_step(int(toks[warmup + n_done]), ctx + warmup + n_done)
+        n_done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
+    n = n_done
     sample = (f"{n} decode step(s) of the same model at positions {ctx + warmup}..{ctx + warmup + n - 1} "
               f"over a {ctx}-token synthetic context, after {warmup} warm-up step(s)")
     return n / dt, n, sample, oracle.num_threads()

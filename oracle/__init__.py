@@ -40,7 +40,8 @@ class _Config(ctypes.Structure):
                 ("moe_renorm", ctypes.c_int)]
 
 
-PROVIDER = ctypes.CFUNCTYPE(None, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+# int provider(layer, expert, which, dst, user): 0 once dst is filled, nonzero on failure
+PROVIDER = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                             ctypes.c_void_p)
 
 _lib = None
@@ -219,16 +220,27 @@ class Model:
         kv_shape = (ctx_cap, cfg.n_kv_heads, cfg.head_dim)
         self.k = [np.zeros(kv_shape, dtype=np.uint16) for _ in range(cfg.n_layers)]
         self.v = [np.zeros(kv_shape, dtype=np.uint16) for _ in range(cfg.n_layers)]
+        self._prov_error: Optional[BaseException] = None
         self._kp = (ctypes.c_void_p * cfg.n_layers)(*[a.ctypes.data for a in self.k])
         self._vp = (ctypes.c_void_p * cfg.n_layers)(*[a.ctypes.data for a in self.v])
         if expert_provider is not None:
             Fe, H = cfg.expert_ffn, cfg.hidden
 
             def _prov(layer, expert, which, dst, user):
+                # an exception cannot cross the C frames: it is kept, the oracle is told
+                # to stop, and the calling method raises it
                 n = Fe * H
-                arr = np.ascontiguousarray(expert_provider(layer, expert, which), dtype=np.uint16)
-                assert arr.size == n
-                ctypes.memmove(dst, arr.ctypes.data, 2 * n)
+                try:
+                    arr = np.ascontiguousarray(expert_provider(layer, expert, which), dtype=np.uint16)
+                    if arr.size != n:
+                        raise ValueError(f"expert provider returned {arr.size} elements for layer {layer}, "
+                                         f"expert {expert}, matrix {which}; expected {n}")
+                    ctypes.memmove(dst, arr.ctypes.data, 2 * n)
+                    return 0
+                except BaseException as exc:       # noqa: BLE001 - re-raised by the caller
+                    if self._prov_error is None:
+                        self._prov_error = exc
+                    return 1
 
             self._prov = PROVIDER(_prov)
         else:
@@ -252,8 +264,7 @@ class Model:
                                   None if ov is None else ov.ctypes.data,
                                   None if sel is None else sel.ctypes.data,
                                   None if wts is None else wts.ctypes.data)
-        if rc != 0:
-            raise ValueError("oracle decode_step: bad argument")
+        self._raise_on(rc, "decode_step")
         out = {"logits": logits}
         if hidden is not None:
             out["hidden"] = hidden
@@ -267,6 +278,12 @@ class Model:
         logits = np.empty((T, self.cfg.vocab), dtype=np.float64)
         rc = lib().oc_forward_nocache(ctypes.byref(self._c), self._wptrs, toks.ctypes.data, T,
                                       logits.ctypes.data, self._prov, None)
-        if rc != 0:
-            raise ValueError("oracle forward_nocache: bad argument")
+        self._raise_on(rc, "forward_nocache")
         return logits
+
+    def _raise_on(self, rc: int, what: str) -> None:
+        err, self._prov_error = self._prov_error, None
+        if rc == -2:
+            raise RuntimeError(f"oracle {what}: the expert provider failed") from err
+        if rc != 0:
+            raise ValueError(f"oracle {what}: bad argument")

@@ -45,8 +45,10 @@ typedef struct {
 } oc_config;
 
 /* Optional supplier of one expert's matrix when the caller does not hold all
- * experts in memory.  which: 0 gate [Fe][H], 1 up [Fe][H], 2 down [H][Fe]. */
-typedef void (*oc_expert_provider)(int layer, int expert, int which, uint16_t* dst, void* user);
+ * experts in memory.  which: 0 gate [Fe][H], 1 up [Fe][H], 2 down [H][Fe].
+ * Returns 0 once dst holds the whole matrix, nonzero on failure; a failure
+ * ends the step with an error code, never with a partly filled matrix. */
+typedef int (*oc_expert_provider)(int layer, int expert, int which, uint16_t* dst, void* user);
 
 /* ------------------------------------------------------------------ scalars */
 
@@ -226,9 +228,10 @@ static const uint16_t* wptr(const oc_config* c, const uint16_t* const* w, int la
 }
 enum { S_ATTN_NORM = 0, S_WQ, S_WK, S_WV, S_WO, S_FFN_NORM };
 
-static void moe_ffn_layer(const oc_config* c, const uint16_t* const* w, int l,
-                          oc_expert_provider prov, void* user, const int* override_sel,
-                          const double* h, double* y, int* sel_out, double* wts_out) {
+/* Returns 0, or -2 when the expert weights are neither held nor supplied. */
+static int moe_ffn_layer(const oc_config* c, const uint16_t* const* w, int l,
+                         oc_expert_provider prov, void* user, const int* override_sel,
+                         const double* h, double* y, int* sel_out, double* wts_out) {
     int H = c->hidden, E = c->n_experts, Fe = c->expert_ffn, K = c->top_k;
     const uint16_t* w_router = wptr(c, w, l, 6);
     const uint16_t* wg_all = wptr(c, w, l, 7);
@@ -239,9 +242,10 @@ static void moe_ffn_layer(const oc_config* c, const uint16_t* const* w, int l,
     oc_moe_route(w_router, E, H, h, K, c->moe_renorm, override_sel, sel, wts, NULL);
     double* ye = (double*)malloc(sizeof(double) * H);
     uint16_t* tmp = NULL;
+    int rc = 0;
     if (!wg_all) tmp = (uint16_t*)malloc(sizeof(uint16_t) * 3 * (size_t)Fe * H);
     for (int i = 0; i < H; ++i) y[i] = 0.0;
-    for (int k = 0; k < K; ++k) {
+    for (int k = 0; k < K && rc == 0; ++k) {
         int e = sel[k];
         const uint16_t *wg, *wu, *wd;
         if (wg_all) {
@@ -249,9 +253,11 @@ static void moe_ffn_layer(const oc_config* c, const uint16_t* const* w, int l,
             wu = wu_all + (size_t)e * Fe * H;
             wd = wd_all + (size_t)e * H * Fe;
         } else {
-            prov(l, e, 0, tmp, user);
-            prov(l, e, 1, tmp + (size_t)Fe * H, user);
-            prov(l, e, 2, tmp + 2 * (size_t)Fe * H, user);
+            if (!prov || prov(l, e, 0, tmp, user) != 0 || prov(l, e, 1, tmp + (size_t)Fe * H, user) != 0 ||
+                prov(l, e, 2, tmp + 2 * (size_t)Fe * H, user) != 0) {
+                rc = -2;
+                break;
+            }
             wg = tmp;
             wu = tmp + (size_t)Fe * H;
             wd = tmp + 2 * (size_t)Fe * H;
@@ -267,6 +273,7 @@ static void moe_ffn_layer(const oc_config* c, const uint16_t* const* w, int l,
     free(ye);
     free(wts);
     free(sel);
+    return rc;
 }
 
 /*
@@ -277,7 +284,8 @@ static void moe_ffn_layer(const oc_config* c, const uint16_t* const* w, int l,
  * stream after the embedding and after each attention / FFN residual add;
  * moe_sel [L][top_k] and moe_wts [L][top_k] the router's choice per layer;
  * moe_override [L][top_k] (entries < 0 mean "no override for this layer")
- * forces a selected set.  Returns 0, or -1 on a bad argument.
+ * forces a selected set.  Returns 0, -1 on a bad argument, or -2 when the
+ * expert provider failed (the outputs are then not valid).
  */
 int oc_decode_step(const oc_config* c, const uint16_t* const* w, uint16_t* const* kcache,
                    uint16_t* const* vcache, int ctx_cap, int token, int pos, double* logits,
@@ -293,12 +301,13 @@ int oc_decode_step(const oc_config* c, const uint16_t* const* w, uint16_t* const
     double* v = (double*)malloc(sizeof(double) * nkv * d);
     double* o = (double*)malloc(sizeof(double) * nq * d);
     double* y = (double*)malloc(sizeof(double) * H);
+    int rc = 0;
 
     const uint16_t* emb = w[0] + (size_t)token * H;
     for (int i = 0; i < H; ++i) x[i] = oc_bf16_to_double(emb[i]);
     if (hidden) memcpy(hidden, x, sizeof(double) * H);
 
-    for (int l = 0; l < L; ++l) {
+    for (int l = 0; l < L && rc == 0; ++l) {
         /* attention block */
         oc_rmsnorm(x, wptr(c, w, l, S_ATTN_NORM), H, c->rms_eps, h);
         oc_gemv(wptr(c, w, l, S_WQ), nq * d, H, h, q);
@@ -322,21 +331,24 @@ int oc_decode_step(const oc_config* c, const uint16_t* const* w, uint16_t* const
         if (c->n_experts > 0) {
             const int* ov = NULL;
             if (moe_override && moe_override[l * c->top_k] >= 0) ov = moe_override + l * c->top_k;
-            moe_ffn_layer(c, w, l, prov, user, ov, h, y, moe_sel ? moe_sel + l * c->top_k : NULL,
-                          moe_wts ? moe_wts + l * c->top_k : NULL);
+            rc = moe_ffn_layer(c, w, l, prov, user, ov, h, y, moe_sel ? moe_sel + l * c->top_k : NULL,
+                               moe_wts ? moe_wts + l * c->top_k : NULL);
+            if (rc != 0) break;
         } else {
             oc_swiglu_ffn(wptr(c, w, l, 6), wptr(c, w, l, 7), wptr(c, w, l, 8), H, c->ffn, h, y);
         }
         for (int i = 0; i < H; ++i) x[i] += y[i];
         if (hidden) memcpy(hidden + (size_t)(2 * l + 2) * H, x, sizeof(double) * H);
     }
-    const uint16_t* final_norm = w[1 + L * layer_slots(c)];
-    const uint16_t* lm_head = w[2 + L * layer_slots(c)];
-    oc_rmsnorm(x, final_norm, H, c->rms_eps, h);
-    oc_gemv(lm_head, c->vocab, H, h, logits);
+    if (rc == 0) {
+        const uint16_t* final_norm = w[1 + L * layer_slots(c)];
+        const uint16_t* lm_head = w[2 + L * layer_slots(c)];
+        oc_rmsnorm(x, final_norm, H, c->rms_eps, h);
+        oc_gemv(lm_head, c->vocab, H, h, logits);
+    }
 
     free(x); free(h); free(q); free(k); free(v); free(o); free(y);
-    return 0;
+    return rc;
 }
 
 /*
@@ -344,7 +356,8 @@ int oc_decode_step(const oc_config* c, const uint16_t* const* w, uint16_t* const
  * (positions 0..T-1) layer by layer, computing every position's K and V
  * afresh (rounded to bf16 as the cache would hold them) and causal attention
  * for every position.  logits [T][vocab].  Used to check that the cached
- * incremental decode reproduces it.  Dense and MoE models.
+ * incremental decode reproduces it.  Dense and MoE models.  Returns 0, -1 on
+ * a bad argument, -2 when the expert provider failed.
  */
 int oc_forward_nocache(const oc_config* c, const uint16_t* const* w, const int* tokens, int T,
                        double* logits, oc_expert_provider prov, void* user) {
@@ -360,11 +373,12 @@ int oc_forward_nocache(const oc_config* c, const uint16_t* const* w, const int* 
     uint16_t* V = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)T * nkv * d);
     double* o = (double*)malloc(sizeof(double) * nq * d);
     double* y = (double*)malloc(sizeof(double) * H);
+    int rc = 0;
 
     for (int t = 0; t < T; ++t)
         for (int i = 0; i < H; ++i) X[(size_t)t * H + i] = oc_bf16_to_double(w[0][(size_t)tokens[t] * H + i]);
 
-    for (int l = 0; l < L; ++l) {
+    for (int l = 0; l < L && rc == 0; ++l) {
         for (int t = 0; t < T; ++t) {
             oc_rmsnorm(X + (size_t)t * H, wptr(c, w, l, S_ATTN_NORM), H, c->rms_eps, h);
             double* qt = q + (size_t)t * nq * d;
@@ -376,28 +390,29 @@ int oc_forward_nocache(const oc_config* c, const uint16_t* const* w, const int* 
             oc_gemv(wptr(c, w, l, S_WV), nkv * d, H, h, kv);
             for (int i = 0; i < nkv * d; ++i) V[(size_t)t * nkv * d + i] = oc_bf16_round(kv[i]);
         }
-        for (int t = 0; t < T; ++t) {
+        for (int t = 0; t < T && rc == 0; ++t) {
             /* causal: position t sees positions 0..t */
             oc_attention(q + (size_t)t * nq * d, K, V, t + 1, nq, nkv, d, o);
             oc_gemv(wptr(c, w, l, S_WO), H, nq * d, o, y);
             double* xt = X + (size_t)t * H;
             for (int i = 0; i < H; ++i) xt[i] += y[i];
             oc_rmsnorm(xt, wptr(c, w, l, S_FFN_NORM), H, c->rms_eps, h);
-            if (c->n_experts > 0)
-                moe_ffn_layer(c, w, l, prov, user, NULL, h, y, NULL, NULL);
-            else
+            if (c->n_experts > 0) {
+                rc = moe_ffn_layer(c, w, l, prov, user, NULL, h, y, NULL, NULL);
+                if (rc != 0) break;
+            } else
                 oc_swiglu_ffn(wptr(c, w, l, 6), wptr(c, w, l, 7), wptr(c, w, l, 8), H, c->ffn, h, y);
             for (int i = 0; i < H; ++i) xt[i] += y[i];
         }
     }
     const uint16_t* final_norm = w[1 + L * layer_slots(c)];
     const uint16_t* lm_head = w[2 + L * layer_slots(c)];
-    for (int t = 0; t < T; ++t) {
+    for (int t = 0; t < T && rc == 0; ++t) {
         oc_rmsnorm(X + (size_t)t * H, final_norm, H, c->rms_eps, h);
         oc_gemv(lm_head, c->vocab, H, h, logits + (size_t)t * c->vocab);
     }
     free(X); free(h); free(q); free(kv); free(K); free(V); free(o); free(y);
-    return 0;
+    return rc;
 }
 
 int oc_num_threads(void) {

@@ -368,3 +368,62 @@ def test_expert_provider_matches_held_experts():
     prov = lambda l, e, which: w[f"layers.{l}." + ("w_gate", "w_up", "w_down")[which]][e]
     lazy = oracle.Model(cfg, lazy_w, 4, _names(cfg), expert_provider=prov).decode_step(9, 0)
     np.testing.assert_array_equal(lazy["logits"], held)
+
+
+def test_dense_ffn_wiring_gate_up_down_closed_form():
+    """Layer 0's dense FFN with W_gate = I, W_up = c·I (on the first H rows) and
+    W_down = I: the residual update is silu(h_i)·c·h_i, h = rmsnorm(x_mid).  Swapping
+    the gate and up slots gives silu(c·h_i)·h_i instead, and a transposed or
+    misplaced down matrix moves the update off the diagonal, so either fails."""
+    cfg = syn.TINY
+    H, F = cfg.hidden, cfg.ffn
+    c = 2.0
+    w = _weights(cfg)
+    z = _zero_like(w)
+    z["tok_emb"] = w["tok_emb"]
+    for name in list(z):
+        if name.endswith("norm"):
+            z[name] = w[name]
+    Wg = np.zeros((F, H), dtype=np.float32)
+    Wg[np.arange(H), np.arange(H)] = 1.0
+    Wd = np.zeros((H, F), dtype=np.float32)
+    Wd[np.arange(H), np.arange(H)] = 1.0
+    z["layers.0.w_gate"], z["layers.0.w_up"], z["layers.0.w_down"] = bits(Wg), bits(c * Wg), bits(Wd)
+    m = oracle.Model(cfg, z, 4, _names(cfg))
+    out = m.decode_step(123, 0, want_hidden=True)
+    x_mid, x_out = out["hidden"][1], out["hidden"][2]
+    # attention weights are zero: x_mid is the embedding row
+    np.testing.assert_array_equal(x_mid, oracle.bf16_to_f64(w["tok_emb"][123]))
+    g = oracle.bf16_to_f64(w["layers.0.ffn_norm"])
+    h = x_mid / np.sqrt(np.mean(x_mid * x_mid) + cfg.rms_eps) * g
+    silu = h / (1.0 + np.exp(-h))
+    np.testing.assert_allclose(x_out - x_mid, silu * c * h, rtol=1e-12, atol=1e-15)
+    swapped = c * h / (1.0 + np.exp(-c * h)) * h
+    assert np.max(np.abs((x_out - x_mid) - swapped)) > 1e-3
+
+
+def test_failing_expert_provider_raises():
+    """A provider that cannot supply a matrix ends the step with an error: the
+    oracle never computes with a partly filled expert buffer."""
+    cfg = syn.TINY_MOE
+    w = _weights(cfg)
+    lazy_w = {k: v for k, v in w.items() if not any(s in k for s in ("w_gate", "w_up", "w_down"))}
+
+    def short(l, e, which):
+        return np.zeros(3, dtype=np.uint16)          # wrong size
+
+    m = oracle.Model(cfg, lazy_w, 4, _names(cfg), expert_provider=short)
+    with pytest.raises(RuntimeError, match="expert provider failed"):
+        m.decode_step(9, 0)
+
+    def boom(l, e, which):
+        raise KeyError("no such expert")
+
+    m = oracle.Model(cfg, lazy_w, 4, _names(cfg), expert_provider=boom)
+    with pytest.raises(RuntimeError) as ei:
+        m.forward_nocache([1, 2])
+    assert isinstance(ei.value.__cause__, KeyError)
+    # a provider that works afterwards still gives the held-weights result
+    prov = lambda l, e, which: w[f"layers.{l}." + ("w_gate", "w_up", "w_down")[which]][e]
+    ok = oracle.Model(cfg, lazy_w, 4, _names(cfg), expert_provider=prov).decode_step(9, 0)["logits"]
+    np.testing.assert_array_equal(ok, oracle.Model(cfg, w, 4, _names(cfg)).decode_step(9, 0)["logits"])
