@@ -219,8 +219,9 @@ void mk_state_destroy(mk_state* state);
  * it sets MK_ERR_TIMEOUT; the kernel then drains and returns. */
 mk_status mk_state_set_timeout(mk_state* state, int64_t timeout_ns);
 
-/* L2 prefetch distance, in tasks ahead of the work-queue head (default 0 =
- * off).  A hint only: results do not depend on it. */
+/* L2 prefetch distance, in tasks ahead of each CTA's latest claim (default 0
+ * = off; every distance measured slower than none on B200).  A hint only:
+ * results do not depend on it. */
 mk_status mk_state_set_prefetch(mk_state* state, int tasks_ahead);
 
 /* Test hook for failure detection: adds `offset` to the target of every

@@ -36,8 +36,11 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
     cmd = nvcc_cmd(True)
     if verbose:
         print(" ".join(cmd))
-    out = subprocess.run(cmd, check=True, capture_output=True, text=True)
+    out = subprocess.run(cmd, capture_output=True, text=True)
     log = out.stdout + out.stderr
+    if out.returncode != 0:
+        errs = [ln for ln in log.splitlines() if "ptxas info" not in ln and "bytes stack frame" not in ln]
+        raise RuntimeError("nvcc failed:\n" + "\n".join(errs[-60:]))
     if ptxas_verbose:
         print(log)
     # The megakernel re-splits its registers between warpgroups at run time

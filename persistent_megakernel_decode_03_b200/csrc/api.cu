@@ -51,7 +51,7 @@ struct mk_state {
     uint32_t wait_offset = 0;
     // device memory
     uint32_t* events = nullptr;
-    unsigned long long* queue = nullptr;   // [0] work queue, [1] L2-prefetch cursor
+    unsigned long long* queue = nullptr;   // [0] work queue ([1] unused)
     uint32_t pf_dist = 0;
     uint32_t* done = nullptr;
     int* err = nullptr;
@@ -189,7 +189,6 @@ mk::Params base_params(mk_state* s) {
     p.thr = s->g->d_thr;
     p.events = s->events;
     p.queue = s->queue;
-    p.pf_head = s->queue + 1;
     p.pf_dist = s->pf_dist;
     p.done = s->done;
     p.err = s->err;

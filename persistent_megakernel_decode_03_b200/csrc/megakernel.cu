@@ -198,6 +198,14 @@ __device__ __forceinline__ int ld_relaxed_int(const int* p) {
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Arrival count with acquire-release semantics at GPU scope: publishes every write
+// that precedes it in causality order (cumulative release) and makes the other
+// arrivals' writes visible to what follows (acquire).  Returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 
 
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
@@ -272,6 +280,7 @@ struct __align__(128) Smem {
     uint32_t tmem_base;                      // TMEM address of the accumulator (batched graphs)
     int mm_last;                             // this CTA's split of a tile arrived last
     int pid[kPidRing];                       // producer: physical page ids read ahead
+    int pf_claimed;                          // producer's latest claimed task (-1: finished), for the prefetcher
     int flag[4];
 };
 
@@ -386,8 +395,11 @@ __device__ __forceinline__ int gemv_chunks(const GemvGeom& g, uint8_t flags) {
 }
 
 // Splits of one (sequence, kv head) actually used this step: about one per
-// kAttnSplitTokens positions of context, at most the graph's split count S.
-constexpr int kAttnSplitTokens = 64;
+// kAttnSplitTokens positions of context, at most the graph's split count S.  A
+// context of up to kAttnSplitTokens positions is one split that writes the
+// normalised output itself: no merge step (measured at 8B, position 300: 3.54 ms
+// per step against 3.73 ms with 64-position splits and their merge).
+constexpr int kAttnSplitTokens = 512;
 __device__ __forceinline__ int attn_active_splits(int n_ctx, int S) {
     int a = (n_ctx + kAttnSplitTokens - 1) / kAttnSplitTokens;
     return a < 1 ? 1 : (a > S ? S : a);
@@ -772,6 +784,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         const unsigned long long q = q_next;
         if (q >= p.n_tasks) break;
         const int ti = (int)q;
+        *reinterpret_cast<volatile int*>(&sm.pf_claimed) = ti;
         const Task t = p.tasks[ti];
         q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
         if constexpr (MM) {
@@ -823,6 +836,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
             }
         }
     }
+    *reinterpret_cast<volatile int*>(&sm.pf_claimed) = -1;   // the prefetcher stops
     int& stage = ring.stage;
     uint32_t& lap = ring.lap;
     auto acquire_slot = [&]() -> bool { return pr_acquire(p, sm, ring); };
@@ -847,21 +861,25 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
 
 // ----------------------------------------------------------------------------- L2 prefetcher
 
-// Walks the task list a bounded distance ahead of the work-queue head and asks
-// L2 to fetch the weight rows (and KV pages) of upcoming tasks, so HBM keeps
-// streaming while the consumers wait on a dependency; the ring copies then hit
-// L2.  Routed-expert weights are unknown until the router runs and are skipped.
-__device__ void prefetch_loop(const Params& p) {
-    if (p.pf_dist == 0 || p.pf_head == nullptr) return;
-    while (true) {
-        const unsigned long long i = atomicAdd(p.pf_head, 1ull) - p.queue_base;
-        if (i >= p.n_tasks) return;
+// Asks L2 to fetch the weight rows (and KV pages) of tasks a bounded distance
+// ahead of the work queue, so HBM could keep streaming while the consumers wait
+// on a dependency.  The task list is dealt to the CTAs statically (CTA c takes
+// tasks c, c + grid, ...), and the distance is measured against this CTA's own
+// latest claim (shared memory), which tracks the global queue head within a
+// wave: no atomics and no polling of global memory.  Off by default: every
+// distance measured slower than none.  Routed-expert weights are unknown until
+// the router runs and are skipped.
+__device__ void prefetch_loop(const Params& p, Smem& sm) {
+    if (p.pf_dist == 0) return;
+    const volatile int* claimed = &sm.pf_claimed;
+    for (uint32_t i = blockIdx.x; i < p.n_tasks; i += gridDim.x) {
         Waiter w{0, 0};
         while (true) {
-            const unsigned long long h = ld_relaxed_u64(p.queue) - p.queue_base;
-            if (h + p.pf_dist > i) break;
-            if (wait_should_stop(p, w)) return;   // an error elsewhere; a slow step is not one
-            __nanosleep(200);
+            const int c = *claimed;
+            if (c < 0 || *reinterpret_cast<volatile int*>(&sm.flag[3])) return;   // producer done or aborting
+            if ((uint32_t)c + p.pf_dist >= i) break;
+            if (wait_should_stop(p, w)) return;          // an error elsewhere; a slow step is not one
+            __nanosleep(128);
         }
         const Task t = p.tasks[i];
         if (t.op == MK_OP_ATTN) {
@@ -1866,6 +1884,41 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
     }
     csync(p, sm, cph);
     if (sm.flag[3]) { abort_all = true; return; }
+    if (valid && attn_active_splits(pos + 1, S) == 1) {
+        // the whole context is in split 0: it writes the normalised output itself and
+        // no merge follows (the other splits only count their arrival, which nobody
+        // waits for; the task's event is signalled by the epilogue warp)
+        if (s == 0) {
+            float* out = p.attn_o + ((size_t)l * p.max_batch + b) * p.nq * HD + (size_t)g * HPG * HD;
+            for (int q = tid; q < HPG * HD / 4; q += kConsumerThreads) {
+                const int h = (q * 4) / HD, c = (q * 4) % HD;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sc[((size_t)w * HPG + h) * (HD + 2)]);
+                float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+                float L = 0.0f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        const float* ww = sc + ((size_t)w * HPG + h) * (HD + 2);
+                        const float f = (ww[0] == -INFINITY) ? 0.0f : exp2f(ww[0] - M);
+                        L = fmaf(ww[1], f, L);
+                        o.x = fmaf(ww[2 + c], f, o.x);
+                        o.y = fmaf(ww[3 + c], f, o.y);
+                        o.z = fmaf(ww[4 + c], f, o.z);
+                        o.w = fmaf(ww[5 + c], f, o.w);
+                    }
+                }
+                const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+                const float4 r = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+                *reinterpret_cast<float4*>(out + (size_t)h * HD + c) = r;
+                if (p.mm) put_operand4(p, kOpAo, l, b, p.nq * HD, g * HPG * HD + h * HD + c, r);
+            }
+            if (p.mm) fence_proxy_async_global();
+        }
+        if (tid == 0) atomicAdd(p.attn_cnt + ((size_t)l * p.max_batch + b) * p.nkv + g, 1u);
+        return;
+    }
     if (valid) {
         for (int idx = tid; idx < HPG * (HD + 2); idx += kConsumerThreads) {
             const int h = idx / (HD + 2), c = idx % (HD + 2);
@@ -1893,12 +1946,13 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
         }
     }
     // arrival of this split (active or not); the split that arrives last for its
-    // (sequence, kv group) merges the partials once, before its completion is signalled
-    __threadfence();
+    // (sequence, kv group) merges the partials once, before its completion is
+    // signalled.  The CTA barrier orders every thread's partial stores before thread
+    // 0's acquire-release arrival (cumulative), and the second barrier orders its
+    // acquire before the merge's loads.
     csync(p, sm, cph);
     if (tid == 0) {
-        const uint32_t old = atomicAdd(p.attn_cnt + ((size_t)l * p.max_batch + b) * p.nkv + g, 1u);
-        __threadfence();
+        const uint32_t old = atom_add_acq_rel(p.attn_cnt + ((size_t)l * p.max_batch + b) * p.nkv + g, 1u);
         sm.attn_last = (old == (uint32_t)S * p.epoch - 1u) ? 1 : 0;
     }
     csync(p, sm, cph);
@@ -2321,9 +2375,11 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
             int r = 1;
             if (lane == 0) {
                 r = event_wait(p, e, p.thr[e] * p.epoch + p.wait_offset, ti) ? 1 : 0;
-                if (r) __threadfence();
             }
+            // lane 0's acquire, then the warp barrier (which orders memory among its
+            // lanes), before any lane reads what the event's producers wrote
             r = __shfl_sync(0xFFFFFFFFu, r, 0);
+            __syncwarp();
             if (!r) { sm.flag[3] = 1; break; }
             ok_evt[3] = ok_evt[2]; ok_evt[2] = ok_evt[1]; ok_evt[1] = ok_evt[0]; ok_evt[0] = e;
         }
@@ -2552,17 +2608,17 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
                                 : (t.flags != kFastNone) ? kConsumerWarps : thread_map(g.K).wpg;
                 gemv_store(p, sm, t, g, wpg, buf, lane);
                 if (t.op == MK_OP_ROUTER) {
-                    // arrival of this router tile; the layer's last tile selects the experts
-                    // and only it signals the router event
-                    __threadfence();
+                    // arrival of this router tile (acquire-release: the warp barrier orders
+                    // the lanes' logit stores before it); the layer's last tile selects the
+                    // experts and only it signals the router event
                     __syncwarp();
                     int last = 0;
                     if (lane == 0) {
-                        const uint32_t old = atomicAdd(p.router_cnt + t.layer, 1u);
-                        __threadfence();
+                        const uint32_t old = atom_add_acq_rel(p.router_cnt + t.layer, 1u);
                         last = (old == (uint32_t)p.n_router_tiles * p.epoch - 1u) ? 1 : 0;
                     }
                     last = __shfl_sync(0xFFFFFFFFu, last, 0);
+                    __syncwarp();
                     if (last) router_finalize(p, sm, t.layer);
                     else evt = MK_NO_EVENT;
                 }
@@ -2572,11 +2628,12 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
             ++nb;
             ++seq;
         } while (nb < kRedBufs && mbar_test_wait(&sm.red_full[seq % kRedBufs], (seq / kRedBufs) & 1));
-        // every lane orders its own stores (and, through the consumers' arrivals, theirs)
-        // before lane 0's releases of the events
-        bool any = false;
-        for (int k = 0; k < nb; ++k) any |= (evts[k] != MK_NO_EVENT);
-        if (any) __threadfence();
+        // The events are released with red.release.gpu by lane 0.  Release is
+        // cumulative: it publishes every write that precedes it in causality order --
+        // the other lanes' stores (ordered by the warp barrier) and the consumer
+        // warps' stores (ordered by their arrivals on red_full, which this warp
+        // acquired).  A full fence here (fence.sc by every lane) cost 0.34 ms of an
+        // 8B step's 3.88 ms and is not needed.
         __syncwarp();
         if (lane == 0) {
             for (int k = 0; k < nb; ++k) {
@@ -2614,6 +2671,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&sm.red_free[i], 1);
         }
         for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
+        sm.pf_claimed = 0;
         // the 128-byte-swizzled tensor-core operands need 1 KB-aligned stages
         if (p.mm && (smem_u32(sm.ring) & 1023u) != 0) {
             set_error(p, kErrFault, -1, -9, (int)(smem_u32(sm.ring) & 1023u), 0);
@@ -2638,7 +2696,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     } else if (warp == kEpilogueWarp) {
         epilogue_loop(p, sm);
     } else if (warp == kPrefetchWarp) {
-        if (lane == 0) prefetch_loop(p);
+        if (lane == 0) prefetch_loop(p, sm);
     }
 }
 
@@ -2649,11 +2707,12 @@ static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream, bool
     auto kern = p.mm ? megakernel<HPG, DPL, true> : megakernel<HPG, DPL, false>;
     // the shared-memory attribute, once per instantiation and device (so that a step
     // can be captured into a CUDA graph without host-side calls in between)
-    static unsigned attr_set[2] = {0u, 0u};
+    // (devices 0..63 are remembered; a higher index sets the attribute every launch)
+    static unsigned long long attr_set[2] = {0ull, 0ull};
     int dev = 0;
     cudaGetDevice(&dev);
-    const unsigned bit = 1u << (dev & 31);
-    if (!(attr_set[p.mm ? 1 : 0] & bit)) {
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (!bit || !(attr_set[p.mm ? 1 : 0] & bit)) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
         if (e != cudaSuccess) return e;
         attr_set[p.mm ? 1 : 0] |= bit;

@@ -160,8 +160,7 @@ struct Params {
     uint32_t* events;
     unsigned long long* queue;   // global work-queue head
     unsigned long long queue_base;
-    unsigned long long* pf_head; // L2-prefetch cursor over the task list (same base as the queue)
-    uint32_t pf_dist;            // prefetch at most this many tasks ahead of the queue head (0: off)
+    uint32_t pf_dist;            // L2 prefetch at most this many tasks ahead of the CTA's claims (0: off)
     uint32_t* done;              // completed-task counter
     int* err;                    // [0] status, [1..4] info
     uint32_t* router_cnt;        // [L] router tile arrivals

@@ -3,6 +3,7 @@
 // forbidden or would disturb a fixed memory budget).  Everything the step needs
 // besides its inputs and outputs lives in one file-scope device array of fixed
 // size, which every GPU that loads this library keeps until the process exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -31,6 +32,7 @@ struct Layout {
 
 struct DeviceCache {
     bool have_base = false;
+    unsigned long long ctx_id = 0;         // CUDA context the address below belongs to
     unsigned char* base = nullptr;         // device address of g_scratch on this device
     bool have_plan = false;
     std::vector<unsigned char> key;        // desc + weight pointers + max_ctx + n_sm
@@ -40,6 +42,32 @@ struct DeviceCache {
 
 std::mutex g_mutex;
 DeviceCache g_cache[kMaxDevices];
+
+// Unique id of the calling thread's current CUDA context (driver calls reached
+// through the runtime's entry-point query: no link against the driver library).
+// A device reset or a new primary context loads the module afresh, and its array
+// then holds nothing of earlier calls: the cache is keyed on this id.
+bool current_ctx_id(unsigned long long* id) {
+    using GetCur = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCur get_cur = nullptr;
+    static GetId get_id = nullptr;
+    if (!get_cur || !get_id) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        get_cur = reinterpret_cast<GetCur>(f);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        get_id = reinterpret_cast<GetId>(f);
+    }
+    CUcontext ctx = nullptr;
+    if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -116,14 +144,28 @@ extern "C" mk_status mk_decode_step_noalloc(const mk_model_desc* desc, const voi
     if (dev < 0 || dev >= kMaxDevices) return nfail(MK_ERR_UNSUPPORTED, "mk_decode_step_noalloc: device index too large");
     cudaStream_t st = (cudaStream_t)stream;
 
+    // the runtime makes the device's primary context current on first use; do that
+    // before asking which context this is (cudaFree(nullptr) allocates nothing)
+    e = cudaFree(nullptr);
+    if (e != cudaSuccess) return nfail(MK_ERR_CUDA, "mk_decode_step_noalloc: no CUDA context");
+    unsigned long long ctx_id = 0;
+    if (!current_ctx_id(&ctx_id)) return nfail(MK_ERR_CUDA, "mk_decode_step_noalloc: context query failed");
+
     std::lock_guard<std::mutex> guard(g_mutex);
     DeviceCache& c = g_cache[dev];
+    if (c.have_base && c.ctx_id != ctx_id) {
+        // another context (after a device reset, or a new primary context): the array
+        // was loaded afresh, so its address is looked up and the plan uploaded again
+        c.have_base = false;
+        c.have_plan = false;
+    }
     if (!c.have_base) {
-        // once per device, with that device current: the device address of the array
+        // once per device and context, with that device current: the array's address
         void* base = nullptr;
         e = cudaGetSymbolAddress(&base, g_scratch);
         if (e != cudaSuccess || !base) return nfail(MK_ERR_CUDA, "mk_decode_step_noalloc: cudaGetSymbolAddress failed");
         c.base = static_cast<unsigned char*>(base);
+        c.ctx_id = ctx_id;
         c.have_base = true;
     }
     // (re)plan when the model, its weights, the context or the device changed
@@ -208,7 +250,6 @@ extern "C" mk_status mk_decode_step_noalloc(const mk_model_desc* desc, const voi
     p.thr = reinterpret_cast<const uint32_t*>(b + lay.thr);
     p.events = reinterpret_cast<uint32_t*>(b + lay.events);
     p.queue = reinterpret_cast<unsigned long long*>(b + lay.queue);
-    p.pf_head = p.queue + 1;
     p.pf_dist = 0;
     p.queue_base = 0;
     p.done = reinterpret_cast<uint32_t*>(b + lay.done);
