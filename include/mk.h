@@ -100,7 +100,11 @@ typedef struct {
 
 /* ---------------------------------------------------------------- model */
 
-/* Records the shape and the weight pointers (device, bf16, row-major
+/* Passage: Cohere page ("Cohere megakerneles kiszolgálót mutatott be a
+ * North Mini Code modellhez"), section "A szűk keresztmetszet a memória-
+ * sávszélesség": the step streams the model's bf16 weights from HBM once per
+ * token; this call registers those weights.
+ * Records the shape and the weight pointers (device, bf16, row-major
  * [out][in]).  Order of weight_ptrs: tok_emb [vocab][hidden]; then per layer
  * attn_norm [hidden], wq [n_q*d][hidden], wk [n_kv*d][hidden], wv
  * [n_kv*d][hidden], wo [hidden][n_q*d], ffn_norm [hidden], then dense:
@@ -114,11 +118,17 @@ typedef struct {
  * hidden, ffn, expert_ffn and n_q*d multiples of 8, top_k <= 16. */
 mk_status mk_load_model(const mk_model_desc* desc, const void* const* weight_ptrs, int n_ptrs,
                         mk_model** out);
+/* Passage: none of its own.  Releases the model record (never the weights). */
 void mk_model_destroy(mk_model* model);
 
 /* ---------------------------------------------------------------- task graph */
 
-/* Builds the task list for batches up to max_batch and contexts up to max_ctx
+/* Passage: MPK digest ("LLM को MegaKernel में compile करके low-latency
+ * inference हासिल करना"), section "Part 1. Compiler": the operator graph is
+ * turned into a fine-grained task graph with events as the
+ * synchronisation points; Cohere page, section "Egyetlen tartós kernelre épül a
+ * kiszolgálás": the blocks work from a task list prepared on the host.
+ * Builds the task list for batches up to max_batch and contexts up to max_ctx
  * tokens (positions 0..max_ctx-1) on the current device (its SM count sets
  * the tile sizes and the grid) and uploads it.  max_batch 1 streams every
  * weight row through CUDA-core GEMV tiles; max_batch 2..64 (dense models
@@ -129,15 +139,18 @@ void mk_model_destroy(mk_model* model);
  * and dependency analysis). */
 mk_status mk_build_taskgraph(mk_model* model, int max_batch, int max_ctx, mk_graph** out);
 
-/* Profiling aid: the graph's tasks of one dense operator kind only (op in
+/* Passage: none of its own (a measurement aid for the per-tile-type evidence).
+ * Profiling aid: the graph's tasks of one dense operator kind only (op in
  * MK_OP_QKV..MK_OP_LMHEAD, every layer), with no dependencies, so one tile type
  * can be timed and profiled alone.  Its outputs are not a decode step. */
 mk_status mk_build_taskgraph_solo(mk_model* model, int max_batch, int max_ctx, int op, mk_graph** out);
 
-/* The same plan on the host only (no device memory, no CUDA call), for an
+/* Passage: MPK digest, "Part 1. Compiler" (as mk_build_taskgraph).
+ * The same plan on the host only (no device memory, no CUDA call), for an
  * SM count given by the caller: for inspecting and checking the graph. */
 mk_status mk_plan_taskgraph(const mk_model_desc* desc, int max_batch, int max_ctx, int n_sm,
                             mk_graph** out);
+/* Passage: none of its own.  Releases a graph (host and device copies). */
 void mk_graph_destroy(mk_graph* graph);
 
 typedef struct {
@@ -147,6 +160,8 @@ typedef struct {
     int64_t weight_bytes_per_step;   /* bf16 weight bytes streamed by one B=1 step (dense: all
                                         but the embedding table; MoE: router + top_k experts) */
 } mk_graph_info;
+/* Passage: MPK digest, "Part 1. Compiler" (the task graph's size).  Copies the
+ * graph's summary to *info (host memory). */
 mk_status mk_graph_get_info(const mk_graph* graph, mk_graph_info* info);
 
 /* Operator kinds of a task. */
@@ -196,9 +211,13 @@ typedef struct {
     uint32_t pointer_wait;
 } mk_task_info;
 
-/* Copies min(cap, n_tasks) tasks in list order; returns the count written via *n. */
+/* Passage: MPK digest, "Part 1. Compiler" (tasks, events and the edges between
+ * them).  Copies min(cap, n_tasks) tasks in list order to out (host memory);
+ * returns the count written via *n. */
 mk_status mk_graph_export_tasks(const mk_graph* graph, mk_task_info* out, int cap, int* n);
-/* thresholds[e] for e < n_events (per step). */
+/* Passage: MPK digest, "Part 2. Runtime", "Event-आधारित execution तरीका" (an
+ * event fires when its counter reaches the threshold).  thresholds[e] for
+ * e < n_events (per step), to host memory. */
 mk_status mk_graph_export_thresholds(const mk_graph* graph, uint32_t* out, int cap, int* n);
 
 /* Wave-quantisation arithmetic used by the tile sizer: n_tiles equal tiles on
@@ -209,28 +228,43 @@ mk_status mk_wave_stats(int n_tiles, int n_sm, int* waves, int* idle_sms_last_wa
 
 /* ---------------------------------------------------------------- state and steps */
 
-/* Allocates the device state of a graph (event counters, work-queue head,
+/* Passage: Cohere page, section "Egyetlen tartós kernelre épül a
+ * kiszolgálás": data dependencies are signalled by counters in global memory;
+ * MPK digest, "Part 2. Runtime" (event counters and thresholds).
+ * Allocates the device state of a graph (event counters, work-queue head,
  * activation buffers, attention partials): library-owned until
  * mk_state_destroy. */
 mk_status mk_state_create(mk_graph* graph, mk_state** out);
+/* Passage: none of its own.  Frees the state's device memory (after the work
+ * queued on its stream has finished: the caller synchronises first). */
 void mk_state_destroy(mk_state* state);
 
-/* Device-side wait limit in nanoseconds (default 2e9).  A wait that exceeds
+/* Passage: none of its own (every device-side wait is bounded).
+ * Device-side wait limit in nanoseconds (default 2e9).  A wait that exceeds
  * it sets MK_ERR_TIMEOUT; the kernel then drains and returns. */
 mk_status mk_state_set_timeout(mk_state* state, int64_t timeout_ns);
 
-/* L2 prefetch distance, in tasks ahead of each CTA's latest claim (default 0
+/* Passage: Cohere page, "Honnan jön a gyorsulás?", last paragraph: weight
+ * tiles are fetched before their activation dependency is met.  The ring
+ * already does that into shared memory; this optional hint also asks L2.
+ * L2 prefetch distance, in tasks ahead of each CTA's latest claim (default 0
  * = off; every distance measured slower than none on B200).  A hint only:
  * results do not depend on it. */
 mk_status mk_state_set_prefetch(mk_state* state, int tasks_ahead);
 
-/* Test hook for failure detection: adds `offset` to the target of every
+/* Passage: none of its own.
+ * Test hook for failure detection: adds `offset` to the target of every
  * device-side event wait of later steps (0 = normal).  With offset 1 no wait
  * can be satisfied, so the step ends with MK_ERR_TIMEOUT after the state's
  * timeout, without faulting or hanging the device. */
 mk_status mk_state_debug_wait_offset(mk_state* state, uint32_t offset);
 
-/* One decode step for `batch` sequences (1 <= batch <= max_batch).
+/* Passage: Cohere page, section "Egyetlen tartós kernelre épül a
+ * kiszolgálás": one persistent kernel runs a whole forward pass, exactly one
+ * threadblock per SM resident for the decode step; section "Folyamatos
+ * batchkezelés, paged attention ...": continuous batching over a paged KV
+ * cache with ragged sequences.
+ * One decode step for `batch` sequences (1 <= batch <= max_batch).
  *   token_ids  device int32 [batch]: the token fed to each sequence
  *   positions  device int32 [batch]: its position = tokens already cached
  *              (0 <= positions[b] < max_ctx); the step writes K/V at that
@@ -242,7 +276,10 @@ mk_status mk_state_debug_wait_offset(mk_state* state, uint32_t offset);
 mk_status mk_decode_step(mk_state* state, const int32_t* token_ids, const int32_t* positions,
                          int batch, const mk_paged_kv* kv, float* logits_out, mk_stream stream);
 
-/* Greedy generation without a host round trip per token: n_steps decode steps
+/* Passage: MPK digest, the benefits list (the launch and host overhead is
+ * paid once, not per operator); Cohere page, "Honnan jön a gyorsulás?", first
+ * reason (launch and synchronisation overhead paid once per step).
+ * Greedy generation without a host round trip per token: n_steps decode steps
  * for `batch` sequences, enqueued at once on `stream`.  Step k feeds each
  * sequence the token chosen at step k - 1 (step 0: first_tokens, device int32
  * [batch]) at position positions[b] + k (positions: device int32 [batch]), and
@@ -253,7 +290,11 @@ mk_status mk_generate(mk_state* state, const int32_t* first_tokens, const int32_
                       int n_steps, const mk_paged_kv* kv, int32_t* tokens_out, float* logits_out,
                       mk_stream stream);
 
-/* The same step as a kernel-per-operator baseline (the pages' comparison point:
+/* Passage: Cohere page, "Honnan jön a gyorsulás?", first reason: between two
+ * kernels every SM must finish before the next grid starts; HN thread
+ * "Compiling LLMs into a MegaKernel", post #51 (CUDA graphs cannot overlap
+ * across layers).
+ * The same step as a kernel-per-operator baseline (the pages' comparison point:
  * kernels with boundaries between operators, MPK digest "Part 1"): one launch per
  * maximal run of tasks of one (operator, layer) in the task list, in order on
  * `stream`, each running the same tiles without the events that let the
@@ -264,28 +305,35 @@ mk_status mk_decode_step_per_op(mk_state* state, const int32_t* token_ids, const
                                 int batch, const mk_paged_kv* kv, float* logits_out, mk_stream stream,
                                 int* n_launches);
 
-/* Same step with HOST inputs and outputs: copies token_ids and positions
+/* Passage: as mk_decode_step (the end-to-end form of the same step).
+ * Same step with HOST inputs and outputs: copies token_ids and positions
  * (host int32 [batch]) to the device, runs the step, copies the logits back
  * to logits_host (host fp32 [batch][vocab]) and waits for the stream. */
 mk_status mk_decode_step_host(mk_state* state, const int32_t* token_ids, const int32_t* positions,
                               int batch, const mk_paged_kv* kv, float* logits_host,
                               mk_stream stream);
 
-/* Runs a prompt through the same graph for ONE sequence whose page-table row
- * is kv->page_table[0]: tokens (device int32 [n_tokens]) at positions
- * pos0 .. pos0+n_tokens-1.  Writes the logits of the last prompt token to
- * last_logits (device fp32 [vocab]).
+/* Passage: MPK digest, "MPK का मुख्य मूल्य" (the measured workload: a
+ * 39-token prompt, then generation); the prompt is one batched operator of the
+ * task graph ("Part 1. Compiler": operators become tile tasks).
+ * Runs the prompt of ONE sequence, the one whose page-table row is
+ * kv->page_table[seq_slot] (0 <= seq_slot < max_batch; 0 for batch-1 graphs),
+ * at positions 0 .. n_tokens-1: tokens is device int32 [n_tokens]; the logits
+ * of the last prompt token go to last_logits (device fp32 [vocab]).
  *  - batch-1 graph: one token per step; the LM head is skipped for all but the
  *    last token;
  *  - batched graph (max_batch > 1): up to max_batch prompt tokens per step, as
- *    the batch rows of the tensor-core tiles (row i at position pos0 + i), with
- *    causal attention over the cache: each row's K/V is appended before any row
- *    attends (MPK digest, Part 1: a prompt's tokens are one batched operator). */
-mk_status mk_prefill(mk_state* state, const int32_t* tokens, int n_tokens, int pos0,
+ *    the batch rows of the tensor-core tiles (row i at position i), with causal
+ *    attention over the cache: each row's K/V is appended before any row
+ *    attends.
+ * Errors: MK_ERR_INVALID_ARG for a null pointer, n_tokens < 1, n_tokens >
+ * max_ctx or seq_slot out of range (returned before any launch). */
+mk_status mk_prefill(mk_state* state, const int32_t* tokens, int n_tokens, int seq_slot,
                      const mk_paged_kv* kv, float* last_logits, mk_stream stream);
 
-/* mk_prefill for the sequence whose page-table row is kv->page_table[seq_slot]
- * (0 <= seq_slot < max_batch; batch-1 graphs: 0). */
+/* Passage: as mk_prefill.  mk_prefill continuing a sequence: the prompt goes
+ * to positions pos0 .. pos0+n_tokens-1 of the sequence whose page-table row is
+ * kv->page_table[seq_slot] (its positions 0..pos0-1 must already be cached). */
 mk_status mk_prefill_seq(mk_state* state, const int32_t* tokens, int n_tokens, int pos0, int seq_slot,
                          const mk_paged_kv* kv, float* last_logits, mk_stream stream);
 
@@ -313,7 +361,10 @@ mk_status mk_decode_step_noalloc(const mk_model_desc* desc, const void* const* w
                                  int max_ctx, const int32_t* token_ids, const int32_t* positions,
                                  int batch, const mk_paged_kv* kv, float* logits_out, mk_stream stream);
 
-/* Waits for the stream and returns the device status word of the last step
+/* Passage: none of its own (error reporting of the persistent kernel's bounded
+ * waits: Cohere page, "Egyetlen tartós kernelre épül a kiszolgálás", counters
+ * in global memory).
+ * Waits for the stream and returns the device status word of the last step
  * (MK_OK, MK_ERR_TIMEOUT, MK_ERR_INVALID_ARG, ...). */
 mk_status mk_sync(mk_state* state, mk_stream stream);
 
@@ -327,12 +378,15 @@ typedef struct {
     int32_t error_info[4];     /* where: task, event, value, detail */
 } mk_state_counters;
 
-/* Synchronises the stream, then copies the counters; events (host uint32
+/* Passage: MPK digest, "Part 2. Runtime", "Event-आधारित execution तरीका": each
+ * finished task increments its event counter up to the threshold.
+ * Synchronises the stream, then copies the counters; events (host uint32
  * [n_events]) may be NULL. */
 mk_status mk_state_read_counters(mk_state* state, mk_stream stream, mk_state_counters* c,
                                  uint32_t* events, int cap);
 
-/* Copies an activation buffer of the last step to host fp32 memory.
+/* Passage: none of its own (inspection of the step's intermediate results).
+ * Copies an activation buffer of the last step to host fp32 memory.
  *   which 0: residual stream after attention [batch][hidden] of `layer`
  *         1: residual stream after the FFN   [batch][hidden] of `layer`
  *            (dense models; an MoE layer keeps its FFN output per expert slot)
@@ -342,20 +396,24 @@ mk_status mk_state_read_counters(mk_state* state, mk_stream stream, mk_state_cou
 mk_status mk_state_read_buffer(mk_state* state, int which, int layer, float* host, size_t n,
                                mk_stream stream);
 
-/* Per-task trace of the last step (needs MK_FLAG_TRACE): host uint64
+/* Passage: none of its own; it measures what the Cohere page's "Honnan jön a
+ * gyorsulás?" describes (idle SMs between dependent tiles).
+ * Per-task trace of the last step (needs MK_FLAG_TRACE): host uint64
  * [n_tasks][4] = {wait start ns, compute start ns, end ns, sm id}. */
 mk_status mk_state_read_trace(mk_state* state, uint64_t* host, int cap_tasks, mk_stream stream);
 
-/* Per-CTA cycle counters accumulated since the last read (needs
+/* Passage: none of its own (as mk_state_read_trace).
+ * Per-CTA cycle counters accumulated since the last read (needs
  * MK_FLAG_TRACE), then cleared: host uint64 [n_sm][8] = {producer waits for a
  * free ring slot, consumer waits for streamed data, dependency waits, kernel
  * cycles, -, signal-slot waits, -, -}. */
 mk_status mk_state_read_stats(mk_state* state, uint64_t* host, int cap, mk_stream stream);
 
-/* Text of the last error of the calling thread ("" if none). */
+/* Passage: none of its own.  Text of the last error of the calling thread
+ * ("" if none); the pointer stays valid until that thread's next call. */
 const char* mk_last_error_string(void);
 
-/* Library version string. */
+/* Passage: none of its own.  Library version string (static storage). */
 const char* mk_version(void);
 
 #ifdef __cplusplus

@@ -256,9 +256,9 @@ def mk_decode_step_host(state: int, token_ids: int, positions: int, batch: int, 
                                      logits_host, stream))
 
 
-def mk_prefill(state: int, tokens: int, n_tokens: int, pos0: int, kv: mk_paged_kv,
+def mk_prefill(state: int, tokens: int, n_tokens: int, seq_slot: int, kv: mk_paged_kv,
                last_logits: int, stream: int = 0) -> None:
-    _check(lib().mk_prefill(state, tokens, n_tokens, pos0, ctypes.byref(kv), last_logits, stream))
+    _check(lib().mk_prefill(state, tokens, n_tokens, seq_slot, ctypes.byref(kv), last_logits, stream))
 
 
 def mk_decode_step_per_op(state: int, token_ids: int, positions: int, batch: int, kv: mk_paged_kv,

@@ -847,9 +847,9 @@ mk_status mk_prefill_seq(mk_state* s, const int32_t* tokens, int n_tokens, int p
     return MK_OK;
 }
 
-mk_status mk_prefill(mk_state* s, const int32_t* tokens, int n_tokens, int pos0, const mk_paged_kv* kv,
+mk_status mk_prefill(mk_state* s, const int32_t* tokens, int n_tokens, int seq_slot, const mk_paged_kv* kv,
                      float* last_logits, mk_stream stream) {
-    return mk_prefill_seq(s, tokens, n_tokens, pos0, 0, kv, last_logits, stream);
+    return mk_prefill_seq(s, tokens, n_tokens, 0, seq_slot, kv, last_logits, stream);
 }
 
 mk_status mk_sync(mk_state* s, mk_stream stream) {

@@ -11,7 +11,8 @@ import torch
 
 from . import (MK_OK, MkError, make_desc, make_kv, mk_build_taskgraph, mk_decode_step,
                mk_decode_step_host, mk_graph_destroy, mk_graph_get_info, mk_last_error_string,
-               mk_load_model, mk_model_destroy, mk_prefill, mk_state_create, mk_state_destroy,
+               mk_load_model, mk_model_destroy, mk_prefill, mk_prefill_seq, mk_state_create,
+               mk_state_destroy,
                mk_sync)
 
 PAGE = 16
@@ -73,12 +74,15 @@ class Decoder:
                             self.kv, ptr(logits_host), self.stream())
 
     def prefill(self, tokens: torch.Tensor, pos0: int = 0, seq: int = 0) -> torch.Tensor:
-        """Prompt of one sequence (row `seq` of the page table); returns last logits [vocab]."""
-        kv = make_kv(self.k_pages.data_ptr(), self.v_pages.data_ptr(),
-                     self.page_table[seq].data_ptr(), self.n_pages, self.max_pages)
+        """Prompt of sequence `seq` (a page-table row) at positions pos0 .. pos0 + n - 1;
+        returns the last token's logits [vocab]."""
         out = self.logits[seq]
-        mk_prefill(self.state, tokens.data_ptr(), tokens.numel(), pos0, kv, out.data_ptr(),
-                   self.stream())
+        if pos0 == 0:
+            mk_prefill(self.state, tokens.data_ptr(), tokens.numel(), seq, self.kv, out.data_ptr(),
+                       self.stream())
+        else:
+            mk_prefill_seq(self.state, tokens.data_ptr(), tokens.numel(), pos0, seq, self.kv,
+                           out.data_ptr(), self.stream())
         return out
 
     def sync(self) -> int:

@@ -60,3 +60,36 @@ def test_noalloc_rejects_too_large_and_bad_arguments():
     assert e.value.status == mk.MK_ERR_UNSUPPORTED
     with pytest.raises(mk.MkError):                # batch > 1
         mk.mk_decode_step_noalloc(desc, ptrs, 64, t.data_ptr(), t.data_ptr(), 2, kv, out.data_ptr())
+
+
+def _noalloc_vs_regular(cfg, seed, max_ctx, tokens):
+    """Runs `tokens` at positions 0.. through both paths (separate KV caches) and
+    compares the logits step by step."""
+    specs, ts = device_weights(cfg, seed)
+    dec = make_decoder(cfg, ts, 1, max_ctx)
+    k2, v2 = torch.zeros_like(dec.k_pages), torch.zeros_like(dec.v_pages)
+    kv2 = mk.make_kv(k2.data_ptr(), v2.data_ptr(), dec.page_table.data_ptr(), dec.n_pages, dec.max_pages)
+    desc = mk.make_desc(**desc_kwargs(cfg))
+    ptrs = [t.data_ptr() for t in ts]
+    out = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    for p, tok in enumerate(tokens):
+        t = torch.tensor([tok], dtype=torch.int32, device="cuda")
+        pos = torch.tensor([p], dtype=torch.int32, device="cuda")
+        ref = dec.step(t, pos).clone()
+        dec.check()
+        mk.mk_decode_step_noalloc(desc, ptrs, max_ctx, t.data_ptr(), pos.data_ptr(), 1, kv2,
+                                  out.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        d, cos, ok = compare_logits(out.cpu().numpy(), ref.cpu().numpy()[0])
+        assert ok, (cfg.name, max_ctx, p, d, cos)
+    np.testing.assert_array_equal(k2.view(torch.int16).cpu().numpy(), dec.k_pages.view(torch.int16).cpu().numpy())
+    dec.close()
+
+
+def test_noalloc_replans_for_another_context_and_a_moe_model():
+    """The array keeps the last plan: a new context length, a routed-expert model
+    (its router, selection and expert buffers live in the array too), and the
+    first model again must each be planned afresh and match the regular path."""
+    _noalloc_vs_regular(syn.TINY, syn.SEED_WEIGHTS + 1, 64, [17, 401, 5])
+    _noalloc_vs_regular(syn.TINY, syn.SEED_WEIGHTS + 1, 200, [9, 33])
+    _noalloc_vs_regular(syn.TINY_MOE, syn.SEED_WEIGHTS + 4, 64, [3, 700, 12])
+    _noalloc_vs_regular(syn.TINY, syn.SEED_WEIGHTS + 2, 64, [1, 2])
