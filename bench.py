@@ -546,8 +546,9 @@ def run_per_op(args, W):
 
 def run_generate(args, W):
     """Greedy generation (the loop after the hot path): 128 new tokens of the 8B
-    model after its 39-token prompt, with mk_generate (each step's argmax chosen on
-    the device, all steps enqueued at once) beside a host loop that copies each
+    model after its 39-token prompt, with mk_generate (each step's argmax taken
+    inside the step by its last LM-head tiles, one launch per token, all enqueued
+    at once) beside a host loop that copies each
     step's logits to the host, takes the argmax there and sends the token back.
     Prints one JSON line; not a decode line."""
     import numpy as np

@@ -53,7 +53,9 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
         if m:
             cur = m.group(1)
         m = re.search(r"Used (\d+) registers", line)
-        if m and cur and "megakernel" in cur and int(m.group(1)) < MIN_LAUNCH_REGS:
+        # (megakernel<HPG, DPL, MM> splits unless MM and DPL == 2: mangled "...Li2ELb1E...")
+        splits = cur is not None and "megakernel" in cur and "ELi2ELb1E" not in cur
+        if m and splits and int(m.group(1)) < MIN_LAUNCH_REGS:
             os.remove(LIB)
             raise RuntimeError(f"{cur} launches with {m.group(1)} registers per thread; the "
                                f"warpgroup register split needs at least {MIN_LAUNCH_REGS}")

@@ -36,13 +36,6 @@ struct mk_graph {
     std::vector<std::pair<int, int>> phases;   // (first task, task count) of each (operator, layer) run
 };
 
-// Greedy generation: per-slice (value, index) pairs of the two-stage argmax.
-constexpr int kArgmaxBlocks = 64;
-struct ArgPair {
-    float v;
-    int i;
-};
-
 struct mk_state {
     mk_graph* g = nullptr;
     uint32_t epoch = 0;
@@ -64,7 +57,9 @@ struct mk_state {
     float* mm_part = nullptr;
     uint32_t* mm_cnt = nullptr;
     void* tmaps = nullptr;         // device copy of the tensor maps (operands, then weights)
-    ArgPair* argmax_part = nullptr;   // greedy generation: per-slice (value, index) pairs
+    mk::ArgVal* lm_arg = nullptr;  // greedy generation: LM-head tiles' (max, index) parts
+    mk::ArgVal* lm_garg = nullptr; // ... and the groups' results
+    uint32_t* lm_cnt = nullptr;    // arrivals per group, then of the groups
     int32_t* tokpos = nullptr;     // host-input variant: [2][max_batch]
     float* logits = nullptr;       // host-output variant: [max_batch][vocab]
     unsigned long long* trace = nullptr;
@@ -238,6 +233,11 @@ mk::Params base_params(mk_state* s) {
     for (int i = 0; i < mk::kNumOperands; ++i) p.opnd[i] = s->opnd[i];
     p.mm_part = s->mm_part;
     p.mm_cnt = s->mm_cnt;
+    p.argmax_out = nullptr;
+    p.n_lm_tiles = P.n_lm_tiles;
+    p.lm_arg = s->lm_arg;
+    p.lm_garg = s->lm_garg;
+    p.lm_cnt = s->lm_cnt;
     return p;
 }
 
@@ -572,7 +572,12 @@ mk_status mk_state_create(mk_graph* g, mk_state** out) {
             }
         }
     }
-    ALLOC(argmax_part, B * kArgmaxBlocks);
+    {
+        const size_t groups = (size_t)(P.n_lm_tiles + mk::kArgGroup - 1) / mk::kArgGroup;
+        ALLOC(lm_arg, (size_t)P.n_lm_tiles * mk::kArgParts * B);
+        ALLOC(lm_garg, groups * B);
+        ALLOC(lm_cnt, groups + 1);
+    }
     ALLOC(tokpos, 2 * B);
     ALLOC(logits, B * (size_t)d.vocab);
     if (d.flags & MK_FLAG_TRACE) ALLOC(trace, P.tasks.size() * 4);
@@ -681,61 +686,6 @@ mk_status mk_decode_step_per_op(mk_state* s, const int32_t* token_ids, const int
     return MK_OK;
 }
 
-// Greedy choice of each sequence's next token from its logits row: the largest
-// logit, ties to the lowest index.  Two kernels: kArgmaxBlocks blocks per
-// sequence each reduce a contiguous slice to one (value, index) pair, then one
-// block per sequence reduces the pairs.
-__device__ __forceinline__ void arg_better(float& v, int& i, float v2, int i2) {
-    if (v2 > v || (v2 == v && i2 < i)) { v = v2; i = i2; }
-}
-__device__ __forceinline__ void block_arg_reduce(float& v, int& i) {
-    __shared__ float sv[256];
-    __shared__ int si[256];
-    const int tid = threadIdx.x;
-    sv[tid] = v;
-    si[tid] = i;
-    __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-        if (tid < w) {
-            float a = sv[tid];
-            int ai = si[tid];
-            arg_better(a, ai, sv[tid + w], si[tid + w]);
-            sv[tid] = a;
-            si[tid] = ai;
-        }
-        __syncthreads();
-    }
-    v = sv[0];
-    i = si[0];
-}
-__global__ void __launch_bounds__(256) argmax_slices_kernel(const float* __restrict__ logits, int vocab,
-                                                            ArgPair* __restrict__ part) {
-    const int b = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x;
-    const int per = (vocab + kArgmaxBlocks - 1) / kArgmaxBlocks;
-    const int lo = blk * per, hi = min(vocab, lo + per);
-    const float* row = logits + (size_t)b * vocab;
-    float best = -INFINITY;
-    int arg = 0x7FFFFFFF;
-    for (int i = lo + tid; i < hi; i += blockDim.x) {
-        const float v = __ldcg(row + i);
-        if (v > best) { best = v; arg = i; }   // i increases: the first of equal values stays
-    }
-    block_arg_reduce(best, arg);
-    if (tid == 0) part[b * kArgmaxBlocks + blk] = ArgPair{best, arg};
-}
-__global__ void __launch_bounds__(256) argmax_final_kernel(const ArgPair* __restrict__ part,
-                                                           int32_t* __restrict__ out) {
-    const int b = blockIdx.x, tid = threadIdx.x;
-    float best = -INFINITY;
-    int arg = 0x7FFFFFFF;
-    if (tid < kArgmaxBlocks) {
-        best = part[b * kArgmaxBlocks + tid].v;
-        arg = part[b * kArgmaxBlocks + tid].i;
-    }
-    block_arg_reduce(best, arg);
-    if (tid == 0) out[b] = (arg == 0x7FFFFFFF) ? 0 : arg;
-}
-
 mk_status mk_generate(mk_state* s, const int32_t* first_tokens, const int32_t* positions, int batch, int n_steps,
                       const mk_paged_kv* kv, int32_t* tokens_out, float* logits_out, mk_stream stream) {
     if (!s || !first_tokens || !positions || !tokens_out || !logits_out)
@@ -745,8 +695,13 @@ mk_status mk_generate(mk_state* s, const int32_t* first_tokens, const int32_t* p
     mk_status r = check_kv(s, kv);
     if (r != MK_OK) return r;
     cudaStream_t st = (cudaStream_t)stream;
-    const int V = s->g->plan.desc.vocab;
+    // the argmax arrivals count from zero for this call
+    const size_t groups = (size_t)(s->g->plan.n_lm_tiles + mk::kArgGroup - 1) / mk::kArgGroup;
+    cudaError_t e = cudaMemsetAsync(s->lm_cnt, 0, sizeof(uint32_t) * (groups + 1), st);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_generate: clearing the argmax counters");
     for (int k = 0; k < n_steps; ++k) {
+        // one launch per token: the step's last LM-head tile writes the argmax to
+        // tokens_out[k], which the next launch reads as its tokens
         mk::Params p = base_params(s);
         p.tokens = (k == 0) ? first_tokens : tokens_out + (size_t)(k - 1) * batch;   // the previous choice
         p.positions = positions;
@@ -759,12 +714,10 @@ mk_status mk_generate(mk_state* s, const int32_t* first_tokens, const int32_t* p
         p.n_pages = kv->n_pages;
         p.max_pages = kv->max_pages_per_seq;
         p.logits = logits_out;
+        p.argmax_out = tokens_out + (size_t)k * batch;
+        p.arg_epoch = (uint32_t)(k + 1);
         r = launch_step(s, p, st);
         if (r != MK_OK) return r;
-        argmax_slices_kernel<<<dim3(kArgmaxBlocks, batch), 256, 0, st>>>(logits_out, V, s->argmax_part);
-        argmax_final_kernel<<<batch, 256, 0, st>>>(s->argmax_part, tokens_out + (size_t)k * batch);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "mk_generate: argmax launch");
     }
     return MK_OK;
 }

@@ -451,6 +451,24 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
         }
     }
     g.n_events = (int)thr.size();
+    // LM-head tiles are numbered for the in-step argmax's partial results: a GEMV
+    // tile in aux, every split of a tensor-core tile in b
+    {
+        int n = 0;
+        for (Task& t : T) {
+            if (t.op == MK_OP_LMHEAD) t.aux = (uint16_t)n++;
+        }
+        // batched LM-head tiles: every split of a tile carries the tile's ordinal in b
+        int nt = 0;
+        uint32_t last_r0 = 0xFFFFFFFFu;
+        for (Task& t : T) {
+            if (t.op != MK_OP_MM_LMHEAD) continue;
+            if (t.r0 != last_r0) { last_r0 = t.r0; ++nt; }
+            t.b = (uint16_t)(nt - 1);
+        }
+        g.n_lm_tiles = std::max(n, nt);
+        if (g.n_lm_tiles > 65535) return fail("too many LM-head tiles");
+    }
 
     // ---- GEMV fast-path variant per task (the device dispatches on it without any
     //      geometry arithmetic)

@@ -24,6 +24,7 @@ struct GraphPlan {
     int bp = 0;                  // padded batch (the MMA's N); 0 for batch-1 graphs
     int mm_slots = 0;            // split partial-sum slots per layer (each bp x 128 floats)
     int mm_counters = 0;         // per-tile split arrival counters
+    int n_lm_tiles = 0;          // LM-head tiles (numbered by their aux)
 };
 
 int64_t ceil_div(int64_t a, int64_t b);

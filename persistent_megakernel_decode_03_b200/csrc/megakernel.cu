@@ -208,6 +208,20 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
 }
 
 
+// (value, index) of a running maximum: a larger value wins, equal values go to the
+// lower index (the greedy rule: ties to the lowest token id).
+__device__ __forceinline__ void arg_better(float& v, int& i, float v2, int i2) {
+    if (v2 > v || (v2 == v && i2 < i)) { v = v2; i = i2; }
+}
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        const int i2 = __shfl_xor_sync(0xFFFFFFFFu, i, o);
+        arg_better(v, i, v2, i2);
+    }
+}
+
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -2018,6 +2032,66 @@ __device__ void router_finalize(const Params& p, Smem& sm, int l) {
     }
 }
 
+// A batch-1 LM-head tile's part of the in-step argmax: the (max, index) of the
+// logits rows it has just stored (this warp's own stores, read back).  One warp.
+__device__ __forceinline__ void lmhead_arg_part(const Params& p, const Task& t, int lane) {
+    __syncwarp();
+    float v = -INFINITY;
+    int i = 0x7FFFFFFF;
+    for (int r = (int)t.r0 + lane; r < (int)t.r1; r += 32) arg_better(v, i, p.logits[r], r);
+    warp_argmax(v, i);
+    if (lane == 0) p.lm_arg[(size_t)t.aux * kArgParts * p.max_batch] = ArgVal{v, i};
+}
+
+// Greedy argmax inside the step (mk_generate).  An LM-head tile has stored the
+// (value, index) of its rows' maximum for every batch row (nparts parts per
+// tile); it arrives on its group of kArgGroup tiles, the group's last tile
+// reduces the group, and the last group writes each batch row's token to
+// argmax_out.  Ties go to the lower index at every level, so the result is the
+// first index of the largest logit whatever the arrival order.  One warp.
+__device__ __forceinline__ void argmax_arrive(const Params& p, int tile, int nparts, int lane) {
+    const int ng = (p.n_lm_tiles + kArgGroup - 1) / kArgGroup;
+    const int g = tile / kArgGroup, t0 = g * kArgGroup, t1 = min(p.n_lm_tiles, t0 + kArgGroup);
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        const uint32_t old = atom_add_acq_rel(p.lm_cnt + g, 1u);
+        last = (old == (uint32_t)(t1 - t0) * p.arg_epoch - 1u) ? 1 : 0;
+    }
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+    if (!last) return;
+    __syncwarp();
+    for (int b = 0; b < p.batch; ++b) {
+        float v = -INFINITY;
+        int i = 0x7FFFFFFF;
+        for (int k = lane; k < (t1 - t0) * nparts; k += 32) {
+            const float2 a = __ldcg(reinterpret_cast<const float2*>(
+                p.lm_arg + ((size_t)(t0 + k / nparts) * kArgParts + k % nparts) * p.max_batch + b));
+            arg_better(v, i, a.x, __float_as_int(a.y));
+        }
+        warp_argmax(v, i);
+        if (lane == 0) p.lm_garg[(size_t)g * p.max_batch + b] = ArgVal{v, i};
+    }
+    __syncwarp();
+    if (lane == 0) {
+        const uint32_t old = atom_add_acq_rel(p.lm_cnt + ng, 1u);
+        last = (old == (uint32_t)ng * p.arg_epoch - 1u) ? 1 : 0;
+    }
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+    if (!last) return;
+    __syncwarp();
+    for (int b = 0; b < p.batch; ++b) {
+        float v = -INFINITY;
+        int i = 0x7FFFFFFF;
+        for (int k = lane; k < ng; k += 32) {
+            const float2 a = __ldcg(reinterpret_cast<const float2*>(p.lm_garg + (size_t)k * p.max_batch + b));
+            arg_better(v, i, a.x, __float_as_int(a.y));
+        }
+        warp_argmax(v, i);
+        if (lane == 0) p.argmax_out[b] = (i == 0x7FFFFFFF) ? 0 : i;
+    }
+}
+
 // ----------------------------------------------------------------------------- consumer loop
 
 // ----------------------------------------------------------------------------- batched tiles
@@ -2166,6 +2240,39 @@ __device__ __noinline__ void mm_epilogue(const Params& p, const Task& t, int tid
                 split_hilo(a, hi, lo);
                 p.opnd[kOpAct][(base + b) * p.F + f] = hi;
                 p.opnd[kOpAct][(base + p.bp + b) * p.F + f] = lo;
+            }
+        }
+        return;
+    }
+    if (t.op == MK_OP_MM_LMHEAD) {
+        // logits, and with the in-step argmax each warp's (max, index) per batch row
+        // (every lane takes part in the shuffles: rows past the tile count as -inf)
+        const int i = tid, w = tid >> 5, lane = tid & 31;
+        const bool row_ok = i < nrows;
+        const int r = (int)t.r0 + i;
+        for (int b0 = 0; b0 < batch; b0 += kEpiRows) {
+            float v[kEpiRows];
+#pragma unroll
+            for (int k = 0; k < kEpiRows; ++k) v[k] = 0.0f;
+            if (row_ok)
+                for (int sp = 0; sp < Sk; ++sp) {
+                    const float* ps = part0 + sp * sstride;
+#pragma unroll
+                    for (int k = 0; k < kEpiRows; ++k)
+                        if (b0 + k < batch) v[k] += __ldcg(ps + (size_t)(b0 + k) * kMmRows + i);
+                }
+#pragma unroll
+            for (int k = 0; k < kEpiRows; ++k) {
+                const int b = b0 + k;
+                if (b >= batch) break;
+                if (row_ok) p.logits[(size_t)b * p.V + r] = v[k];
+                if (p.argmax_out) {
+                    float bv = row_ok ? v[k] : -INFINITY;
+                    int bi = row_ok ? r : 0x7FFFFFFF;
+                    warp_argmax(bv, bi);
+                    if (lane == 0)
+                        p.lm_arg[((size_t)t.b * kArgParts + w) * p.max_batch + b] = ArgVal{bv, bi};
+                }
             }
         }
         return;
@@ -2321,6 +2428,10 @@ __device__ __noinline__ bool mm_task(const Params& p, Smem& sm, const Task& t, i
         mm_epilogue(p, t, etid);
         fence_proxy_async_global();
         __threadfence();
+        if (t.op == MK_OP_MM_LMHEAD && p.argmax_out) {
+            if (!msync4(p, sm, mph)) return false;       // the four warps' parts are stored
+            if (etid < 32) argmax_arrive(p, t.b, kArgParts, lane);
+        }
     }
     if (etid == 0) sm.ep_task[buf].sig = last ? t.sig : MK_NO_EVENT;
     return true;
@@ -2523,6 +2634,13 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
 
 // ----------------------------------------------------------------------------- epilogue warp
 
+// The in-step argmax of a batch-1 LM-head tile, run by the epilogue warp after it
+// stored the tile's logits (out of line: it keeps the epilogue loop's registers).
+__device__ __noinline__ void lmhead_argmax(const Params& p, const Task& t, int lane) {
+    lmhead_arg_part(p, t, lane);
+    argmax_arrive(p, t.aux, 1, lane);
+}
+
 // Output rows of a finished GEMV task: the consumer warps' partial sums reduced in
 // a fixed order (bit-identical from run to run), then the operator's tail.
 __device__ __forceinline__ void gemv_store(const Params& p, const Smem& sm, const Task& t, const GemvGeom& g,
@@ -2607,6 +2725,7 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
                 const int wpg = is_warp_row(t.flags) ? 1
                                 : (t.flags != kFastNone) ? kConsumerWarps : thread_map(g.K).wpg;
                 gemv_store(p, sm, t, g, wpg, buf, lane);
+                if (t.op == MK_OP_LMHEAD && p.argmax_out) lmhead_argmax(p, t, lane);
                 if (t.op == MK_OP_ROUTER) {
                     // arrival of this router tile (acquire-release: the warp barrier orders
                     // the lanes' logit stores before it); the layer's last tile selects the
@@ -2649,6 +2768,12 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
 
 // ----------------------------------------------------------------------------- kernel
 
+// Instantiations that re-split their registers between the warpgroups: the batch-1
+// kernels (GEMV tiles keep the input slice and row sums in registers) and the
+// batched kernels with 128-wide heads (attention staging); the batched kernels with
+// 64-wide heads need fewer than the launch allows, and ptxas launches them with less.
+__host__ __device__ constexpr bool splits_registers(bool mm, int dpl) { return !mm || dpl == 4; }
+
 template <int HPG, int DPL, bool MM>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -2682,15 +2807,18 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     __syncthreads();
     // Hand registers from the support warpgroup to the two consumer warpgroups.
     // The two branches never meet again (each returns), so the register limit of
-    // one never constrains the code of the other.
+    // one never constrains the code of the other.  The split is only valid when the
+    // kernel launches with at least kMinLaunchRegs registers per thread (the build
+    // and the launch both check that); instantiations whose code needs fewer keep
+    // the launch's even split (splits_registers).
     if (warp < kConsumerWarps) {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
+        if constexpr (splits_registers(MM, DPL)) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
         const long long k0 = clock64();
         consumer_loop<HPG, DPL, MM>(p, sm);
         if (threadIdx.x == 0) stat_add(p, 3, (unsigned long long)(clock64() - k0));
         return;
     }
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSupportRegs));
+    if constexpr (splits_registers(MM, DPL)) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSupportRegs));
     if (warp == kProducerWarp) {
         if (lane == 0) producer_loop<MM>(p, sm);
     } else if (warp == kEpilogueWarp) {
@@ -2715,6 +2843,12 @@ static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream, bool
     if (!bit || !(attr_set[p.mm ? 1 : 0] & bit)) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
         if (e != cudaSuccess) return e;
+        // a register split (setmaxnreg) needs the launch's registers: with fewer, the
+        // consumers' increase would wait forever, so such a build is never launched
+        cudaFuncAttributes fa{};
+        e = cudaFuncGetAttributes(&fa, (const void*)kern);
+        if (e != cudaSuccess) return e;
+        if (splits_registers(p.mm != 0, DPL) && fa.numRegs < kMinLaunchRegs) return cudaErrorInvalidConfiguration;
         attr_set[p.mm ? 1 : 0] |= bit;
     }
     void* args[] = {const_cast<Params*>(&p)};

@@ -137,6 +137,12 @@ struct Task {
 };
 static_assert(sizeof(Task) == 64, "task record is 64 bytes");
 
+// (value, index) of a partial maximum (the in-step argmax), 8 bytes.
+struct alignas(8) ArgVal {
+    float v;
+    int i;
+};
+
 // Per-layer weight pointers (bf16 bits).
 struct LayerW {
     const uint16_t* attn_norm;
@@ -213,7 +219,21 @@ struct Params {
     uint16_t* opnd[kNumOperands];   // bf16 [rows][K]: per layer 2 * bp rows (hi, then lo)
     float* mm_part;              // split partial sums: [slot][bp][128]
     uint32_t* mm_cnt;            // per-tile split arrivals
+
+    // greedy argmax inside the step (mk_generate): each LM-head tile leaves the
+    // (value, index) of its rows' maximum per batch row, groups of kArgGroup tiles
+    // are reduced by their last tile, and the last group writes the token
+    int* argmax_out;             // device int32 [batch], or null: no argmax this step
+    uint32_t arg_epoch;          // 1-based count of argmax steps since the counters were cleared
+    int n_lm_tiles;              // LM-head tiles (their aux is the tile's ordinal)
+    ArgVal* lm_arg;              // [n_lm_tiles * kArgParts][max_batch]
+    ArgVal* lm_garg;             // [groups][max_batch]
+    uint32_t* lm_cnt;            // [groups + 1] arrivals: per group, then of the groups
 };
+// Parts per LM-head tile (a batched tile reduces its 128 rows in 4 warps) and tiles
+// per reduction group of the in-step argmax.
+constexpr int kArgParts = 4;
+constexpr int kArgGroup = 32;
 
 // Sets the text returned by mk_last_error_string() for the calling thread.
 void set_last_error(const char* msg);

@@ -83,3 +83,31 @@ def test_batched_greedy_generation_on_device():
     for b in range(B):
         assert got[:, b].tolist() == want[b], b
     dec.close()
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_in_step_argmax_over_a_large_vocabulary(B):
+    """8B shapes (2 layers, 128256-token vocabulary: thousands of LM-head tiles, many
+    argmax groups): after each enqueued step the token written on the device is the
+    first index of the largest logit of that step (torch's argmax picks the first
+    maximum too), for every sequence."""
+    import dataclasses
+    cfg = dataclasses.replace(syn.LLAMA8B, n_layers=2)
+    specs, ts = device_weights(cfg, syn.SEED_WEIGHTS + 71)
+    dec = make_decoder(cfg, ts, B, 64)
+    firsts = torch.tensor([int(t) for t in syn.host_tokens(B, 71, cfg.vocab)], dtype=torch.int32, device="cuda")
+    pos = torch.tensor([3 * b for b in range(B)], dtype=torch.int32, device="cuda")
+    n = 3
+    out = torch.full((n, B), -1, dtype=torch.int32, device="cuda")
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    for k in range(n):
+        # one step at a time, so each step's logits can be checked
+        first_k = firsts if k == 0 else out[k - 1].clone()
+        pos_k = pos + k                                  # (held until the step has run)
+        mk.mk_generate(dec.state, first_k.data_ptr(), pos_k.data_ptr(), B, 1, dec.kv,
+                       out[k].data_ptr(), logits.data_ptr(), dec.stream())
+        torch.cuda.synchronize()
+        dec.check()
+        assert out[k].cpu().tolist() == torch.argmax(logits[:B], dim=1).int().cpu().tolist(), k
+    check_counters(dec)
+    dec.close()
