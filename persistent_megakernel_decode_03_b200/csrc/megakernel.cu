@@ -1044,10 +1044,16 @@ __device__ void attn_merge_group(const Params& p, Smem& sm, uint32_t& cph, int l
     const int hd = p.hd, hpg = hpg_of(p), tid = threadIdx.x;
     int pos = position_of(p, b);
     if (pos < 0 || pos >= p.max_ctx) pos = 0;
-    const int sa = attn_active_splits(pos + 1, p.S);      // (S + 1) * hpg floats fit the scratch
-    float* f = sm.attn;                                     // [sa][hpg] weights, then [hpg] 1/L
+    const int sa = attn_active_splits(pos + 1, p.S);      // (2 S + 1) * hpg floats fit the scratch
+    float* f = sm.attn;                                     // [sa][hpg] weights, then [hpg] 1/L, then [sa][hpg] l
+    float* fl = f + (sa + 1) * hpg;
     const size_t i0 = attn_part_index(p, l, b, g, 0, 0);   // split s, head h at i0 + s*hpg + h
-    for (int k = tid; k < sa * hpg; k += kConsumerThreads) f[k] = __ldcg(attn_part_ml(p, i0 + k));
+    // every split's (m, l) in one parallel pass: the loop below reads only shared memory
+    for (int k = tid; k < sa * hpg; k += kConsumerThreads) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(attn_part_ml(p, i0 + k)));
+        f[k] = ml.x;
+        fl[k] = ml.y;
+    }
     csync(p, sm, cph);
     if (tid < hpg) {
         float M = -INFINITY;
@@ -1056,7 +1062,7 @@ __device__ void attn_merge_group(const Params& p, Smem& sm, uint32_t& cph, int l
         for (int sp = 0; sp < sa; ++sp) {
             const float mm = f[sp * hpg + tid];
             const float w = (mm == -INFINITY) ? 0.0f : exp2f(mm - M);
-            L = fmaf(__ldcg(attn_part_ml(p, i0 + (size_t)sp * hpg + tid) + 1), w, L);
+            L = fmaf(fl[sp * hpg + tid], w, L);
             f[sp * hpg + tid] = w;
         }
         f[sa * hpg + tid] = (L > 0.0f) ? 1.0f / L : 0.0f;
