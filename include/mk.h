@@ -186,8 +186,11 @@ enum {
     MK_OP_MM_GATEUP = 13, /* FFN rows [r0, r1) (<= 64): silu(Wg h) * (Wu h) */
     MK_OP_MM_DOWN = 14,   /* rows of Wd . a plus the residual */
     MK_OP_MM_LMHEAD = 15, /* rows of Wlm . rmsnorm(x) */
-    MK_OP_KVAPPEND = 16   /* batched graphs: K (rotated) and V of batch rows [r0, r1) into
+    MK_OP_KVAPPEND = 16,  /* batched graphs: K (rotated) and V of batch rows [r0, r1) into
                              their pages; the attention tasks of the layer wait for them */
+    MK_OP_ATTN_MERGE = 17 /* long-context batch-1 graphs: q heads [r0, r1) of sequence b, the
+                             splits' softmax partials merged (their attention tasks cover every
+                             KV head of a page, exported with aux = -1) */
 };
 
 #define MK_NO_EVENT 0xFFFFFFFFu

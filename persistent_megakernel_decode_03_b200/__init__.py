@@ -35,9 +35,10 @@ MK_OP_NORM, MK_OP_MM_QKV, MK_OP_MM_OPROJ, MK_OP_MM_GATEUP, MK_OP_MM_DOWN, MK_OP_
     10, 11, 12, 13, 14, 15)
 MM_OPS = (MK_OP_MM_QKV, MK_OP_MM_OPROJ, MK_OP_MM_GATEUP, MK_OP_MM_DOWN, MK_OP_MM_LMHEAD)
 MK_OP_KVAPPEND = 16
+MK_OP_ATTN_MERGE = 17
 OP_NAMES = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
             8: "exp_gateup", 9: "exp_down", 10: "norm", 11: "mm_qkv", 12: "mm_oproj", 13: "mm_gateup",
-            14: "mm_down", 15: "mm_lmhead", 16: "kvappend"}
+            14: "mm_down", 15: "mm_lmhead", 16: "kvappend", 17: "attn_merge"}
 
 # Exported symbols (declared in include/mk.h).
 SYMBOLS = (

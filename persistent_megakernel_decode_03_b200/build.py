@@ -53,7 +53,7 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
         if m:
             cur = m.group(1)
         m = re.search(r"Used (\d+) registers", line)
-        # (megakernel<HPG, DPL, MM> splits unless MM and DPL == 2: mangled "...Li2ELb1E...")
+        # (megakernel<HPG, DPL, MM, WIDE> splits unless MM and DPL == 2: mangled "...ELi2ELb1E...")
         splits = cur is not None and "megakernel" in cur and "ELi2ELb1E" not in cur
         if m and splits and int(m.group(1)) < MIN_LAUNCH_REGS:
             os.remove(LIB)

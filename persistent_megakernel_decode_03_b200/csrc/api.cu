@@ -228,6 +228,7 @@ mk::Params base_params(mk_state* s) {
     p.seq_row = -1;
     p.pos_stride = 0;
     p.mm = P.bp > 0 ? 1 : 0;
+    p.wide = P.wide_attn ? 1 : 0;
     p.bp = P.bp;
     p.tmaps = s->tmaps;
     for (int i = 0; i < mk::kNumOperands; ++i) p.opnd[i] = s->opnd[i];
@@ -490,6 +491,7 @@ mk_status mk_graph_export_tasks(const mk_graph* g, mk_task_info* out, int cap, i
         out[i].wait[1] = T[i].wait1;
         out[i].signal = T[i].sig;
         out[i].pointer_wait = T[i].pad;
+        if (T[i].op == MK_OP_ATTN && (T[i].flags & mk::kAttnWide)) out[i].aux = -1;   // every KV head
         if (mk::is_mm_op(T[i].op)) {          // split s of a tile with nblk splits
             out[i].b = T[i].chunk_rows;
             out[i].aux = T[i].nblk;

@@ -28,6 +28,7 @@ namespace {
 
 // Tensor kinds for the region-overlap analysis.
 enum TensorKind { T_XIN = 1, T_QKV, T_O, T_XMID, T_ACT, T_ACTE, T_SEL, T_LOGITS,
+                  T_PART,                     // wide attention: the splits' softmax partials
                   T_XQOP, T_XFOP, T_XLOP,     // bf16 hi/lo operands of batched tiles
                   T_KV };                     // batched graphs: this step's K/V rows in the cache
 
@@ -146,7 +147,11 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     // make the splits unequal; the dynamic queue evens them out), with splits of at
     // least ~512 positions of a half-full context (shorter ones cost more in fixed
     // per-task work than they gain in balance).
-    int S = (B == 1) ? n_sm / (B * nkv)
+    // Long contexts at batch 1: one task per split covers every KV head (its pages'
+    // blocks of all heads are contiguous: large copies), one wave of splits over the
+    // SMs, and merge tasks per q head combine the splits.
+    g.wide_attn = (B == 1) && max_ctx >= kWideAttnCtx && kConsumerWarps % nkv == 0;   // warps per head
+    int S = (B == 1) ? n_sm / (g.wide_attn ? 1 : nkv)
                      : (int)std::min<int64_t>(std::lround(4.0 * n_sm / (double)(B * nkv)), ceil_div(max_ctx, 1024));
     S = std::max(1, std::min<int>(S, (int)ceil_div(max_ctx, 64)));
     g.S = S;
@@ -225,6 +230,21 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
                 own_entity(t, {Region{tensor_key(T_QKV, l, 0), 0, B, r0, r1}});
                 r0 = r1;
             }
+    };
+    // wide attention of a layer: per split, every KV head; then per q head a merge task
+    auto attn_wide = [&](int l) {
+        const int64_t qkv_rows = (int64_t)(nq + 2 * nkv) * hd;
+        for (int s = 0; s < S; ++s) {
+            int t = new_task(MK_OP_ATTN, l, 0, 0, (uint32_t)s, (uint32_t)S);
+            T[t].flags = kAttnWide;
+            task_in[t] = {Region{tensor_key(T_QKV, l, 0), 0, B, 0, qkv_rows}};
+            own_entity(t, {Region{tensor_key(T_PART, l, 0), 0, B, s, s + 1}});
+        }
+        for (int qh = 0; qh < nq; ++qh) {
+            int t = new_task(MK_OP_ATTN_MERGE, l, 0, 0, (uint32_t)qh, (uint32_t)(qh + 1));
+            task_in[t] = {Region{tensor_key(T_PART, l, 0), 0, B, 0, S}};
+            own_entity(t, {Region{tensor_key(T_O, l, 0), 0, B, (int64_t)qh * hd, (int64_t)(qh + 1) * hd}});
+        }
     };
     // attention of one KV group: per (sequence, split); each split writes its softmax
     // partial, and the O-projection's input stage merges the splits
@@ -348,7 +368,9 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
         // stream.  Attention follows all QKV tiles: a CTA that claimed a task still
         // waiting on its inputs streams nothing meanwhile.
         for (int kh = 0; kh < nkv; ++kh) qkv_group(l, kh);
-        for (int kh = 0; kh < nkv; ++kh) attn_group(l, kh);
+        if (g.wide_attn) attn_wide(l);
+        else
+            for (int kh = 0; kh < nkv; ++kh) attn_group(l, kh);
         gemv_op(MK_OP_OPROJ, l, H, R_o, T_XMID, l, {all_rows(T_O, l, 0, (int64_t)nq * hd)});
         if (!moe) {
             gemv_op(MK_OP_GATEUP, l, d.ffn, R_gu, T_ACT, l, {all_rows(T_XMID, l, 0, H)});
@@ -482,7 +504,7 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
             case MK_OP_EXP_DOWN: K = d.expert_ffn; break;
             default: break;
         }
-        t.flags = K ? fast_path_for(K, (int)(t.r1 - t.r0), nblk) : 0;
+        if (K) t.flags = fast_path_for(K, (int)(t.r1 - t.r0), nblk);   // (attention keeps its own flags)
     }
 
     // ---- bytes streamed per B=1 step

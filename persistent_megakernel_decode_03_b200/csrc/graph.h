@@ -14,6 +14,7 @@ struct GraphPlan {
     mk_model_desc desc{};
     int max_batch = 0, max_ctx = 0, n_sm = 0;
     int S = 1;                   // attention splits per (sequence, kv head)
+    bool wide_attn = false;      // attention tasks cover every KV head (long contexts, batch 1)
     int n_router_tiles = 0;
     int n_events = 0;
     int64_t weight_bytes = 0;    // bf16 bytes streamed per B=1 step

@@ -550,6 +550,83 @@ __device__ __forceinline__ void pr_advance(PRing& r) {
     if (++r.stage == kStages) { r.stage = 0; ++r.lap; }
 }
 
+// The pages of a wide attention task: per page, stages of hps KV heads each (2 at
+// d = 128), a stage holding the heads' key blocks then their value blocks (the page
+// holds the heads' 16 x d blocks back to back, so each half is one contiguous copy):
+// a warp finds both halves of its head in one stage.  The stage's info.aux is the
+// logical page.  Page ids are read 8 at a time, a batch ahead, into the shared ring
+// of ids; an id out of range is reported and its stages go out empty.
+__device__ __noinline__ bool produce_wide_pages(const Params& p, Smem& sm, const Task& t, int ti, PRing& ring,
+                                                uint64_t pol) {
+    // the split's cached positions (the new token is attended from registers)
+    int npages = 0, lp0 = 0;
+    if (t.b < p.batch) {
+        const int pos = position_of(p, t.b);
+        if (pos >= 0 && pos < p.max_ctx && pos / kPageSize < p.max_pages) {
+            int j0 = 0, j1 = 0;
+            const int sa = attn_active_splits(pos + 1, (int)t.r1);
+            if ((int)t.r0 < sa) attn_range(pos + 1, sa, (int)t.r0, j0, j1);
+            const int jc = min(j1, pos);
+            if (jc > j0) {
+                lp0 = j0 / kPageSize;
+                npages = (jc - 1) / kPageSize - lp0 + 1;
+            }
+        }
+    }
+    const int nkv = p.nkv, n_pages = p.n_pages;
+    const uint32_t blk = (uint32_t)(kPageSize * p.hd * 2);
+    const size_t blk_elems = (size_t)kPageSize * p.hd;
+    const int hps = kStageBytes / (2 * (int)blk);           // KV heads per stage (keys and values)
+    const int spp = (nkv + hps - 1) / hps;                  // stages per page
+    const int nch = npages * spp;
+    if (nch == 0) {
+        if (!pr_acquire(p, sm, ring)) return false;
+        sm.info[ring.stage] = StageInfo{ti, 0, 0, 0, t};
+        mbar_arrive(&sm.full[ring.stage]);
+        pr_advance(ring);
+        return true;
+    }
+    const int* prow = page_row(p, t.b);
+    int pid_have = 0;
+    for (int c = 0; c < nch; ++c) {
+        const int pg = c / spp, q = c % spp;
+        if (q == 0) {
+            while (pid_have < min(npages, pg + 1 + kPidBatch)) {
+                int v[kPidBatch];
+#pragma unroll
+                for (int i = 0; i < kPidBatch; ++i) {
+                    const int k = pid_have + i;
+                    v[i] = (k < npages) ? __ldg(prow + lp0 + k) : 0;
+                }
+#pragma unroll
+                for (int i = 0; i < kPidBatch; ++i) sm.pid[(pid_have + i) % kPidRing] = v[i];
+                pid_have += kPidBatch;
+            }
+        }
+        if (!pr_acquire(p, sm, ring)) return false;
+        StageInfo& inf = sm.info[ring.stage];
+        inf.task = ti;
+        inf.chunk = c;
+        inf.nchunks = nch;
+        inf.aux = lp0 + pg;
+        if (c == 0) inf.rec = t;
+        const int ph = sm.pid[pg % kPidRing];
+        if (ph < 0 || ph >= n_pages) {                       // validated before any copy of the page
+            set_error(p, kErrInvalid, ti, -2, lp0 + pg, t.b);
+            mbar_arrive(&sm.full[ring.stage]);
+            pr_advance(ring);
+            continue;
+        }
+        const int h0 = q * hps, nh = min(hps, nkv - h0);
+        mbar_arrive_expect_tx(&sm.full[ring.stage], 2u * (uint32_t)nh * blk);
+        const size_t off = (((size_t)t.layer * n_pages + ph) * nkv + h0) * blk_elems;
+        bulk_g2s(sm.ring[ring.stage], p.k_pages + off, (uint32_t)nh * blk, &sm.full[ring.stage], pol);
+        bulk_g2s(sm.ring[ring.stage] + (size_t)nh * blk, p.v_pages + off, (uint32_t)nh * blk, &sm.full[ring.stage], pol);
+        pr_advance(ring);
+    }
+    return true;
+}
+
 // Tasks whose streamed data is only known on the device: attention (KV pages of
 // this step's positions) and routed experts (weights of the expert the router
 // picked).  Out of line: it keeps the producer's hot loop small.
@@ -780,7 +857,7 @@ __device__ __noinline__ bool produce_mm(const Params& p, Smem& sm, const Task& t
     return true;
 }
 
-template <bool MM>
+template <bool MM, bool WIDE>
 __device__ void producer_loop(const Params& p, Smem& sm) {
     const uint64_t pol = l2_evict_first_policy();
     PRing ring{0, 0};
@@ -807,7 +884,14 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
                 continue;
             }
         }
-        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm) || t.op == MK_OP_NORM || t.op == MK_OP_KVAPPEND;
+        if constexpr (WIDE) {
+            if (t.op == MK_OP_ATTN) {
+                ok = produce_wide_pages(p, sm, t, ti, ring, pol);
+                continue;
+            }
+        }
+        const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm) || t.op == MK_OP_NORM || t.op == MK_OP_KVAPPEND ||
+                          t.op == MK_OP_ATTN_MERGE;
         if (skip) {                                      // nothing to stream: a marker stage
             if (!pr_acquire(p, sm, ring)) { ok = false; break; }
             sm.info[ring.stage] = StageInfo{ti, 0, 0, 0, t};
@@ -1980,6 +2064,273 @@ __device__ void attention_task(const Params& p, Smem& sm, uint32_t& cph, const T
     if (sm.attn_last && active_row) attn_merge_group(p, sm, cph, l, b, g);
 }
 
+// ---- wide attention (long contexts, batch 1): one task per split covers every KV
+// head.  Warp w serves KV head w / (8 / n_kv); with fewer than 8 KV heads the
+// warps of a head take its pages in turn.  Each page arrives as stage-sized blocks
+// of all heads' keys, then values (produce_wide_pages).  The split owning the new
+// position appends and attends the new token's k and v.  The split writes its
+// softmax partial per (KV head, q head); merge tasks combine the splits.
+
+// Row 0 of the warp's staging page from one head's fp32 vector in global memory
+// (k: rotated at the position's (cos, sin) pairs; v: as is), rounded to bf16; rows
+// 1..15 zero.  With `append`, the bf16 row is also written to the cache slot.
+template <int HD>
+__device__ __forceinline__ void stage_new_row(const float* src, const float* rope, bool rotate, uint8_t* stg,
+                                              uint16_t* append) {
+    constexpr int CPR = HD / 8;
+    const int lane = threadIdx.x & 31;
+    for (int q = lane; q < kPageSize * CPR; q += 32) {
+        const int r = q / CPR, c = q % CPR;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r == 0) {
+            float e[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int col = 8 * c + k;
+                float x = __ldcg(src + col);
+                if (rotate) {
+                    const int i = col % (HD / 2);
+                    const float2 cs = __ldg(reinterpret_cast<const float2*>(rope) + i);
+                    const float other = __ldcg(src + (col < HD / 2 ? col + HD / 2 : col - HD / 2));
+                    x = (col < HD / 2) ? x * cs.x - other * cs.y : x * cs.x + other * cs.y;
+                }
+                e[k] = bf16_to_f32(f32_to_bf16_rne(x));
+            }
+            v = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
+                           pack_bf16x2(e[6], e[7]));
+            if (append) *reinterpret_cast<uint4*>(append + 8 * c) = v;
+        }
+        sts128(smem_u32(stg) + stg_off<HD>(r, c), v);
+    }
+}
+
+template <int HPG, int DPL>
+__device__ void attention_wide_task(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti, int& stage,
+                                    uint32_t& lap, bool& abort_all) {
+    constexpr int HD = DPL * 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = t.b, s = (int)t.r0, S = (int)t.r1, l = t.layer;
+    const int nkv = p.nkv, wph = kConsumerWarps / nkv;
+    const int head = warp / wph, sub = warp % wph;
+    int pos = position_of(p, b);
+    const bool valid = b < p.batch && pos >= 0 && pos < p.max_ctx && pos / kPageSize < p.max_pages;
+    if (b < p.batch && !valid && tid == 0) set_error(p, kErrInvalid, ti, -3, pos, b);
+    if (!valid) pos = 0;
+    int j0 = 0, j1 = 0;
+    if (valid) {
+        const int sa = attn_active_splits(pos + 1, S);
+        if (s < sa) attn_range(pos + 1, sa, s, j0, j1);
+    }
+    const bool has_new = valid && pos >= j0 && pos < j1;
+    const float qscale = 1.4426950408889634f / sqrtf((float)HD);   // log2(e) / sqrt(d)
+
+    AttnMma<HPG, DPL> st;
+    st.m = -INFINITY;
+    st.l = 0.0f;
+#pragma unroll
+    for (int j = 0; j < AttnMma<HPG, DPL>::NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.o[j][e] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < AttnMma<HPG, DPL>::KS; ++ks)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.qa[ks][e] = 0u;
+    uint8_t* stg = reinterpret_cast<uint8_t*>(sm.attn) + warp * (kPageSize * HD * 2);   // staging page
+    csync(p, sm, cph);                                   // shared scratch of the previous task is free
+    const float* qkv = p.qkv + ((size_t)l * p.max_batch + b) * ((p.nq + 2 * p.nkv) * HD);
+    const float* rope = p.rope + (size_t)pos * HD;       // [HD/2][2] = cos, sin
+    if (valid && j1 > j0) {
+        // q of this warp's head group, rotated at pos and pre-scaled, through the
+        // staging page (fp32 [HPG][HD]) into the hi/lo A fragments
+        float* qf = reinterpret_cast<float*>(stg);
+        for (int idx = lane; idx < HPG * (HD / 2); idx += 32) {
+            const int h = idx / (HD / 2), i = idx % (HD / 2);
+            const float* src = qkv + (size_t)(head * HPG + h) * HD;
+            const float x0 = __ldcg(src + i), x1 = __ldcg(src + i + HD / 2);
+            const float2 cs = __ldg(reinterpret_cast<const float2*>(rope) + i);
+            qf[h * HD + i] = (x0 * cs.x - x1 * cs.y) * qscale;
+            qf[h * HD + i + HD / 2] = (x1 * cs.x + x0 * cs.y) * qscale;
+        }
+        __syncwarp();
+        const int g4 = lane >> 2, t4 = lane & 3;
+        if (g4 < HPG) {
+#pragma unroll
+            for (int ks = 0; ks < AttnMma<HPG, DPL>::KS; ++ks) {
+                const float* qh = qf + g4 * HD + 16 * ks + 2 * t4;
+                split_bf16x2(qh[0], qh[1], st.qa[ks][0], st.qa[ks][1]);
+                split_bf16x2(qh[8], qh[9], st.qa[ks][2], st.qa[ks][3]);
+            }
+        }
+        __syncwarp();
+        if (has_new && sub == 0) {
+            // the new token of this head: k rotated, both rounded to bf16, appended to the
+            // cache and attended as a one-token page
+            uint16_t* kapp = nullptr;
+            uint16_t* vapp = nullptr;
+            const int* prow = page_row(p, b);
+            const int ph = prow[pos / kPageSize];
+            if (ph >= 0 && ph < p.n_pages) {
+                const size_t off = ((((size_t)l * p.n_pages + ph) * nkv + head) * kPageSize + pos % kPageSize) * HD;
+                kapp = p.k_pages + off;
+                vapp = p.v_pages + off;
+            } else if (lane == 0) {
+                set_error(p, kErrInvalid, ti, -2, pos / kPageSize, b);
+            }
+            stage_new_row<HD>(qkv + (size_t)(p.nq + head) * HD, rope, true, stg, kapp);
+            __syncwarp();
+            float s0[4], s1[4];
+            attn_qk<HPG, DPL>(st, stg, s0, s1);
+            uint32_t pa[4];
+            attn_softmax<HPG, DPL>(st, s0, s1, 0, 1, pa);
+            __syncwarp();
+            stage_new_row<HD>(qkv + (size_t)(p.nq + nkv + head) * HD, rope, false, stg, vapp);
+            __syncwarp();
+            attn_pv<HPG, DPL>(st, stg, pa);
+            __syncwarp();
+        }
+    }
+
+    // the cached pages: per page spp stages of hps heads (their keys, then values)
+    const int jc = min(j1, pos);
+    const int blk_elems = kPageSize * HD;
+    const int hps = kStageBytes / (blk_elems * 2 * 2), spp = (nkv + hps - 1) / hps;
+    const int my_q = head / hps, my_slot = head % hps;
+    for (int c = 0;; ++c) {
+        if (c == 0) {
+            seen_complete_wait(p, &sm.full[stage], lap & 1, &sm.flag[3]);
+        } else if (!mbar_wait_bounded(p, &sm.full[stage], lap & 1, 3)) {
+            sm.flag[3] = 1;
+            break;
+        }
+        const StageInfo inf = sm.info[stage];
+        if (inf.task != ti) {
+            set_error(p, kErrFault, ti, -4, inf.task, 1);
+            sm.flag[3] = 1;
+            break;
+        }
+        if (inf.nchunks > 0) {
+            const int q = inf.chunk % spp;
+            const int lp = inf.aux;                          // logical page
+            if (q == my_q && (lp % wph) == sub) {
+                const int pf = lp * kPageSize;
+                const int k_lo = max(j0 - pf, 0), k_hi = min(jc - pf, kPageSize);
+                if (k_hi > k_lo) {
+                    const int nh = min(hps, nkv - q * hps);
+                    const uint16_t* kb = reinterpret_cast<const uint16_t*>(sm.ring[stage]) + (size_t)my_slot * blk_elems;
+                    attn_page<HPG, DPL>(st, kb, kb + (size_t)nh * blk_elems, k_lo, k_hi, stg);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        const bool last = inf.nchunks == 0 || inf.chunk == inf.nchunks - 1;
+        if (++stage == kStages) { stage = 0; ++lap; }
+        if (last) break;
+    }
+    st.l += __shfl_xor_sync(0xFFFFFFFFu, st.l, 1);
+    st.l += __shfl_xor_sync(0xFFFFFFFFu, st.l, 2);
+    csync(p, sm, cph);                                   // every warp is done with its staging page
+    float* sc = sm.attn;                                 // [warp][HPG][m, l, o]
+    {
+        const int g4 = lane >> 2, t4 = lane & 3;
+        if (g4 < HPG) {
+            float* w = sc + ((size_t)warp * HPG + g4) * (HD + 2);
+            if (t4 == 0) { w[0] = st.m; w[1] = st.l; }
+#pragma unroll
+            for (int j = 0; j < AttnMma<HPG, DPL>::NT; ++j) {
+                w[2 + 8 * j + 2 * t4] = st.o[j][0] + st.o[j][2];
+                w[2 + 8 * j + 2 * t4 + 1] = st.o[j][1] + st.o[j][3];
+            }
+        }
+    }
+    csync(p, sm, cph);
+    if (sm.flag[3]) { abort_all = true; return; }
+    if (!valid) return;
+    // this split's partial per (KV head, q head): the head's warps combined in order
+    for (int idx = tid; idx < nkv * HPG * (HD + 2); idx += kConsumerThreads) {
+        const int g = idx / (HPG * (HD + 2)), r = idx % (HPG * (HD + 2)), h = r / (HD + 2), c = r % (HD + 2);
+        float M = -INFINITY;
+        for (int u = 0; u < wph; ++u) M = fmaxf(M, sc[((size_t)(g * wph + u) * HPG + h) * (HD + 2)]);
+        float val;
+        if (c == 0) {
+            val = M;
+        } else {
+            float acc = 0.0f;
+            if (M != -INFINITY)
+                for (int u = 0; u < wph; ++u) {
+                    const float* ww = sc + ((size_t)(g * wph + u) * HPG + h) * (HD + 2);
+                    const float f = (ww[0] == -INFINITY) ? 0.0f : exp2f(ww[0] - M);
+                    acc = fmaf(ww[c], f, acc);
+                }
+            val = acc;
+        }
+        const size_t pidx = attn_part_index(p, l, b, g, s, h);
+        if (c < 2) attn_part_ml(p, pidx)[c] = val;
+        else attn_part_o(p, pidx)[c - 2] = val;
+    }
+}
+
+// Merge task of wide attention: q head t.r0 of sequence t.b, the active splits'
+// partials combined (m* = max m_s; o = sum 2^(m_s - m*) o_s / sum 2^(m_s - m*) l_s),
+// normalised and stored.  Warp 0 forms the weights; then thread (j, c4) sums splits
+// j, j + 8, ... over four columns, and the eight partial sums are added in order.
+__device__ void attn_merge_head(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti) {
+    const int tid = threadIdx.x, lane = tid & 31, hd = p.hd, hpg = hpg_of(p);
+    const int b = t.b, l = t.layer, qh = (int)t.r0, g = qh / hpg, h = qh % hpg;
+    int pos = (b < p.batch) ? position_of(p, b) : -1;
+    if (pos < 0 || pos >= p.max_ctx) return;             // (the attention task reported it)
+    const int sa = attn_active_splits(pos + 1, p.S);
+    float* f = sm.attn;                                  // [sa] weights, [sa] l, then [8][hd] sums
+    float* fl = f + sa;
+    float* part = f + ((2 * sa + 3) & ~3);               // 16-byte aligned (float4 stores)
+    csync(p, sm, cph);                                   // the scratch of the previous task is free
+    for (int k = tid; k < sa; k += kConsumerThreads) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(attn_part_ml(p, attn_part_index(p, l, b, g, k, h))));
+        f[k] = ml.x;
+        fl[k] = ml.y;
+    }
+    csync(p, sm, cph);
+    if (tid < 32) {
+        float M = -INFINITY;
+        for (int k = lane; k < sa; k += 32) M = fmaxf(M, f[k]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+        float L = 0.0f;
+        for (int k = lane; k < sa; k += 32) {
+            const float w = (f[k] == -INFINITY) ? 0.0f : exp2f(f[k] - M);
+            f[k] = w;
+            L = fmaf(fl[k], w, L);
+        }
+        L = warp_sum(L);
+        if (lane == 0) fl[0] = (L > 0.0f) ? 1.0f / L : 0.0f;   // (fl is no longer needed)
+    }
+    csync(p, sm, cph);
+    const int j = tid >> 5, c4 = lane;
+    if (4 * c4 < hd) {
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int k = j; k < sa; k += kConsumerWarps) {
+            const float w = f[k];
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(attn_part_o(p, attn_part_index(p, l, b, g, k, h)) + 4 * c4));
+            o.x = fmaf(v.x, w, o.x); o.y = fmaf(v.y, w, o.y); o.z = fmaf(v.z, w, o.z); o.w = fmaf(v.w, w, o.w);
+        }
+        *reinterpret_cast<float4*>(part + (size_t)j * hd + 4 * c4) = o;
+    }
+    const float inv = fl[0];
+    csync(p, sm, cph);
+    if (tid < hd / 4) {
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int jj = 0; jj < kConsumerWarps; ++jj) {
+            const float4 v = *reinterpret_cast<const float4*>(part + (size_t)jj * hd + 4 * tid);
+            o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+        }
+        float* out = p.attn_o + ((size_t)l * p.max_batch + b) * p.nq * hd + (size_t)qh * hd;
+        *reinterpret_cast<float4*>(out + 4 * tid) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+    }
+    (void)ti;
+}
+
 // ----------------------------------------------------------------------------- consumer: router top-k
 
 // Last router tile of a layer: softmax over the experts, top-k (ties to the
@@ -2445,7 +2796,7 @@ __device__ __noinline__ bool mm_task(const Params& p, Smem& sm, const Task& t, i
 
 // MM: the instantiation for batched graphs (norm tasks, tensor-core tiles,
 // attention); the batch-1 instantiation holds the GEMV tiles and none of that.
-template <int HPG, int DPL, bool MM>
+template <int HPG, int DPL, bool MM, bool WIDE>
 __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int stage = 0;
@@ -2539,9 +2890,23 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
             continue;
         }
         }
+        if constexpr (WIDE) {
+        if (t.op == MK_OP_ATTN_MERGE) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);     // the marker stage
+            if (++stage == kStages) { stage = 0; ++lap; }
+            attn_merge_head(p, sm, cph, t, ti);
+            if (sm.flag[3]) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.red_full[buf]);
+            ++seq;
+            continue;
+        }
+        }
         if (t.op == MK_OP_ATTN) {
             bool abort_all = false;
-            attention_task<HPG, DPL, MM>(p, sm, cph, t, ti, stage, lap, abort_all);
+            if constexpr (WIDE) attention_wide_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
+            else attention_task<HPG, DPL, MM>(p, sm, cph, t, ti, stage, lap, abort_all);
             if (abort_all) break;
             x_key_op = -1;
             // the input slice in registers is dead across an attention task (saves registers)
@@ -2780,7 +3145,10 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
 // 64-wide heads need fewer than the launch allows, and ptxas launches them with less.
 __host__ __device__ constexpr bool splits_registers(bool mm, int dpl) { return !mm || dpl == 4; }
 
-template <int HPG, int DPL, bool MM>
+// MM: batched graphs (tensor-core tiles); WIDE: batch-1 graphs whose attention tasks
+// cover every KV head (long contexts).  Each graph kind has its own instantiation,
+// so one kind's code never costs another registers.
+template <int HPG, int DPL, bool MM, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
@@ -2820,13 +3188,13 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     if (warp < kConsumerWarps) {
         if constexpr (splits_registers(MM, DPL)) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
         const long long k0 = clock64();
-        consumer_loop<HPG, DPL, MM>(p, sm);
+        consumer_loop<HPG, DPL, MM, WIDE>(p, sm);
         if (threadIdx.x == 0) stat_add(p, 3, (unsigned long long)(clock64() - k0));
         return;
     }
     if constexpr (splits_registers(MM, DPL)) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSupportRegs));
     if (warp == kProducerWarp) {
-        if (lane == 0) producer_loop<MM>(p, sm);
+        if (lane == 0) producer_loop<MM, WIDE>(p, sm);
     } else if (warp == kEpilogueWarp) {
         epilogue_loop(p, sm);
     } else if (warp == kPrefetchWarp) {
@@ -2838,15 +3206,17 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 
 template <int HPG, int DPL>
 static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream, bool cooperative) {
-    auto kern = p.mm ? megakernel<HPG, DPL, true> : megakernel<HPG, DPL, false>;
+    const int kind = p.mm ? 1 : (p.wide ? 2 : 0);
+    auto kern = p.mm ? megakernel<HPG, DPL, true, false>
+                     : (p.wide ? megakernel<HPG, DPL, false, true> : megakernel<HPG, DPL, false, false>);
     // the shared-memory attribute, once per instantiation and device (so that a step
     // can be captured into a CUDA graph without host-side calls in between)
     // (devices 0..63 are remembered; a higher index sets the attribute every launch)
-    static unsigned long long attr_set[2] = {0ull, 0ull};
+    static unsigned long long attr_set[3] = {0ull, 0ull, 0ull};
     int dev = 0;
     cudaGetDevice(&dev);
     const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
-    if (!bit || !(attr_set[p.mm ? 1 : 0] & bit)) {
+    if (!bit || !(attr_set[kind] & bit)) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
         if (e != cudaSuccess) return e;
         // a register split (setmaxnreg) needs the launch's registers: with fewer, the
@@ -2855,7 +3225,7 @@ static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream, bool
         e = cudaFuncGetAttributes(&fa, (const void*)kern);
         if (e != cudaSuccess) return e;
         if (splits_registers(p.mm != 0, DPL) && fa.numRegs < kMinLaunchRegs) return cudaErrorInvalidConfiguration;
-        attr_set[p.mm ? 1 : 0] |= bit;
+        attr_set[kind] |= bit;
     }
     void* args[] = {const_cast<Params*>(&p)};
     if (cooperative)
@@ -2894,15 +3264,15 @@ cudaError_t megakernel_occupancy(int hpg, int hd, int* blocks_per_sm) {
     const int dpl = hd / 32;
     const void* f = nullptr;
     if (dpl == 4) {
-        if (hpg == 1) f = (const void*)megakernel<1, 4, false>;
-        if (hpg == 2) f = (const void*)megakernel<2, 4, false>;
-        if (hpg == 4) f = (const void*)megakernel<4, 4, false>;
-        if (hpg == 8) f = (const void*)megakernel<8, 4, false>;
+        if (hpg == 1) f = (const void*)megakernel<1, 4, false, false>;
+        if (hpg == 2) f = (const void*)megakernel<2, 4, false, false>;
+        if (hpg == 4) f = (const void*)megakernel<4, 4, false, false>;
+        if (hpg == 8) f = (const void*)megakernel<8, 4, false, false>;
     } else {
-        if (hpg == 1) f = (const void*)megakernel<1, 2, false>;
-        if (hpg == 2) f = (const void*)megakernel<2, 2, false>;
-        if (hpg == 4) f = (const void*)megakernel<4, 2, false>;
-        if (hpg == 8) f = (const void*)megakernel<8, 2, false>;
+        if (hpg == 1) f = (const void*)megakernel<1, 2, false, false>;
+        if (hpg == 2) f = (const void*)megakernel<2, 2, false, false>;
+        if (hpg == 4) f = (const void*)megakernel<4, 2, false, false>;
+        if (hpg == 8) f = (const void*)megakernel<8, 2, false, false>;
     }
     if (!f) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));

@@ -105,6 +105,13 @@ __host__ __device__
 #endif
 inline bool is_mm_op(int op) { return op >= MK_OP_MM_QKV && op <= MK_OP_MM_LMHEAD; }
 
+// Decode attention over every KV head of a page at once ("wide" tasks, batch-1
+// graphs from kWideAttnCtx positions of context): per split, the pages' keys and
+// values of all heads stream as contiguous blocks (a page holds each head's 16 x d
+// block back to back), and separate merge tasks combine the splits per q head.
+constexpr int kWideAttnCtx = 32768;
+constexpr uint8_t kAttnWide = 1;       // Task::flags of a wide attention task
+
 // Device task record (32 bytes).
 struct Task {
     uint8_t op;
@@ -212,6 +219,7 @@ struct Params {
     int n_pages, max_pages;
     float* logits;
 
+    int wide;                    // 1: the graph's attention tasks cover every KV head
     // batched projection tiles (max_batch > 1)
     int mm;                      // 1: the graph uses tensor-core tiles
     int bp;                      // padded batch: the MMA's N (16, 32 or 64)

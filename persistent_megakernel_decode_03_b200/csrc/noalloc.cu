@@ -272,6 +272,7 @@ extern "C" mk_status mk_decode_step_noalloc(const mk_model_desc* desc, const voi
     p.act = reinterpret_cast<float*>(b + lay.act);
     p.part = reinterpret_cast<float*>(b + lay.part);
     p.attn_o = reinterpret_cast<float*>(b + lay.attn_o);
+    p.wide = P.wide_attn ? 1 : 0;
     if (d.n_experts > 0) {
         p.rlogits = reinterpret_cast<float*>(b + lay.rlogits);
         p.moe_w = reinterpret_cast<float*>(b + lay.moe_w);

@@ -18,6 +18,10 @@ Read/write sets per operator mirror the megakernel's tiles:
   exp_gu   reads sel[l], x_mid[l] (all)        writes acte[l][k][rows]
   exp_dn   reads sel[l], acte[l][k] (all)      writes ypart[l][k][rows]
   lmhead   reads x_in[L] (all)                 writes logits[rows]
+Long-context batch-1 graphs ("wide" attention, exported with aux = -1):
+  attn     reads qkv[l] (all)                  writes part[l][b, g, s] for every kv head g
+  attn_merge  q head r0: reads part[l][b, its kv head, all splits]   writes ao[l][r0]
+  oproj    then reads ao[l] (all) instead of the partials
 For MoE models x_in[l+1][i] is x_mid[l][i] combined with ypart[l][k][i] for all k
 and the routing weights sel[l].
 
@@ -44,7 +48,7 @@ import numpy as np
 
 OP = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
       8: "exp_gu", 9: "exp_dn", 10: "norm", 11: "mm_qkv", 12: "mm_oproj", 13: "mm_gu", 14: "mm_down",
-      15: "mm_lm", 16: "kvappend"}
+      15: "mm_lm", 16: "kvappend", 17: "attn_merge"}
 NO_EVENT = 0xFFFFFFFF
 M64 = (1 << 64) - 1
 
@@ -95,6 +99,7 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
     for l in range(L):
         T[("qkv", l)] = Tensor(qkv_rows)
         T[("part", l)] = Tensor(B * nkv * 4096)
+        T[("ao", l)] = Tensor(nq)
         T[("x_mid", l)] = Tensor(B * H)
         if moe:
             T[("rlog", l)] = Tensor(E)
@@ -113,6 +118,7 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
         T[("kv", l)] = Tensor(B)
     T[("logits",)] = Tensor(V)
     mm_arrivals = defaultdict(int)
+    wide = any(tk.op == 17 for tk in tasks)
     tasks_split = {tk.layer: tk.r1 for tk in tasks if tk.op == 2}
     router_arr = defaultdict(int)
     n_router = defaultdict(int)
@@ -167,6 +173,19 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
             d = read_xin(l, 0, H, who)
             t("qkv", l).write(r0, r1, _mix(base ^ d), who)
             signal(tk.signal)
+        elif op == "attn" and tk.aux == -1:               # every kv head of split r0
+            b = tk.b
+            d = t("qkv", l).read(0, qkv_rows, who)
+            for g in range(nkv):
+                idx = (b * nkv + g) * 4096 + r0
+                t("part", l).write(idx, idx + 1, _mix(base ^ d ^ g), who)
+            signal(tk.signal)
+        elif op == "attn_merge":
+            g, b = r0 // hpg, tk.b
+            lo = (b * nkv + g) * 4096
+            d = t("part", l).read(lo, lo + tasks_split[l], who)
+            t("ao", l).write(r0, r1, _mix(base ^ d), who)
+            signal(tk.signal)
         elif op == "attn":
             g, b = tk.aux, tk.b
             qkv = t("qkv", l)
@@ -181,10 +200,13 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
         elif op == "oproj":
             n_split = tasks_split[l]
             d = read_xin(l, r0, r1, who)
-            for bb in range(B):
-                for gg in range(nkv):
-                    lo = (bb * nkv + gg) * 4096
-                    d += t("part", l).read(lo, lo + n_split, who)
+            if wide:
+                d += t("ao", l).read(0, nq, who)
+            else:
+                for bb in range(B):
+                    for gg in range(nkv):
+                        lo = (bb * nkv + gg) * 4096
+                        d += t("part", l).read(lo, lo + n_split, who)
             t("x_mid", l).write(r0, r1, _mix(base ^ (d & M64)), who)
             signal(tk.signal)
         elif op == "gateup":

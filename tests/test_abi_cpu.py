@@ -3,6 +3,7 @@
 No compute call is made here (there is no GPU); the task graph is planned on
 the host with mk_plan_taskgraph and checked symbolically.
 """
+import copy
 import json
 import os
 import re
@@ -149,6 +150,37 @@ def test_random_orders_on_8b_shaped_graph():
     ref = dataflow.run(tasks, thr, shape_of(cfg), seed=0)
     for s in (1, 2):
         assert (dataflow.run(tasks, thr, shape_of(cfg), seed=s)["logits"] == ref["logits"]).all()
+
+
+def test_long_context_graph_wide_attention_random_orders():
+    """Long contexts at batch 1: one attention task per split covers every KV head,
+    merge tasks per q head combine the splits, and the O-projection waits on the
+    merges; the graph runs in random valid orders with identical digests, and a
+    dropped merge wait is caught."""
+    cfg = syn.TINY
+    info, tasks, thr = plan(cfg, max_ctx=40000, n_sm=16)
+    attn = [t for t in tasks if t.op == mk.MK_OP_ATTN]
+    merges = [t for t in tasks if t.op == mk.MK_OP_ATTN_MERGE]
+    assert attn and all(t.aux == -1 for t in attn)
+    assert len(merges) == cfg.n_layers * cfg.n_q_heads
+    assert len(attn) == cfg.n_layers * info.attn_splits == cfg.n_layers * 16
+    ref = dataflow.run(tasks, thr, shape_of(cfg), seed=0)
+    for s in range(1, 20):
+        assert (dataflow.run(tasks, thr, shape_of(cfg), seed=s)["logits"] == ref["logits"]).all()
+    broken = [copy.copy(t) for t in tasks]
+    victim = next(i for i, t in enumerate(broken) if t.op == mk.MK_OP_ATTN_MERGE)
+    broken[victim].wait[0] = mk.MK_NO_EVENT
+    caught = 0
+    for s in range(40):
+        try:
+            dataflow.run(broken, thr, shape_of(cfg), seed=s)
+        except dataflow.Violation:
+            caught += 1
+    assert caught > 0
+    # short contexts keep one task per (KV head, split)
+    info2, tasks2, _ = plan(cfg, max_ctx=600, n_sm=16)
+    assert all(t.aux >= 0 for t in tasks2 if t.op == mk.MK_OP_ATTN)
+    assert not any(t.op == mk.MK_OP_ATTN_MERGE for t in tasks2)
 
 
 def test_executor_detects_a_missing_dependency():
