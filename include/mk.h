@@ -188,9 +188,12 @@ enum {
     MK_OP_MM_LMHEAD = 15, /* rows of Wlm . rmsnorm(x) */
     MK_OP_KVAPPEND = 16,  /* batched graphs: K (rotated) and V of batch rows [r0, r1) into
                              their pages; the attention tasks of the layer wait for them */
-    MK_OP_ATTN_MERGE = 17 /* long-context batch-1 graphs: q heads [r0, r1) of sequence b, the
+    MK_OP_ATTN_MERGE = 17,/* long-context batch-1 graphs: q heads [r0, r1) of sequence b, the
                              splits' softmax partials merged (their attention tasks cover every
                              KV head of a page, exported with aux = -1) */
+    MK_OP_TP_REDUCE = 18  /* tensor-parallel graphs: rows [r0, r1) of the residual stream after
+                             attention (aux 0) or the FFN (aux 1): waits until every rank has
+                             pushed its partial sums of those rows, adds them in rank order */
 };
 
 #define MK_NO_EVENT 0xFFFFFFFFu
@@ -285,10 +288,12 @@ mk_status mk_decode_step(mk_state* state, const int32_t* token_ids, const int32_
  * Greedy generation without a host round trip per token: n_steps decode steps
  * for `batch` sequences, enqueued at once on `stream`.  Step k feeds each
  * sequence the token chosen at step k - 1 (step 0: first_tokens, device int32
- * [batch]) at position positions[b] + k (positions: device int32 [batch]), and
- * after it a small kernel writes the argmax of each logits row (ties to the
- * lowest index) to tokens_out[k][b] (device int32 [n_steps][batch]).
- * logits_out (device fp32 [batch][vocab]) holds each step's logits in turn. */
+ * [batch]) at position positions[b] + k (positions: device int32 [batch]).
+ * Inside the same launch the step's last LM-head tile writes the argmax of each
+ * logits row (ties to the lowest index) to tokens_out[k][b] (device int32
+ * [n_steps][batch]), so generation is one launch per token.
+ * logits_out (device fp32 [batch][vocab]) holds each step's logits in turn.
+ * Not for tensor-parallel states (each rank holds a vocabulary shard). */
 mk_status mk_generate(mk_state* state, const int32_t* first_tokens, const int32_t* positions, int batch,
                       int n_steps, const mk_paged_kv* kv, int32_t* tokens_out, float* logits_out,
                       mk_stream stream);
@@ -339,6 +344,77 @@ mk_status mk_prefill(mk_state* state, const int32_t* tokens, int n_tokens, int s
  * kv->page_table[seq_slot] (its positions 0..pos0-1 must already be cached). */
 mk_status mk_prefill_seq(mk_state* state, const int32_t* tokens, int n_tokens, int pos0, int seq_slot,
                          const mk_paged_kv* kv, float* last_logits, mk_stream stream);
+
+/* ---------------------------------------------------------------- tensor parallelism
+ *
+ * Passage: MPK digest, section "Part 1. Compiler": an all-reduce after a
+ * matrix multiplication is a task of the graph like any other, and it can start
+ * on the parts of the product that are done instead of after the whole
+ * operator; the runtime of the same digest (one kernel per GPU computing and
+ * communicating).  Russian MPK overview, the task-graph pseudocode (an
+ * all-reduce task waiting on the matmul's event).
+ *
+ * A dense model split over tp ranks (one GPU each): rank r holds q heads
+ * [r*nq/tp, (r+1)*nq/tp) with their KV heads, FFN rows [r*F/tp, (r+1)*F/tp)
+ * and vocabulary rows [r*V/tp, (r+1)*V/tp) of the LM head.  Each O-projection
+ * and down-projection tile stores its partial sums of its residual rows into
+ * every rank's receive buffer (plain stores into peer memory) and raises that
+ * tile's arrival flag on every rank (system-scope release); a reduce task per
+ * tile on each rank waits for tp arrivals and adds the ranks' parts in rank
+ * order, then the residual.  No multicast of any kind. */
+
+#define MK_TP_IPC_HANDLE_BYTES 64
+
+/* Registers rank tp_rank's shard of the model described by desc (the WHOLE
+ * model's shape).  weight_ptrs follows mk_load_model's order with the shard's
+ * shapes: tok_emb [vocab][hidden] whole; wq [nq/tp*d][hidden], wk and wv
+ * [nkv/tp*d][hidden], wo [hidden][nq/tp*d] (the rank's columns), w_gate and
+ * w_up [ffn/tp][hidden], w_down [hidden][ffn/tp], norms whole, lm_head
+ * [vocab/tp][hidden].  Needs a dense model, 2 <= tp_size <= 8, n_kv_heads,
+ * ffn (in multiples of 8 per rank) and vocab divisible by tp_size.
+ * Errors: MK_ERR_UNSUPPORTED when the model does not divide; as mk_load_model
+ * otherwise.  Graphs built from the model are batch-1 tensor-parallel graphs;
+ * a state's KV cache holds the rank's nkv/tp heads and its logits the rank's
+ * vocab/tp rows. */
+mk_status mk_load_model_tp(const mk_model_desc* desc, int tp_size, int tp_rank, const void* const* weight_ptrs,
+                           int n_ptrs, mk_model** out);
+
+/* Host-only plan of rank tp_rank's batch-1 task graph (for inspection and
+ * tests; no device needed), with the shard shapes mk_load_model_tp derives from
+ * the whole model's desc.  The O- and down-projection tiles of each layer are
+ * followed by one MK_OP_TP_REDUCE task per tile (same rows; aux 0 after
+ * attention, 1 after the FFN), whose signal the next operator waits on; the
+ * reduce tasks themselves wait on arrival flags, not events. */
+mk_status mk_plan_taskgraph_tp(const mk_model_desc* desc, int tp_size, int tp_rank, int max_ctx, int n_sm,
+                               mk_graph** out);
+
+/* The state's own receive buffer and arrival flags (one device allocation of
+ * *bytes bytes at *base, owned by the state).  Errors: MK_ERR_INVALID_ARG for a
+ * state that is not tensor-parallel. */
+mk_status mk_state_tp_buffer(mk_state* state, void** base, size_t* bytes);
+
+/* Rank `rank`'s buffer (its mk_state_tp_buffer base) as addressable from this
+ * state's device: a peer pointer after cudaDeviceEnablePeerAccess, or the same
+ * device's pointer when the ranks are emulated on one GPU.  Borrowed.  Every
+ * other rank must be set before a step. */
+mk_status mk_state_tp_set_peer(mk_state* state, int rank, void* peer_base);
+
+/* For ranks in separate processes: the IPC handle (MK_TP_IPC_HANDLE_BYTES
+ * bytes to handle_out, host memory) of this state's buffer, and the opening of
+ * a peer's handle (kept open until mk_state_destroy). */
+mk_status mk_state_tp_ipc_handle(mk_state* state, void* handle_out);
+mk_status mk_state_tp_open_peer(mk_state* state, int rank, const void* handle);
+
+/* A tensor-parallel decode step on every rank: each rank launches
+ * mk_decode_step on its own GPU with the same token and position (the ranks'
+ * kernels meet through the flags).  For n ranks on ONE GPU this call runs the
+ * n ranks' steps in a single cooperative launch, each rank on n_sm/n of the
+ * SMs (states[r] is rank r of n, 2 <= n <= 4, head_dim 128; kvs[r] and
+ * logits_out[r] are the rank's cache and logits shard).  token_ids and
+ * positions: device int32 [1]. */
+mk_status mk_decode_step_tp_emulated(mk_state* const* states, int n, const int32_t* token_ids,
+                                     const int32_t* positions, const mk_paged_kv* const* kvs,
+                                     float* const* logits_out, mk_stream stream);
 
 /* The decode step of mk_decode_step for callers that cannot allocate device
  * memory: code running where cudaMalloc is not allowed (inside a host callback,

@@ -36,9 +36,11 @@ MK_OP_NORM, MK_OP_MM_QKV, MK_OP_MM_OPROJ, MK_OP_MM_GATEUP, MK_OP_MM_DOWN, MK_OP_
 MM_OPS = (MK_OP_MM_QKV, MK_OP_MM_OPROJ, MK_OP_MM_GATEUP, MK_OP_MM_DOWN, MK_OP_MM_LMHEAD)
 MK_OP_KVAPPEND = 16
 MK_OP_ATTN_MERGE = 17
+MK_OP_TP_REDUCE = 18
+MK_TP_IPC_HANDLE_BYTES = 64
 OP_NAMES = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
             8: "exp_gateup", 9: "exp_down", 10: "norm", 11: "mm_qkv", 12: "mm_oproj", 13: "mm_gateup",
-            14: "mm_down", 15: "mm_lmhead", 16: "kvappend", 17: "attn_merge"}
+            14: "mm_down", 15: "mm_lmhead", 16: "kvappend", 17: "attn_merge", 18: "tp_reduce"}
 
 # Exported symbols (declared in include/mk.h).
 SYMBOLS = (
@@ -51,6 +53,8 @@ SYMBOLS = (
     "mk_state_read_counters",
     "mk_state_read_buffer", "mk_state_read_trace", "mk_state_read_stats", "mk_last_error_string",
     "mk_version",
+    "mk_load_model_tp", "mk_plan_taskgraph_tp", "mk_state_tp_buffer", "mk_state_tp_set_peer", "mk_state_tp_ipc_handle",
+    "mk_state_tp_open_peer", "mk_decode_step_tp_emulated",
 )
 
 
@@ -138,6 +142,13 @@ def lib() -> ctypes.CDLL:
             "mk_state_read_stats": ([vp, vp, i32, vp], st),
             "mk_last_error_string": ([], ctypes.c_char_p),
             "mk_version": ([], ctypes.c_char_p),
+            "mk_load_model_tp": ([P(mk_model_desc), i32, i32, vp, i32, P(vp)], st),
+            "mk_plan_taskgraph_tp": ([P(mk_model_desc), i32, i32, i32, i32, P(vp)], st),
+            "mk_state_tp_buffer": ([vp, P(vp), P(ctypes.c_size_t)], st),
+            "mk_state_tp_set_peer": ([vp, i32, vp], st),
+            "mk_state_tp_ipc_handle": ([vp, vp], st),
+            "mk_state_tp_open_peer": ([vp, i32, vp], st),
+            "mk_decode_step_tp_emulated": ([vp, i32, vp, vp, vp, vp, vp], st),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -290,6 +301,58 @@ def mk_decode_step_noalloc(desc: mk_model_desc, weight_ptrs: Sequence[int], max_
     arr = (ctypes.c_void_p * len(weight_ptrs))(*weight_ptrs)
     _check(lib().mk_decode_step_noalloc(ctypes.byref(desc), arr, len(weight_ptrs), max_ctx, token_ids,
                                         positions, batch, ctypes.byref(kv), logits_out, stream))
+
+
+def mk_load_model_tp(desc: mk_model_desc, tp_size: int, tp_rank: int, weight_ptrs: Sequence[int]) -> int:
+    """Rank tp_rank's shard of the model `desc` describes (weights: the shard's, in
+    mk_load_model's order)."""
+    arr = (ctypes.c_void_p * len(weight_ptrs))(*weight_ptrs)
+    out = ctypes.c_void_p()
+    _check(lib().mk_load_model_tp(ctypes.byref(desc), int(tp_size), int(tp_rank), arr, len(weight_ptrs),
+                                  ctypes.byref(out)))
+    return out.value
+
+
+def mk_plan_taskgraph_tp(desc: mk_model_desc, tp_size: int, tp_rank: int, max_ctx: int, n_sm: int) -> int:
+    """Host-only plan of one rank's tensor-parallel graph (no device needed)."""
+    out = ctypes.c_void_p()
+    _check(lib().mk_plan_taskgraph_tp(ctypes.byref(desc), int(tp_size), int(tp_rank), int(max_ctx), int(n_sm),
+                                      ctypes.byref(out)))
+    return out.value
+
+
+def mk_state_tp_buffer(state: int) -> Tuple[int, int]:
+    """(device address, bytes) of the state's receive buffer and arrival flags."""
+    base, n = ctypes.c_void_p(), ctypes.c_size_t()
+    _check(lib().mk_state_tp_buffer(state, ctypes.byref(base), ctypes.byref(n)))
+    return base.value, n.value
+
+
+def mk_state_tp_set_peer(state: int, rank: int, peer_base: int) -> None:
+    _check(lib().mk_state_tp_set_peer(state, int(rank), peer_base))
+
+
+def mk_state_tp_ipc_handle(state: int) -> bytes:
+    buf = ctypes.create_string_buffer(MK_TP_IPC_HANDLE_BYTES)
+    _check(lib().mk_state_tp_ipc_handle(state, buf))
+    return buf.raw
+
+
+def mk_state_tp_open_peer(state: int, rank: int, handle: bytes) -> None:
+    if len(handle) != MK_TP_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle is 64 bytes")
+    buf = ctypes.create_string_buffer(bytes(handle), MK_TP_IPC_HANDLE_BYTES)
+    _check(lib().mk_state_tp_open_peer(state, int(rank), buf))
+
+
+def mk_decode_step_tp_emulated(states: Sequence[int], token_ids: int, positions: int,
+                               kvs: Sequence[mk_paged_kv], logits_out: Sequence[int], stream: int = 0) -> None:
+    """len(states) ranks of one tensor-parallel model in one launch on this GPU."""
+    n = len(states)
+    st = (ctypes.c_void_p * n)(*states)
+    kp = (ctypes.POINTER(mk_paged_kv) * n)(*[ctypes.pointer(k) for k in kvs])
+    lo = (ctypes.c_void_p * n)(*logits_out)
+    _check(lib().mk_decode_step_tp_emulated(st, n, token_ids, positions, kp, lo, stream))
 
 
 def mk_sync(state: int, stream: int = 0) -> int:

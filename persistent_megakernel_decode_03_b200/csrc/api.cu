@@ -18,8 +18,10 @@
 using mk::GraphPlan;
 
 struct mk_model {
-    mk_model_desc desc{};
+    mk_model_desc desc{};        // this rank's shapes (tensor parallelism: the shard's)
     int device = 0;
+    int tp = 1, tp_rank = 0;     // tensor-parallel size and rank
+    int vocab_full = 0;          // rows of the token embedding (the whole vocabulary)
     std::vector<const void*> w;
     std::vector<mk::LayerW> h_layers;
     mk::LayerW* d_layers = nullptr;
@@ -64,6 +66,14 @@ struct mk_state {
     float* logits = nullptr;       // host-output variant: [max_batch][vocab]
     unsigned long long* trace = nullptr;
     unsigned long long* stats = nullptr;
+    int ncta = 0;                  // CTAs of the last step (the queue head advances by tasks + CTAs)
+    // tensor parallelism: this rank's receive buffer [tp][L][2][H] floats followed by
+    // its arrival flags [L][2][tiles] (one allocation, so one IPC handle covers it),
+    // and every rank's copy as mapped here (own included)
+    void* tp_buf = nullptr;
+    size_t tp_recv_bytes = 0, tp_bytes = 0;
+    void* tp_peer[mk::kMaxTp] = {};
+    bool tp_ipc[mk::kMaxTp] = {};  // opened through an IPC handle (closed on destroy)
     std::vector<void*> allocs;
 };
 
@@ -138,8 +148,17 @@ mk_status dev_alloc(mk_state* s, T** p, size_t count) {
 }
 
 void free_state_memory(mk_state* s) {
+    for (int q = 0; q < mk::kMaxTp; ++q)
+        if (s->tp_ipc[q] && s->tp_peer[q]) cudaIpcCloseMemHandle(s->tp_peer[q]);
     for (void* v : s->allocs) cudaFree(v);
     s->allocs.clear();
+}
+
+bool tp_ready(const mk_state* s) {
+    const int tp = s->g->model ? s->g->model->tp : 1;
+    for (int q = 0; q < tp; ++q)
+        if (!s->tp_peer[q]) return false;
+    return true;
 }
 
 mk_status reset_counters(mk_state* s, cudaStream_t st) {
@@ -155,6 +174,10 @@ mk_status reset_counters(mk_state* s, cudaStream_t st) {
                             sizeof(uint32_t) * d.n_layers * s->g->plan.max_batch * d.n_kv_heads, st);
     if (e == cudaSuccess && s->mm_cnt)
         e = cudaMemsetAsync(s->mm_cnt, 0, sizeof(uint32_t) * std::max(1, s->g->plan.mm_counters), st);
+    // the arrival flags count from zero again (every rank resets together: the flags
+    // are raised by all ranks against the same step count)
+    if (e == cudaSuccess && s->tp_buf)
+        e = cudaMemsetAsync(static_cast<char*>(s->tp_buf) + s->tp_recv_bytes, 0, s->tp_bytes - s->tp_recv_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "reset");
     s->epoch = 0;
     s->needs_reset = false;
@@ -204,7 +227,7 @@ mk::Params base_params(mk_state* s) {
     p.nkv = d.n_kv_heads;
     p.hd = d.head_dim;
     p.F = d.ffn;
-    p.V = d.vocab;
+    p.V = m->vocab_full;             // embedding rows (the LM head's rows are the graph's)
     p.E = d.n_experts;
     p.topk = d.top_k;
     p.Fe = d.expert_ffn;
@@ -239,18 +262,40 @@ mk::Params base_params(mk_state* s) {
     p.lm_arg = s->lm_arg;
     p.lm_garg = s->lm_garg;
     p.lm_cnt = s->lm_cnt;
+    p.tp = m->tp;
+    p.tp_rank = m->tp_rank;
+    p.tp_tiles = P.tp_tiles;
+    for (int q = 0; q < m->tp && q < mk::kMaxTp; ++q) {
+        char* b = static_cast<char*>(s->tp_peer[q]);
+        p.tp_recv[q] = reinterpret_cast<float*>(b);
+        p.tp_flag[q] = b ? reinterpret_cast<uint32_t*>(b + s->tp_recv_bytes) : nullptr;
+    }
     return p;
 }
 
-mk_status launch_step(mk_state* s, mk::Params& p, cudaStream_t st) {
+// Starts a step of `ncta` CTAs: the epoch and the queue base (the queue head moved
+// by tasks + CTAs in every earlier step since the last reset).
+mk_status begin_step(mk_state* s, mk::Params& p, int ncta, cudaStream_t st) {
+    if (s->ncta != ncta && s->epoch > 0) s->needs_reset = true;
     if (s->needs_reset) {
         mk_status r = reset_counters(s, st);
         if (r != MK_OK) return r;
     }
-    const GraphPlan& P = s->g->plan;
+    s->ncta = ncta;
     s->epoch += 1;
     p.epoch = s->epoch;
-    p.queue_base = (unsigned long long)(s->epoch - 1) * (P.tasks.size() + (size_t)P.n_sm);
+    p.queue_base = (unsigned long long)(s->epoch - 1) * (s->g->plan.tasks.size() + (size_t)ncta);
+    p.cta0 = 0;
+    p.ncta = ncta;
+    return MK_OK;
+}
+
+mk_status launch_step(mk_state* s, mk::Params& p, cudaStream_t st) {
+    const GraphPlan& P = s->g->plan;
+    if (P.tp > 1 && !tp_ready(s))
+        return fail(MK_ERR_INVALID_ARG, "tensor-parallel step: the peers' receive buffers are not all set");
+    mk_status r = begin_step(s, p, P.n_sm, st);
+    if (r != MK_OK) return r;
     cudaError_t e = mk::megakernel_launch(p, P.n_sm, st);
     if (e != cudaSuccess) {
         s->needs_reset = true;
@@ -278,9 +323,8 @@ mk_status mk_wave_stats(int n_tiles, int n_sm, int* waves, int* idle) {
 
 // ---------------------------------------------------------------- model
 
-mk_status mk_load_model(const mk_model_desc* desc, const void* const* wp, int n_ptrs, mk_model** out) {
-    if (!desc || !wp || !out) return fail(MK_ERR_INVALID_ARG, "mk_load_model: null argument");
-    *out = nullptr;
+static mk_status load_model(const mk_model_desc* desc, const void* const* wp, int n_ptrs, int tp, int tp_rank,
+                            int vocab_full, mk_model** out) {
     const mk_model_desc& d = *desc;
     std::string err;
     if (!mk::validate_desc(d, err)) return fail(MK_ERR_UNSUPPORTED, "mk_load_model: %s", err.c_str());
@@ -295,6 +339,9 @@ mk_status mk_load_model(const mk_model_desc* desc, const void* const* wp, int n_
     mk_model* m = new (std::nothrow) mk_model;
     if (!m) return fail(MK_ERR_OOM, "mk_load_model: host allocation");
     m->desc = d;
+    m->tp = tp;
+    m->tp_rank = tp_rank;
+    m->vocab_full = vocab_full;
     cudaGetDevice(&m->device);
     m->w.assign(wp, wp + n_ptrs);
     const int S = slots_per_layer(d);
@@ -332,6 +379,23 @@ mk_status mk_load_model(const mk_model_desc* desc, const void* const* wp, int n_
     return MK_OK;
 }
 
+mk_status mk_load_model(const mk_model_desc* desc, const void* const* wp, int n_ptrs, mk_model** out) {
+    if (!desc || !wp || !out) return fail(MK_ERR_INVALID_ARG, "mk_load_model: null argument");
+    *out = nullptr;
+    return load_model(desc, wp, n_ptrs, 1, 0, desc->vocab, out);
+}
+
+mk_status mk_load_model_tp(const mk_model_desc* desc, int tp_size, int tp_rank, const void* const* wp, int n_ptrs,
+                           mk_model** out) {
+    if (!desc || !wp || !out) return fail(MK_ERR_INVALID_ARG, "mk_load_model_tp: null argument");
+    *out = nullptr;
+    mk_model_desc d;
+    std::string err;
+    if (!mk::tp_shard_desc(*desc, tp_size, tp_rank, d, err))
+        return fail(MK_ERR_UNSUPPORTED, "mk_load_model_tp: %s", err.c_str());
+    return load_model(&d, wp, n_ptrs, tp_size, tp_rank, desc->vocab, out);
+}
+
 void mk_model_destroy(mk_model* m) {
     if (!m) return;
     if (m->d_layers) cudaFree(m->d_layers);
@@ -349,6 +413,24 @@ mk_status mk_plan_taskgraph(const mk_model_desc* desc, int max_batch, int max_ct
     if (!mk::plan_graph(*desc, max_batch, max_ctx, n_sm, g->plan, err)) {
         delete g;
         return fail(MK_ERR_UNSUPPORTED, "mk_plan_taskgraph: %s", err.c_str());
+    }
+    *out = g;
+    return MK_OK;
+}
+
+mk_status mk_plan_taskgraph_tp(const mk_model_desc* desc, int tp_size, int tp_rank, int max_ctx, int n_sm,
+                               mk_graph** out) {
+    if (!desc || !out) return fail(MK_ERR_INVALID_ARG, "mk_plan_taskgraph_tp: null argument");
+    *out = nullptr;
+    mk_model_desc d;
+    std::string err;
+    if (!mk::tp_shard_desc(*desc, tp_size, tp_rank, d, err))
+        return fail(MK_ERR_UNSUPPORTED, "mk_plan_taskgraph_tp: %s", err.c_str());
+    mk_graph* g = new (std::nothrow) mk_graph;
+    if (!g) return fail(MK_ERR_OOM, "mk_plan_taskgraph_tp: host allocation");
+    if (!mk::plan_graph(d, 1, max_ctx, n_sm, g->plan, err, tp_size)) {
+        delete g;
+        return fail(MK_ERR_UNSUPPORTED, "mk_plan_taskgraph_tp: %s", err.c_str());
     }
     *out = g;
     return MK_OK;
@@ -383,8 +465,13 @@ static mk_status build_graph(mk_model* model, int max_batch, int max_ctx, int so
     if (e != cudaSuccess) return cuda_fail(e, "mk_build_taskgraph: occupancy query");
     if (per_sm < 1) return fail(MK_ERR_UNSUPPORTED, "mk_build_taskgraph: megakernel does not fit on one SM");
     mk_graph* g = nullptr;
-    mk_status st = mk_plan_taskgraph(&d, max_batch, max_ctx, n_sm, &g);
-    if (st != MK_OK) return st;
+    g = new (std::nothrow) mk_graph;
+    if (!g) return fail(MK_ERR_OOM, "mk_build_taskgraph: host allocation");
+    std::string perr;
+    if (!mk::plan_graph(d, max_batch, max_ctx, n_sm, g->plan, perr, model->tp)) {
+        delete g;
+        return fail(MK_ERR_UNSUPPORTED, "mk_build_taskgraph: %s", perr.c_str());
+    }
     g->model = model;
     g->device = dev;
     if (solo_op && g->plan.bp > 0) {
@@ -492,6 +579,9 @@ mk_status mk_graph_export_tasks(const mk_graph* g, mk_task_info* out, int cap, i
         out[i].signal = T[i].sig;
         out[i].pointer_wait = T[i].pad;
         if (T[i].op == MK_OP_ATTN && (T[i].flags & mk::kAttnWide)) out[i].aux = -1;   // every KV head
+        // tensor parallelism: pad is a projection tile's ordinal (its arrival flag)
+        if (g->plan.tp > 1 && (T[i].op == MK_OP_OPROJ || T[i].op == MK_OP_DOWN || T[i].op == MK_OP_TP_REDUCE))
+            out[i].pointer_wait = MK_NO_EVENT;
         if (mk::is_mm_op(T[i].op)) {          // split s of a tile with nblk splits
             out[i].b = T[i].chunk_rows;
             out[i].aux = T[i].nblk;
@@ -584,6 +674,16 @@ mk_status mk_state_create(mk_graph* g, mk_state** out) {
     ALLOC(logits, B * (size_t)d.vocab);
     if (d.flags & MK_FLAG_TRACE) ALLOC(trace, P.tasks.size() * 4);
     if (d.flags & MK_FLAG_TRACE) ALLOC(stats, (size_t)P.n_sm * 8);
+    if (P.tp > 1 && st == MK_OK) {
+        // receive buffer (every rank's partial sums of both phases of every layer) and
+        // the arrival flags; the flags start at zero
+        s->tp_recv_bytes = sizeof(float) * (size_t)P.tp * L * 2 * H;
+        s->tp_bytes = s->tp_recv_bytes + sizeof(uint32_t) * L * 2 * (size_t)std::max(1, P.tp_tiles);
+        unsigned char* b = nullptr;
+        st = dev_alloc(s, &b, s->tp_bytes);
+        s->tp_buf = b;
+        s->tp_peer[g->model->tp_rank] = b;
+    }
 #undef ALLOC
     if (st != MK_OK) {
         free_state_memory(s);
@@ -648,6 +748,8 @@ mk_status mk_decode_step_per_op(mk_state* s, const int32_t* token_ids, const int
         return fail(MK_ERR_INVALID_ARG, "mk_decode_step_per_op: batch %d outside 1..%d", batch, s->g->plan.max_batch);
     mk_status r = check_kv(s, kv);
     if (r != MK_OK) return r;
+    if (s->g->plan.tp > 1)
+        return fail(MK_ERR_UNSUPPORTED, "mk_decode_step_per_op: tensor-parallel graphs run as one launch per step");
     cudaStream_t st = (cudaStream_t)stream;
     // counters from zero, epoch 1 in every launch: each launch's waits are met by the
     // launches before it on the stream, and the next megakernel step starts afresh
@@ -694,6 +796,8 @@ mk_status mk_generate(mk_state* s, const int32_t* first_tokens, const int32_t* p
         return fail(MK_ERR_INVALID_ARG, "mk_generate: null argument");
     if (batch < 1 || batch > s->g->plan.max_batch || n_steps < 1)
         return fail(MK_ERR_INVALID_ARG, "mk_generate: batch %d or steps %d out of range", batch, n_steps);
+    if (s->g->plan.tp > 1)
+        return fail(MK_ERR_UNSUPPORTED, "mk_generate: a tensor-parallel rank holds only its vocabulary shard");
     mk_status r = check_kv(s, kv);
     if (r != MK_OK) return r;
     cudaStream_t st = (cudaStream_t)stream;
@@ -805,6 +909,110 @@ mk_status mk_prefill_seq(mk_state* s, const int32_t* tokens, int n_tokens, int p
 mk_status mk_prefill(mk_state* s, const int32_t* tokens, int n_tokens, int seq_slot, const mk_paged_kv* kv,
                      float* last_logits, mk_stream stream) {
     return mk_prefill_seq(s, tokens, n_tokens, 0, seq_slot, kv, last_logits, stream);
+}
+
+// ---------------------------------------------------------------- tensor parallelism
+
+mk_status mk_state_tp_buffer(mk_state* s, void** base, size_t* bytes) {
+    if (!s || !base || !bytes) return fail(MK_ERR_INVALID_ARG, "mk_state_tp_buffer: null argument");
+    if (!s->tp_buf) return fail(MK_ERR_INVALID_ARG, "mk_state_tp_buffer: not a tensor-parallel state");
+    *base = s->tp_buf;
+    *bytes = s->tp_bytes;
+    return MK_OK;
+}
+
+mk_status mk_state_tp_set_peer(mk_state* s, int rank, void* peer_base) {
+    if (!s || !s->tp_buf) return fail(MK_ERR_INVALID_ARG, "mk_state_tp_set_peer: not a tensor-parallel state");
+    const mk_model* m = s->g->model;
+    if (rank < 0 || rank >= m->tp || rank == m->tp_rank || !peer_base || ((uintptr_t)peer_base & 15))
+        return fail(MK_ERR_INVALID_ARG, "mk_state_tp_set_peer: bad rank or pointer");
+    if (s->tp_ipc[rank] && s->tp_peer[rank]) cudaIpcCloseMemHandle(s->tp_peer[rank]);
+    s->tp_ipc[rank] = false;
+    s->tp_peer[rank] = peer_base;
+    return MK_OK;
+}
+
+mk_status mk_state_tp_ipc_handle(mk_state* s, void* handle_out) {
+    if (!s || !s->tp_buf || !handle_out) return fail(MK_ERR_INVALID_ARG, "mk_state_tp_ipc_handle: bad argument");
+    cudaIpcMemHandle_t h;
+    cudaError_t e = cudaIpcGetMemHandle(&h, s->tp_buf);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_state_tp_ipc_handle");
+    static_assert(sizeof(h) == MK_TP_IPC_HANDLE_BYTES, "IPC handle size");
+    std::memcpy(handle_out, &h, sizeof(h));
+    return MK_OK;
+}
+
+mk_status mk_state_tp_open_peer(mk_state* s, int rank, const void* handle) {
+    if (!s || !s->tp_buf || !handle) return fail(MK_ERR_INVALID_ARG, "mk_state_tp_open_peer: bad argument");
+    const mk_model* m = s->g->model;
+    if (rank < 0 || rank >= m->tp || rank == m->tp_rank)
+        return fail(MK_ERR_INVALID_ARG, "mk_state_tp_open_peer: bad rank");
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    void* ptr = nullptr;
+    cudaError_t e = cudaIpcOpenMemHandle(&ptr, h, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return cuda_fail(e, "mk_state_tp_open_peer");
+    if (s->tp_ipc[rank] && s->tp_peer[rank]) cudaIpcCloseMemHandle(s->tp_peer[rank]);
+    s->tp_peer[rank] = ptr;
+    s->tp_ipc[rank] = true;
+    return MK_OK;
+}
+
+mk_status mk_decode_step_tp_emulated(mk_state* const* states, int n, const int32_t* token_ids,
+                                     const int32_t* positions, const mk_paged_kv* const* kvs,
+                                     float* const* logits_out, mk_stream stream) {
+    if (!states || !token_ids || !positions || !kvs || !logits_out)
+        return fail(MK_ERR_INVALID_ARG, "mk_decode_step_tp_emulated: null argument");
+    if (n < 2 || n > mk::kMaxTpEmulated)
+        return fail(MK_ERR_INVALID_ARG, "mk_decode_step_tp_emulated: %d ranks (2..4 in one launch)", n);
+    int dev = 0, n_sm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    const int per = n_sm / n;
+    bool reset = false;
+    for (int r = 0; r < n; ++r) {
+        const mk_state* s = states[r];
+        if (!s || !s->tp_buf || !logits_out[r])
+            return fail(MK_ERR_INVALID_ARG, "mk_decode_step_tp_emulated: rank %d: not a tensor-parallel state", r);
+        const mk_model* m = s->g->model;
+        if (m->tp != n || m->tp_rank != r || s->g->device != dev)
+            return fail(MK_ERR_INVALID_ARG, "mk_decode_step_tp_emulated: state %d is not rank %d of %d on this device",
+                        r, r, n);
+        if (!tp_ready(s)) return fail(MK_ERR_INVALID_ARG, "mk_decode_step_tp_emulated: rank %d: peers not set", r);
+        mk_status st = check_kv(s, kvs[r]);
+        if (st != MK_OK) return st;
+        if (s->needs_reset || s->epoch != states[0]->epoch || (s->ncta != per && s->epoch > 0)) reset = true;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    mk::TpLaunch L;
+    std::memset(&L, 0, sizeof(L));
+    L.n = n;
+    for (int r = 0; r < n; ++r) {
+        mk_state* s = states[r];
+        if (reset) s->needs_reset = true;      // the ranks count their steps together
+        mk::Params p = base_params(s);
+        p.tokens = token_ids;
+        p.positions = positions;
+        p.pos_offset = 0;
+        p.batch = 1;
+        p.skip_lm = 0;
+        p.k_pages = static_cast<uint16_t*>(kvs[r]->k_pages);
+        p.v_pages = static_cast<uint16_t*>(kvs[r]->v_pages);
+        p.page_table = kvs[r]->page_table;
+        p.n_pages = kvs[r]->n_pages;
+        p.max_pages = kvs[r]->max_pages_per_seq;
+        p.logits = logits_out[r];
+        mk_status rs = begin_step(s, p, per, st);
+        if (rs != MK_OK) return rs;
+        p.cta0 = r * per;
+        L.r[r] = p;
+    }
+    cudaError_t e = mk::megakernel_launch_tp_emulated(L, per * n, st);
+    if (e != cudaSuccess) {
+        for (int r = 0; r < n; ++r) states[r]->needs_reset = true;
+        return cuda_fail(e, "mk_decode_step_tp_emulated: launch");
+    }
+    return MK_OK;
 }
 
 mk_status mk_sync(mk_state* s, mk_stream stream) {

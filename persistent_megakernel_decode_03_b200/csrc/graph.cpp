@@ -30,7 +30,8 @@ namespace {
 enum TensorKind { T_XIN = 1, T_QKV, T_O, T_XMID, T_ACT, T_ACTE, T_SEL, T_LOGITS,
                   T_PART,                     // wide attention: the splits' softmax partials
                   T_XQOP, T_XFOP, T_XLOP,     // bf16 hi/lo operands of batched tiles
-                  T_KV };                     // batched graphs: this step's K/V rows in the cache
+                  T_KV,                       // batched graphs: this step's K/V rows in the cache
+                  T_TPP };                    // tensor parallelism: a rank's partial sums (pushed to peers)
 
 struct Region {
     int tensor;         // encoded (kind, layer, slot)
@@ -119,7 +120,7 @@ bool validate_desc(const mk_model_desc& d, std::string& err) {
 }
 
 bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, GraphPlan& g,
-                std::string& err) {
+                std::string& err, int tp) {
     auto fail = [&](const std::string& m) { err = m; return false; };
     if (!validate_desc(d, err)) return false;
     const int L = d.n_layers, H = d.hidden, nq = d.n_q_heads, nkv = d.n_kv_heads, hd = d.head_dim;
@@ -129,12 +130,15 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     if (max_batch > 1 && moe) return fail("max_batch > 1 needs a dense model (MoE decode is batch 1)");
     if (max_ctx < 1 || max_ctx > (1 << 22)) return fail("max_ctx must be in 1..4194304");
     if (n_sm < 1) return fail("n_sm must be >= 1");
+    if (tp < 1 || tp > kMaxTp) return fail("tensor-parallel size must be in 1..8");
+    if (tp > 1 && (max_batch != 1 || moe)) return fail("tensor parallelism needs a dense model at batch 1");
 
     g = GraphPlan();
     g.desc = d;
     g.max_batch = max_batch;
     g.max_ctx = max_ctx;
     g.n_sm = n_sm;
+    g.tp = tp;
     const int B = max_batch;
     const int hpg = nq / nkv;
     const int64_t qkv_rows = (int64_t)(nq + 2 * nkv) * hd;
@@ -150,7 +154,7 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     // Long contexts at batch 1: one task per split covers every KV head (its pages'
     // blocks of all heads are contiguous: large copies), one wave of splits over the
     // SMs, and merge tasks per q head combine the splits.
-    g.wide_attn = (B == 1) && max_ctx >= kWideAttnCtx && kConsumerWarps % nkv == 0;   // warps per head
+    g.wide_attn = (B == 1) && tp == 1 && max_ctx >= kWideAttnCtx && kConsumerWarps % nkv == 0;   // warps per head
     int S = (B == 1) ? n_sm / (g.wide_attn ? 1 : nkv)
                      : (int)std::min<int64_t>(std::lround(4.0 * n_sm / (double)(B * nkv)), ceil_div(max_ctx, 1024));
     S = std::max(1, std::min<int>(S, (int)ceil_div(max_ctx, 64)));
@@ -265,6 +269,22 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
             }
     };
 
+    // tensor parallelism: the projection tiles since task `first` wrote this rank's
+    // partial sums of their rows (pushed to every rank); one reduce task per tile adds
+    // the ranks' parts and the residual into the residual stream.  The tile's ordinal
+    // (pad) names its arrival flag; the reduce task waits on that flag, not on an event.
+    auto tp_reduce = [&](int l, int phase, int first, int out_kind, int out_layer) {
+        const int last = (int)T.size();
+        int ord = 0;
+        for (int i = first; i < last; ++i, ++ord) {
+            T[i].pad = (uint32_t)ord;
+            int t = new_task(MK_OP_TP_REDUCE, l, 0, phase, T[i].r0, T[i].r1);
+            T[t].pad = (uint32_t)ord;
+            own_entity(t, {Region{tensor_key(out_kind, out_layer, 0), 0, B, (int64_t)T[i].r0, (int64_t)T[i].r1}});
+        }
+        g.tp_tiles = std::max(g.tp_tiles, ord);
+    };
+
     if (B > 1) {
         // ---- batched step: tensor-core tiles of 128 weight rows x all batch rows.
         // A tile's K range is cut into splits so that (tiles x splits) fills the SMs;
@@ -371,6 +391,16 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
         if (g.wide_attn) attn_wide(l);
         else
             for (int kh = 0; kh < nkv; ++kh) attn_group(l, kh);
+        if (tp > 1) {
+            int first = (int)T.size();
+            gemv_op(MK_OP_OPROJ, l, H, R_o, T_TPP, l, {all_rows(T_O, l, 0, (int64_t)nq * hd)});
+            tp_reduce(l, 0, first, T_XMID, l);
+            gemv_op(MK_OP_GATEUP, l, d.ffn, R_gu, T_ACT, l, {all_rows(T_XMID, l, 0, H)});
+            first = (int)T.size();
+            gemv_op(MK_OP_DOWN, l, H, R_dn, T_TPP, l, {all_rows(T_ACT, l, 0, d.ffn)});
+            tp_reduce(l, 1, first, T_XIN, l + 1);
+            continue;
+        }
         gemv_op(MK_OP_OPROJ, l, H, R_o, T_XMID, l, {all_rows(T_O, l, 0, (int64_t)nq * hd)});
         if (!moe) {
             gemv_op(MK_OP_GATEUP, l, d.ffn, R_gu, T_ACT, l, {all_rows(T_XMID, l, 0, H)});
@@ -518,6 +548,23 @@ bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, Gr
     wb += 2LL * H + 2LL * d.vocab * H;
     g.weight_bytes = wb;
     return true;
+}
+
+bool tp_shard_desc(const mk_model_desc& full, int tp, int rank, mk_model_desc& out, std::string& err) {
+    auto fail = [&](const std::string& m) { err = m; return false; };
+    if (!validate_desc(full, err)) return false;
+    if (tp < 2 || tp > kMaxTp) return fail("tensor-parallel size must be in 2..8");
+    if (rank < 0 || rank >= tp) return fail("tensor-parallel rank outside 0..tp-1");
+    if (full.n_experts > 0) return fail("tensor parallelism covers dense models");
+    if (full.n_kv_heads % tp) return fail("KV heads must divide evenly over the ranks");
+    if (full.ffn % tp || (full.ffn / tp) % 8) return fail("FFN rows per rank must be a multiple of 8");
+    if (full.vocab % tp) return fail("vocabulary rows must divide evenly over the ranks");
+    out = full;
+    out.n_q_heads = full.n_q_heads / tp;
+    out.n_kv_heads = full.n_kv_heads / tp;
+    out.ffn = full.ffn / tp;
+    out.vocab = full.vocab / tp;
+    return validate_desc(out, err);
 }
 
 void attach_weights(GraphPlan& g, const void* const* w) {

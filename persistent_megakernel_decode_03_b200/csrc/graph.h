@@ -26,6 +26,8 @@ struct GraphPlan {
     int mm_slots = 0;            // split partial-sum slots per layer (each bp x 128 floats)
     int mm_counters = 0;         // per-tile split arrival counters
     int n_lm_tiles = 0;          // LM-head tiles (numbered by their aux)
+    int tp = 1;                  // tensor-parallel ranks (desc holds this rank's shard shapes)
+    int tp_tiles = 0;            // row tiles of the residual stream per reduce phase
 };
 
 int64_t ceil_div(int64_t a, int64_t b);
@@ -34,7 +36,11 @@ int choose_tile_rows(int64_t rows, int64_t row_bytes, int n_blocks, int n_sm, in
                      int divide);
 bool validate_desc(const mk_model_desc& d, std::string& err);
 bool plan_graph(const mk_model_desc& d, int max_batch, int max_ctx, int n_sm, GraphPlan& g,
-                std::string& err);
+                std::string& err, int tp = 1);
+// The shapes of rank `rank`'s shard under tensor parallelism of `tp` ranks: q and
+// KV heads, FFN rows and LM-head (vocabulary) rows divided evenly; false (with the
+// reason) when the model does not divide.
+bool tp_shard_desc(const mk_model_desc& full, int tp, int rank, mk_model_desc& out, std::string& err);
 // Keeps only the tasks of operator `op` (all layers), without dependencies:
 // a list for timing and profiling one tile type alone.
 void make_solo(GraphPlan& g, int op);

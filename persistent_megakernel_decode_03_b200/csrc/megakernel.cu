@@ -198,6 +198,16 @@ __device__ __forceinline__ int ld_relaxed_int(const int* p) {
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Tensor-parallel arrival flags live in the receiving rank's memory and are raised
+// by every rank's GPU: system scope on both sides.
+__device__ __forceinline__ void red_release_add_sys(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.sys.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 // Arrival count with acquire-release semantics at GPU scope: publishes every write
 // that precedes it in causality order (cumulative release) and makes the other
 // arrivals' writes visible to what follows (acquire).  Returns the old value.
@@ -453,7 +463,7 @@ __device__ __forceinline__ bool wait_should_stop(const Params& p, Waiter& w) {
 // free ring slot, [1] consumer thread 0 waits for data, [2] dependency waits,
 // [3] kernel cycles, [4] tasks run, [5] signal-slot waits.
 __device__ __forceinline__ void stat_add(const Params& p, int i, unsigned long long v) {
-    if (p.stats) atomicAdd(&p.stats[(size_t)blockIdx.x * 8 + i], v);   // reduction, no return value
+    if (p.stats) atomicAdd(&p.stats[(size_t)(blockIdx.x - p.cta0) * 8 + i], v);   // reduction, no return value
 }
 
 __device__ __forceinline__ void wait_stat(const Params& p, int where, long long c0) {
@@ -468,7 +478,7 @@ __device__ bool mbar_wait_slow(const Params& p, uint64_t* bar, uint32_t parity, 
     const long long c0 = p.stats ? clock64() : 0;
     while (!mbar_try_wait(bar, parity)) {
         if (wait_should_stop(p, w)) {
-            if (ld_relaxed_int(p.err) == 0) set_error(p, kErrTimeout, -1, -1, where, (int)blockIdx.x);
+            if (ld_relaxed_int(p.err) == 0) set_error(p, kErrTimeout, -1, -1, where, (int)(blockIdx.x - p.cta0));
             wait_stat(p, where, c0);
             return false;
         }
@@ -511,7 +521,7 @@ __device__ __forceinline__ bool msync4(const Params& p, Smem& sm, uint32_t& phas
 __device__ __forceinline__ void seen_complete_wait(const Params& p, uint64_t* bar, uint32_t parity, int* abort_flag) {
     for (int i = 0; i < (1 << 22); ++i)
         if (mbar_try_wait(bar, parity)) return;
-    set_error(p, kErrFault, -1, -6, (int)parity, (int)blockIdx.x);
+    set_error(p, kErrFault, -1, -6, (int)parity, (int)(blockIdx.x - p.cta0));
     *abort_flag = 1;
 }
 
@@ -532,6 +542,21 @@ __device__ bool event_wait(const Params& p, uint32_t e, uint32_t target, int tas
     }
     if (p.stats && threadIdx.x == 0) stat_add(p, 2, (unsigned long long)(clock64() - c0));
     return ok;
+}
+
+// Spin (acquire, system scope) until a tensor-parallel arrival flag reaches target.
+// Single thread; bounded like every other wait.
+__device__ bool tp_flag_wait(const Params& p, const uint32_t* f, uint32_t target, int task) {
+    Waiter w{0, 0};
+    while (true) {
+        const uint32_t v = ld_acquire_sys(f);
+        if ((int32_t)(v - target) >= 0) return true;
+        if (wait_should_stop(p, w)) {
+            if (ld_relaxed_int(p.err) == 0) set_error(p, kErrTimeout, task, -11, (int)v, (int)target);
+            return false;
+        }
+        __nanosleep(32);
+    }
 }
 
 // ----------------------------------------------------------------------------- producer
@@ -891,7 +916,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
             }
         }
         const bool skip = (t.op == MK_OP_LMHEAD && p.skip_lm) || t.op == MK_OP_NORM || t.op == MK_OP_KVAPPEND ||
-                          t.op == MK_OP_ATTN_MERGE;
+                          t.op == MK_OP_ATTN_MERGE || t.op == MK_OP_TP_REDUCE;
         if (skip) {                                      // nothing to stream: a marker stage
             if (!pr_acquire(p, sm, ring)) { ok = false; break; }
             sm.info[ring.stage] = StageInfo{ti, 0, 0, 0, t};
@@ -970,7 +995,7 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
 __device__ void prefetch_loop(const Params& p, Smem& sm) {
     if (p.pf_dist == 0) return;
     const volatile int* claimed = &sm.pf_claimed;
-    for (uint32_t i = blockIdx.x; i < p.n_tasks; i += gridDim.x) {
+    for (uint32_t i = blockIdx.x - p.cta0; i < p.n_tasks; i += p.ncta) {
         Waiter w{0, 0};
         while (true) {
             const int c = *claimed;
@@ -2492,6 +2517,31 @@ __device__ __noinline__ void kvappend_task(const Params& p, const Task& t, int t
     }
 }
 
+// Tensor-parallel reduction of rows [r0, r1) of the residual stream (aux 0: after
+// attention, into x_mid; aux 1: after the FFN, into x_out): once every rank has
+// pushed its partial sums of these rows (the tile's arrival flag in this rank's
+// memory reaches tp per step), the parts are added in rank order and the residual
+// last -- every rank computes the same sums in the same order, so the replicated
+// residual stream stays bit-identical across ranks.  The reads go around L1: the
+// receive buffer is written by other GPUs.
+__device__ __noinline__ void tp_reduce_task(const Params& p, Smem& sm, uint32_t& cph, const Task& t, int ti) {
+    const int tid = threadIdx.x, l = t.layer, ph = t.aux;
+    if (tid == 0) {
+        const uint32_t* f = p.tp_flag[p.tp_rank] + ((size_t)l * 2 + ph) * p.tp_tiles + t.pad;
+        if (!tp_flag_wait(p, f, (uint32_t)p.tp * p.epoch + p.wait_offset, ti)) sm.flag[3] = 1;
+    }
+    // thread 0's acquire, then the consumers' barrier, before any thread reads the parts
+    csync(p, sm, cph);
+    if (sm.flag[3]) return;
+    const float* recv = p.tp_recv[p.tp_rank];
+    for (int r = (int)t.r0 + tid; r < (int)t.r1; r += kConsumerThreads) {
+        float y = 0.0f;
+        for (int q = 0; q < p.tp; ++q) y += __ldcg(recv + (((size_t)q * p.L + l) * 2 + ph) * p.H + r);
+        if (ph == 0) p.x_mid[((size_t)l * p.max_batch) * p.H + r] = x_in(p, l, 0, r) + y;
+        else p.x_out[((size_t)l * p.max_batch) * p.H + r] = x_mid_at(p, l, 0, r) + y;
+    }
+}
+
 // RMSNorm of one batch row into the operand of the next projection, by all 256
 // consumer threads: h = x / sqrt(mean(x^2) + eps) * g (kind 0: attention norm of
 // the residual entering layer l, the token embedding at l = 0; kind 1: FFN norm
@@ -2853,7 +2903,7 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
         }
         if (p.trace && tid == 0) {
             p.trace[(size_t)ti * 4 + 1] = globaltimer();
-            p.trace[(size_t)ti * 4 + 3] = (uint64_t)blockIdx.x;
+            p.trace[(size_t)ti * 4 + 3] = (uint64_t)(blockIdx.x - p.cta0);
         }
         const int buf = (int)(seq % kRedBufs);
         // buffer set `buf` is reused once the epilogue warp has finished the task that
@@ -2903,6 +2953,19 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
             continue;
         }
         }
+        if constexpr (!MM && !WIDE) {
+        if (t.op == MK_OP_TP_REDUCE) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[stage]);     // the marker stage
+            if (++stage == kStages) { stage = 0; ++lap; }
+            tp_reduce_task(p, sm, cph, t, ti);
+            if (sm.flag[3]) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.red_full[buf]);
+            ++seq;
+            continue;
+        }
+        }
         if (t.op == MK_OP_ATTN) {
             bool abort_all = false;
             if constexpr (WIDE) attention_wide_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
@@ -2943,7 +3006,7 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
             m = thread_map(g.K);
         }
         const int rows_total = g.rows * g.nblk;
-        const bool resid = !skip && warp == 0 && (t.op == MK_OP_OPROJ || t.op == MK_OP_DOWN);
+        const bool resid = !skip && warp == 0 && (t.op == MK_OP_OPROJ || t.op == MK_OP_DOWN) && p.tp <= 1;
         float resid0 = 0.0f, resid1 = 0.0f;
         if (!skip) {
             if (t.op == MK_OP_QKV && t.layer == 0 && tid == 0) {
@@ -3012,6 +3075,34 @@ __device__ __noinline__ void lmhead_argmax(const Params& p, const Task& t, int l
     argmax_arrive(p, t.aux, 1, lane);
 }
 
+// Row r of a finished GEMV task: the consumer warps' partial sums added in a fixed
+// order (bit-identical from run to run).
+__device__ __forceinline__ float gemv_row_sum(const Smem& sm, int buf, int r, int wpg) {
+    float y = 0.0f;
+    if (wpg == kConsumerWarps) {
+        const float4 a = *reinterpret_cast<const float4*>(&sm.red[buf][r][0]);
+        const float4 c = *reinterpret_cast<const float4*>(&sm.red[buf][r][4]);
+        y = a.x; y += a.y; y += a.z; y += a.w; y += c.x; y += c.y; y += c.z; y += c.w;
+    } else {
+        for (int w = 0; w < wpg; ++w) y += sm.red[buf][r][w];
+    }
+    return y;
+}
+
+// Tensor parallelism: a finished O- or down-projection tile's rows are this rank's
+// partial sums of those residual rows; each goes into every rank's receive buffer
+// at this rank's slot (plain stores; the peers' buffers are mapped into this GPU's
+// address space).  Out of line: the epilogue warp's register budget is small.
+__device__ __noinline__ void tp_store_tile(const Params& p, const Smem& sm, const Task& t, int rows, int wpg,
+                                           int buf, int lane) {
+    const int ph = (t.op == MK_OP_DOWN) ? 1 : 0;
+    const size_t base = (((size_t)p.tp_rank * p.L + t.layer) * 2 + ph) * p.H + t.r0;
+    for (int r = lane; r < rows; r += 32) {
+        const float y = gemv_row_sum(sm, buf, r, wpg);
+        for (int q = 0; q < p.tp; ++q) p.tp_recv[q][base + r] = y;
+    }
+}
+
 // Output rows of a finished GEMV task: the consumer warps' partial sums reduced in
 // a fixed order (bit-identical from run to run), then the operator's tail.
 __device__ __forceinline__ void gemv_store(const Params& p, const Smem& sm, const Task& t, const GemvGeom& g,
@@ -3019,17 +3110,7 @@ __device__ __forceinline__ void gemv_store(const Params& p, const Smem& sm, cons
     const int l = t.layer, b = t.b;
     const int rows_total = g.rows * g.nblk;
     const int nout = (g.nblk == 2) ? g.rows : rows_total;
-    auto row_sum = [&](int r) -> float {
-        float y = 0.0f;
-        if (wpg == kConsumerWarps) {
-            const float4 a = *reinterpret_cast<const float4*>(&sm.red[buf][r][0]);
-            const float4 c = *reinterpret_cast<const float4*>(&sm.red[buf][r][4]);
-            y = a.x; y += a.y; y += a.z; y += a.w; y += c.x; y += c.y; y += c.z; y += c.w;
-        } else {
-            for (int w = 0; w < wpg; ++w) y += sm.red[buf][r][w];
-        }
-        return y;
-    };
+    auto row_sum = [&](int r) -> float { return gemv_row_sum(sm, buf, r, wpg); };
     for (int r = lane; r < nout; r += 32) {
         const float y = row_sum(r);
         const int row = (int)t.r0 + r;
@@ -3095,7 +3176,10 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
                 gemv_geom(p, t, g, false);
                 const int wpg = is_warp_row(t.flags) ? 1
                                 : (t.flags != kFastNone) ? kConsumerWarps : thread_map(g.K).wpg;
-                gemv_store(p, sm, t, g, wpg, buf, lane);
+                if (p.tp > 1 && (t.op == MK_OP_OPROJ || t.op == MK_OP_DOWN))
+                    tp_store_tile(p, sm, t, g.rows, wpg, buf, lane);
+                else
+                    gemv_store(p, sm, t, g, wpg, buf, lane);
                 if (t.op == MK_OP_LMHEAD && p.argmax_out) lmhead_argmax(p, t, lane);
                 if (t.op == MK_OP_ROUTER) {
                     // arrival of this router tile (acquire-release: the warp barrier orders
@@ -3113,6 +3197,9 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
                     else evt = MK_NO_EVENT;
                 }
             }
+            // tensor parallelism: a projection tile raises its arrival flag on every rank
+            if (p.tp > 1 && (t.op == MK_OP_OPROJ || t.op == MK_OP_DOWN))
+                evt = kTpFlagBit | (((uint32_t)t.layer * 2u + (t.op == MK_OP_DOWN ? 1u : 0u)) * (uint32_t)p.tp_tiles + t.pad);
             evts[nb] = evt;
             tis[nb] = ti;
             ++nb;
@@ -3127,7 +3214,15 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
         __syncwarp();
         if (lane == 0) {
             for (int k = 0; k < nb; ++k) {
-                if (evts[k] != MK_NO_EVENT) red_release_add(&p.events[evts[k]], 1u);
+                if (evts[k] != MK_NO_EVENT) {
+                    if (evts[k] & kTpFlagBit) {
+                        // system-scope release: cumulative over the lanes' stores to the
+                        // peers' buffers (ordered before it by the warp barrier)
+                        for (int q = 0; q < p.tp; ++q) red_release_add_sys(p.tp_flag[q] + (evts[k] & ~kTpFlagBit), 1u);
+                    } else {
+                        red_release_add(&p.events[evts[k]], 1u);
+                    }
+                }
                 atomicAdd(p.done, 1u);
                 if (p.trace) p.trace[(size_t)tis[k] * 4 + 2] = globaltimer();
                 mbar_arrive(&sm.red_free[(seq - nb + k) % kRedBufs]);
@@ -3149,7 +3244,7 @@ __host__ __device__ constexpr bool splits_registers(bool mm, int dpl) { return !
 // cover every KV head (long contexts).  Each graph kind has its own instantiation,
 // so one kind's code never costs another registers.
 template <int HPG, int DPL, bool MM, bool WIDE>
-__global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
+__device__ __forceinline__ void megakernel_body(const Params& p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -3202,6 +3297,22 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     }
 }
 
+template <int HPG, int DPL, bool MM, bool WIDE>
+__global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ Params p) {
+    megakernel_body<HPG, DPL, MM, WIDE>(p);
+}
+
+// Tensor parallelism emulated on one GPU: the ranks' steps in one launch, the grid's
+// CTAs dealt out to the ranks in equal consecutive runs (rank r: CTAs
+// [r * per, (r + 1) * per)).  All CTAs are co-resident (a cooperative launch), so
+// a rank's reduce tasks waiting on another rank's tiles always make progress.
+template <int HPG, int DPL>
+__global__ void __launch_bounds__(kThreads, 1) megakernel_tp(const __grid_constant__ TpLaunch L) {
+    const int per = (int)gridDim.x / L.n;
+    const int r = min((int)blockIdx.x / per, L.n - 1);
+    megakernel_body<HPG, DPL, false, false>(L.r[r]);
+}
+
 // ----------------------------------------------------------------------------- host launch
 
 template <int HPG, int DPL>
@@ -3227,7 +3338,10 @@ static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream, bool
         if (splits_registers(p.mm != 0, DPL) && fa.numRegs < kMinLaunchRegs) return cudaErrorInvalidConfiguration;
         attr_set[kind] |= bit;
     }
-    void* args[] = {const_cast<Params*>(&p)};
+    Params q = p;                 // this launch's CTAs: all of the grid
+    q.cta0 = 0;
+    q.ncta = grid;
+    void* args[] = {&q};
     if (cooperative)
         return cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kThreads), args, sizeof(Smem), stream);
     return cudaLaunchKernel((const void*)kern, dim3(grid), dim3(kThreads), args, sizeof(Smem), stream);
@@ -3251,6 +3365,34 @@ cudaError_t megakernel_launch(const Params& p, int grid, cudaStream_t stream, bo
             case 2: return launch_t<2, 2>(p, grid, stream, cooperative);
             case 4: return launch_t<4, 2>(p, grid, stream, cooperative);
             case 8: return launch_t<8, 2>(p, grid, stream, cooperative);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <int HPG, int DPL>
+static cudaError_t launch_tp_t(const TpLaunch& L, int grid, cudaStream_t stream) {
+    auto kern = megakernel_tp<HPG, DPL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, (const void*)kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kMinLaunchRegs) return cudaErrorInvalidConfiguration;
+    void* args[] = {const_cast<TpLaunch*>(&L)};
+    return cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kThreads), args, sizeof(Smem), stream);
+}
+
+cudaError_t megakernel_launch_tp_emulated(const TpLaunch& L, int grid, cudaStream_t stream) {
+    if (L.n < 1 || L.n > kMaxTpEmulated || grid < L.n || grid % L.n) return cudaErrorInvalidValue;
+    const Params& p = L.r[0];
+    const int hpg = p.nq / p.nkv, dpl = p.hd / 32;
+    if (dpl == 4) {
+        switch (hpg) {
+            case 1: return launch_tp_t<1, 4>(L, grid, stream);
+            case 2: return launch_tp_t<2, 4>(L, grid, stream);
+            case 4: return launch_tp_t<4, 4>(L, grid, stream);
+            case 8: return launch_tp_t<8, 4>(L, grid, stream);
         }
     }
     return cudaErrorInvalidValue;

@@ -112,6 +112,12 @@ inline bool is_mm_op(int op) { return op >= MK_OP_MM_QKV && op <= MK_OP_MM_LMHEA
 constexpr int kWideAttnCtx = 32768;
 constexpr uint8_t kAttnWide = 1;       // Task::flags of a wide attention task
 
+// Tensor parallelism (dense batch-1 graphs): up to kMaxTp ranks; a launch that
+// emulates the ranks on one GPU runs up to kMaxTpEmulated of them side by side.
+constexpr int kMaxTp = 8;
+constexpr int kMaxTpEmulated = 4;
+constexpr uint32_t kTpFlagBit = 0x80000000u;   // epilogue: "raise tensor-parallel flag i" marker
+
 // Device task record (32 bytes).
 struct Task {
     uint8_t op;
@@ -220,6 +226,14 @@ struct Params {
     float* logits;
 
     int wide;                    // 1: the graph's attention tasks cover every KV head
+    int cta0, ncta;              // this step's CTAs: blockIdx.x - cta0 in [0, ncta) (several ranks
+                                 // share a launch when tensor parallelism is emulated)
+    // tensor parallelism: rank tp_rank of tp; the O- and down-projection tiles push
+    // their partial sums into every rank's receive buffer and raise the tile's flag
+    // there; reduce tasks wait on their own rank's flags and add the ranks in order
+    int tp, tp_rank, tp_tiles;
+    float* tp_recv[kMaxTp];      // rank q's receive buffer [tp][L][2][H]
+    uint32_t* tp_flag[kMaxTp];   // rank q's flags [L][2][tp_tiles]
     // batched projection tiles (max_batch > 1)
     int mm;                      // 1: the graph uses tensor-core tiles
     int bp;                      // padded batch: the MMA's N (16, 32 or 64)
@@ -237,6 +251,12 @@ struct Params {
     ArgVal* lm_arg;              // [n_lm_tiles * kArgParts][max_batch]
     ArgVal* lm_garg;             // [groups][max_batch]
     uint32_t* lm_cnt;            // [groups + 1] arrivals: per group, then of the groups
+};
+// The launch parameters of emulated tensor parallelism: the ranks' parameter
+// blocks; the grid's CTAs are shared out among them.
+struct TpLaunch {
+    Params r[kMaxTpEmulated];
+    int n;
 };
 // Parts per LM-head tile (a batched tile reduces its 128 rows in 4 warps) and tiles
 // per reduction group of the in-step argmax.

@@ -25,6 +25,14 @@ Long-context batch-1 graphs ("wide" attention, exported with aux = -1):
 For MoE models x_in[l+1][i] is x_mid[l][i] combined with ypart[l][k][i] for all k
 and the routing weights sel[l].
 
+Tensor-parallel batch-1 graphs (run_tp: every rank's list, each rank its own tensors):
+  oproj    reads part[l] (all)                 writes recv[q][r, l, 0][rows] on EVERY rank q
+           (r = this rank) and raises flag[q][l, 0, rows] there
+  down     reads act[l] (all)                  the same with phase 1
+  tp_reduce  (aux = phase) runs once flag[r][l, aux, rows] == tp; reads recv[r][q, l, aux][rows]
+           for every q and x_in[l][rows] (aux 0) or x_mid[l][rows] (aux 1); writes x_mid[l][rows]
+           (aux 0) or x_in[l+1][rows] (aux 1)
+
 Batched graphs (tensor-core tiles; x_in, x_mid hold B rows of H):
   norm     reads its batch rows [r0, r1) of x_in[l] (aux 0), x_mid[l] (aux 1)
            or x_in[L] (aux 2)              writes those rows of opq[l] / opf[l] / opl
@@ -48,7 +56,7 @@ import numpy as np
 
 OP = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "router",
       8: "exp_gu", 9: "exp_dn", 10: "norm", 11: "mm_qkv", 12: "mm_oproj", 13: "mm_gu", 14: "mm_down",
-      15: "mm_lm", 16: "kvappend", 17: "attn_merge"}
+      15: "mm_lm", 16: "kvappend", 17: "attn_merge", 18: "tp_reduce"}
 NO_EVENT = 0xFFFFFFFF
 M64 = (1 << 64) - 1
 
@@ -291,3 +299,123 @@ def run(tasks, thr: List[int], shape: dict, seed: int) -> Dict[str, np.ndarray]:
     if not T[("logits",)].ok.all():
         raise Violation("logits not fully written")
     return {"logits": T[("logits",)].val.copy()}
+
+
+def run_tp(rank_tasks, rank_thr, shape: dict, tp: int, seed: int, workers: int = 4, ahead: int = 2):
+    """Executes the ranks' task lists together, the way the kernels claim them: each
+    rank has `workers` CTAs taking tasks from its own list IN ORDER, each holding up
+    to `ahead` claimed tasks and running only the oldest (a CTA finishes its tasks
+    in claim order).  Every step picks a random (rank, CTA) that can move.  Raises
+    Violation on a read of unwritten data, a double write, or a deadlock (tasks
+    left, no CTA can move).  Returns each rank's logits digests."""
+    L, H, nq, nkv, hd = shape["L"], shape["H"], shape["nq"], shape["nkv"], shape["hd"]
+    F, V = shape["F"], shape["V"]
+    hpg = nq // nkv
+    qkv_rows = (nq + 2 * nkv) * hd
+    rng = random.Random(seed)
+    T = []
+    for r in range(tp):
+        d = {("x_in", 0): Tensor(H, ready=True)}
+        for l in range(L):
+            d[("qkv", l)] = Tensor(qkv_rows)
+            d[("part", l)] = Tensor(nkv * 4096)
+            d[("x_mid", l)] = Tensor(H)
+            d[("act", l)] = Tensor(F)
+            d[("x_in", l + 1)] = Tensor(H)
+            for q in range(tp):
+                for ph in range(2):
+                    d[("recv", q, l, ph)] = Tensor(H)
+        d[("logits",)] = Tensor(V)
+        T.append(d)
+    flags = [defaultdict(int) for _ in range(tp)]
+    counters = [[0] * len(th) for th in rank_thr]
+    splits = [{tk.layer: tk.r1 for tk in tasks if tk.op == 2} for tasks in rank_tasks]
+    nxt = [0] * tp                                   # next unclaimed task of each rank
+    held = [[[] for _ in range(workers)] for _ in range(tp)]
+    done = [0] * tp
+
+    def ready(r: int, i: int) -> bool:
+        tk = rank_tasks[r][i]
+        for e in (tk.wait[0], tk.wait[1]):
+            if e != NO_EVENT and counters[r][e] < rank_thr[r][e]:
+                return False
+        if OP[tk.op] == "tp_reduce" and flags[r][(tk.layer, tk.aux, tk.r0)] < tp:
+            return False
+        return True
+
+    def execute(r: int, i: int) -> None:
+        tk = rank_tasks[r][i]
+        t = T[r]
+        op, l, r0, r1 = OP[tk.op], tk.layer, tk.r0, tk.r1
+        who = f"rank {r} task {i} ({op} l{l} aux{tk.aux} {r0}:{r1})"
+        base = _mix(i + 1)
+        if op == "qkv":
+            t[("qkv", l)].write(r0, r1, _mix(base ^ t[("x_in", l)].read(0, H, who)), who)
+        elif op == "attn":
+            g = tk.aux
+            qkv = t[("qkv", l)]
+            d = qkv.read(g * hpg * hd, (g + 1) * hpg * hd, who)
+            d += qkv.read(nq * hd + g * hd, nq * hd + (g + 1) * hd, who)
+            d += qkv.read((nq + nkv) * hd + g * hd, (nq + nkv) * hd + (g + 1) * hd, who)
+            t[("part", l)].write(g * 4096 + r0, g * 4096 + r0 + 1, _mix(base ^ (d & M64)), who)
+        elif op in ("oproj", "down"):
+            ph = 0 if op == "oproj" else 1
+            if ph == 0:
+                d = 0
+                for g in range(nkv):
+                    d += t[("part", l)].read(g * 4096, g * 4096 + splits[r][l], who)
+            else:
+                d = t[("act", l)].read(0, F, who)
+            for q in range(tp):
+                T[q][("recv", r, l, ph)].write(r0, r1, _mix(base ^ (d & M64)), who)
+                flags[q][(l, ph, r0)] += 1
+                if flags[q][(l, ph, r0)] > tp:
+                    raise Violation(f"{who}: flag raised beyond tp")
+        elif op == "tp_reduce":
+            d = 0
+            for q in range(tp):
+                d += t[("recv", q, l, tk.aux)].read(r0, r1, who)
+            if tk.aux == 0:
+                d += t[("x_in", l)].read(r0, r1, who)
+                t[("x_mid", l)].write(r0, r1, _mix(d & M64), who)
+            else:
+                d += t[("x_mid", l)].read(r0, r1, who)
+                t[("x_in", l + 1)].write(r0, r1, _mix(d & M64), who)
+        elif op == "gateup":
+            t[("act", l)].write(r0, r1, _mix(base ^ t[("x_mid", l)].read(0, H, who)), who)
+        elif op == "lmhead":
+            t[("logits",)].write(r0, r1, _mix(base ^ t[("x_in", L)].read(0, H, who)), who)
+        else:
+            raise Violation(f"{who}: not an operator of a tensor-parallel graph")
+        e = tk.signal
+        if e != NO_EVENT:
+            counters[r][e] += 1
+            if counters[r][e] > rank_thr[r][e]:
+                raise Violation(f"{who}: event {e} signalled beyond its threshold")
+        done[r] += 1
+
+    total = sum(len(x) for x in rank_tasks)
+    while sum(done) < total:
+        moves = []
+        for r in range(tp):
+            for w in range(workers):
+                h = held[r][w]
+                if len(h) < ahead and nxt[r] < len(rank_tasks[r]):
+                    moves.append((r, w, "claim"))
+                if h and ready(r, h[0]):
+                    moves.append((r, w, "run"))
+        if not moves:
+            raise Violation(f"deadlock: {sum(done)} of {total} tasks ran")
+        r, w, kind = moves[rng.randrange(len(moves))]
+        if kind == "claim":
+            held[r][w].append(nxt[r])
+            nxt[r] += 1
+        else:
+            execute(r, held[r][w].pop(0))
+    for r in range(tp):
+        for e, (c, th) in enumerate(zip(counters[r], rank_thr[r])):
+            if c != th:
+                raise Violation(f"rank {r} event {e}: counter {c} != threshold {th}")
+        if not T[r][("logits",)].ok.all():
+            raise Violation(f"rank {r}: logits not fully written")
+    return [T[r][("logits",)].val.copy() for r in range(tp)]
