@@ -305,6 +305,9 @@ struct __align__(128) Smem {
     int mm_last;                             // this CTA's split of a tile arrived last
     int pid[kPidRing];                       // producer: physical page ids read ahead
     int pf_claimed;                          // producer's latest claimed task (-1: finished), for the prefetcher
+    int pf_wait;                             // 1 while consumer warp 0 waits on a dependency (the prefetcher runs)
+    int started;                             // latest task the consumers have started (past its event wait)
+    int attn_hold;                           // this step's attention splits hold the next claim (-1: not yet known)
     int flag[4];
 };
 
@@ -652,6 +655,10 @@ __device__ __noinline__ bool produce_wide_pages(const Params& p, Smem& sm, const
     return true;
 }
 
+// Attention splits of at least this many ring stages hold the producer's next claim
+// until the consumers start them.
+constexpr int kHoldStages = 6;
+
 // Tasks whose streamed data is only known on the device: attention (KV pages of
 // this step's positions) and routed experts (weights of the expert the router
 // picked).  Out of line: it keeps the producer's hot loop small.
@@ -882,6 +889,56 @@ __device__ __noinline__ bool produce_mm(const Params& p, Smem& sm, const Task& t
     return true;
 }
 
+// Whether this step's attention splits hold the producer's next claim (see
+// producer_loop): batched graphs' splits (ragged, long contexts) always; a batch-1
+// step's splits when its first split streams kHoldStages stages or more (all its
+// splits are equal to within a page).  Decided once per step, so that no attention
+// task's claim waits on a load of the position.  (Wide steps always hold.)
+template <bool MM>
+__device__ __forceinline__ bool attn_hold_this_step(const Params& p) {
+    if (MM) return true;
+    const int pos = position_of(p, 0);
+    if (pos < 0 || pos >= p.max_ctx) return false;
+    const int sa = attn_active_splits(pos + 1, p.S);
+    int j0, j1;
+    attn_range(pos + 1, sa, 0, j0, j1);
+    const int jc = min(j1, pos);
+    if (jc <= j0) return false;
+    const int npages = (jc - 1) / kPageSize - j0 / kPageSize + 1;
+    const int pps = pages_per_stage(p);
+    return (npages + pps - 1) / pps >= kHoldStages;
+}
+
+// Producer: waits (bounded) until the consumers have started task ti.
+__device__ bool wait_started(const Params& p, Smem& sm, int ti) {
+    const volatile int* st = &sm.started;
+    Waiter w{0, 0};
+    while (*st < ti) {
+        if (*reinterpret_cast<volatile int*>(&sm.flag[3])) return false;
+        if (wait_should_stop(p, w)) {
+            if (ld_relaxed_int(p.err) == 0) set_error(p, kErrTimeout, ti, -12, 0, (int)(blockIdx.x - p.cta0));
+            return false;
+        }
+        __nanosleep(32);
+    }
+    return true;
+}
+
+// An attention task of a step whose splits hold: its pages, then a wait until the
+// consumers have started it (the caller claims the next task after that).
+template <bool MM, bool WIDE>
+__device__ __forceinline__ bool produce_attention_held(const Params& p, Smem& sm, const Task& t, int ti, PRing& ring,
+                                                    uint64_t pol) {
+    bool ok;
+    if (WIDE && (t.flags & kAttnWide)) {
+        ok = produce_wide_pages(p, sm, t, ti, ring, pol);
+    } else {
+        uint32_t no_router = MK_NO_EVENT;
+        ok = produce_special<MM>(p, sm, t, ti, ring, no_router, pol);
+    }
+    return ok && wait_started(p, sm, ti);
+}
+
 template <bool MM, bool WIDE>
 __device__ void producer_loop(const Params& p, Smem& sm) {
     const uint64_t pol = l2_evict_first_policy();
@@ -891,6 +948,16 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
     // The next task is claimed while the current one's copies are issued, so the
     // atomic's round trip overlaps useful work.  Still exactly one failing claim
     // per CTA, which keeps the queue head at (n_tasks + grid) per step.
+    // In the batched and long-attention kernels, attention tasks are the exception
+    // when this step's splits are long (kHoldStages ring stages or more, every wide
+    // split; attn_hold_this_step): after issuing one, the producer claims the next
+    // task only once the consumers have started it.  Otherwise a CTA that reaches a
+    // layer's attention early claims two or three of its tasks (their pages fit the
+    // ring) and runs them one after another while other CTAs, whose next claims are
+    // the O-projection tiles waiting for all attention, stay idle (30B MoE at an
+    // 8192-token context: 6.37 -> 5.7 ms per step; 8B at 131072 tokens: 13.74 ->
+    // 10.8 ms).
+    if constexpr (MM || WIDE) sm.attn_hold = -1;     // decided at the step's first attention task
     unsigned long long q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
     uint32_t n_claimed = 0;
     while (ok) {
@@ -902,6 +969,15 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
         const int ti = (int)q;
         *reinterpret_cast<volatile int*>(&sm.pf_claimed) = ti;
         const Task t = p.tasks[ti];
+        if constexpr (MM || WIDE) {
+            // a step whose attention splits hold: the claim after an attention task
+            // waits until the consumers have started it
+            if (sm.attn_hold > 0 && t.op == MK_OP_ATTN) {
+                ok = produce_attention_held<MM, WIDE>(p, sm, t, ti, ring, pol);
+                if (ok) q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
+                continue;
+            }
+        }
         q_next = atomicAdd(p.queue, 1ull) - p.queue_base;
         if constexpr (MM) {
             if (is_mm_op(t.op)) {
@@ -910,7 +986,8 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
             }
         }
         if constexpr (WIDE) {
-            if (t.op == MK_OP_ATTN) {
+            if (t.op == MK_OP_ATTN && (t.flags & kAttnWide)) {
+                sm.attn_hold = 1;                            // every wide step holds
                 ok = produce_wide_pages(p, sm, t, ti, ring, pol);
                 continue;
             }
@@ -925,6 +1002,10 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
             continue;
         }
         if (t.nchunks == 0 || t.op == MK_OP_ATTN) {
+            if constexpr (MM || WIDE) {
+                // (the step's first attention task decides whether its splits hold)
+                if (t.op == MK_OP_ATTN && sm.attn_hold < 0) sm.attn_hold = attn_hold_this_step<MM>(p) ? 1 : 0;
+            }
             ok = produce_special<MM>(p, sm, t, ti, ring, last_router_evt, pol);
             continue;
         }
@@ -985,25 +1066,32 @@ __device__ void producer_loop(const Params& p, Smem& sm) {
 // ----------------------------------------------------------------------------- L2 prefetcher
 
 // Asks L2 to fetch the weight rows (and KV pages) of tasks a bounded distance
-// ahead of the work queue, so HBM could keep streaming while the consumers wait
-// on a dependency.  The task list is dealt to the CTAs statically (CTA c takes
-// tasks c, c + grid, ...), and the distance is measured against this CTA's own
-// latest claim (shared memory), which tracks the global queue head within a
-// wave: no atomics and no polling of global memory.  Off by default: every
-// distance measured slower than none.  Routed-expert weights are unknown until
-// the router runs and are skipped.
+// ahead of the work queue, so that HBM keeps streaming while this CTA's consumers
+// wait on a dependency (at an operator boundary the ring holds the next tile, and
+// HBM would otherwise idle until the event fires).  It issues prefetches ONLY while
+// consumer warp 0 is waiting: at any other time the stream is HBM-bound already and
+// a prefetch would only compete with the tiles the next event waits for.  The task
+// list is dealt to the CTAs statically (CTA c covers tasks c, c + grid, ...; the
+// union over the CTAs covers every task of the window whoever claims it), tasks
+// already claimed are skipped, and the window ends pf_dist tasks past this CTA's
+// latest claim (shared memory): no atomics and no polling of global memory.
+// Routed-expert weights are unknown until the router runs and are skipped.
 __device__ void prefetch_loop(const Params& p, Smem& sm) {
     if (p.pf_dist == 0) return;
     const volatile int* claimed = &sm.pf_claimed;
+    const volatile int* waiting = &sm.pf_wait;
     for (uint32_t i = blockIdx.x - p.cta0; i < p.n_tasks; i += p.ncta) {
         Waiter w{0, 0};
+        bool skip = false;
         while (true) {
             const int c = *claimed;
             if (c < 0 || *reinterpret_cast<volatile int*>(&sm.flag[3])) return;   // producer done or aborting
-            if ((uint32_t)c + p.pf_dist >= i) break;
+            if (i <= (uint32_t)c) { skip = true; break; }                         // claimed: streaming already
+            if ((uint32_t)c + p.pf_dist >= i && *waiting) break;
             if (wait_should_stop(p, w)) return;          // an error elsewhere; a slow step is not one
-            __nanosleep(128);
+            __nanosleep(64);
         }
+        if (skip) continue;
         const Task t = p.tasks[i];
         if (t.op == MK_OP_ATTN) {
             const int b = t.b;
@@ -2892,7 +2980,9 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
         if (e != MK_NO_EVENT && e != ok_evt[0] && e != ok_evt[1] && e != ok_evt[2] && e != ok_evt[3]) {
             int r = 1;
             if (lane == 0) {
+                if (warp == 0) *reinterpret_cast<volatile int*>(&sm.pf_wait) = 1;   // the prefetcher may run
                 r = event_wait(p, e, p.thr[e] * p.epoch + p.wait_offset, ti) ? 1 : 0;
+                if (warp == 0) *reinterpret_cast<volatile int*>(&sm.pf_wait) = 0;
             }
             // lane 0's acquire, then the warp barrier (which orders memory among its
             // lanes), before any lane reads what the event's producers wrote
@@ -2901,6 +2991,7 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
             if (!r) { sm.flag[3] = 1; break; }
             ok_evt[3] = ok_evt[2]; ok_evt[2] = ok_evt[1]; ok_evt[1] = ok_evt[0]; ok_evt[0] = e;
         }
+        if (tid == 0) *reinterpret_cast<volatile int*>(&sm.started) = ti;   // the producer may claim on
         if (p.trace && tid == 0) {
             p.trace[(size_t)ti * 4 + 1] = globaltimer();
             p.trace[(size_t)ti * 4 + 3] = (uint64_t)(blockIdx.x - p.cta0);
@@ -2968,7 +3059,7 @@ __device__ __forceinline__ void consumer_loop(const Params& p, Smem& sm) {
         }
         if (t.op == MK_OP_ATTN) {
             bool abort_all = false;
-            if constexpr (WIDE) attention_wide_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
+            if (WIDE && (t.flags & kAttnWide)) attention_wide_task<HPG, DPL>(p, sm, cph, t, ti, stage, lap, abort_all);
             else attention_task<HPG, DPL, MM>(p, sm, cph, t, ti, stage, lap, abort_all);
             if (abort_all) break;
             x_key_op = -1;
@@ -3240,9 +3331,12 @@ __device__ void epilogue_loop(const Params& p, Smem& sm) {
 // 64-wide heads need fewer than the launch allows, and ptxas launches them with less.
 __host__ __device__ constexpr bool splits_registers(bool mm, int dpl) { return !mm || dpl == 4; }
 
-// MM: batched graphs (tensor-core tiles); WIDE: batch-1 graphs whose attention tasks
-// cover every KV head (long contexts).  Each graph kind has its own instantiation,
-// so one kind's code never costs another registers.
+// MM: batched graphs (tensor-core tiles); WIDE: batch-1 graphs with a long attention
+// phase -- attention tasks that cover every KV head (long contexts) or MoE graphs --
+// whose steps may hold the producer's claims after attention tasks.  Each graph
+// kind has its own instantiation, so one kind's code never costs another registers
+// (the dense batch-1 kernel keeps the plain claim loop: the hold logic in it cost
+// the 8B step 2% even where no split held).
 template <int HPG, int DPL, bool MM, bool WIDE>
 __device__ __forceinline__ void megakernel_body(const Params& p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -3266,6 +3360,8 @@ __device__ __forceinline__ void megakernel_body(const Params& p) {
         }
         for (int i = 0; i < 4; ++i) sm.flag[i] = 0;
         sm.pf_claimed = 0;
+        sm.pf_wait = 0;
+        sm.started = -1;
         // the 128-byte-swizzled tensor-core operands need 1 KB-aligned stages
         if (p.mm && (smem_u32(sm.ring) & 1023u) != 0) {
             set_error(p, kErrFault, -1, -9, (int)(smem_u32(sm.ring) & 1023u), 0);
@@ -3317,9 +3413,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel_tp(const __grid_consta
 
 template <int HPG, int DPL>
 static cudaError_t launch_t(const Params& p, int grid, cudaStream_t stream, bool cooperative) {
-    const int kind = p.mm ? 1 : (p.wide ? 2 : 0);
+    const bool long_attn = p.wide || p.E > 0;
+    const int kind = p.mm ? 1 : (long_attn ? 2 : 0);
     auto kern = p.mm ? megakernel<HPG, DPL, true, false>
-                     : (p.wide ? megakernel<HPG, DPL, false, true> : megakernel<HPG, DPL, false, false>);
+                     : (long_attn ? megakernel<HPG, DPL, false, true> : megakernel<HPG, DPL, false, false>);
     // the shared-memory attribute, once per instantiation and device (so that a step
     // can be captured into a CUDA graph without host-side calls in between)
     // (devices 0..63 are remembered; a higher index sets the attribute every launch)
