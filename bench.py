@@ -680,6 +680,73 @@ def run_solo(args, W):
     dec.close()
 
 
+def run_trace(args, W):
+    """Per-task timestamps of a few steps (the state's trace flag): for each operator,
+    the time its tasks waited on their dependency events, summed per SM; and for a
+    middle layer, when each operator's first task started and its last task ended.
+    The gap between one operator's last end and the next one's first start is the
+    boundary cost the persistent kernel pays.  Timestamps are the GPU's global
+    timer (ns) taken by the consumer warps (claim seen, dependency met) and the
+    epilogue warp (signalled).  Evidence for where a step's time goes; not the
+    metric (tracing slows the step a little)."""
+    import numpy as np
+    import torch
+    import synthetic as syn
+    import persistent_megakernel_decode_03_b200 as mk
+    from persistent_megakernel_decode_03_b200.runner import Decoder
+
+    cfg = W["cfg"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    seed = syn.SEED_WEIGHTS + W["seed"]
+    ts = []
+    for s in syn.tensor_specs(cfg):
+        t = torch.empty(s.shape, dtype=torch.bfloat16, device=dev)
+        syn.dev_fill_tensor(t, s, seed)
+        ts.append(t)
+    desc = dict(n_layers=cfg.n_layers, hidden=cfg.hidden, n_q_heads=cfg.n_q_heads,
+                n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, ffn=cfg.ffn, vocab=cfg.vocab,
+                rms_eps=cfg.rms_eps, rope_theta=cfg.rope_theta, n_experts=cfg.n_experts, top_k=cfg.top_k,
+                expert_ffn=cfg.expert_ffn, moe_renorm=cfg.moe_renorm, flags=mk.MK_FLAG_TRACE)
+    n_steps = 4
+    ctx = W["prompt"] + max(0, min(60, W["gen"] - n_steps - 1))
+    dec = Decoder(desc, [t.data_ptr() for t in ts], 1, W["prompt"] + W["gen"], device="cuda:0")
+    tok = torch.tensor([7], dtype=torch.int32, device=dev)
+    ms = []
+    for i in range(n_steps):
+        pos = torch.tensor([ctx + i], dtype=torch.int32, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dec.step(tok, pos)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms.append(e0.elapsed_time(e1))
+    dec.check()
+    tasks = mk.mk_graph_export_tasks(dec.graph)
+    tr = np.array(mk.mk_state_read_trace(dec.state, dec.info.n_tasks), dtype=np.uint64)
+    tr = tr.reshape(-1, 4).astype(np.int64)        # seen, go, signalled (ns), CTA of the last step
+    ops = np.array([t.op for t in tasks])
+    layers = np.array([t.layer for t in tasks])
+    t0 = tr[:, 0].min()
+    n_cta = int(tr[:, 3].max()) + 1
+    wait_us = (tr[:, 1] - tr[:, 0]) / 1e3
+    out = {"trace": W["desc"], "position": ctx + len(ms) - 1, "step_ms_traced": ms[-1],
+           "makespan_us": float(tr[:, 2].max() - t0) / 1e3, "ops": {}, "layer": {}}
+    for op in sorted(set(ops.tolist())):
+        m = ops == op
+        out["ops"][mk.OP_NAMES[op]] = {"tasks": int(m.sum()), "dep_wait_us_per_sm": float(wait_us[m].sum() / n_cta),
+                                       "mean_wait_us": float(wait_us[m].mean())}
+    l = cfg.n_layers // 2
+    for op in sorted(set(ops[layers == l].tolist())):
+        m = (ops == op) & (layers == l)
+        out["layer"][mk.OP_NAMES[op]] = {"first_go_us": float((tr[m, 1].min() - t0) / 1e3),
+                                         "last_end_us": float((tr[m, 2].max() - t0) / 1e3),
+                                         "median_go_to_end_us": float(np.median((tr[m, 2] - tr[m, 1]) / 1e3))}
+    out["layer_index"] = l
+    print(json.dumps(out), flush=True)
+    dec.close()
+
+
 def kernel_source_sha() -> str:
     import hashlib
     h = hashlib.sha256()
@@ -708,6 +775,8 @@ def main(argv=None):
                     help="time greedy generation with the device-side loop beside a host loop instead")
     ap.add_argument("--per-op", action="store_true",
                     help="time the kernel-per-operator baseline of the step beside the megakernel instead")
+    ap.add_argument("--trace", action="store_true",
+                    help="print the per-operator dependency waits and one layer's timeline from the kernel's task trace")
     ap.add_argument("--prefill", action="store_true",
                     help="time the 39-token prompt's prefill (batched vs token by token) instead")
     ap.add_argument("--ref-budget", type=float, default=120.0,
@@ -722,6 +791,8 @@ def main(argv=None):
         W["desc"] += f" [first {W['cfg'].n_layers} layers only: profiling case]"
     if args.solo:
         run_solo(args, W)
+    elif args.trace:
+        run_trace(args, W)
     elif args.prefill:
         run_prefill(args, W)
     elif args.per_op:
