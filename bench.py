@@ -356,7 +356,7 @@ def run_gpu(args, W):
     # end to end through the host-buffer entry point: H2D of token+position, D2H of logits
     e2e = None
     if not args.no_e2e:
-        k_e2e = min(args.steps, 100)
+        k_e2e = args.steps                 # the same steps (positions) as the timed region
         tok_h = torch.tensor(gen_toks, dtype=torch.int32).pin_memory()
         pos_h = torch.tensor(positions, dtype=torch.int32).pin_memory()
         logits_h = torch.empty((B, cfg.vocab), dtype=torch.float32).pin_memory()

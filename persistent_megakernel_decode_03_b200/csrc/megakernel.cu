@@ -421,14 +421,21 @@ __device__ __forceinline__ int gemv_chunks(const GemvGeom& g, uint8_t flags) {
     return per_blk * g.nblk;
 }
 
-// Splits of one (sequence, kv head) actually used this step: about one per
-// kAttnSplitTokens positions of context, at most the graph's split count S.  A
-// context of up to kAttnSplitTokens positions is one split that writes the
-// normalised output itself: no merge step (measured at 8B, position 300: 3.54 ms
-// per step against 3.73 ms with 64-position splits and their merge).
-constexpr int kAttnSplitTokens = 512;
+// Splits of one (sequence, kv head) actually used this step, at most the graph's
+// split count S (one wave of tasks over the SMs):
+//  - up to kAttnLongCtx positions, one split per kAttnShortSplit positions: a
+//    context of up to 512 is one split that writes the normalised output itself,
+//    with no merge step (8B, position 300: 3.54 ms per step against 3.73 ms with
+//    64-position splits and their merge);
+//  - longer contexts, one split per kAttnSplitTokens positions, so that every SM
+//    gets a split (30B MoE at 8192 tokens: 5.59 -> 5.42 ms per step against
+//    512-position splits).
+constexpr int kAttnShortSplit = 512;
+constexpr int kAttnLongCtx = 2048;
+constexpr int kAttnSplitTokens = 64;
 __device__ __forceinline__ int attn_active_splits(int n_ctx, int S) {
-    int a = (n_ctx + kAttnSplitTokens - 1) / kAttnSplitTokens;
+    const int per = n_ctx < kAttnLongCtx ? kAttnShortSplit : kAttnSplitTokens;
+    const int a = (n_ctx + per - 1) / per;
     return a < 1 ? 1 : (a > S ? S : a);
 }
 
