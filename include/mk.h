@@ -361,7 +361,7 @@ mk_status mk_prefill_seq(mk_state* state, const int32_t* tokens, int n_tokens, i
  * every rank's receive buffer (plain stores into peer memory) and raises that
  * tile's arrival flag on every rank (system-scope release); a reduce task per
  * tile on each rank waits for tp arrivals and adds the ranks' parts in rank
- * order, then the residual.  No multicast of any kind. */
+ * order, then the residual.  Only plain stores and reductions cross GPUs. */
 
 #define MK_TP_IPC_HANDLE_BYTES 64
 
